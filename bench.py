@@ -1,0 +1,407 @@
+#!/usr/bin/env python3
+"""Benchmark: all-reduce algbw / busbw and % of the HBM roofline for 8
+virtual ranks x 256 MiB fp32 on one B200 (per GPU; N GPUs run N independent
+copies of the workload, weak scaling).
+
+One step = one ``all_reduce`` call through the library's public API (algo
+AUTO, op AVG, in place) on 8 rank buffers of 64 Mi fp32 each: the chunk
+partition, the ring-order fold with AVG's division, and the store of the
+result to all 8 buffers.  Prints one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+``--impl reference`` times the CPU oracle (the plain ring all-reduce written
+from the pages) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "all-reduce algbw/busbw GB/s and % of HBM peak, 8 virtual ranks x 256 MB fp32"
+WORKLOAD = "allreduce-8x256MiB-f32"
+NRANKS = 8
+COUNT = 1 << 26  # fp32 elements per rank: 256 MiB
+ELEM = 4
+SEED = 0
+FALLBACK_HBM_GBS = 6650.0
+
+# DRAM traffic of one launch of the dominant kernel per algorithmic byte,
+# from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), with the
+# hash of the kernel sources it was taken on.  The summary with its command is
+# in profiles/oneshot_ring_kernel_allreduce-8x64MiB-f32.md.
+NCU_TRAFFIC = {"per_algorithmic_byte": None, "sources_sha1": None}
+
+
+def sources_sha1() -> str:
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "ring_all_reduce_virtual_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=8)
+    ap.add_argument("--cpu-seconds", type=float, default=8.0, help="CPU-baseline sample budget")
+    ap.add_argument("--no-extra", action="store_true", help="skip the per-algorithm extra timings")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------- plumbing --
+
+class Dist:
+    """Rank/world from the launcher's environment; NCCL only for the
+    barrier and the max over ranks of the measured time."""
+
+    def __init__(self):
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+
+    def init(self, backend: str):
+        import torch.distributed as dist
+
+        if self.world > 1 and not self.pg:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+            self.pg = True
+
+    def barrier(self):
+        if self.pg:
+            import torch.distributed as dist
+
+            dist.barrier()
+
+    def max(self, x: float, device) -> float:
+        if not self.pg:
+            return x
+        import torch
+        import torch.distributed as dist
+
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+            self.pg = False
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed
+    region."""
+
+    FIELDS = ["uuid", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, uuid: str | None):
+        self.uuid = self._norm(uuid)
+        self.proc = None
+        self.path = None
+
+    @staticmethod
+    def _norm(u) -> str:
+        u = str(u or "").lower()
+        return u[4:].replace("-", "") if u.startswith("gpu-") else u.replace("-", "")
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="rr_clocks_", suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) != len(self.FIELDS):
+                    continue
+                if self.uuid and self._norm(parts[0]) != self.uuid:
+                    continue
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- inputs --
+
+def host_inputs(rank_offset: int):
+    from ring_all_reduce_virtual_b200 import synth
+
+    return [synth.rank_values(SEED + rank_offset, r, COUNT, "normal", "f32") for r in range(NRANKS)]
+
+
+# ------------------------------------------------------------ cpu oracle --
+
+def cpu_baseline(budget_s: float):
+    """The oracle's ring all-reduce on a bounded sample (8 ranks x m fp32),
+    single-threaded and with each step's transfers on all host cores."""
+    import oracle
+    from ring_all_reduce_virtual_b200 import synth
+
+    m = 1 << 20
+    x = synth.ranks(SEED, NRANKS, m, "normal", "f32")
+    t0 = time.perf_counter()
+    oracle.ring_allreduce(x, "avg")
+    one = time.perf_counter() - t0
+    reps = max(1, int(budget_s / 2 / max(one, 1e-6)))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.ring_allreduce(x, "avg")
+    t1 = (time.perf_counter() - t0) / reps
+    cores = os.cpu_count() or 1
+    oracle.ring_allreduce_omp(x, "avg", cores)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.ring_allreduce_omp(x, "avg", cores)
+    tp = (time.perf_counter() - t0) / reps
+    S = m * ELEM
+    return {
+        "value": round(S / t1 / 1e9, 4), "unit": "GB/s (algbw)", "cores": 1, "kind": "oracle",
+        "sample": f"{reps} ring all-reduce calls (AVG) of {NRANKS} ranks x {m} fp32 ({S >> 20} MiB per rank), "
+                  f"single-threaded C oracle",
+        "parallel": {"value": round(S / tp / 1e9, 4), "cores": cores,
+                     "kind": "oracle, each step's N transfers on host threads (OpenMP)"},
+        "cpu_model": _cpu_model(),
+    }
+
+
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def run_reference(args, d: Dist):
+    """The reference arm: the CPU oracle, as it stands, on a bounded sample
+    of this workload per step (rank 0 only)."""
+    if d.rank != 0:
+        return
+    import oracle
+    from ring_all_reduce_virtual_b200 import synth
+
+    steps, warm = args.steps, args.warmup
+    m = 1 << 16
+    x = synth.ranks(SEED, NRANKS, m, "normal", "f32")
+    t0 = time.perf_counter()
+    oracle.ring_allreduce(x, "avg")
+    one = max(time.perf_counter() - t0, 1e-6)
+    budget = 90.0 / max(steps + warm, 1)  # whole run in about a minute and a half
+    m = int(min(COUNT, max(4096, m * budget / one)))
+    m -= m % NRANKS
+    x = synth.ranks(SEED, NRANKS, m, "normal", "f32")
+    for _ in range(warm):
+        oracle.ring_allreduce(x, "avg")
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle.ring_allreduce(x, "avg")
+    dt = (time.perf_counter() - t0) / max(steps, 1)
+    S = m * ELEM
+    algbw = S / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(algbw, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": steps, "warmup": warm, "ms_per_step": round(dt * 1e3, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic: normal(0, 1e-3) fp32 from numpy default_rng([seed, rank])",
+        "config": {"workload": WORKLOAD, "nranks_virtual": NRANKS, "count_per_rank": m,
+                   "sample_of_count_per_rank": COUNT, "op": "avg", "algo": "ring (CPU oracle)"},
+        "busbw": round(algbw * 2 * (NRANKS - 1) / NRANKS, 4),
+        "cpu_baseline": {"value": round(algbw, 4), "unit": "GB/s (algbw)", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: ring all-reduce (AVG) of {NRANKS} ranks x {m} fp32, "
+                                   f"single-threaded C oracle", "cpu_model": _cpu_model()},
+        "e2e": {"value": round(algbw, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ ours --
+
+def run_ours(args, d: Dist):
+    import torch
+
+    import ring_all_reduce_virtual_b200 as rrv
+    from ring_all_reduce_virtual_b200.build import build
+
+    if d.rank == 0:
+        build()
+    d.barrier()
+    torch.cuda.set_device(d.local_rank)
+    dev = torch.device("cuda", d.local_rank)
+    d.init("nccl")
+    stream = torch.cuda.current_stream(dev)
+
+    host = host_inputs(d.rank * NRANKS)
+    bufs = [torch.from_numpy(a).to(dev) for a in host]
+    S = COUNT * ELEM
+    alg_bytes = 2 * NRANKS * S  # one-shot: read N*S, write N*S
+
+    def step():
+        rrv.all_reduce(bufs, "avg", "auto", stream)
+
+    # warm-up, then exactly K timed steps between barriers and syncs
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    picked = rrv.last_stats()
+    clocks = Clocks(getattr(torch.cuda.get_device_properties(dev), "uuid", None))
+    clocks.start()
+    d.barrier()
+    torch.cuda.synchronize(dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    d.barrier()
+    clk = clocks.stop()
+    ms_local = ev0.elapsed_time(ev1) / max(args.steps, 1)
+    ms = d.max(ms_local, dev)
+    t = ms / 1e3
+    algbw = S / t / 1e9  # per GPU
+    value = algbw * d.world  # whole job: every GPU reduces its own 8 x 256 MiB
+    busbw = algbw * 2 * (NRANKS - 1) / NRANKS
+    achieved = alg_bytes / t / 1e9
+    peak, peak_kind = hbm_peak()
+    traffic = None
+    if NCU_TRAFFIC["per_algorithmic_byte"] and NCU_TRAFFIC["sources_sha1"] == sources_sha1():
+        traffic = int(NCU_TRAFFIC["per_algorithmic_byte"] * alg_bytes)
+
+    # end to end through the public API with host buffers: H2D + all-reduce + D2H
+    pinned = [torch.from_numpy(a).pin_memory() for a in host]
+    for _ in range(2):
+        rrv.all_reduce_host(pinned, bufs, "avg", "auto", stream)
+    torch.cuda.synchronize(dev)
+    d.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        rrv.all_reduce_host(pinned, bufs, "avg", "auto", stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    d.barrier()
+    e2e_ms = d.max(e0.elapsed_time(e1) / max(args.e2e_steps, 1), dev)
+    e2e = {"value": round(S / (e2e_ms / 1e3) / 1e9 * d.world, 3), "unit": "GB/s",
+           "h2d_bytes_per_step": NRANKS * S, "d2h_bytes_per_step": NRANKS * S,
+           "ms_per_step": round(e2e_ms, 3), "host_memory": "pinned"}
+
+    extra = {}
+    if not args.no_extra:
+        for name, op, algo, reps in (("oneshot_sum", "sum", "oneshot", 20), ("ring_sum", "sum", "ring", 10),
+                                     ("tree_oneshot_sum", "sum", "tree_oneshot", 10), ("tree_sum", "sum", "tree", 10)):
+            fresh = [torch.from_numpy(a).to(dev) for a in host]
+            rrv.all_reduce(fresh, op, algo, stream)
+            st = rrv.last_stats()
+            torch.cuda.synchronize(dev)
+            a0 = torch.cuda.Event(enable_timing=True)
+            a1 = torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for _ in range(reps):
+                rrv.all_reduce(fresh, op, algo, stream)
+            a1.record(stream)
+            torch.cuda.synchronize(dev)
+            tm = a0.elapsed_time(a1) / reps / 1e3
+            extra[name] = {"ms": round(tm * 1e3, 4), "algbw_gbs": round(S / tm / 1e9, 2),
+                           "hbm_gbs": round(st["hbm_bytes"] / tm / 1e9, 1),
+                           "hbm_frac": round(st["hbm_bytes"] / tm / 1e9 / peak, 4), "launches": st["launches"]}
+            del fresh
+
+    cpu = cpu_baseline(args.cpu_seconds) if (d.rank == 0 and d.world == 1) else None
+    if d.rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": d.world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic: normal(0, 1e-3) fp32 from numpy default_rng([seed, rank]), generated on the host",
+            "config": {"workload": WORKLOAD, "nranks_virtual": NRANKS, "count_per_rank": COUNT,
+                       "bytes_per_rank": S, "op": "avg", "algo": "auto -> " + str(picked["algo"]),
+                       "in_place": True, "value_is": "algbw = S / T summed over GPUs",
+                       "l2": "inputs 2 GiB per GPU > 126 MB L2; no flush needed"},
+            "algbw_per_gpu": round(algbw, 3), "busbw": round(busbw, 3),
+            "hbm_gbs": round(achieved, 1), "hbm_frac": round(achieved / peak, 4),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "kernel": "oneshot_ring_kernel<F32T, AVG>",
+                         "algorithmic_bytes_per_launch": alg_bytes, "peak_kind": peak_kind + " (burst copy)"},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": int(picked["launches"]) * args.steps,
+            "clocks": clk,
+            "extra": extra,
+        }
+        print(json.dumps(line), flush=True)
+    d.close()
+
+
+def main():
+    args = parse_args()
+    d = Dist()
+    if args.impl == "reference":
+        run_reference(args, d)
+        return
+    run_ours(args, d)
+
+
+if __name__ == "__main__":
+    main()

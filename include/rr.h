@@ -1,0 +1,269 @@
+/*
+ * rr.h -- C ABI of the ring all-reduce library for N virtual ranks on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * A "virtual rank" is one device buffer in the GPU's HBM.  The library runs
+ * the collectives that data-parallel training uses for gradient sync between
+ * N such buffers: the ring all-reduce (a reduce-scatter of N chunks over N-1
+ * ring steps, then an all-gather over N-1 steps), a fused one-shot all-reduce
+ * that gives the ring's bits in one pass, tree-order variants, standalone
+ * reduce-scatter, all-gather and all-to-all, and DDP-style gradient buckets.
+ *
+ * Sources (four web pages on ring all-reduce), cited by tag:
+ *   [P1] "How all-reduce keeps every card identical" (mhpq.cn, news 451051)
+ *   [P2] "AllReduce from principle to tuning" (xxqk.cn, news 376101)
+ *   [P3] "Training gradient sync and collective communication: from parameter
+ *        server to Ring AllReduce" (geek-doc.cn)
+ *   [P4] "Collective communication primitives" (ai-infra-handbooks,
+ *        train/basics/collectives)
+ *
+ * Conventions for every call below
+ *   - Pointers named bufs/send/recv/grads/buckets are HOST arrays of DEVICE
+ *     pointers, one per rank (nranks entries; grads has nranks*ntensors).
+ *     The library copies the pointer values into kernel parameters and does
+ *     not keep them.  The caller owns all device memory and the stream.
+ *   - No call allocates device memory or synchronises the host; work is
+ *     enqueued on `stream` and the call returns.  A CUDA launch error is
+ *     returned as RR_ERR_CUDA (detail in rr_last_error()).
+ *   - Argument errors are returned before anything is enqueued:
+ *     RR_ERR_INVALID_ARG for a NULL or repeated device pointer, nranks
+ *     outside 1..RR_MAX_RANKS, overlapping buffers, a bad enum or a count
+ *     that the operation cannot split; RR_ERR_UNSUPPORTED for a valid but
+ *     unsupported combination (AVG on int32).
+ *   - count == 0 is RR_OK and enqueues nothing.  Any pointer alignment is
+ *     accepted; buffers whose addresses agree modulo 16 bytes take the
+ *     128-bit vector path, the rest a scalar path.
+ *   - Chunking: chunk size C = ceil(count / N); chunk k is the element range
+ *     [k*C, min((k+1)*C, count)), possibly short or empty ([P4] "Ring
+ *     all-reduce and communication volume": the tensor is split with
+ *     tensor.chunk(n)).
+ *   - Reduction order ("ring order"): element i of chunk c = i / C reduces as
+ *     ((x_c[i] op x_{c+1}[i]) op x_{c+2}[i]) ... op x_{c+N-1}[i], rank indices
+ *     mod N, the partial on the left; this is the order in which the ring
+ *     schedule folds chunk c (its partial starts on rank c and gains one rank
+ *     per hop).  AVG is that SUM divided once by N.  MAX keeps the left
+ *     operand unless it is smaller, MIN unless it is larger.
+ *   - Precision: fp32 and bf16 reduce in fp32 ([P1] s5.3: reduce
+ *     low-precision gradients in fp32); bf16 results are rounded once to
+ *     nearest-even, except in the RING and TREE schedules, whose partials
+ *     live in the bf16 buffers between steps and are rounded at every hop.
+ *     int32 SUM and PROD wrap modulo 2^32.
+ */
+#ifndef RR_H_
+#define RR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RR_MAX_RANKS 64
+#define RR_VERSION 1
+
+typedef enum rr_status {
+    RR_OK = 0,
+    RR_ERR_INVALID_ARG = 1,
+    RR_ERR_UNSUPPORTED = 2,
+    RR_ERR_CUDA = 3,
+    RR_ERR_TIMEOUT = 4 /* reserved: no kernel of this library waits on another */
+} rr_status_t;
+
+/* Element types of the rank buffers. */
+typedef enum rr_dtype { RR_F32 = 0, RR_BF16 = 1, RR_I32 = 2 } rr_dtype_t;
+
+/* Reductions of [P1] s2.1: SUM, AVG (sum then divide by N), MAX, MIN, PROD. */
+typedef enum rr_op { RR_SUM = 0, RR_AVG = 1, RR_MAX = 2, RR_MIN = 3, RR_PROD = 4 } rr_op_t;
+
+/* Algorithms.
+ *   RING         the ring schedule: 2(N-1) launches, one per ring step
+ *                ([P4] "Ring all-reduce and communication volume"; [P3] s3)
+ *   ONESHOT      one launch that reads all N buffers once, folds in ring
+ *                order and writes the result to all N ([P4] "alpha-beta
+ *                model": one-shot reads every peer's buffer directly)
+ *   TREE         the tree schedule: ceil(log2 N) pairwise reduce levels,
+ *                then as many broadcast levels ([P3] s6)
+ *   TREE_ONESHOT one launch that folds in the tree's pairwise order
+ *   AUTO         the picker's choice between RING and ONESHOT (never a tree
+ *                order, whose bits differ); env RR_ALGO=ring|oneshot|tree|
+ *                tree_oneshot overrides it. */
+typedef enum rr_algo {
+    RR_ALGO_AUTO = 0,
+    RR_ALGO_RING = 1,
+    RR_ALGO_ONESHOT = 2,
+    RR_ALGO_TREE = 3,
+    RR_ALGO_TREE_ONESHOT = 4
+} rr_algo_t;
+
+/* The two phases of the ring ([P3] s3; [P4]). */
+typedef enum rr_phase { RR_PHASE_REDUCE_SCATTER = 0, RR_PHASE_ALL_GATHER = 1 } rr_phase_t;
+
+/* What the last call on this host thread did. */
+typedef struct rr_stats {
+    int32_t algo;              /* rr_algo_t that ran (never AUTO) */
+    int32_t steps;             /* communication steps: ring 2(N-1), tree 2 ceil(log2 N), one-shot 1 */
+    int32_t launches;          /* kernel launches enqueued */
+    int32_t nranks;
+    uint64_t bytes_per_rank;   /* S = count * element size */
+    uint64_t bytes_sent_max;   /* most bytes any one rank sent (ring: 2(N-1)/N*S when N | count) */
+    uint64_t bytes_sent_total; /* bytes sent by all ranks together */
+    uint64_t hbm_bytes;        /* algorithmic HBM bytes read + written by the kernels */
+} rr_stats_t;
+
+/* One transfer of the ring schedule: at (phase, step), `rank` sends chunk
+ * send_idx to its right neighbour dst and receives chunk recv_idx from its
+ * left neighbour; `bytes` is the size of the sent chunk. */
+typedef struct rr_ring_event {
+    int32_t phase;
+    int32_t step;
+    int32_t rank;
+    int32_t dst;
+    int32_t send_idx;
+    int32_t recv_idx;
+    uint64_t bytes;
+} rr_ring_event_t;
+
+/* Terms of the alpha-beta cost model ([P3] s4: T = 2(N-1) alpha +
+ * 2(N-1)/N M / beta for the ring; [P4] "alpha-beta model"). */
+typedef struct rr_cost {
+    double steps;       /* sequential steps, each paying alpha */
+    double bytes_sent;  /* bytes on the busiest rank's link */
+    double latency_s;   /* steps * alpha */
+    double bandwidth_s; /* bytes_sent / beta */
+    double total_s;     /* latency_s + bandwidth_s */
+} rr_cost_t;
+
+/* ---------------------------------------------------------------- calls -- */
+
+/* All-reduce in place over bufs[0..nranks): afterwards every buffer holds the
+ * reduction of all inputs, element by element ([P4] "The five primitives";
+ * [P1] s2.1).  count elements per rank.  Bits: RING, ONESHOT and AUTO give
+ * the ring order for fp32 and int32; for bf16, ONESHOT rounds once and RING
+ * rounds per hop.  TREE and TREE_ONESHOT give the tree order.  Buffers must
+ * not overlap.  nranks == 1 enqueues nothing. */
+rr_status_t rr_allreduce(void* const* bufs, int nranks, size_t count, rr_dtype_t dtype, rr_op_t op,
+                         rr_algo_t algo, cudaStream_t stream);
+
+/* All-reduce of HOST buffers through caller-provided device buffers: copies
+ * host_bufs[r] -> dev_bufs[r] (cudaMemcpyAsync on `stream`), runs
+ * rr_allreduce on dev_bufs, and copies the result back into every
+ * host_bufs[r].  Host buffers should be page-locked for the copies to be
+ * asynchronous.  Same arguments, results and errors as rr_allreduce; the
+ * device buffers must not overlap.  The host buffers hold the result once
+ * `stream` has been synchronised. */
+rr_status_t rr_allreduce_host(void* const* host_bufs, void* const* dev_bufs, int nranks, size_t count,
+                              rr_dtype_t dtype, rr_op_t op, rr_algo_t algo, cudaStream_t stream);
+
+/* One step of the ring schedule for all ranks at once (one launch), in place:
+ * reduce-scatter step s has every rank r fold chunk (r-s-1) mod N received
+ * from rank r-1 into its own copy (received partial on the left; AVG divides
+ * by N in step N-2); all-gather step s has every rank r overwrite chunk
+ * (r-s) mod N with rank r-1's copy ([P4] ring_allreduce.py; [P3] s3, the
+ * 4-GPU walkthrough).  step in 0..N-2.  Running the 2(N-1) steps in order is
+ * exactly rr_allreduce(..., RR_ALGO_RING). */
+rr_status_t rr_ring_step(void* const* bufs, int nranks, size_t count, rr_dtype_t dtype, rr_op_t op,
+                         rr_phase_t phase, int step, cudaStream_t stream);
+
+/* The ring schedule as data (host only): fills events[0..2(N-1)N) in the order
+ * phase, step, rank -- exactly the transfers rr_ring_step launches.  *nevents
+ * receives the number of events (also when capacity is too small, which
+ * returns RR_ERR_INVALID_ARG). */
+rr_status_t rr_ring_schedule(int nranks, size_t count, rr_dtype_t dtype, rr_ring_event_t* events,
+                             size_t capacity, size_t* nevents);
+
+/* Reduce-scatter ([P4] "The five primitives"; [P3] s6): send[p] holds
+ * nranks*recvcount elements; recv[r] receives chunk r reduced over all ranks
+ * in ring order (the fold of chunk r starts on rank r), so reduce-scatter
+ * followed by all-gather equals the all-reduce bit for bit.  algo: AUTO or
+ * ONESHOT (one launch).  recv buffers must not overlap the send buffers. */
+rr_status_t rr_reduce_scatter(const void* const* send, void* const* recv, int nranks, size_t recvcount,
+                              rr_dtype_t dtype, rr_op_t op, rr_algo_t algo, cudaStream_t stream);
+
+/* All-gather ([P4] "The five primitives"): recv[r][p*sendcount + i] =
+ * send[p][i] for every r and p.  algo: AUTO or ONESHOT (one launch: each
+ * input element read once, written N times). */
+rr_status_t rr_all_gather(const void* const* send, void* const* recv, int nranks, size_t sendcount,
+                          rr_dtype_t dtype, rr_algo_t algo, cudaStream_t stream);
+
+/* All-to-all ([P4] "The five primitives": rank r's p-th block goes to rank
+ * p, a transpose): recv[r][p*C + i] = send[p][r*C + i], C = count_per_peer;
+ * each buffer holds nranks*C elements.  Out of place, one launch. */
+rr_status_t rr_all_to_all(const void* const* send, void* const* recv, int nranks, size_t count_per_peer,
+                          rr_dtype_t dtype, cudaStream_t stream);
+
+/* --------------------------------------------------------------- buckets -- */
+
+/* Opaque bucket plan (host memory owned by the library). */
+typedef struct rr_bucket_plan rr_bucket_plan_t;
+
+/* DDP-style bucket plan ([P2] s3.3: gradients go into buckets in the order
+ * given, and a bucket is reduced once it reaches the threshold; [P1] s5.2:
+ * bucket_cap_mb, default 25).  Greedy over numels[0..ntensors) in the order
+ * given, never splitting a tensor: each tensor joins the open bucket, which
+ * closes as soon as its bytes (in grad_dtype) reach cap_bytes.  grad_dtype is
+ * RR_BF16 or RR_F32; buckets are fp32.  Host only; free with
+ * rr_bucket_plan_free. */
+rr_status_t rr_bucket_plan(const size_t* numels, int ntensors, rr_dtype_t grad_dtype, size_t cap_bytes,
+                           rr_bucket_plan_t** out);
+void rr_bucket_plan_free(rr_bucket_plan_t* plan);
+
+/* Plan queries (host only).  rr_bucket_info gives a bucket's first tensor,
+ * its number of tensors and its length in fp32 elements; rr_bucket_tensor
+ * gives a tensor's bucket and its element offset inside it. */
+int rr_bucket_count(const rr_bucket_plan_t* plan);
+rr_status_t rr_bucket_info(const rr_bucket_plan_t* plan, int bucket, int* first_tensor, int* ntensors,
+                           size_t* numel);
+rr_status_t rr_bucket_tensor(const rr_bucket_plan_t* plan, int tensor, int* bucket, size_t* offset);
+
+/* Pack one bucket for every rank: buckets[r][offset(t) + j] = fp32(grads[r *
+ * ntensors + t][j]) for each tensor t of the bucket (exact widening).  grads
+ * holds nranks*ntensors device pointers (entries of tensors outside the
+ * bucket are ignored); buckets holds nranks fp32 buffers of at least the
+ * bucket's numel.  One launch. */
+rr_status_t rr_bucket_pack(const rr_bucket_plan_t* plan, int bucket, const void* const* grads,
+                           void* const* buckets, int nranks, cudaStream_t stream);
+
+/* Unpack one reduced bucket: grads[r * ntensors + t][j] =
+ * round(buckets[r][offset(t) + j] / N) for AVG (no division for SUM), one
+ * round-to-nearest-even to the gradient dtype.  One launch. */
+rr_status_t rr_bucket_unpack(const rr_bucket_plan_t* plan, int bucket, const void* const* buckets,
+                             void* const* grads, int nranks, rr_op_t op, cudaStream_t stream);
+
+/* Fused bucket sync: reduces one bucket's gradients across ranks in place,
+ * with the bits of pack -> rr_allreduce(SUM, ring order over the bucket's
+ * flat index) -> unpack(op), but reading and writing each gradient once
+ * (4 bytes per bf16 parameter per rank instead of 20).  op: SUM or AVG.
+ * One launch. */
+rr_status_t rr_bucket_allreduce(const rr_bucket_plan_t* plan, int bucket, void* const* grads,
+                                int nranks, rr_op_t op, cudaStream_t stream);
+
+/* ----------------------------------------------------- picker and model -- */
+
+/* The alpha-beta model of one algorithm for N ranks and M bytes per rank
+ * ([P3] s4-s6; [P4] "alpha-beta model"): RING 2(N-1) steps moving 2(N-1)/N M
+ * per rank; TREE 2 ceil(log2 N) steps each moving M; ONESHOT 1 step in which
+ * each rank reads (N-1) M.  alpha in seconds, beta in bytes/second. */
+rr_status_t rr_cost_model(rr_algo_t algo, int nranks, double bytes_per_rank, double alpha_s,
+                          double beta_bytes_per_s, rr_cost_t* out);
+
+/* The algorithm AUTO runs for this call shape (RING or ONESHOT), from the
+ * same model applied to one GPU's launch cost and HBM traffic, with the
+ * parameters set by rr_set_picker_params (defaults: 4 us, 6.5 TB/s). */
+rr_algo_t rr_pick_algo(int nranks, size_t count, rr_dtype_t dtype);
+rr_status_t rr_set_picker_params(double launch_s, double hbm_bytes_per_s);
+
+/* ------------------------------------------------------------ utilities -- */
+
+rr_status_t rr_get_stats(rr_stats_t* out); /* last call on this host thread */
+const char* rr_status_string(rr_status_t status);
+const char* rr_last_error(void); /* detail of the last failure on this thread */
+int rr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RR_H_ */

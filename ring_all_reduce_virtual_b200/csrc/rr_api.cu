@@ -1,0 +1,841 @@
+// rr_api.cu -- the C ABI (include/rr.h): argument checks, the ring and tree
+// schedules as launch tables, the per-size picker, bucket plans, call
+// statistics.  Host code only; every data movement runs in the kernels.
+//
+// Sources, cited by tag in the comments below:
+//   [P1] "How all-reduce keeps every card identical" (mhpq.cn, news 451051)
+//   [P2] "AllReduce from principle to tuning" (xxqk.cn, news 376101)
+//   [P3] "Training gradient sync and collective communication: from parameter
+//        server to Ring AllReduce" (geek-doc.cn)
+//   [P4] "Collective communication primitives" (ai-infra-handbooks)
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "rr.h"
+#include "rr_internal.h"
+
+using namespace rr;
+
+struct rr_bucket_plan {
+    int ntensors = 0;
+    int grad_dtype = RR_BF16;
+    size_t cap_bytes = 0;
+    std::vector<uint64_t> numel;   // per tensor
+    std::vector<uint64_t> offset;  // per tensor: element offset in its bucket
+    std::vector<int> bucket_of;    // per tensor
+    std::vector<int> first;        // per bucket: first tensor
+    std::vector<int> count;        // per bucket: number of tensors
+    std::vector<uint64_t> bnumel;  // per bucket: elements
+};
+
+namespace {
+
+thread_local rr_stats_t t_stats{};
+thread_local std::string t_error;
+
+double g_launch_s = 4e-6;         // picker: cost of one launch
+double g_hbm_bps = 6.5e12;        // picker: effective HBM bytes/s
+
+rr_status_t fail(rr_status_t st, const std::string& why)
+{
+    t_error = why;
+    return st;
+}
+
+rr_status_t cuda_fail(cudaError_t e, const char* where)
+{
+    t_error = std::string(where) + ": " + cudaGetErrorString(e);
+    return RR_ERR_CUDA;
+}
+
+bool env_flag(const char* name)
+{
+    const char* v = std::getenv(name);
+    return v && *v && std::strcmp(v, "0") != 0;
+}
+
+size_t esize(rr_dtype_t d) { return d == RR_BF16 ? 2u : 4u; }
+
+bool dtype_ok(rr_dtype_t d) { return d == RR_F32 || d == RR_BF16 || d == RR_I32; }
+bool op_ok(rr_op_t o) { return o >= RR_SUM && o <= RR_PROD; }
+
+const char* algo_name(int a)
+{
+    switch (a) {
+    case RR_ALGO_AUTO: return "auto";
+    case RR_ALGO_RING: return "ring";
+    case RR_ALGO_ONESHOT: return "oneshot";
+    case RR_ALGO_TREE: return "tree";
+    case RR_ALGO_TREE_ONESHOT: return "tree_oneshot";
+    }
+    return "?";
+}
+
+// Common checks of dtype, op and rank count.
+rr_status_t check_basic(int n, rr_dtype_t dtype, rr_op_t op)
+{
+    if (n < 1 || n > RR_MAX_RANKS) return fail(RR_ERR_INVALID_ARG, "nranks must be in 1..64");
+    if (!dtype_ok(dtype)) return fail(RR_ERR_INVALID_ARG, "unknown dtype");
+    if (!op_ok(op)) return fail(RR_ERR_INVALID_ARG, "unknown op");
+    if (dtype == RR_I32 && op == RR_AVG) return fail(RR_ERR_UNSUPPORTED, "AVG is not defined for int32");
+    return RR_OK;
+}
+
+struct Span {
+    uintptr_t lo, hi;
+    bool out;
+};
+
+// Every output span must be non-NULL and overlap no other span; inputs may
+// overlap one another (they are only read).
+rr_status_t check_spans(std::vector<Span>& s)
+{
+    for (const Span& a : s)
+        if (a.lo == 0) return fail(RR_ERR_INVALID_ARG, "NULL buffer pointer");
+    std::sort(s.begin(), s.end(), [](const Span& a, const Span& b) { return a.lo < b.lo; });
+    for (size_t i = 0; i < s.size(); ++i)
+        for (size_t j = i + 1; j < s.size() && s[j].lo < s[i].hi; ++j)
+            if (s[i].out || s[j].out) return fail(RR_ERR_INVALID_ARG, "buffers overlap (or repeat)");
+    return RR_OK;
+}
+
+// True when all pointers agree modulo 16 bytes.
+bool same_phase(const void* const* p, int n)
+{
+    for (int i = 1; i < n; ++i)
+        if (((uintptr_t)p[i] & 15u) != ((uintptr_t)p[0] & 15u)) return false;
+    return true;
+}
+
+// Optional (RR_DEBUG=1): reject pointers the driver does not know as device
+// or managed memory, before any launch.
+rr_status_t check_device_ptrs(const void* const* p, int n)
+{
+    if (!env_flag("RR_DEBUG")) return RR_OK;
+    for (int i = 0; i < n; ++i) {
+        cudaPointerAttributes a{};
+        if (cudaPointerGetAttributes(&a, p[i]) != cudaSuccess ||
+            (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)) {
+            cudaGetLastError();
+            return fail(RR_ERR_INVALID_ARG, "pointer is not device memory");
+        }
+    }
+    return RR_OK;
+}
+
+uint64_t ceil_div(uint64_t a, uint64_t b) { return b ? (a + b - 1) / b : 0; }
+
+uint64_t chunk_len(uint64_t count, int n, int k)
+{
+    const uint64_t C = ceil_div(count, (uint64_t)n), lo = (uint64_t)k * C;
+    if (lo >= count) return 0;
+    return std::min(C, count - lo);
+}
+
+int imod(int a, int n) { return ((a % n) + n) % n; }
+
+// Ring schedule ([P4] "Ring all-reduce and communication volume",
+// ring_allreduce.py; [P3] section 3, steps 1-2 of the 4-GPU walkthrough):
+// at reduce-scatter step s rank r sends chunk (r - s) and receives chunk
+// (r - s - 1) from its left neighbour; at all-gather step s it sends
+// (r + 1 - s) and receives (r - s).
+int ring_send_chunk(int phase, int r, int s, int n)
+{
+    return phase == RR_PHASE_REDUCE_SCATTER ? imod(r - s, n) : imod(r + 1 - s, n);
+}
+
+void log_call(const char* what, int n, size_t count, rr_dtype_t dtype, int op, int algo)
+{
+    static const bool on = env_flag("RR_LOG");
+    if (on)
+        std::fprintf(stderr, "[rr] %s nranks=%d count=%zu dtype=%d op=%d algo=%s launches=%d\n", what, n,
+                     count, (int)dtype, op, algo_name(algo), t_stats.launches);
+}
+
+void stats_begin(int algo, int n, uint64_t S)
+{
+    t_stats = rr_stats_t{};
+    t_stats.algo = algo;
+    t_stats.nranks = n;
+    t_stats.bytes_per_rank = S;
+}
+
+// Build and launch one ring step (all ranks at once).
+rr_status_t ring_step_launch(void* const* bufs, int n, size_t count, rr_dtype_t dtype, rr_op_t op, int phase,
+                             int step, cudaStream_t stream)
+{
+    const size_t es = esize(dtype);
+    const uint64_t C = ceil_div(count, (uint64_t)n);
+    StepParams p{};
+    p.nseg = n;
+    p.nin = phase == RR_PHASE_REDUCE_SCATTER ? 2 : 1;
+    p.vec_ok = same_phase(bufs, n);
+    p.divisor = (float)n;
+    uint64_t maxlen = 0;
+    for (int r = 0; r < n; ++r) {
+        const int left = imod(r - 1, n);
+        const int k = ring_send_chunk(phase, left, step, n);  // the chunk r receives
+        const uint64_t lo = (uint64_t)k * C, len = chunk_len(count, n, k);
+        p.seg[r].in0 = static_cast<const char*>(bufs[left]) + lo * es;
+        p.seg[r].in1 = p.nin == 2 ? static_cast<const char*>(bufs[r]) + lo * es : nullptr;
+        p.seg[r].out = static_cast<char*>(bufs[r]) + lo * es;
+        p.seg[r].len = len;
+        maxlen = std::max(maxlen, len);
+    }
+    p.tps = std::max<uint64_t>(1, ceil_div(maxlen, tile_elems(dtype)));
+    // AVG divides once, in the step that completes each chunk's fold
+    int op_eff = op;
+    if (op == RR_AVG && !(phase == RR_PHASE_REDUCE_SCATTER && step == n - 2)) op_eff = RR_SUM;
+    if (maxlen == 0) return RR_OK;
+    cudaError_t e = launch_step(dtype, op_eff, p, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "ring step launch");
+    t_stats.launches += 1;
+    return RR_OK;
+}
+
+rr_status_t run_ring(void* const* bufs, int n, size_t count, rr_dtype_t dtype, rr_op_t op, cudaStream_t stream)
+{
+    const size_t es = esize(dtype);
+    std::vector<uint64_t> sent(n, 0);
+    for (int phase = RR_PHASE_REDUCE_SCATTER; phase <= RR_PHASE_ALL_GATHER; ++phase)
+        for (int s = 0; s < n - 1; ++s) {
+            rr_status_t st = ring_step_launch(bufs, n, count, dtype, op, phase, s, stream);
+            if (st != RR_OK) return st;
+            for (int r = 0; r < n; ++r) sent[r] += chunk_len(count, n, ring_send_chunk(phase, r, s, n)) * es;
+        }
+    t_stats.steps = 2 * (n - 1);
+    for (int r = 0; r < n; ++r) {
+        t_stats.bytes_sent_max = std::max<uint64_t>(t_stats.bytes_sent_max, sent[r]);
+        t_stats.bytes_sent_total += sent[r];
+    }
+    // each reduce-scatter step reads 2 and writes 1 chunk per rank, each
+    // all-gather step reads and writes 1: 5 (N-1) S in all
+    t_stats.hbm_bytes = 5ull * (uint64_t)(n - 1) * count * es;
+    return RR_OK;
+}
+
+int tree_levels(int n)
+{
+    int l = 0;
+    while ((1 << l) < n) ++l;
+    return l;
+}
+
+// Tree schedule ([P3] section 6): pairwise reduce levels up to rank 0, then
+// broadcast levels back down.
+rr_status_t run_tree(void* const* bufs, int n, size_t count, rr_dtype_t dtype, rr_op_t op, cudaStream_t stream)
+{
+    const size_t es = esize(dtype);
+    const int L = tree_levels(n);
+    const bool vec = same_phase(bufs, n);
+    std::vector<uint64_t> sent(n, 0);
+    uint64_t pairs_total = 0;
+    for (int pass = 0; pass < 2; ++pass) {
+        for (int i = 0; i < L; ++i) {
+            const int l = pass == 0 ? i : L - 1 - i;
+            const int h = 1 << l;
+            StepParams p{};
+            p.nin = pass == 0 ? 2 : 1;
+            p.vec_ok = vec;
+            p.divisor = (float)n;
+            p.tps = std::max<uint64_t>(1, ceil_div(count, tile_elems(dtype)));
+            for (int a = 0; a + h < n; a += 2 * h) {
+                StepSeg& sg = p.seg[p.nseg++];
+                if (pass == 0) {  // x_a <- x_a op x_{a+h}
+                    sg.in0 = bufs[a];
+                    sg.in1 = bufs[a + h];
+                    sg.out = bufs[a];
+                    sent[a + h] += count * es;
+                } else {          // x_{a+h} <- x_a
+                    sg.in0 = bufs[a];
+                    sg.out = bufs[a + h];
+                    sent[a] += count * es;
+                }
+                sg.len = count;
+                ++pairs_total;
+            }
+            int op_eff = op;
+            if (op == RR_AVG && !(pass == 0 && l == L - 1)) op_eff = RR_SUM;
+            cudaError_t e = launch_step(dtype, op_eff, p, stream);
+            if (e != cudaSuccess) return cuda_fail(e, "tree level launch");
+            t_stats.launches += 1;
+        }
+    }
+    t_stats.steps = 2 * L;
+    for (int r = 0; r < n; ++r) {
+        t_stats.bytes_sent_max = std::max<uint64_t>(t_stats.bytes_sent_max, sent[r]);
+        t_stats.bytes_sent_total += sent[r];
+    }
+    // reduce: 3 S per pair, broadcast: 2 S per pair, N-1 pairs each way
+    t_stats.hbm_bytes = 5ull * (pairs_total / 2) * count * es;
+    return RR_OK;
+}
+
+rr_status_t run_rank_kernel(int kind, const void* const* in, void* const* out, int n, uint64_t C,
+                            uint64_t count, uint64_t nseg, uint64_t tps, rr_dtype_t dtype, int op, bool vec,
+                            cudaStream_t stream)
+{
+    RankParams p{};
+    for (int r = 0; r < n; ++r) {
+        p.in[r] = in[r];
+        p.out[r] = out[r];
+    }
+    p.n = n;
+    p.vec_ok = vec;
+    p.divisor = (float)n;
+    p.C = C;
+    p.count = count;
+    p.nseg = nseg;
+    p.tps = tps;
+    cudaError_t e = launch_rank_kernel(kind, dtype, op, p, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    t_stats.launches += 1;
+    return RR_OK;
+}
+
+rr_algo_t resolve_algo(rr_algo_t algo, int n, size_t count, rr_dtype_t dtype)
+{
+    if (algo != RR_ALGO_AUTO) return algo;
+    static const int forced = [] {
+        const char* v = std::getenv("RR_ALGO");
+        if (!v) return -1;
+        if (!std::strcmp(v, "ring")) return (int)RR_ALGO_RING;
+        if (!std::strcmp(v, "oneshot")) return (int)RR_ALGO_ONESHOT;
+        if (!std::strcmp(v, "tree")) return (int)RR_ALGO_TREE;
+        if (!std::strcmp(v, "tree_oneshot")) return (int)RR_ALGO_TREE_ONESHOT;
+        return -1;
+    }();
+    if (forced >= 0) return (rr_algo_t)forced;
+    return rr_pick_algo(n, count, dtype);
+}
+
+}  // namespace
+
+// ================================================================ C ABI ==
+
+extern "C" {
+
+int rr_version(void) { return RR_VERSION; }
+
+const char* rr_status_string(rr_status_t s)
+{
+    switch (s) {
+    case RR_OK: return "ok";
+    case RR_ERR_INVALID_ARG: return "invalid argument";
+    case RR_ERR_UNSUPPORTED: return "unsupported";
+    case RR_ERR_CUDA: return "CUDA error";
+    case RR_ERR_TIMEOUT: return "timeout";
+    }
+    return "unknown status";
+}
+
+const char* rr_last_error(void) { return t_error.c_str(); }
+
+rr_status_t rr_get_stats(rr_stats_t* out)
+{
+    if (!out) return fail(RR_ERR_INVALID_ARG, "NULL stats pointer");
+    *out = t_stats;
+    return RR_OK;
+}
+
+rr_status_t rr_allreduce(void* const* bufs, int nranks, size_t count, rr_dtype_t dtype, rr_op_t op,
+                         rr_algo_t algo, cudaStream_t stream)
+{
+    rr_status_t st = check_basic(nranks, dtype, op);
+    if (st != RR_OK) return st;
+    if (algo < RR_ALGO_AUTO || algo > RR_ALGO_TREE_ONESHOT) return fail(RR_ERR_INVALID_ARG, "unknown algo");
+    if (!bufs) return fail(RR_ERR_INVALID_ARG, "NULL bufs array");
+    const int n = nranks;
+    const size_t es = esize(dtype);
+    const rr_algo_t a = resolve_algo(algo, n, count, dtype);
+    stats_begin(a, n, (uint64_t)count * es);
+    if (count == 0) return RR_OK;
+    std::vector<Span> spans;
+    for (int r = 0; r < n; ++r)
+        spans.push_back({(uintptr_t)bufs[r], (uintptr_t)bufs[r] + count * es, true});
+    if ((st = check_spans(spans)) != RR_OK) return st;
+    if ((st = check_device_ptrs(bufs, n)) != RR_OK) return st;
+    if (n == 1) return RR_OK;  // one rank already holds the reduction (AVG: x / 1 == x)
+    const uint64_t S = (uint64_t)count * es;
+    switch (a) {
+    case RR_ALGO_RING:
+        st = run_ring(bufs, n, count, dtype, op, stream);
+        break;
+    case RR_ALGO_TREE:
+        st = run_tree(bufs, n, count, dtype, op, stream);
+        break;
+    case RR_ALGO_ONESHOT: {
+        const uint64_t C = ceil_div(count, (uint64_t)n);
+        const uint64_t tps = std::max<uint64_t>(1, ceil_div(C, tile_elems(dtype)));
+        st = run_rank_kernel(kOneshotRing, bufs, bufs, n, C, count, (uint64_t)n, tps, dtype, op,
+                             same_phase(bufs, n), stream);
+        t_stats.steps = 1;
+        t_stats.bytes_sent_max = (uint64_t)(n - 1) * S;  // each buffer is read by N-1 peers
+        t_stats.bytes_sent_total = (uint64_t)n * (n - 1) * S;
+        t_stats.hbm_bytes = 2ull * n * S;
+        break;
+    }
+    case RR_ALGO_TREE_ONESHOT: {
+        const uint64_t tps = std::max<uint64_t>(1, ceil_div(count, tile_elems(dtype)));
+        st = run_rank_kernel(kOneshotTree, bufs, bufs, n, count, count, 1, tps, dtype, op, same_phase(bufs, n),
+                             stream);
+        t_stats.steps = 1;
+        t_stats.bytes_sent_max = (uint64_t)(n - 1) * S;
+        t_stats.bytes_sent_total = (uint64_t)n * (n - 1) * S;
+        t_stats.hbm_bytes = 2ull * n * S;
+        break;
+    }
+    default:
+        return fail(RR_ERR_INVALID_ARG, "unknown algo");
+    }
+    log_call("allreduce", n, count, dtype, op, a);
+    return st;
+}
+
+rr_status_t rr_allreduce_host(void* const* host_bufs, void* const* dev_bufs, int nranks, size_t count,
+                              rr_dtype_t dtype, rr_op_t op, rr_algo_t algo, cudaStream_t stream)
+{
+    rr_status_t st = check_basic(nranks, dtype, op);
+    if (st != RR_OK) return st;
+    if (!host_bufs || !dev_bufs) return fail(RR_ERR_INVALID_ARG, "NULL pointer array");
+    const size_t bytes = count * esize(dtype);
+    for (int r = 0; r < nranks && count; ++r)
+        if (!host_bufs[r]) return fail(RR_ERR_INVALID_ARG, "NULL host buffer");
+    std::vector<Span> spans;
+    for (int r = 0; r < nranks && count; ++r)
+        spans.push_back({(uintptr_t)dev_bufs[r], (uintptr_t)dev_bufs[r] + bytes, true});
+    if ((st = check_spans(spans)) != RR_OK) return st;
+    if (count == 0) return rr_allreduce(dev_bufs, nranks, 0, dtype, op, algo, stream);
+    for (int r = 0; r < nranks; ++r) {
+        cudaError_t e = cudaMemcpyAsync(dev_bufs[r], host_bufs[r], bytes, cudaMemcpyHostToDevice, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+    }
+    if ((st = rr_allreduce(dev_bufs, nranks, count, dtype, op, algo, stream)) != RR_OK) return st;
+    for (int r = 0; r < nranks; ++r) {
+        cudaError_t e = cudaMemcpyAsync(host_bufs[r], dev_bufs[r], bytes, cudaMemcpyDeviceToHost, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+    }
+    return RR_OK;
+}
+
+rr_status_t rr_ring_step(void* const* bufs, int nranks, size_t count, rr_dtype_t dtype, rr_op_t op,
+                         rr_phase_t phase, int step, cudaStream_t stream)
+{
+    rr_status_t st = check_basic(nranks, dtype, op);
+    if (st != RR_OK) return st;
+    if (phase != RR_PHASE_REDUCE_SCATTER && phase != RR_PHASE_ALL_GATHER)
+        return fail(RR_ERR_INVALID_ARG, "unknown phase");
+    if (step < 0 || step > nranks - 2) return fail(RR_ERR_INVALID_ARG, "step must be in 0..nranks-2");
+    if (!bufs) return fail(RR_ERR_INVALID_ARG, "NULL bufs array");
+    const size_t es = esize(dtype);
+    stats_begin(RR_ALGO_RING, nranks, (uint64_t)count * es);
+    if (count == 0) return RR_OK;
+    std::vector<Span> spans;
+    for (int r = 0; r < nranks; ++r)
+        spans.push_back({(uintptr_t)bufs[r], (uintptr_t)bufs[r] + count * es, true});
+    if ((st = check_spans(spans)) != RR_OK) return st;
+    if ((st = check_device_ptrs(bufs, nranks)) != RR_OK) return st;
+    st = ring_step_launch(bufs, nranks, count, dtype, op, phase, step, stream);
+    t_stats.steps = 1;
+    for (int r = 0; r < nranks; ++r) {
+        const uint64_t b = chunk_len(count, nranks, ring_send_chunk(phase, r, step, nranks)) * es;
+        t_stats.bytes_sent_max = std::max(t_stats.bytes_sent_max, b);
+        t_stats.bytes_sent_total += b;
+    }
+    t_stats.hbm_bytes = (phase == RR_PHASE_REDUCE_SCATTER ? 3ull : 2ull) * count * es;
+    log_call("ring_step", nranks, count, dtype, op, RR_ALGO_RING);
+    return st;
+}
+
+rr_status_t rr_ring_schedule(int nranks, size_t count, rr_dtype_t dtype, rr_ring_event_t* events,
+                             size_t capacity, size_t* nevents)
+{
+    if (nranks < 1 || nranks > RR_MAX_RANKS) return fail(RR_ERR_INVALID_ARG, "nranks must be in 1..64");
+    if (!dtype_ok(dtype)) return fail(RR_ERR_INVALID_ARG, "unknown dtype");
+    const int n = nranks;
+    const size_t total = 2ull * (size_t)(n - 1) * (size_t)n;
+    if (nevents) *nevents = total;
+    if (total > capacity || (total && !events)) return fail(RR_ERR_INVALID_ARG, "events capacity too small");
+    size_t i = 0;
+    for (int phase = RR_PHASE_REDUCE_SCATTER; phase <= RR_PHASE_ALL_GATHER; ++phase)
+        for (int s = 0; s < n - 1; ++s)
+            for (int r = 0; r < n; ++r) {
+                rr_ring_event_t& e = events[i++];
+                e.phase = phase;
+                e.step = s;
+                e.rank = r;
+                e.dst = imod(r + 1, n);
+                e.send_idx = ring_send_chunk(phase, r, s, n);
+                e.recv_idx = ring_send_chunk(phase, imod(r - 1, n), s, n);
+                e.bytes = chunk_len(count, n, e.send_idx) * esize(dtype);
+            }
+    return RR_OK;
+}
+
+rr_status_t rr_reduce_scatter(const void* const* send, void* const* recv, int nranks, size_t recvcount,
+                              rr_dtype_t dtype, rr_op_t op, rr_algo_t algo, cudaStream_t stream)
+{
+    rr_status_t st = check_basic(nranks, dtype, op);
+    if (st != RR_OK) return st;
+    if (algo != RR_ALGO_AUTO && algo != RR_ALGO_ONESHOT)
+        return fail(RR_ERR_UNSUPPORTED, "reduce-scatter runs AUTO or ONESHOT");
+    if (!send || !recv) return fail(RR_ERR_INVALID_ARG, "NULL pointer array");
+    const int n = nranks;
+    const size_t es = esize(dtype);
+    const uint64_t S = (uint64_t)n * recvcount * es;
+    stats_begin(RR_ALGO_ONESHOT, n, S);
+    if (recvcount == 0) return RR_OK;
+    std::vector<Span> spans;
+    for (int r = 0; r < n; ++r) {
+        spans.push_back({(uintptr_t)send[r], (uintptr_t)send[r] + S, false});
+        spans.push_back({(uintptr_t)recv[r], (uintptr_t)recv[r] + recvcount * es, true});
+    }
+    if ((st = check_spans(spans)) != RR_OK) return st;
+    if ((st = check_device_ptrs(send, n)) != RR_OK || (st = check_device_ptrs(recv, n)) != RR_OK) return st;
+    const uint64_t tps = std::max<uint64_t>(1, ceil_div(recvcount, tile_elems(dtype)));
+    st = run_rank_kernel(kReduceScatter, send, recv, n, recvcount, (uint64_t)n * recvcount, (uint64_t)n, tps,
+                         dtype, op, same_phase(send, n) && same_phase(recv, n), stream);
+    t_stats.steps = 1;
+    t_stats.bytes_sent_max = (uint64_t)(n - 1) * recvcount * es;  // (N-1)/N S ([P4])
+    t_stats.bytes_sent_total = (uint64_t)n * t_stats.bytes_sent_max;
+    t_stats.hbm_bytes = (uint64_t)(n + 1) * S;
+    log_call("reduce_scatter", n, recvcount, dtype, op, RR_ALGO_ONESHOT);
+    return st;
+}
+
+rr_status_t rr_all_gather(const void* const* send, void* const* recv, int nranks, size_t sendcount,
+                          rr_dtype_t dtype, rr_algo_t algo, cudaStream_t stream)
+{
+    rr_status_t st = check_basic(nranks, dtype, RR_SUM);
+    if (st != RR_OK) return st;
+    if (algo != RR_ALGO_AUTO && algo != RR_ALGO_ONESHOT)
+        return fail(RR_ERR_UNSUPPORTED, "all-gather runs AUTO or ONESHOT");
+    if (!send || !recv) return fail(RR_ERR_INVALID_ARG, "NULL pointer array");
+    const int n = nranks;
+    const size_t es = esize(dtype);
+    const uint64_t S = (uint64_t)n * sendcount * es;
+    stats_begin(RR_ALGO_ONESHOT, n, S);
+    if (sendcount == 0) return RR_OK;
+    std::vector<Span> spans;
+    for (int r = 0; r < n; ++r) {
+        spans.push_back({(uintptr_t)send[r], (uintptr_t)send[r] + sendcount * es, false});
+        spans.push_back({(uintptr_t)recv[r], (uintptr_t)recv[r] + S, true});
+    }
+    if ((st = check_spans(spans)) != RR_OK) return st;
+    if ((st = check_device_ptrs(send, n)) != RR_OK || (st = check_device_ptrs(recv, n)) != RR_OK) return st;
+    const uint64_t tps = std::max<uint64_t>(1, ceil_div(sendcount, tile_elems(dtype)));
+    st = run_rank_kernel(kAllGather, send, recv, n, sendcount, (uint64_t)n * sendcount, (uint64_t)n, tps, dtype,
+                         RR_SUM, same_phase(send, n) && same_phase(recv, n), stream);
+    t_stats.steps = 1;
+    t_stats.bytes_sent_max = (uint64_t)(n - 1) * sendcount * es;
+    t_stats.bytes_sent_total = (uint64_t)n * t_stats.bytes_sent_max;
+    t_stats.hbm_bytes = (uint64_t)(n + 1) * S;
+    log_call("all_gather", n, sendcount, dtype, RR_SUM, RR_ALGO_ONESHOT);
+    return st;
+}
+
+rr_status_t rr_all_to_all(const void* const* send, void* const* recv, int nranks, size_t count_per_peer,
+                          rr_dtype_t dtype, cudaStream_t stream)
+{
+    rr_status_t st = check_basic(nranks, dtype, RR_SUM);
+    if (st != RR_OK) return st;
+    if (!send || !recv) return fail(RR_ERR_INVALID_ARG, "NULL pointer array");
+    const int n = nranks;
+    const size_t es = esize(dtype);
+    const uint64_t S = (uint64_t)n * count_per_peer * es;
+    stats_begin(RR_ALGO_ONESHOT, n, S);
+    if (count_per_peer == 0) return RR_OK;
+    std::vector<Span> spans;
+    for (int r = 0; r < n; ++r) {
+        spans.push_back({(uintptr_t)send[r], (uintptr_t)send[r] + S, false});
+        spans.push_back({(uintptr_t)recv[r], (uintptr_t)recv[r] + S, true});
+    }
+    if ((st = check_spans(spans)) != RR_OK) return st;
+    if ((st = check_device_ptrs(send, n)) != RR_OK || (st = check_device_ptrs(recv, n)) != RR_OK) return st;
+    const uint64_t tps = std::max<uint64_t>(1, ceil_div(count_per_peer, tile_elems(dtype)));
+    st = run_rank_kernel(kAllToAll, send, recv, n, count_per_peer, (uint64_t)n * count_per_peer,
+                         (uint64_t)n * n, tps, dtype, RR_SUM, true, stream);
+    t_stats.steps = 1;
+    t_stats.bytes_sent_max = (uint64_t)(n - 1) * count_per_peer * es;  // own block stays ([P4])
+    t_stats.bytes_sent_total = (uint64_t)n * t_stats.bytes_sent_max;
+    t_stats.hbm_bytes = 2ull * n * S;
+    log_call("all_to_all", n, count_per_peer, dtype, RR_SUM, RR_ALGO_ONESHOT);
+    return st;
+}
+
+// ------------------------------------------------------------- buckets --
+
+rr_status_t rr_bucket_plan(const size_t* numels, int ntensors, rr_dtype_t grad_dtype, size_t cap_bytes,
+                           rr_bucket_plan_t** out)
+{
+    if (!out) return fail(RR_ERR_INVALID_ARG, "NULL plan output");
+    *out = nullptr;
+    if (ntensors < 0 || (ntensors > 0 && !numels)) return fail(RR_ERR_INVALID_ARG, "bad tensor list");
+    if (grad_dtype != RR_BF16 && grad_dtype != RR_F32)
+        return fail(RR_ERR_UNSUPPORTED, "gradients must be bf16 or fp32");
+    auto* p = new rr_bucket_plan_t();
+    p->ntensors = ntensors;
+    p->grad_dtype = grad_dtype;
+    p->cap_bytes = cap_bytes;
+    const uint64_t es = esize(grad_dtype);
+    uint64_t off = 0, bytes = 0;
+    int b = 0, open = 0;
+    for (int t = 0; t < ntensors; ++t) {
+        if (!open) {
+            p->first.push_back(t);
+            p->count.push_back(0);
+            p->bnumel.push_back(0);
+            open = 1;
+        }
+        p->numel.push_back(numels[t]);
+        p->offset.push_back(off);
+        p->bucket_of.push_back(b);
+        p->count[b] += 1;
+        off += numels[t];
+        p->bnumel[b] = off;
+        bytes += numels[t] * es;
+        if (bytes >= cap_bytes) {  // the bucket reached the cap: close it
+            ++b;
+            off = 0;
+            bytes = 0;
+            open = 0;
+        }
+    }
+    *out = p;
+    return RR_OK;
+}
+
+void rr_bucket_plan_free(rr_bucket_plan_t* plan) { delete plan; }
+
+int rr_bucket_count(const rr_bucket_plan_t* plan) { return plan ? (int)plan->first.size() : 0; }
+
+rr_status_t rr_bucket_info(const rr_bucket_plan_t* plan, int bucket, int* first_tensor, int* ntensors,
+                           size_t* numel)
+{
+    if (!plan || bucket < 0 || bucket >= (int)plan->first.size()) return fail(RR_ERR_INVALID_ARG, "bad bucket");
+    if (first_tensor) *first_tensor = plan->first[bucket];
+    if (ntensors) *ntensors = plan->count[bucket];
+    if (numel) *numel = plan->bnumel[bucket];
+    return RR_OK;
+}
+
+rr_status_t rr_bucket_tensor(const rr_bucket_plan_t* plan, int tensor, int* bucket, size_t* offset)
+{
+    if (!plan || tensor < 0 || tensor >= plan->ntensors) return fail(RR_ERR_INVALID_ARG, "bad tensor");
+    if (bucket) *bucket = plan->bucket_of[tensor];
+    if (offset) *offset = plan->offset[tensor];
+    return RR_OK;
+}
+
+namespace {
+
+// Checks shared by the bucket calls; fills the bucket's tensor range.
+rr_status_t bucket_check(const rr_bucket_plan_t* plan, int bucket, const void* const* grads, int nranks, int* t0,
+                         int* nt)
+{
+    if (!plan) return fail(RR_ERR_INVALID_ARG, "NULL plan");
+    if (nranks < 1 || nranks > RR_MAX_RANKS) return fail(RR_ERR_INVALID_ARG, "nranks must be in 1..64");
+    if (bucket < 0 || bucket >= (int)plan->first.size()) return fail(RR_ERR_INVALID_ARG, "bad bucket");
+    if (!grads) return fail(RR_ERR_INVALID_ARG, "NULL gradient array");
+    *t0 = plan->first[bucket];
+    *nt = plan->count[bucket];
+    const uint64_t es = esize((rr_dtype_t)plan->grad_dtype);
+    std::vector<Span> spans;
+    for (int r = 0; r < nranks; ++r)
+        for (int t = *t0; t < *t0 + *nt; ++t) {
+            const void* g = grads[(size_t)r * plan->ntensors + t];
+            if (plan->numel[t] == 0) continue;
+            spans.push_back({(uintptr_t)g, (uintptr_t)g + plan->numel[t] * es, true});
+        }
+    return check_spans(spans);
+}
+
+}  // namespace
+
+static rr_status_t bucket_copy(const rr_bucket_plan_t* plan, int bucket, const void* const* grads,
+                               void* const* buckets, int nranks, int op, bool pack, cudaStream_t stream)
+{
+    int t0 = 0, nt = 0;
+    rr_status_t st = bucket_check(plan, bucket, grads, nranks, &t0, &nt);
+    if (st != RR_OK) return st;
+    if (!buckets) return fail(RR_ERR_INVALID_ARG, "NULL bucket array");
+    const int n = nranks;
+    const uint64_t es = esize((rr_dtype_t)plan->grad_dtype);
+    stats_begin(RR_ALGO_ONESHOT, n, plan->bnumel[bucket] * 4);
+    std::vector<Span> spans;
+    for (int r = 0; r < n; ++r)
+        spans.push_back({(uintptr_t)buckets[r], (uintptr_t)buckets[r] + plan->bnumel[bucket] * 4, true});
+    if (plan->bnumel[bucket] && (st = check_spans(spans)) != RR_OK) return st;
+    bool vec = same_phase(buckets, n);
+    const int per_launch = std::max(1, std::min(kMaxBucketTensors, kMaxBucketPtrs / n));
+    auto* p = new BucketCopyParams();
+    for (int g0 = 0; g0 < nt; g0 += per_launch) {
+        const int g1 = std::min(nt, g0 + per_launch);
+        *p = BucketCopyParams{};
+        p->n = n;
+        p->nt = g1 - g0;
+        p->divisor = (float)n;
+        uint64_t maxlen = 0;
+        bool v = vec;
+        for (int t = g0; t < g1; ++t) {
+            const int gt = t0 + t;
+            for (int r = 0; r < n; ++r) p->grad[(t - g0) * n + r] = grads[(size_t)r * plan->ntensors + gt];
+            v = v && same_phase(&p->grad[(t - g0) * n], n);
+            p->toff[t - g0] = plan->offset[gt];
+            p->tlen[t - g0] = plan->numel[gt];
+            maxlen = std::max<uint64_t>(maxlen, plan->numel[gt]);
+        }
+        for (int r = 0; r < n; ++r) p->bucket[r] = buckets[r];
+        p->vec_ok = v;
+        p->tps = std::max<uint64_t>(1, ceil_div(maxlen, bucket_tile_elems(plan->grad_dtype)));
+        if (maxlen == 0) continue;
+        cudaError_t e = pack ? launch_bucket_pack(plan->grad_dtype, *p, stream)
+                             : launch_bucket_unpack(plan->grad_dtype, op, *p, stream);
+        if (e != cudaSuccess) {
+            delete p;
+            return cuda_fail(e, pack ? "bucket pack launch" : "bucket unpack launch");
+        }
+        t_stats.launches += 1;
+    }
+    delete p;
+    t_stats.steps = 1;
+    t_stats.hbm_bytes = (uint64_t)n * plan->bnumel[bucket] * (es + 4);
+    return RR_OK;
+}
+
+rr_status_t rr_bucket_pack(const rr_bucket_plan_t* plan, int bucket, const void* const* grads,
+                           void* const* buckets, int nranks, cudaStream_t stream)
+{
+    rr_status_t st = bucket_copy(plan, bucket, grads, buckets, nranks, RR_SUM, true, stream);
+    log_call("bucket_pack", nranks, plan ? (size_t)plan->bnumel[std::max(0, bucket)] : 0, RR_F32, RR_SUM,
+             RR_ALGO_ONESHOT);
+    return st;
+}
+
+rr_status_t rr_bucket_unpack(const rr_bucket_plan_t* plan, int bucket, const void* const* buckets,
+                             void* const* grads, int nranks, rr_op_t op, cudaStream_t stream)
+{
+    if (op != RR_SUM && op != RR_AVG) return fail(RR_ERR_UNSUPPORTED, "bucket unpack takes SUM or AVG");
+    return bucket_copy(plan, bucket, grads, const_cast<void* const*>(buckets), nranks, op, false, stream);
+}
+
+rr_status_t rr_bucket_allreduce(const rr_bucket_plan_t* plan, int bucket, void* const* grads, int nranks,
+                                rr_op_t op, cudaStream_t stream)
+{
+    if (op != RR_SUM && op != RR_AVG) return fail(RR_ERR_UNSUPPORTED, "bucket all-reduce takes SUM or AVG");
+    int t0 = 0, nt = 0;
+    rr_status_t st = bucket_check(plan, bucket, grads, nranks, &t0, &nt);
+    if (st != RR_OK) return st;
+    const int n = nranks;
+    const uint64_t es = esize((rr_dtype_t)plan->grad_dtype);
+    const uint64_t total = plan->bnumel[bucket];
+    stats_begin(RR_ALGO_ONESHOT, n, total * es);
+    if (n == 1 || total == 0) return RR_OK;
+    const uint64_t C = ceil_div(total, (uint64_t)n);  // the bucket's chunk size
+    auto* p = new BucketFoldParams();
+    auto flush = [&](int ntens) -> rr_status_t {
+        if (p->nseg == 0) return RR_OK;
+        uint64_t maxlen = 0;
+        for (int s = 0; s < p->nseg; ++s) maxlen = std::max(maxlen, p->seg[s].len);
+        p->n = n;
+        p->divisor = (float)n;
+        p->tps = std::max<uint64_t>(1, ceil_div(maxlen, tile_elems(plan->grad_dtype)));
+        bool v = true;
+        for (int t = 0; t < ntens; ++t) v = v && same_phase(&p->grad[t * n], n);
+        p->vec_ok = v;
+        cudaError_t e = launch_bucket_fold(plan->grad_dtype, op, *p, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "bucket all-reduce launch");
+        t_stats.launches += 1;
+        return RR_OK;
+    };
+    int lt = 0;  // tensors in the current launch
+    *p = BucketFoldParams{};
+    for (int t = t0; t < t0 + nt && st == RR_OK; ++t) {
+        const uint64_t lo = plan->offset[t], hi = lo + plan->numel[t];
+        const int nsegs_t = hi > lo ? (int)((hi - 1) / C - lo / C + 1) : 0;
+        if (lt + 1 > kMaxBucketTensors || (lt + 1) * n > kMaxBucketPtrs || p->nseg + nsegs_t > kMaxBucketSegs) {
+            st = flush(lt);
+            *p = BucketFoldParams{};
+            lt = 0;
+        }
+        for (int r = 0; r < n; ++r) p->grad[lt * n + r] = grads[(size_t)r * plan->ntensors + t];
+        for (uint64_t pos = lo; pos < hi;) {  // split the tensor at the bucket's chunk boundaries
+            const uint64_t c = pos / C, end = std::min(hi, (c + 1) * C);
+            p->seg[p->nseg++] = BucketSeg{(uint32_t)lt, (uint32_t)c, pos - lo, end - pos};
+            pos = end;
+        }
+        ++lt;
+    }
+    if (st == RR_OK) st = flush(lt);
+    delete p;
+    t_stats.steps = 1;
+    t_stats.bytes_sent_max = (uint64_t)(n - 1) * total * es;
+    t_stats.bytes_sent_total = (uint64_t)n * t_stats.bytes_sent_max;
+    t_stats.hbm_bytes = 2ull * n * total * es;
+    log_call("bucket_allreduce", n, total, (rr_dtype_t)plan->grad_dtype, op, RR_ALGO_ONESHOT);
+    return st;
+}
+
+// ------------------------------------------------------ model, picker --
+
+rr_status_t rr_cost_model(rr_algo_t algo, int nranks, double bytes, double alpha_s, double beta,
+                          rr_cost_t* out)
+{
+    if (!out || nranks < 1 || beta <= 0) return fail(RR_ERR_INVALID_ARG, "bad cost-model arguments");
+    const double n = nranks;
+    rr_cost_t c{};
+    switch (algo) {
+    case RR_ALGO_RING:  // [P3] section 4: 2(N-1) steps, 2(N-1)/N M per rank
+        c.steps = 2 * (n - 1);
+        c.bytes_sent = 2 * (n - 1) / n * bytes;
+        break;
+    case RR_ALGO_TREE:  // [P3] section 6: 2 log2 N steps, the whole message per level
+    {
+        const double L = std::ceil(std::log2(n));
+        c.steps = 2 * L;
+        c.bytes_sent = 2 * L * bytes;
+        break;
+    }
+    case RR_ALGO_ONESHOT:  // [P4]: one step, read every peer's buffer
+    case RR_ALGO_TREE_ONESHOT:
+        c.steps = nranks > 1 ? 1 : 0;
+        c.bytes_sent = (n - 1) * bytes;
+        break;
+    default:
+        return fail(RR_ERR_INVALID_ARG, "unknown algo");
+    }
+    c.latency_s = c.steps * alpha_s;
+    c.bandwidth_s = c.bytes_sent / beta;
+    c.total_s = c.latency_s + c.bandwidth_s;
+    *out = c;
+    return RR_OK;
+}
+
+rr_status_t rr_set_picker_params(double launch_s, double hbm_bytes_per_s)
+{
+    if (!(launch_s >= 0) || !(hbm_bytes_per_s > 0)) return fail(RR_ERR_INVALID_ARG, "bad picker parameters");
+    g_launch_s = launch_s;
+    g_hbm_bps = hbm_bytes_per_s;
+    return RR_OK;
+}
+
+// On one GPU every "link" is HBM: a step costs one launch, and its bytes are
+// the HBM bytes it reads and writes (ring 5(N-1) S over 2(N-1) launches,
+// one-shot 2 N S in one).  bf16 always takes ONESHOT: the ring rounds its
+// bf16 partials at every hop, the fp32-accumulating one-shot does not
+// ([P1] s5.3).
+rr_algo_t rr_pick_algo(int nranks, size_t count, rr_dtype_t dtype)
+{
+    if (dtype == RR_BF16 || nranks <= 1) return RR_ALGO_ONESHOT;
+    const double n = nranks, S = (double)count * (double)esize(dtype);
+    const double ring = 2 * (n - 1) * g_launch_s + 5 * (n - 1) * S / g_hbm_bps;
+    const double one = g_launch_s + 2 * n * S / g_hbm_bps;
+    return ring < one ? RR_ALGO_RING : RR_ALGO_ONESHOT;
+}
+
+}  // extern "C"

@@ -1,0 +1,199 @@
+// rr_bucket.cu -- DDP-style gradient buckets: pack (gradients -> fp32
+// bucket), unpack (fp32 bucket -> gradients, with AVG's division and one
+// rounding) and the fused bucket sync that does pack + ring-order all-reduce
+// + unpack in one pass over the gradients.
+//
+// Sources: [P1] "How all-reduce keeps every card identical" (mhpq.cn),
+// s5.1-5.2 (DDP buckets, bucket_cap_mb = 25) and s5.3 (reduce low-precision
+// gradients in fp32); [P2] "AllReduce from principle to tuning" (xxqk.cn),
+// s3.3 (gradients fill buckets in order; a full bucket triggers its
+// all-reduce); [P3] "Training gradient sync and collective communication"
+// (geek-doc.cn), section 5 (bucketing hides the per-message latency).
+#include "rr_device.cuh"
+#include "rr_internal.h"
+
+namespace rr {
+
+namespace {
+
+constexpr int kUnitsPerThread = 2;
+
+// Convert one tile of a segment from In's element type to Out's, dividing by
+// `divisor` first when OP is AVG.  A unit is U elements, one 16-byte vector
+// of the narrower type; both sides must reach a 16-byte boundary after the
+// same scalar head, otherwise the whole segment is scalar.
+template <class In, class Out, int OP>
+__device__ __forceinline__ void convert_tile(const typename In::T* src, typename Out::T* dst, uint64_t len,
+                                             uint64_t tile, bool vec_ok, float divisor)
+{
+    constexpr int U = In::L > Out::L ? In::L : Out::L;
+    constexpr int NI = U / In::L, NO = U / Out::L;
+    constexpr uint64_t TU = (uint64_t)kThreads * kUnitsPerThread;
+    const int tid = threadIdx.x;
+    const int ps = phase_of(src, In::L), pd = phase_of(dst, Out::L);
+    int h = In::L == U ? (U - ps) % U : (U - pd) % U;
+    const bool vec = vec_ok && ((ps + h) % In::L == 0) && ((pd + h) % Out::L == 0);
+    auto one = [&](uint64_t e) { Out::st1(dst + e, finish<OP>((float)In::ld1(src + e), divisor)); };
+    if (!vec) {
+        const uint64_t e0 = tile * TU * U;
+#pragma unroll 4
+        for (int k = 0; k < kUnitsPerThread * U; ++k) {
+            const uint64_t e = e0 + (uint64_t)k * kThreads + tid;
+            if (e < len) one(e);
+        }
+        return;
+    }
+    uint64_t head = (uint64_t)h;
+    if (head > len) head = len;
+    const uint64_t nu = (len - head) / U;
+    const uint64_t tail = len - head - nu * U;
+    if (tile == 0 && (uint64_t)tid < head + tail)
+        one((uint64_t)tid < head ? (uint64_t)tid : head + nu * U + ((uint64_t)tid - head));
+#pragma unroll
+    for (int k = 0; k < kUnitsPerThread; ++k) {
+        const uint64_t u = tile * TU + (uint64_t)k * kThreads + tid;
+        if (u >= nu) continue;
+        const uint64_t e = head + u * U;
+        float a[U];
+#pragma unroll
+        for (int i = 0; i < NI; ++i) {
+            typename In::Acc t[In::L];
+            In::unpack(ldv(src + e + (uint64_t)i * In::L), t);
+#pragma unroll
+            for (int l = 0; l < In::L; ++l) a[i * In::L + l] = finish<OP>((float)t[l], divisor);
+        }
+#pragma unroll
+        for (int i = 0; i < NO; ++i) {
+            typename Out::Acc t[Out::L];
+#pragma unroll
+            for (int l = 0; l < Out::L; ++l) t[l] = a[i * Out::L + l];
+            stv(dst + e + (uint64_t)i * Out::L, Out::pack(t));
+        }
+    }
+}
+
+// Pack: segment (t, r) copies rank r's tensor t into rank r's fp32 bucket at
+// the tensor's offset (exact widening).
+template <class G>
+__global__ void __launch_bounds__(kThreads) bucket_pack_kernel(const __grid_constant__ BucketCopyParams p)
+{
+    const uint64_t nseg = (uint64_t)p.nt * (uint64_t)p.n;
+    const uint64_t total = nseg * p.tps;
+    for (uint64_t w = blockIdx.x; w < total; w += gridDim.x) {
+        const uint64_t s = w / p.tps, tile = w - s * p.tps;
+        const uint64_t t = s / (uint64_t)p.n, r = s - t * (uint64_t)p.n;
+        const auto* src = static_cast<const typename G::T*>(p.grad[s]);
+        float* dst = static_cast<float*>(p.bucket[r]) + p.toff[t];
+        convert_tile<G, F32T, kSum>(src, dst, p.tlen[t], tile, p.vec_ok, 1.0f);
+    }
+}
+
+// Unpack: segment (t, r) writes round(bucket[r][toff + j] / N) (AVG) or
+// round(bucket[r][toff + j]) (SUM) into rank r's tensor t.
+template <class G, int OP>
+__global__ void __launch_bounds__(kThreads) bucket_unpack_kernel(const __grid_constant__ BucketCopyParams p)
+{
+    const uint64_t nseg = (uint64_t)p.nt * (uint64_t)p.n;
+    const uint64_t total = nseg * p.tps;
+    for (uint64_t w = blockIdx.x; w < total; w += gridDim.x) {
+        const uint64_t s = w / p.tps, tile = w - s * p.tps;
+        const uint64_t t = s / (uint64_t)p.n, r = s - t * (uint64_t)p.n;
+        const float* src = static_cast<const float*>(p.bucket[r]) + p.toff[t];
+        auto* dst = static_cast<typename G::T*>(const_cast<void*>(p.grad[s]));
+        convert_tile<F32T, G, OP>(src, dst, p.tlen[t], tile, p.vec_ok, p.divisor);
+    }
+}
+
+// Fused bucket sync: segment = a run of one tensor inside one chunk c of the
+// bucket's flat index; every rank's copy is read once, folded in fp32 in ring
+// order from rank c, divided (AVG), rounded once and written back to every
+// rank.  Same bits as pack -> one-shot all-reduce (SUM) -> unpack.
+template <class G, int OP>
+__global__ void __launch_bounds__(kThreads) bucket_fold_kernel(const __grid_constant__ BucketFoldParams p)
+{
+    using T = typename G::T;
+    const uint64_t total = (uint64_t)p.nseg * p.tps;
+    for (uint64_t w = blockIdx.x; w < total; w += gridDim.x) {
+        const uint64_t s = w / p.tps, tile = w - s * p.tps;
+        const BucketSeg& sg = p.seg[s];
+        const int n = p.n;
+        const int base = (int)sg.t * n;
+        const int start = (int)sg.c;
+        auto in = [&](int j) {
+            int r = start + j;
+            if (r >= n) r -= n;
+            return static_cast<const T*>(p.grad[base + r]) + sg.off;
+        };
+        auto out = [&](int o) { return static_cast<T*>(p.grad[base + o]) + sg.off; };
+        fold_tile<G, OP>(in, n, out, n, sg.len, tile, p.vec_ok, p.divisor);
+    }
+}
+
+int sm_count_b()
+{
+    static int sms = [] {
+        int dev = 0, v = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        return v > 0 ? v : 148;
+    }();
+    return sms;
+}
+
+template <class P>
+cudaError_t launch_wave_b(void (*kernel)(P), const P& p, uint64_t work, cudaStream_t s)
+{
+    if (work == 0) return cudaSuccess;
+    int occ = 0;
+    cudaError_t e = resident_ctas(reinterpret_cast<const void*>(kernel), &occ);
+    if (e != cudaSuccess) return e;
+    uint64_t grid = (uint64_t)sm_count_b() * (uint64_t)occ;
+    if (grid > work) grid = work;
+    kernel<<<(unsigned)grid, kThreads, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// Elements one pack/unpack tile covers: kThreads * kUnitsPerThread units of
+// U elements (U = 8 for bf16 gradients, 4 for fp32).
+uint64_t bucket_tile_elems(int grad_dtype)
+{
+    return (uint64_t)kThreads * kUnitsPerThread * (grad_dtype == kBF16 ? 8u : 4u);
+}
+
+cudaError_t launch_bucket_pack(int grad_dtype, const BucketCopyParams& p, cudaStream_t s)
+{
+    const uint64_t work = (uint64_t)p.nt * (uint64_t)p.n * p.tps;
+    if (grad_dtype == kBF16) return launch_wave_b(bucket_pack_kernel<BF16T>, p, work, s);
+    if (grad_dtype == kF32) return launch_wave_b(bucket_pack_kernel<F32T>, p, work, s);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_bucket_unpack(int grad_dtype, int op, const BucketCopyParams& p, cudaStream_t s)
+{
+    const uint64_t work = (uint64_t)p.nt * (uint64_t)p.n * p.tps;
+    const bool avg = op == kAvg;
+    if (grad_dtype == kBF16)
+        return avg ? launch_wave_b(bucket_unpack_kernel<BF16T, kAvg>, p, work, s)
+                   : launch_wave_b(bucket_unpack_kernel<BF16T, kSum>, p, work, s);
+    if (grad_dtype == kF32)
+        return avg ? launch_wave_b(bucket_unpack_kernel<F32T, kAvg>, p, work, s)
+                   : launch_wave_b(bucket_unpack_kernel<F32T, kSum>, p, work, s);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p, cudaStream_t s)
+{
+    const uint64_t work = (uint64_t)p.nseg * p.tps;
+    const bool avg = op == kAvg;
+    if (grad_dtype == kBF16)
+        return avg ? launch_wave_b(bucket_fold_kernel<BF16T, kAvg>, p, work, s)
+                   : launch_wave_b(bucket_fold_kernel<BF16T, kSum>, p, work, s);
+    if (grad_dtype == kF32)
+        return avg ? launch_wave_b(bucket_fold_kernel<F32T, kAvg>, p, work, s)
+                   : launch_wave_b(bucket_fold_kernel<F32T, kSum>, p, work, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace rr

@@ -1,0 +1,285 @@
+// rr_device.cuh -- device building blocks shared by the kernels: element
+// types, the reduction operators, 128-bit memory access and the tile routine
+// that folds (or copies) one tile of one segment.
+//
+// A "segment" is a run of `len` elements that all reduce in the same order:
+// a chunk of the all-reduce (its fold starts on rank c, [P4] "Ring all-reduce
+// and communication volume"), one rank's part of a reduce-scatter, one ring
+// step's chunk transfer, one tensor of a bucket.  A segment has `nin` input
+// pointers in fold order and `nout` output pointers; the fold of element e is
+// op(...op(op(in0[e], in1[e]), in2[e])..., in_{nin-1}[e]), then AVG's division
+// by the rank count, then a store to every output.
+//
+// Sources: [P4] "Collective communication primitives" (ai-infra-handbooks);
+// [P1] "How all-reduce keeps every card identical" (mhpq.cn), s2.1 for the
+// operators and s5.3 for reducing low-precision gradients in fp32.
+#pragma once
+
+#include <cstdint>
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace rr {
+
+constexpr int kMaxRanks = 64;
+constexpr int kThreads = 256;  // threads per CTA of every kernel
+constexpr int kGroup = 8;      // input ranks whose loads are issued together
+
+enum OpCode : int { kSum = 0, kAvg = 1, kMax = 2, kMin = 3, kProd = 4 };
+
+// ------------------------------------------------------------ element types
+
+// fp32 buffers, fp32 arithmetic; 4 elements per 16-byte vector.
+struct F32T {
+    using T = float;
+    using Acc = float;
+    static constexpr int L = 4;
+    __device__ static __forceinline__ Acc ld1(const T* p) { return *p; }
+    __device__ static __forceinline__ void st1(T* p, Acc v) { *p = v; }
+    __device__ static __forceinline__ void unpack(const uint4& r, Acc (&a)[L])
+    {
+        a[0] = __uint_as_float(r.x);
+        a[1] = __uint_as_float(r.y);
+        a[2] = __uint_as_float(r.z);
+        a[3] = __uint_as_float(r.w);
+    }
+    __device__ static __forceinline__ uint4 pack(const Acc (&a)[L])
+    {
+        return make_uint4(__float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]),
+                          __float_as_uint(a[3]));
+    }
+};
+
+// bf16 buffers (raw 16-bit patterns), fp32 arithmetic; widening is the exact
+// shift into the top half of a binary32, narrowing rounds to nearest even.
+struct BF16T {
+    using T = uint16_t;
+    using Acc = float;
+    static constexpr int L = 8;
+    __device__ static __forceinline__ Acc ld1(const T* p) { return __uint_as_float((uint32_t)*p << 16); }
+    __device__ static __forceinline__ void st1(T* p, Acc v)
+    {
+        *p = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    }
+    __device__ static __forceinline__ void unpack2(uint32_t w, Acc& lo, Acc& hi)
+    {
+        lo = __uint_as_float(w << 16);
+        hi = __uint_as_float(w & 0xffff0000u);
+    }
+    __device__ static __forceinline__ uint32_t pack2(Acc lo, Acc hi)
+    {
+        __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half), .y = hi
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+    __device__ static __forceinline__ void unpack(const uint4& r, Acc (&a)[L])
+    {
+        unpack2(r.x, a[0], a[1]);
+        unpack2(r.y, a[2], a[3]);
+        unpack2(r.z, a[4], a[5]);
+        unpack2(r.w, a[6], a[7]);
+    }
+    __device__ static __forceinline__ uint4 pack(const Acc (&a)[L])
+    {
+        return make_uint4(pack2(a[0], a[1]), pack2(a[2], a[3]), pack2(a[4], a[5]), pack2(a[6], a[7]));
+    }
+};
+
+// int32 buffers; SUM and PROD wrap modulo 2^32.
+struct I32T {
+    using T = int32_t;
+    using Acc = int32_t;
+    static constexpr int L = 4;
+    __device__ static __forceinline__ Acc ld1(const T* p) { return *p; }
+    __device__ static __forceinline__ void st1(T* p, Acc v) { *p = v; }
+    __device__ static __forceinline__ void unpack(const uint4& r, Acc (&a)[L])
+    {
+        a[0] = (int32_t)r.x;
+        a[1] = (int32_t)r.y;
+        a[2] = (int32_t)r.z;
+        a[3] = (int32_t)r.w;
+    }
+    __device__ static __forceinline__ uint4 pack(const Acc (&a)[L])
+    {
+        return make_uint4((uint32_t)a[0], (uint32_t)a[1], (uint32_t)a[2], (uint32_t)a[3]);
+    }
+};
+
+// -------------------------------------------------------------- operators
+
+// One binary step of the fold, partial on the left.  __fadd_rn/__fmul_rn are
+// never contracted into an FMA; MAX/MIN keep the left operand on ties.
+template <int OP>
+__device__ __forceinline__ float apply(float a, float b)
+{
+    if constexpr (OP == kSum || OP == kAvg) return __fadd_rn(a, b);
+    else if constexpr (OP == kProd) return __fmul_rn(a, b);
+    else if constexpr (OP == kMax) return (a < b) ? b : a;
+    else return (b < a) ? b : a;
+}
+
+template <int OP>
+__device__ __forceinline__ int32_t apply(int32_t a, int32_t b)
+{
+    if constexpr (OP == kSum) return (int32_t)((uint32_t)a + (uint32_t)b);
+    else if constexpr (OP == kProd) return (int32_t)((uint32_t)a * (uint32_t)b);
+    else if constexpr (OP == kMax) return (a < b) ? b : a;
+    else return (b < a) ? b : a;
+}
+
+// AVG's last step: one IEEE division of the full fold by the rank count.
+template <int OP>
+__device__ __forceinline__ float finish(float a, float divisor)
+{
+    if constexpr (OP == kAvg) return __fdiv_rn(a, divisor);
+    else return a;
+}
+
+template <int OP>
+__device__ __forceinline__ int32_t finish(int32_t a, float) { return a; }
+
+// ------------------------------------------------------------------ memory
+
+// 128-bit streaming access: every byte is touched once per call, so hint the
+// caches to evict it first.  Plain (coherent) loads: in-place calls read and
+// write the same buffers.
+__device__ __forceinline__ uint4 ldv(const void* p) { return __ldcs(reinterpret_cast<const uint4*>(p)); }
+__device__ __forceinline__ void stv(void* p, const uint4& v) { __stcs(reinterpret_cast<uint4*>(p), v); }
+
+template <class T>
+__device__ __forceinline__ int phase_of(const T* p, int L)
+{
+    return (int)(((uintptr_t)p / sizeof(T)) & (uintptr_t)(L - 1));
+}
+
+// --------------------------------------------------------------- the tile
+
+// Scalar fold of element e of a segment.
+template <class Ty, int OP, class InF, class OutF>
+__device__ __forceinline__ void fold_one(const InF& in, int nin, const OutF& out, int nout, uint64_t e,
+                                         float divisor)
+{
+    using Acc = typename Ty::Acc;
+    Acc acc = Ty::ld1(in(0) + e);
+    for (int j = 1; j < nin; ++j) acc = apply<OP>(acc, Ty::ld1(in(j) + e));
+    if (nin > 1) acc = finish<OP>(acc, divisor);
+    for (int o = 0; o < nout; ++o) Ty::st1(out(o) + e, acc);
+}
+
+// Vectors per tile per thread.
+template <class Ty>
+struct Vpt {
+    static constexpr int value = 2;
+};
+
+// Fold (nin > 1) or copy (nin == 1) tile `tile` of a segment of `len`
+// elements.  in(j) / out(o) return the segment's base pointers.  vec_ok says
+// that every in(j) has the same address modulo 16 as in(0), and every out(o)
+// the same as out(0) (checked by the host); when in(0) and out(0) also agree,
+// the segment splits into a scalar head up to the first 16-byte boundary, a
+// body of 16-byte vectors and a scalar tail, otherwise every element is
+// scalar.  Tile t covers body vectors [t*TV, (t+1)*TV), TV = kThreads*VPT, or
+// the same number of elements on the scalar path; tile 0 also does the head
+// and tail.
+template <class Ty, int OP, class InF, class OutF>
+__device__ __forceinline__ void fold_tile(const InF& in, int nin, const OutF& out, int nout, uint64_t len,
+                                          uint64_t tile, bool vec_ok, float divisor)
+{
+    using T = typename Ty::T;
+    using Acc = typename Ty::Acc;
+    constexpr int L = Ty::L;
+    constexpr int VPT = Vpt<Ty>::value;
+    constexpr uint64_t TV = (uint64_t)kThreads * VPT;
+    const int tid = threadIdx.x;
+    const int pin = phase_of(in(0), L);
+    const int pout = phase_of(out(0), L);
+    if (!(vec_ok && pin == pout)) {
+        const uint64_t e0 = tile * TV * L;
+#pragma unroll 4
+        for (int k = 0; k < VPT * L; ++k) {
+            uint64_t e = e0 + (uint64_t)k * kThreads + tid;
+            if (e < len) fold_one<Ty, OP>(in, nin, out, nout, e, divisor);
+        }
+        return;
+    }
+    uint64_t head = (uint64_t)((L - pin) & (L - 1));
+    if (head > len) head = len;
+    const uint64_t nv = (len - head) / L;
+    const uint64_t tail = len - head - nv * L;
+    if (tile == 0 && (uint64_t)tid < head + tail) {
+        uint64_t e = (uint64_t)tid < head ? (uint64_t)tid : head + nv * L + ((uint64_t)tid - head);
+        fold_one<Ty, OP>(in, nin, out, nout, e, divisor);
+    }
+    const uint64_t v0 = tile * TV;
+    if (v0 >= nv) return;
+    uint64_t off[VPT];
+    bool ok[VPT];
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) {
+        uint64_t v = v0 + (uint64_t)u * kThreads + tid;
+        ok[u] = v < nv;
+        off[u] = head + v * L;
+    }
+    if (nin == 1) {  // a copy: move the raw bits
+        uint4 raw[VPT];
+        const T* p = in(0);
+#pragma unroll
+        for (int u = 0; u < VPT; ++u)
+            if (ok[u]) raw[u] = ldv(p + off[u]);
+#pragma unroll 4
+        for (int o = 0; o < nout; ++o) {
+            T* q = out(o);
+#pragma unroll
+            for (int u = 0; u < VPT; ++u)
+                if (ok[u]) stv(q + off[u], raw[u]);
+        }
+        return;
+    }
+    Acc a[VPT][L];
+    {
+        const T* p = in(0);
+#pragma unroll
+        for (int u = 0; u < VPT; ++u)
+            if (ok[u]) Ty::unpack(ldv(p + off[u]), a[u]);
+    }
+    for (int g = 1; g < nin; g += kGroup) {
+        uint4 raw[kGroup][VPT];
+#pragma unroll
+        for (int k = 0; k < kGroup; ++k) {
+            if (g + k < nin) {
+                const T* p = in(g + k);
+#pragma unroll
+                for (int u = 0; u < VPT; ++u)
+                    if (ok[u]) raw[k][u] = ldv(p + off[u]);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kGroup; ++k) {
+            if (g + k < nin) {
+#pragma unroll
+                for (int u = 0; u < VPT; ++u) {
+                    Acc b[L];
+                    Ty::unpack(raw[k][u], b);
+#pragma unroll
+                    for (int l = 0; l < L; ++l) a[u][l] = apply<OP>(a[u][l], b[l]);
+                }
+            }
+        }
+    }
+    uint4 res[VPT];
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) {
+#pragma unroll
+        for (int l = 0; l < L; ++l) a[u][l] = finish<OP>(a[u][l], divisor);
+        res[u] = Ty::pack(a[u]);
+    }
+#pragma unroll 4
+    for (int o = 0; o < nout; ++o) {
+        T* q = out(o);
+#pragma unroll
+        for (int u = 0; u < VPT; ++u)
+            if (ok[u]) stv(q + off[u], res[u]);
+    }
+}
+
+}  // namespace rr

@@ -1,0 +1,104 @@
+// rr_internal.h -- kernel parameter blocks and launchers shared between the
+// host dispatcher (rr_api.cu) and the kernels (rr_kernels.cu, rr_bucket.cu).
+// Not part of the C ABI.
+#pragma once
+
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+namespace rr {
+
+constexpr int kMaxRanksH = 64;
+
+// Rule-driven collectives over N rank buffers (one-shot all-reduce in ring
+// or tree order, reduce-scatter, all-gather, all-to-all).
+struct RankParams {
+    const void* in[kMaxRanksH];
+    void* out[kMaxRanksH];
+    int n;          // ranks
+    int vec_ok;     // all in[] agree modulo 16 bytes, and all out[] do
+    float divisor;  // AVG's divisor (the rank count)
+    int pad_;
+    uint64_t C;     // chunk / part length in elements
+    uint64_t count; // elements per rank buffer (all-reduce)
+    uint64_t nseg;  // segments
+    uint64_t tps;   // tiles per segment
+};
+
+// One segment of a table-driven step (a ring step, a tree level): fold
+// in0 op in1 (in0 on the left) into out, or copy in0 into out when the step
+// has one input.
+struct StepSeg {
+    const void* in0;
+    const void* in1;
+    void* out;
+    uint64_t len;
+};
+
+struct StepParams {
+    StepSeg seg[kMaxRanksH];
+    int nseg;
+    int nin;        // 2: fold, 1: copy
+    int vec_ok;     // every segment's pointers agree modulo 16 bytes
+    float divisor;  // AVG's divisor when this step finishes the fold
+    uint64_t tps;
+};
+
+// Bucket launches: one launch covers up to kMaxBucketTensors tensors of one
+// bucket and up to kMaxBucketPtrs gradient pointers (tensor-major: entry
+// t * n + r is rank r's copy of the launch's t-th tensor).
+constexpr int kMaxBucketPtrs = 2048;
+constexpr int kMaxBucketTensors = 384;
+constexpr int kMaxBucketSegs = kMaxBucketTensors + kMaxRanksH;
+
+struct BucketCopyParams {
+    const void* grad[kMaxBucketPtrs];  // pack: sources; unpack: destinations
+    void* bucket[kMaxRanksH];          // fp32 bucket of each rank
+    uint64_t toff[kMaxBucketTensors];  // element offset of tensor t in the bucket
+    uint64_t tlen[kMaxBucketTensors];  // elements of tensor t
+    int n;
+    int nt;
+    int vec_ok;
+    float divisor;
+    uint64_t tps;
+};
+
+// A fused bucket segment: elements [off, off + len) of launch tensor t, all
+// in the bucket's chunk c (their fold starts on rank c).
+struct BucketSeg {
+    uint32_t t;
+    uint32_t c;
+    uint64_t off;
+    uint64_t len;
+};
+
+struct BucketFoldParams {
+    void* grad[kMaxBucketPtrs];
+    BucketSeg seg[kMaxBucketSegs];
+    int n;
+    int nseg;
+    int vec_ok;
+    float divisor;
+    uint64_t tps;
+};
+
+enum DType : int { kF32 = 0, kBF16 = 1, kI32 = 2 };
+enum Kind : int { kOneshotRing = 0, kOneshotTree = 1, kReduceScatter = 2, kAllGather = 3, kAllToAll = 4 };
+
+// Elements one fold tile covers (for sizing tiles per segment on the host),
+// and one bucket pack/unpack tile.
+uint64_t tile_elems(int dtype);
+uint64_t bucket_tile_elems(int grad_dtype);
+
+// Resident CTAs per SM of a kernel at kThreads threads (cached per kernel).
+cudaError_t resident_ctas(const void* kernel, int* out);
+
+// Launchers: return the launch's cudaError_t.  `op` is an rr_op_t value.
+cudaError_t launch_rank_kernel(int kind, int dtype, int op, const RankParams& p, cudaStream_t s);
+cudaError_t launch_step(int dtype, int op, const StepParams& p, cudaStream_t s);
+cudaError_t launch_bucket_pack(int grad_dtype, const BucketCopyParams& p, cudaStream_t s);
+cudaError_t launch_bucket_unpack(int grad_dtype, int op, const BucketCopyParams& p, cudaStream_t s);
+cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p, cudaStream_t s);
+
+}  // namespace rr

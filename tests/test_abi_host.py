@@ -1,0 +1,204 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+The library must load and export every function ``include/rr.h`` declares.
+Its host logic (ring schedule, bucket plan, cost model, picker, argument
+checks) is compared with the oracle and the pages' figures.  No call here
+launches a kernel: every call either computes on the host only or fails
+argument checks before anything is enqueued.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+import ring_all_reduce_virtual_b200 as rrv
+from conftest import ROOT, golden_lines
+from ring_all_reduce_virtual_b200 import _lib, synth
+from ring_all_reduce_virtual_b200.build import build
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "rr.h"), encoding="utf-8").read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(rr_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("rr_allreduce", "rr_reduce_scatter", "rr_all_gather", "rr_all_to_all", "rr_bucket_plan",
+              "rr_bucket_pack", "rr_bucket_unpack", "rr_bucket_plan_free", "rr_get_stats",
+              "rr_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.lib()
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (rr_\w+)", out))
+    for name in _declared():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_library_uses_sm100a_code():
+    out = subprocess.run(["cuobjdump", "--list-elf", _lib.LIB_PATH], capture_output=True, text=True).stdout
+    assert "sm_100a" in out
+
+
+def test_version_and_status_strings():
+    lib = _lib.lib()
+    assert lib.rr_version() == 1
+    assert lib.rr_status_string(0) == b"ok"
+    assert lib.rr_status_string(1) == b"invalid argument"
+
+
+# ------------------------------------------------------- ring schedule --
+
+@pytest.mark.parametrize("n,count", [(1, 7), (2, 2), (4, 4096), (4, 1024), (3, 10), (8, 3), (16, 1000), (64, 130)])
+def test_ring_schedule_equals_oracle_trace(n, count):
+    x = synth.ranks(0, n, count, "uniform")
+    sent, trace = oracle.ring_allreduce(x, trace=True)
+    ours = rrv.ring_schedule(n, count, "f32")
+    assert ours == trace
+    per_rank = np.zeros(n, dtype=np.uint64)
+    for e in ours:
+        per_rank[e["rank"]] += e["bytes"]
+    assert np.array_equal(per_rank, sent)
+
+
+def test_ring_schedule_bytes_golden():
+    g = dict(ln.split(":", 1) for ln in golden_lines("ring_bytes_4rank.txt"))
+    n, m = int(g["ranks"]), int(g["elements_per_rank"])
+    ev = rrv.ring_schedule(n, m, "f32")
+    sent = [sum(e["bytes"] for e in ev if e["rank"] == r) for r in range(n)]
+    assert sent == [int(v) for v in g["sent"].split()]
+
+
+# --------------------------------------------------------- bucket plan --
+
+@pytest.mark.parametrize("cap", [0, 1, 700, 25 * (1 << 20)])
+def test_bucket_plan_equals_oracle(cap):
+    if cap == 25 * (1 << 20):
+        numels = [m for _, m in synth.grad_ready_order(synth.gpt_grad_tensors())]
+    else:
+        numels = np.random.default_rng(cap).integers(0, 400, size=50).tolist()
+    b, off, nb = oracle.bucket_plan(numels, 2, cap)
+    plan = rrv.BucketPlan(numels, "bf16", cap)
+    assert plan.num_buckets == nb
+    for t in range(len(numels)):
+        assert plan.tensor(t) == (int(b[t]), int(off[t]))
+    for k in range(nb):
+        first, cnt, numel = plan.info(k)
+        members = [t for t in range(len(numels)) if b[t] == k]
+        assert (first, cnt) == (members[0], len(members))
+        assert numel == sum(numels[t] for t in members)
+
+
+# ---------------------------------------------------------- cost model --
+
+def _parse_ab(line):
+    name, rest = line.split(":", 1)
+    lhs, rhs = rest.split("->")
+    args = dict(kv.split("=") for kv in lhs.split())
+    val, tol = rhs.split()
+    return name, {k: float(v) for k, v in args.items()}, float(val), float(tol.split("=")[1])
+
+
+def test_cost_model_matches_the_pages():
+    for line in golden_lines("alpha_beta.txt"):
+        name, a, want, rel = _parse_ab(line)
+        n = int(a["N"])
+        if name == "volume":
+            got = rrv.cost_model("ring", n, a["M"], 0.0, 1.0)["bytes_sent"]
+        elif name == "latency_term":
+            got = rrv.cost_model("ring", n, 1.0, a["alpha"], 1.0)["latency_s"]
+        elif name == "bandwidth_term":
+            got = rrv.cost_model("ring", n, a["M"], 0.0, a["beta"])["bandwidth_s"]
+        elif name == "ring_time":
+            got = rrv.cost_model("ring", n, a["M"], a["alpha"], a["beta"])["total_s"]
+        elif name == "ps_centre":
+            # the parameter server's centre receives and sends (N-1) M each
+            got = 2 * (n - 1) * a["M"]
+        elif name == "ps_time":
+            got = 2 * (n - 1) * a["M"] / a["beta"]
+        else:
+            raise AssertionError(name)
+        assert abs(got - want) <= rel * want, (line, got)
+
+
+def test_cost_model_tree_and_oneshot_steps():
+    # [P3] section 6 table: the tree takes 2 log2 N steps, the ring 2(N-1)
+    for n in (2, 4, 8, 16, 64):
+        assert rrv.cost_model("tree", n, 1.0, 1.0, 1.0)["steps"] == 2 * np.log2(n)
+        assert rrv.cost_model("ring", n, 1.0, 1.0, 1.0)["steps"] == 2 * (n - 1)
+        assert rrv.cost_model("oneshot", n, 1.0, 1.0, 1.0)["steps"] == 1
+
+
+def test_picker_is_size_aware_and_exact():
+    # AUTO only ever picks schedules with the ring's bits
+    for n in (2, 4, 8, 16, 64):
+        for count in (1, 256, 1 << 20, 1 << 28):
+            assert rrv.pick_algo(n, count, "f32") in ("ring", "oneshot")
+            assert rrv.pick_algo(n, count, "bf16") == "oneshot"
+    # with launches free and bandwidth the only cost, fewer bytes win
+    rrv.set_picker_params(0.0, 1e12)
+    assert rrv.pick_algo(8, 1 << 20, "f32") == "oneshot"
+    rrv.set_picker_params(4e-6, 6.5e12)
+
+
+# -------------------------------------------------- argument checking --
+
+def _fake(n, stride=1 << 20, base=1 << 40):
+    arr = (ctypes.c_void_p * n)()
+    for i in range(n):
+        arr[i] = base + i * stride
+    return arr
+
+
+def test_argument_errors_return_before_any_launch():
+    lib = _lib.lib()
+    s = ctypes.c_void_p(0)
+    assert lib.rr_allreduce(_fake(4), 0, 16, 0, 0, 0, s) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_allreduce(_fake(4), 65, 16, 0, 0, 0, s) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_allreduce(_fake(4), 4, 16, 7, 0, 0, s) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_allreduce(_fake(4), 4, 16, 0, 9, 0, s) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_allreduce(_fake(4), 4, 16, 0, 0, 9, s) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_allreduce(_fake(4), 4, 16, 2, 1, 0, s) == _lib.RR_ERR_UNSUPPORTED  # int32 AVG
+    assert lib.rr_allreduce(None, 4, 16, 0, 0, 0, s) == _lib.RR_ERR_INVALID_ARG
+    overlapping = _fake(4, stride=32)  # 16 fp32 = 64 bytes apart by 32
+    assert lib.rr_allreduce(overlapping, 4, 16, 0, 0, 0, s) == _lib.RR_ERR_INVALID_ARG
+    assert b"overlap" in lib.rr_last_error()
+    repeated = _fake(4, stride=0)
+    assert lib.rr_allreduce(repeated, 4, 16, 0, 0, 0, s) == _lib.RR_ERR_INVALID_ARG
+    nulls = (ctypes.c_void_p * 2)(None, None)
+    assert lib.rr_allreduce(nulls, 2, 16, 0, 0, 0, s) == _lib.RR_ERR_INVALID_ARG
+    # bad ring steps
+    assert lib.rr_ring_step(_fake(4), 4, 16, 0, 0, 0, 3, s) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_ring_step(_fake(4), 4, 16, 0, 0, 2, 0, s) == _lib.RR_ERR_INVALID_ARG
+    # reduce-scatter output overlapping an input
+    send, recv = _fake(2), _fake(2, base=(1 << 40) + 8)
+    assert lib.rr_reduce_scatter(send, recv, 2, 4, 0, 0, 0, s) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_reduce_scatter(_fake(2), _fake(2, base=1 << 41), 2, 4, 0, 0, 1, s) == _lib.RR_ERR_UNSUPPORTED
+
+
+def test_trivial_calls_enqueue_nothing():
+    lib = _lib.lib()
+    s = ctypes.c_void_p(0)
+    assert lib.rr_allreduce(_fake(4), 4, 0, 0, 0, 0, s) == 0  # count == 0
+    assert rrv.last_stats()["launches"] == 0
+    assert lib.rr_allreduce(_fake(1), 1, 1000, 0, 1, 0, s) == 0  # one rank: identity
+    assert rrv.last_stats()["launches"] == 0
+
+
+def test_bucket_plan_rejects_bad_dtype():
+    with pytest.raises(rrv.RRError):
+        rrv.BucketPlan([1, 2, 3], "i32", 100)

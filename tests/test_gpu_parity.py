@@ -1,0 +1,296 @@
+"""GPU parity: every CUDA path, called through the C ABI, against the CPU
+oracle on the same seeded inputs, element by element.
+
+The bar is bit-exactness for every dtype: fp32 and int32 reduce in the ring
+order on both sides; bf16 is folded in fp32 and rounded once by the one-shot
+paths and rounded per hop by the ring and tree schedules, on both sides
+alike.  bf16 results are also checked against an fp64 reduction within the
+stated tolerance (abs 1e-2, rel 1e-2).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ring_all_reduce_virtual_b200 as rrv
+from conftest import golden_lines
+from gpu_util import assert_bits_equal, empty_like_ranks, to_dev, to_host
+from ring_all_reduce_virtual_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+ALGOS = ["ring", "oneshot", "tree", "tree_oneshot", "auto"]
+ORACLE = {
+    "ring": oracle.ring_allreduce,
+    "oneshot": oracle.fold_ring_order,
+    "auto": oracle.fold_ring_order,
+    "tree": oracle.tree_schedule,
+    "tree_oneshot": oracle.tree_fold,
+}
+TILE = {"f32": 2048, "bf16": 4096, "i32": 2048}  # elements per tile of the fold kernels
+
+
+def _dist(op, dtype):
+    if dtype == "i32":
+        return "int"
+    return "prod" if op == "prod" else "uniform"
+
+
+def _run(n, count, dtype, op, algo, seed=0, offsets=None):
+    x = synth.ranks(seed, n, count, _dist(op, dtype), dtype)
+    want = [a.copy() for a in x]
+    ORACLE[algo](want, op)
+    d = to_dev(x, offsets)
+    rrv.all_reduce(d, op, algo)
+    got = to_host(d)
+    assert_bits_equal(got, want, f"{algo} {dtype} {op} n={n} count={count}")
+    return x, got
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from ring_all_reduce_virtual_b200.build import build
+
+    build()
+
+
+# -------------------------------------------------------- worked example --
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_worked_example(algo):
+    exp = {}
+    for ln in golden_lines("five_primitives_4rank.txt"):
+        head, rest = ln.split(":", 1)
+        p = head.split()
+        if len(p) == 2:
+            exp.setdefault(p[0], {})[int(p[1])] = [float(v) for v in rest.split()]
+    x = synth.ranks(0, 4, 4, "arange")
+    d = to_dev(x)
+    rrv.all_reduce(d, "sum", algo)
+    for r, t in enumerate(to_host(d)):
+        assert t.tolist() == exp["all_reduce"][r]
+    d = to_dev(x)
+    rs = empty_like_ranks(4, 1, "f32")
+    rrv.reduce_scatter(d, rs)
+    ag = empty_like_ranks(4, 4, "f32")
+    rrv.all_gather(rs, ag)
+    a2a = empty_like_ranks(4, 4, "f32")
+    rrv.all_to_all(d, a2a)
+    for r in range(4):
+        assert to_host(rs)[r].tolist() == exp["reduce_scatter"][r]
+        assert to_host(ag)[r].tolist() == exp["all_gather"][r]
+        assert to_host(a2a)[r].tolist() == exp["all_to_all"][r]
+
+
+# ------------------------------------------------------ all-reduce parity --
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "i32"])
+@pytest.mark.parametrize("op", ["sum", "avg", "max", "min", "prod"])
+def test_allreduce_every_op_and_dtype(algo, dtype, op):
+    if dtype == "i32" and op == "avg":
+        pytest.skip("AVG is not defined for int32")
+    n = 5
+    count = 3 * TILE[dtype] * n + 37  # several tiles per chunk and a ragged tail
+    x, got = _run(n, count, dtype, op, algo, seed=1)
+    if dtype == "bf16" and op in ("sum", "avg"):
+        ref = np.stack([oracle.bf16_to_f32(v) for v in x]).astype(np.float64).sum(0)
+        if op == "avg":
+            ref /= n
+        assert np.allclose(oracle.bf16_to_f32(got[0]), ref, atol=1e-2, rtol=1e-2)
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("n", [1, 2, 3, 4, 7, 8, 16])
+@pytest.mark.parametrize("count", [0, 1, 3, 4, 5, 17, 1000, 4096, 70001])
+def test_allreduce_sizes(algo, n, count):
+    _run(n, count, "f32", "sum", algo, seed=2)
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_allreduce_64_ranks(algo, dtype):
+    _run(64, 64 * 700 + 3, dtype, "sum", algo, seed=3)
+
+
+@pytest.mark.parametrize("algo", ["ring", "oneshot", "tree_oneshot"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_allreduce_shared_misalignment(algo, dtype):
+    # every base 1 element past a 16-byte boundary: vector path after a head
+    n = 4
+    _run(n, 5 * TILE[dtype] + 11, dtype, "sum", algo, seed=4, offsets=[1] * n)
+
+
+@pytest.mark.parametrize("algo", ["ring", "oneshot", "tree", "tree_oneshot"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_allreduce_mixed_misalignment(algo, dtype):
+    # bases disagree modulo 16 bytes: the scalar path
+    n = 4
+    _run(n, 3 * TILE[dtype] + 5, dtype, "avg", algo, seed=5, offsets=[0, 1, 2, 3])
+
+
+def test_fold_order_fixture():
+    # the hand-derived rounding fixture: ring order gives 0 everywhere,
+    # a pairwise tree gives 1 for element 0
+    g = {ln.split(":")[0]: [float(v) for v in ln.split(":")[1].split()] for ln in golden_lines("fold_order.txt")}
+    big = np.float32(2.0 ** 24)
+    x = [np.zeros(4, dtype=np.float32) for _ in range(4)]
+    for i in range(4):
+        for k, v in enumerate([np.float32(1), big, np.float32(1), -big]):
+            x[(i + k) % 4][i] = v
+    for algo in ("ring", "oneshot", "auto"):
+        d = to_dev(x)
+        rrv.all_reduce(d, "sum", algo)
+        for t in to_host(d):
+            assert t.tolist() == g["ring_order"]
+    d = to_dev(x)
+    rrv.all_reduce(d, "sum", "tree_oneshot")
+    assert to_host(d)[0][0] == 1.0
+
+
+def test_max_signed_zero_ties_follow_the_fold():
+    n = 4
+    x = [np.full(n, -1.0, dtype=np.float32) for _ in range(n)]
+    for i in range(n):
+        x[i][i] = 0.0
+        x[(i + 1) % n][i] = -0.0
+    for algo in ("ring", "oneshot"):
+        want = [a.copy() for a in x]
+        ORACLE[algo](want, "max")
+        d = to_dev(x)
+        rrv.all_reduce(d, "max", algo)
+        assert_bits_equal(to_host(d), want, algo)
+
+
+# ----------------------------------------------------------- ring steps --
+
+@pytest.mark.parametrize("n", [2, 3, 4, 8])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("op", ["sum", "avg"])
+def test_ring_steps_track_the_oracle_state(n, dtype, op):
+    # after every one of the 2(N-1) steps the device buffers equal the
+    # oracle's per-rank chunk arrays bit for bit
+    count = 2 * TILE[dtype] * n + 13
+    x = synth.ranks(6, n, count, "uniform", dtype)
+    d = to_dev(x)
+    host = [a.copy() for a in x]
+    for phase in ("reduce_scatter", "all_gather"):
+        for s in range(n - 1):
+            oracle.ring_step(host, op, oracle.PHASE_RS if phase == "reduce_scatter" else oracle.PHASE_AG, s)
+            rrv.ring_step(d, op, phase, s)
+            assert_bits_equal(to_host(d), host, f"{phase} step {s}")
+            st = rrv.last_stats()
+            assert st["launches"] == 1
+
+
+def test_ring_stats_match_the_schedule():
+    n, count = 4, 1024
+    d = to_dev(synth.ranks(7, n, count, "uniform"))
+    rrv.all_reduce(d, "sum", "ring")
+    st = rrv.last_stats()
+    assert st["algo"] == "ring" and st["steps"] == 6 and st["launches"] == 6
+    assert st["bytes_sent_max"] == 6144  # [P4]: 2(n-1)/n x 4096 bytes
+    assert st["hbm_bytes"] == 5 * 3 * 4096
+    rrv.all_reduce(d, "sum", "oneshot")
+    st = rrv.last_stats()
+    assert st["launches"] == 1 and st["hbm_bytes"] == 2 * 4 * 4096
+
+
+# --------------------------------------------- reduce-scatter, all-gather --
+
+@pytest.mark.parametrize("n", [1, 2, 3, 4, 8, 64])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "i32"])
+def test_reduce_scatter_all_gather_all_to_all(n, dtype):
+    per = 2 * TILE[dtype] + 9
+    x = synth.ranks(8, n, n * per, "int" if dtype == "i32" else "uniform", dtype)
+    d = to_dev(x)
+    for op in ("sum", "max") if dtype != "bf16" else ("sum", "avg"):
+        rs = empty_like_ranks(n, per, dtype)
+        rrv.reduce_scatter(d, rs, op)
+        assert_bits_equal(to_host(rs), oracle.reduce_scatter([a.copy() for a in x], op), f"rs {op}")
+    ag = empty_like_ranks(n, n * per, dtype)
+    rrv.all_gather(rs, ag)
+    assert_bits_equal(to_host(ag), oracle.all_gather(to_host(rs)), "ag")
+    a2a = empty_like_ranks(n, n * per, dtype)
+    rrv.all_to_all(d, a2a)
+    assert_bits_equal(to_host(a2a), oracle.all_to_all(x), "a2a")
+
+
+@pytest.mark.parametrize("op", ["sum", "avg", "min", "prod"])
+def test_rs_then_ag_equals_allreduce(op):
+    n, per = 8, 3000
+    x = synth.ranks(9, n, n * per, "prod" if op == "prod" else "uniform")
+    d = to_dev(x)
+    rs = empty_like_ranks(n, per, "f32")
+    ag = empty_like_ranks(n, n * per, "f32")
+    rrv.reduce_scatter(d, rs, op)
+    rrv.all_gather(rs, ag)
+    rrv.all_reduce(d, op, "ring")
+    assert_bits_equal(to_host(ag), to_host(d), op)
+
+
+# --------------------------------------------------------------- buckets --
+
+def _grad_set(seed, n, numels, dtype="bf16"):
+    return [synth.rank_grads(seed, r, numels, "normal", dtype) for r in range(n)]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("op", ["avg", "sum"])
+def test_bucket_staged_and_fused_match_the_oracle(dtype, op):
+    n = 8
+    numels = [5, 3000, 64, 1, 9000, 77, 0, 20000, 333, 4096]
+    cap = 4 * 4096 * (2 if dtype == "bf16" else 4)
+    host = _grad_set(10, n, numels, dtype)
+    want = [[g.copy() for g in rank] for rank in host]
+    oracle.bucket_sync(want, cap, op)
+    plan = rrv.BucketPlan(numels, dtype, cap)
+    # staged: pack -> one-shot SUM on the fp32 buckets -> unpack
+    grads = [to_dev(rank) for rank in host]
+    for b in range(plan.num_buckets):
+        numel = plan.info(b)[2]
+        buckets = [torch.empty(max(numel, 1), dtype=torch.float32, device="cuda") for _ in range(n)]
+        plan.pack(b, grads, buckets)
+        packed = to_host(buckets)
+        rrv.all_reduce([t[:numel] for t in buckets], "sum", "oneshot")
+        plan.unpack(b, buckets, grads, op)
+        # the packed bucket is the exact widening of the gradients
+        bo, off = [], []
+        first, cnt, _ = plan.info(b)
+        for t in range(first, first + cnt):
+            w = oracle.bf16_to_f32(host[0][t]) if dtype == "bf16" else host[0][t]
+            assert np.array_equal(packed[0][plan.tensor(t)[1]:plan.tensor(t)[1] + numels[t]], w)
+    for r in range(n):
+        assert_bits_equal(to_host(grads[r]), want[r], f"staged rank {r}")
+    # fused: one pass over the gradients
+    grads = [to_dev(rank) for rank in host]
+    for b in range(plan.num_buckets):
+        plan.all_reduce(b, grads, op)
+    for r in range(n):
+        assert_bits_equal(to_host(grads[r]), want[r], f"fused rank {r}")
+
+
+def test_bucket_fused_misaligned_tensors():
+    # tensors carved out of one flat allocation at odd element offsets
+    n = 4
+    numels = [7, 1001, 3, 2500, 64]
+    host = _grad_set(11, n, numels)
+    want = [[g.copy() for g in rank] for rank in host]
+    oracle.bucket_sync(want, 1000, "avg")
+    plan = rrv.BucketPlan(numels, "bf16", 1000)
+    grads = []
+    for r in range(n):
+        flat = torch.zeros(sum(numels) + 8 * len(numels), dtype=torch.bfloat16, device="cuda")
+        ts, o = [], 1 + r
+        for g in host[r]:
+            t = flat[o:o + g.size]
+            t.copy_(torch.from_numpy(g.view(np.int16)).cuda().view(torch.bfloat16))
+            ts.append(t)
+            o += g.size + 3
+        grads.append(ts)
+    for b in range(plan.num_buckets):
+        plan.all_reduce(b, grads, "avg")
+    for r in range(n):
+        assert_bits_equal(to_host(grads[r]), want[r], f"rank {r}")
