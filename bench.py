@@ -61,7 +61,12 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--cpu-seconds", type=float, default=8.0, help="CPU-baseline sample budget")
+    ap.add_argument("--ref-seconds", type=float, default=90.0, help="reference-arm time budget")
     ap.add_argument("--no-extra", action="store_true", help="skip the per-algorithm extra timings")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end host-buffer timing")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--count", type=int, default=COUNT,
+                    help="fp32 elements per virtual rank (default 2^26 = 256 MiB); smaller for profiling")
     return ap.parse_args()
 
 
@@ -156,16 +161,22 @@ class Clocks:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.out.close()
-        rows = []
         with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) != len(self.FIELDS):
-                    continue
-                if self.uuid and self._norm(parts[0]) != self.uuid:
-                    continue
-                rows.append(parts)
+            lines = f.readlines()
         os.unlink(self.path)
+        return self.parse(lines, self.uuid)
+
+    @classmethod
+    def parse(cls, lines, uuid: str = ""):
+        """Median SM clock, max clock and the throttle reasons seen."""
+        rows = []
+        for line in lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != len(cls.FIELDS):
+                continue
+            if uuid and cls._norm(parts[0]) != uuid:
+                continue
+            rows.append(parts)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -178,10 +189,10 @@ class Clocks:
 
 # ---------------------------------------------------------------- inputs --
 
-def host_inputs(rank_offset: int):
+def host_inputs(rank_offset: int, count: int):
     from ring_all_reduce_virtual_b200 import synth
 
-    return [synth.rank_values(SEED + rank_offset, r, COUNT, "normal", "f32") for r in range(NRANKS)]
+    return [synth.rank_values(SEED + rank_offset, r, count, "normal", "f32") for r in range(NRANKS)]
 
 
 # ------------------------------------------------------------ cpu oracle --
@@ -244,7 +255,7 @@ def run_reference(args, d: Dist):
     t0 = time.perf_counter()
     oracle.ring_allreduce(x, "avg")
     one = max(time.perf_counter() - t0, 1e-6)
-    budget = 90.0 / max(steps + warm, 1)  # whole run in about a minute and a half
+    budget = 0.5 * args.ref_seconds / max(steps + warm, 1)  # whole run within the budget (time grows faster than m)
     m = int(min(COUNT, max(4096, m * budget / one)))
     m -= m % NRANKS
     x = synth.ranks(SEED, NRANKS, m, "normal", "f32")
@@ -289,9 +300,10 @@ def run_ours(args, d: Dist):
     d.init("nccl")
     stream = torch.cuda.current_stream(dev)
 
-    host = host_inputs(d.rank * NRANKS)
+    count = args.count
+    host = host_inputs(d.rank * NRANKS, count)
     bufs = [torch.from_numpy(a).to(dev) for a in host]
-    S = COUNT * ELEM
+    S = count * ELEM
     alg_bytes = 2 * NRANKS * S  # one-shot: read N*S, write N*S
 
     def step():
@@ -328,56 +340,22 @@ def run_ours(args, d: Dist):
         traffic = int(NCU_TRAFFIC["per_algorithmic_byte"] * alg_bytes)
 
     # end to end through the public API with host buffers: H2D + all-reduce + D2H
-    pinned = [torch.from_numpy(a).pin_memory() for a in host]
-    for _ in range(2):
-        rrv.all_reduce_host(pinned, bufs, "avg", "auto", stream)
-    torch.cuda.synchronize(dev)
-    d.barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        rrv.all_reduce_host(pinned, bufs, "avg", "auto", stream)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    d.barrier()
-    e2e_ms = d.max(e0.elapsed_time(e1) / max(args.e2e_steps, 1), dev)
-    e2e = {"value": round(S / (e2e_ms / 1e3) / 1e9 * d.world, 3), "unit": "GB/s",
-           "h2d_bytes_per_step": NRANKS * S, "d2h_bytes_per_step": NRANKS * S,
-           "ms_per_step": round(e2e_ms, 3), "host_memory": "pinned"}
-
-    extra = {}
-    if not args.no_extra:
-        for name, op, algo, reps in (("oneshot_sum", "sum", "oneshot", 20), ("ring_sum", "sum", "ring", 10),
-                                     ("tree_oneshot_sum", "sum", "tree_oneshot", 10), ("tree_sum", "sum", "tree", 10)):
-            fresh = [torch.from_numpy(a).to(dev) for a in host]
-            rrv.all_reduce(fresh, op, algo, stream)
-            st = rrv.last_stats()
-            torch.cuda.synchronize(dev)
-            a0 = torch.cuda.Event(enable_timing=True)
-            a1 = torch.cuda.Event(enable_timing=True)
-            a0.record(stream)
-            for _ in range(reps):
-                rrv.all_reduce(fresh, op, algo, stream)
-            a1.record(stream)
-            torch.cuda.synchronize(dev)
-            tm = a0.elapsed_time(a1) / reps / 1e3
-            extra[name] = {"ms": round(tm * 1e3, 4), "algbw_gbs": round(S / tm / 1e9, 2),
-                           "hbm_gbs": round(st["hbm_bytes"] / tm / 1e9, 1),
-                           "hbm_frac": round(st["hbm_bytes"] / tm / 1e9 / peak, 4), "launches": st["launches"]}
-            del fresh
-
-    cpu = cpu_baseline(args.cpu_seconds) if (d.rank == 0 and d.world == 1) else None
+    e2e = None
+    if not args.no_e2e:
+        e2e = time_e2e(args, d, dev, stream, host, bufs, S)
+    extra = {} if args.no_extra else time_extra(dev, stream, host, S, hbm_peak()[0])
+    cpu = cpu_baseline(args.cpu_seconds) if (d.rank == 0 and d.world == 1 and not args.no_cpu) else None
     if d.rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": d.world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32",
             "data": "synthetic: normal(0, 1e-3) fp32 from numpy default_rng([seed, rank]), generated on the host",
-            "config": {"workload": WORKLOAD, "nranks_virtual": NRANKS, "count_per_rank": COUNT,
-                       "bytes_per_rank": S, "op": "avg", "algo": "auto -> " + str(picked["algo"]),
-                       "in_place": True, "value_is": "algbw = S / T summed over GPUs",
-                       "l2": "inputs 2 GiB per GPU > 126 MB L2; no flush needed"},
+            "config": {"workload": WORKLOAD if count == COUNT else f"allreduce-8x{count}-f32", "nranks_virtual": NRANKS,
+                       "count_per_rank": count, "bytes_per_rank": S, "op": "avg",
+                       "algo": "auto -> " + str(picked["algo"]), "in_place": True,
+                       "value_is": "algbw = S / T summed over GPUs",
+                       "l2": f"inputs {NRANKS * S / 2**30:.2f} GiB per GPU vs 126 MB L2; no flush between steps"},
             "algbw_per_gpu": round(algbw, 3), "busbw": round(busbw, 3),
             "hbm_gbs": round(achieved, 1), "hbm_frac": round(achieved / peak, 4),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
@@ -392,6 +370,58 @@ def run_ours(args, d: Dist):
         }
         print(json.dumps(line), flush=True)
     d.close()
+
+
+def time_e2e(args, d, dev, stream, host, bufs, S):
+    import torch
+
+    import ring_all_reduce_virtual_b200 as rrv
+
+    pinned = [torch.from_numpy(a).pin_memory() for a in host]
+    for _ in range(2):
+        rrv.all_reduce_host(pinned, bufs, "avg", "auto", stream)
+    torch.cuda.synchronize(dev)
+    d.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        rrv.all_reduce_host(pinned, bufs, "avg", "auto", stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    d.barrier()
+    e2e_ms = d.max(e0.elapsed_time(e1) / max(args.e2e_steps, 1), dev)
+    return {"value": round(S / (e2e_ms / 1e3) / 1e9 * d.world, 3), "unit": "GB/s",
+            "h2d_bytes_per_step": NRANKS * S, "d2h_bytes_per_step": NRANKS * S,
+            "ms_per_step": round(e2e_ms, 3), "host_memory": "pinned"}
+
+
+def time_extra(dev, stream, host, S, peak):
+    """The other algorithms on the same workload (a few calls each)."""
+    import torch
+
+    import ring_all_reduce_virtual_b200 as rrv
+
+    extra = {}
+    for name, op, algo, reps in (("oneshot_sum", "sum", "oneshot", 20), ("ring_sum", "sum", "ring", 10),
+                                 ("tree_oneshot_sum", "sum", "tree_oneshot", 10), ("tree_sum", "sum", "tree", 10)):
+        fresh = [torch.from_numpy(a).to(dev) for a in host]
+        rrv.all_reduce(fresh, op, algo, stream)
+        st = rrv.last_stats()
+        torch.cuda.synchronize(dev)
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(reps):
+            rrv.all_reduce(fresh, op, algo, stream)
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        tm = a0.elapsed_time(a1) / reps / 1e3
+        extra[name] = {"ms": round(tm * 1e3, 4), "algbw_gbs": round(S / tm / 1e9, 2),
+                       "hbm_gbs": round(st["hbm_bytes"] / tm / 1e9, 1),
+                       "hbm_frac": round(st["hbm_bytes"] / tm / 1e9 / peak, 4), "launches": st["launches"]}
+        del fresh
+    return extra
 
 
 def main():
