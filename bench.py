@@ -65,6 +65,9 @@ def parse_args():
     ap.add_argument("--no-extra", action="store_true", help="skip the per-algorithm extra timings")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end host-buffer timing")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--workload", choices=[WORKLOAD, "sweep", "gpt-buckets", "64x256MiB"], default=WORKLOAD,
+                    help="the headline workload (default), the message-size sweep, or the bucketed "
+                         "gradient sync of a GPT-like model; the last two print one JSON line per point")
     ap.add_argument("--count", type=int, default=COUNT,
                     help="fp32 elements per virtual rank (default 2^26 = 256 MiB); smaller for profiling")
     return ap.parse_args()
@@ -424,11 +427,195 @@ def time_extra(dev, stream, host, S, peak):
     return extra
 
 
+def run_sweep(args):
+    """Message-size sweep: 1 KiB .. 1 GiB per rank, N in {2, 4, 8, 16}, fp32
+    SUM, every algorithm.  Per point: median per-call device time over 20
+    calls after 5 warm-ups, and for sizes up to 1 MiB the per-call time of a
+    CUDA graph holding 100 calls.  Points whose 2 N S bytes fit in L2 are
+    flagged."""
+    import torch
+
+    import ring_all_reduce_virtual_b200 as rrv
+    from ring_all_reduce_virtual_b200.build import build
+
+    build()
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.Stream(dev)
+    peak, _ = hbm_peak()
+    for n in (2, 4, 8, 16):
+        for e in range(10, 31):
+            nbytes = 1 << e
+            count = nbytes // ELEM
+            bufs = [torch.randn(count, device=dev) for _ in range(n)]
+            for algo in ("ring", "oneshot", "tree", "tree_oneshot"):
+                with torch.cuda.stream(stream):
+                    for _ in range(5):
+                        rrv.all_reduce(bufs, "sum", algo, stream)
+                    st = rrv.last_stats()
+                    times = []
+                    for _ in range(20):
+                        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        a.record(stream)
+                        rrv.all_reduce(bufs, "sum", algo, stream)
+                        b.record(stream)
+                        times.append((a, b))
+                    stream.synchronize()
+                    t = statistics.median(x.elapsed_time(y) for x, y in times) / 1e3
+                    graph_us = None
+                    if nbytes <= 1 << 20:
+                        g = torch.cuda.CUDAGraph()
+                        with torch.cuda.graph(g, stream=stream):
+                            for _ in range(100):
+                                rrv.all_reduce(bufs, "sum", algo, stream)
+                        g.replay()
+                        stream.synchronize()
+                        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        a.record(stream)
+                        for _ in range(5):
+                            g.replay()
+                        b.record(stream)
+                        stream.synchronize()
+                        graph_us = a.elapsed_time(b) * 1e3 / 500
+                        del g
+                algbw = nbytes / t / 1e9
+                print(json.dumps({
+                    "workload": "size-sweep-f32-sum", "nranks_virtual": n, "bytes_per_rank": nbytes, "algo": algo,
+                    "latency_us": round(t * 1e6, 3), "graph_latency_us": None if graph_us is None else round(graph_us, 3),
+                    "algbw_gbs": round(algbw, 3), "busbw_gbs": round(algbw * 2 * (n - 1) / n, 3),
+                    "hbm_gbs": round(st["hbm_bytes"] / t / 1e9, 1), "hbm_frac": round(st["hbm_bytes"] / t / 1e9 / peak, 4),
+                    "launches": st["launches"], "l2_resident": 2 * n * nbytes <= 126 * 10**6}), flush=True)
+            del bufs
+            torch.cuda.empty_cache()
+
+
+def run_gpt_buckets(args):
+    """Bucketed gradient sync of a GPT-like model (24 layers, d_model 2048,
+    4x MLP, 32k vocab: 293 bf16 tensors, 1.34 B parameters per rank) over 8
+    virtual ranks with 25 MiB buckets and AVG: the fused path (4 bytes per
+    parameter per rank) and the staged pack -> all-reduce -> unpack path (20
+    bytes).  Gradients are normal(0, 1e-3) drawn on the device (timing does
+    not depend on the values)."""
+    import torch
+
+    import ring_all_reduce_virtual_b200 as rrv
+    from ring_all_reduce_virtual_b200 import synth
+    from ring_all_reduce_virtual_b200.build import build
+
+    build()
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    n = 8
+    numels = [m for _, m in synth.grad_ready_order(synth.gpt_grad_tensors())]
+    params = sum(numels)
+    gen = torch.Generator(device=dev).manual_seed(SEED)
+    grads = [[(torch.randn(m, device=dev, generator=gen) * 1e-3).to(torch.bfloat16) for m in numels]
+             for _ in range(n)]
+    plan = rrv.BucketPlan(numels, "bf16", synth.BUCKET_CAP_BYTES)
+    nb = plan.num_buckets
+    biggest = max(plan.info(b)[2] for b in range(nb))
+    buckets = [torch.empty(biggest, dtype=torch.float32, device=dev) for _ in range(n)]
+    peak, _ = hbm_peak()
+
+    def fused():
+        for b in range(nb):
+            plan.all_reduce(b, grads, "avg", stream)
+
+    def staged():
+        for b in range(nb):
+            numel = plan.info(b)[2]
+            plan.pack(b, grads, buckets, stream)
+            rrv.all_reduce([t[:numel] for t in buckets], "sum", "auto", stream)
+            plan.unpack(b, buckets, grads, "avg", stream)
+
+    for name, fn, bpp in (("fused", fused, 4), ("staged", staged, 20)):
+        for _ in range(max(args.warmup, 3)):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 10
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        t = a.elapsed_time(b) / reps / 1e3
+        hbm = n * params * bpp
+        print(json.dumps({
+            "workload": "gpt-24x2048-buckets-bf16-avg", "path": name, "nranks_virtual": n, "params_per_rank": params,
+            "tensors": len(numels), "buckets": nb, "bucket_cap_bytes": synth.BUCKET_CAP_BYTES,
+            "ms_per_sync": round(t * 1e3, 3), "grad_bytes_per_rank": params * 2,
+            "algbw_gbs": round(params * 2 / t / 1e9, 2), "hbm_bytes_per_param_per_rank": bpp,
+            "hbm_gbs": round(hbm / t / 1e9, 1), "hbm_frac": round(hbm / t / 1e9 / peak, 4),
+            "launches_per_sync": nb * (1 if name == "fused" else 3)}), flush=True)
+
+
+def run_64_ranks(args):
+    """64 virtual ranks x 64 Mi fp32 (16 GiB): all-reduce SUM/MAX/MIN/PROD
+    (PROD on [0.99, 1.01]) and reduce-scatter, all-gather, all-to-all, each
+    timed over 10 calls.  Inputs are drawn on the device (timing does not
+    depend on the values)."""
+    import torch
+
+    import ring_all_reduce_virtual_b200 as rrv
+    from ring_all_reduce_virtual_b200.build import build
+
+    build()
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    n, count = 64, COUNT
+    S = count * ELEM
+    peak, _ = hbm_peak()
+    gen = torch.Generator(device=dev).manual_seed(SEED)
+    x = [torch.rand(count, device=dev, generator=gen) * 2 - 1 for _ in range(n)]
+
+    def timed(fn, reps=10):
+        fn()
+        st = rrv.last_stats()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / reps / 1e3, st
+
+    def emit(what, t, st):
+        print(json.dumps({"workload": "64x256MiB-f32", "call": what, "nranks_virtual": n, "bytes_per_rank": S,
+                          "ms": round(t * 1e3, 3), "algbw_gbs": round(S / t / 1e9, 2),
+                          "hbm_gbs": round(st["hbm_bytes"] / t / 1e9, 1),
+                          "hbm_frac": round(st["hbm_bytes"] / t / 1e9 / peak, 4), "launches": st["launches"]}),
+              flush=True)
+
+    for op in ("sum", "max", "min"):
+        emit(f"all_reduce {op}", *timed(lambda: rrv.all_reduce(x, op, "auto", stream)))
+    prod = [torch.rand(count, device=dev, generator=gen) * 0.02 + 0.99 for _ in range(4)]
+    for i in range(4):  # PROD inputs for the first ranks; the rest stay uniform[-1, 1)
+        x[i].copy_(prod[i])
+    del prod
+    emit("all_reduce prod", *timed(lambda: rrv.all_reduce(x, "prod", "auto", stream)))
+    per = count // n
+    rs = [torch.empty(per, device=dev) for _ in range(n)]
+    emit("reduce_scatter sum", *timed(lambda: rrv.reduce_scatter(x, rs, "sum", "auto", stream)))
+    out = [torch.empty(count, device=dev) for _ in range(n)]
+    emit("all_gather", *timed(lambda: rrv.all_gather(rs, out, "auto", stream)))
+    emit("all_to_all", *timed(lambda: rrv.all_to_all(x, out, stream)))
+
+
 def main():
     args = parse_args()
     d = Dist()
     if args.impl == "reference":
         run_reference(args, d)
+        return
+    if args.workload == "sweep":
+        run_sweep(args)
+        return
+    if args.workload == "gpt-buckets":
+        run_gpt_buckets(args)
+        return
+    if args.workload == "64x256MiB":
+        run_64_ranks(args)
         return
     run_ours(args, d)
 

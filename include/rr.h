@@ -148,12 +148,18 @@ rr_status_t rr_allreduce(void* const* bufs, int nranks, size_t count, rr_dtype_t
                          rr_algo_t algo, cudaStream_t stream);
 
 /* All-reduce of HOST buffers through caller-provided device buffers: copies
- * host_bufs[r] -> dev_bufs[r] (cudaMemcpyAsync on `stream`), runs
- * rr_allreduce on dev_bufs, and copies the result back into every
- * host_bufs[r].  Host buffers should be page-locked for the copies to be
+ * host_bufs[r] -> dev_bufs[r], reduces dev_bufs as rr_allreduce does, and
+ * copies the result back into every host_bufs[r]; dev_bufs hold the result
+ * too.  For the one-shot algorithms (AUTO's choice) above 8 MiB per rank the
+ * work is pipelined in 8 MiB slices: uploads run on an internal stream,
+ * folds on `stream`, downloads on a second internal stream, so uploads and
+ * downloads overlap; the internal streams wait for `stream` first and
+ * `stream` waits for them at the end, so the call is ordered on `stream`
+ * like any other.  Host buffers should be page-locked for the copies to be
  * asynchronous.  Same arguments, results and errors as rr_allreduce; the
  * device buffers must not overlap.  The host buffers hold the result once
- * `stream` has been synchronised. */
+ * `stream` has been synchronised.  The first call on a device creates the two
+ * streams and four events it keeps until exit. */
 rr_status_t rr_allreduce_host(void* const* host_bufs, void* const* dev_bufs, int nranks, size_t count,
                               rr_dtype_t dtype, rr_op_t op, rr_algo_t algo, cudaStream_t stream);
 

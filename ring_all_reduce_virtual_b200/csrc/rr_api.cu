@@ -13,7 +13,9 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <string>
+#include <unordered_map>
 #include <vector>
 
 #include "rr.h"
@@ -187,7 +189,7 @@ rr_status_t ring_step_launch(void* const* bufs, int n, size_t count, rr_dtype_t 
         p.seg[r].len = len;
         maxlen = std::max(maxlen, len);
     }
-    p.tps = std::max<uint64_t>(1, ceil_div(maxlen, tile_elems(dtype)));
+    p.tps = std::max<uint64_t>(1, ceil_div(maxlen, tile_elems(dtype, kVptMove)));
     // AVG divides once, in the step that completes each chunk's fold
     int op_eff = op;
     if (op == RR_AVG && !(phase == RR_PHASE_REDUCE_SCATTER && step == n - 2)) op_eff = RR_SUM;
@@ -243,7 +245,7 @@ rr_status_t run_tree(void* const* bufs, int n, size_t count, rr_dtype_t dtype, r
             p.nin = pass == 0 ? 2 : 1;
             p.vec_ok = vec;
             p.divisor = (float)n;
-            p.tps = std::max<uint64_t>(1, ceil_div(count, tile_elems(dtype)));
+            p.tps = std::max<uint64_t>(1, ceil_div(count, tile_elems(dtype, kVptMove)));
             for (int a = 0; a + h < n; a += 2 * h) {
                 StepSeg& sg = p.seg[p.nseg++];
                 if (pass == 0) {  // x_a <- x_a op x_{a+h}
@@ -278,7 +280,7 @@ rr_status_t run_tree(void* const* bufs, int n, size_t count, rr_dtype_t dtype, r
 
 rr_status_t run_rank_kernel(int kind, const void* const* in, void* const* out, int n, uint64_t C,
                             uint64_t count, uint64_t nseg, uint64_t tps, rr_dtype_t dtype, int op, bool vec,
-                            cudaStream_t stream)
+                            cudaStream_t stream, uint64_t lo = 0, uint64_t hi = UINT64_MAX)
 {
     RankParams p{};
     for (int r = 0; r < n; ++r) {
@@ -292,6 +294,8 @@ rr_status_t run_rank_kernel(int kind, const void* const* in, void* const* out, i
     p.count = count;
     p.nseg = nseg;
     p.tps = tps;
+    p.lo = lo;
+    p.hi = hi;
     cudaError_t e = launch_rank_kernel(kind, dtype, op, p, stream);
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     t_stats.launches += 1;
@@ -312,6 +316,45 @@ rr_algo_t resolve_algo(rr_algo_t algo, int n, size_t count, rr_dtype_t dtype)
     }();
     if (forced >= 0) return (rr_algo_t)forced;
     return rr_pick_algo(n, count, dtype);
+}
+
+// Slice size of the pipelined host-buffer all-reduce, per rank.
+constexpr uint64_t kHostSliceBytes = 8ull << 20;
+
+// Two copy streams and the events that order them against the caller's
+// stream; created once per device and kept until exit.
+struct HostPipe {
+    cudaStream_t in = nullptr, out = nullptr;
+    cudaEvent_t start = nullptr, arrived = nullptr, reduced = nullptr, done = nullptr;
+};
+
+rr_status_t host_pipe(HostPipe** out)
+{
+    static std::mutex mu;
+    static std::unordered_map<int, HostPipe*> pipes;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = pipes.find(dev);
+    if (it != pipes.end()) {
+        *out = it->second;
+        return RR_OK;
+    }
+    auto* hp = new HostPipe();
+    const unsigned ef = cudaEventDisableTiming;
+    if ((e = cudaStreamCreateWithFlags(&hp->in, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaStreamCreateWithFlags(&hp->out, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&hp->start, ef)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&hp->arrived, ef)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&hp->reduced, ef)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&hp->done, ef)) != cudaSuccess) {
+        delete hp;
+        return cuda_fail(e, "creating the copy streams");
+    }
+    pipes.emplace(dev, hp);
+    *out = hp;
+    return RR_OK;
 }
 
 }  // namespace
@@ -371,7 +414,7 @@ rr_status_t rr_allreduce(void* const* bufs, int nranks, size_t count, rr_dtype_t
         break;
     case RR_ALGO_ONESHOT: {
         const uint64_t C = ceil_div(count, (uint64_t)n);
-        const uint64_t tps = std::max<uint64_t>(1, ceil_div(C, tile_elems(dtype)));
+        const uint64_t tps = std::max<uint64_t>(1, ceil_div(C, tile_elems(dtype, kVptReduce)));
         st = run_rank_kernel(kOneshotRing, bufs, bufs, n, C, count, (uint64_t)n, tps, dtype, op,
                              same_phase(bufs, n), stream);
         t_stats.steps = 1;
@@ -381,7 +424,7 @@ rr_status_t rr_allreduce(void* const* bufs, int nranks, size_t count, rr_dtype_t
         break;
     }
     case RR_ALGO_TREE_ONESHOT: {
-        const uint64_t tps = std::max<uint64_t>(1, ceil_div(count, tile_elems(dtype)));
+        const uint64_t tps = std::max<uint64_t>(1, ceil_div(count, tile_elems(dtype, kVptReduce)));
         st = run_rank_kernel(kOneshotTree, bufs, bufs, n, count, count, 1, tps, dtype, op, same_phase(bufs, n),
                              stream);
         t_stats.steps = 1;
@@ -402,24 +445,86 @@ rr_status_t rr_allreduce_host(void* const* host_bufs, void* const* dev_bufs, int
 {
     rr_status_t st = check_basic(nranks, dtype, op);
     if (st != RR_OK) return st;
+    if (algo < RR_ALGO_AUTO || algo > RR_ALGO_TREE_ONESHOT) return fail(RR_ERR_INVALID_ARG, "unknown algo");
     if (!host_bufs || !dev_bufs) return fail(RR_ERR_INVALID_ARG, "NULL pointer array");
-    const size_t bytes = count * esize(dtype);
-    for (int r = 0; r < nranks && count; ++r)
+    const int n = nranks;
+    const size_t es = esize(dtype), bytes = count * es;
+    for (int r = 0; r < n && count; ++r)
         if (!host_bufs[r]) return fail(RR_ERR_INVALID_ARG, "NULL host buffer");
     std::vector<Span> spans;
-    for (int r = 0; r < nranks && count; ++r)
+    for (int r = 0; r < n && count; ++r)
         spans.push_back({(uintptr_t)dev_bufs[r], (uintptr_t)dev_bufs[r] + bytes, true});
     if ((st = check_spans(spans)) != RR_OK) return st;
-    if (count == 0) return rr_allreduce(dev_bufs, nranks, 0, dtype, op, algo, stream);
-    for (int r = 0; r < nranks; ++r) {
-        cudaError_t e = cudaMemcpyAsync(dev_bufs[r], host_bufs[r], bytes, cudaMemcpyHostToDevice, stream);
-        if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+    const rr_algo_t a = resolve_algo(algo, n, count, dtype);
+    if (count == 0) return rr_allreduce(dev_bufs, n, 0, dtype, op, a, stream);
+    const bool sliced = n > 1 && (a == RR_ALGO_ONESHOT || a == RR_ALGO_TREE_ONESHOT) && bytes > kHostSliceBytes;
+    if (!sliced) {  // copy in, reduce, copy out, all on the caller's stream
+        for (int r = 0; r < n; ++r) {
+            cudaError_t e = cudaMemcpyAsync(dev_bufs[r], host_bufs[r], bytes, cudaMemcpyHostToDevice, stream);
+            if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+        }
+        if ((st = rr_allreduce(dev_bufs, n, count, dtype, op, a, stream)) != RR_OK) return st;
+        for (int r = 0; r < n; ++r) {
+            cudaError_t e = cudaMemcpyAsync(host_bufs[r], dev_bufs[r], bytes, cudaMemcpyDeviceToHost, stream);
+            if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+        }
+        return RR_OK;
     }
-    if ((st = rr_allreduce(dev_bufs, nranks, count, dtype, op, algo, stream)) != RR_OK) return st;
-    for (int r = 0; r < nranks; ++r) {
-        cudaError_t e = cudaMemcpyAsync(host_bufs[r], dev_bufs[r], bytes, cudaMemcpyDeviceToHost, stream);
-        if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+    // Pipelined: slice k of every rank is uploaded on one stream, reduced on
+    // the caller's stream once it has arrived, and downloaded on another
+    // stream, so uploads and downloads of different slices overlap.  The
+    // one-shot fold is element-local, so each slice reduces on its own with
+    // the chunk rule of the whole buffer.
+    HostPipe* hp = nullptr;
+    if ((st = host_pipe(&hp)) != RR_OK) return st;
+    auto ck = [&](cudaError_t e, const char* where) { return e == cudaSuccess ? RR_OK : cuda_fail(e, where); };
+    if ((st = ck(cudaEventRecord(hp->start, stream), "event record")) != RR_OK) return st;
+    if ((st = ck(cudaStreamWaitEvent(hp->in, hp->start, 0), "stream wait")) != RR_OK) return st;
+    if ((st = ck(cudaStreamWaitEvent(hp->out, hp->start, 0), "stream wait")) != RR_OK) return st;
+    const uint64_t slice = std::max<uint64_t>(1, kHostSliceBytes / es);
+    const uint64_t C = ceil_div(count, (uint64_t)n);
+    const bool vec = same_phase(dev_bufs, n);
+    int launches = 0;
+    for (uint64_t lo = 0; lo < count; lo += slice) {
+        const uint64_t hi = std::min<uint64_t>(count, lo + slice), len = hi - lo;
+        for (int r = 0; r < n; ++r) {
+            cudaError_t e = cudaMemcpyAsync(static_cast<char*>(dev_bufs[r]) + lo * es,
+                                            static_cast<const char*>(host_bufs[r]) + lo * es, len * es,
+                                            cudaMemcpyHostToDevice, hp->in);
+            if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+        }
+        if ((st = ck(cudaEventRecord(hp->arrived, hp->in), "event record")) != RR_OK) return st;
+        if ((st = ck(cudaStreamWaitEvent(stream, hp->arrived, 0), "stream wait")) != RR_OK) return st;
+        if (a == RR_ALGO_ONESHOT) {
+            const uint64_t tps = std::max<uint64_t>(1, ceil_div(std::min(C, len), tile_elems(dtype, kVptReduce)));
+            st = run_rank_kernel(kOneshotRing, dev_bufs, dev_bufs, n, C, count, (uint64_t)n, tps, dtype, op, vec,
+                                 stream, lo, hi);
+        } else {
+            void* off[RR_MAX_RANKS];
+            for (int r = 0; r < n; ++r) off[r] = static_cast<char*>(dev_bufs[r]) + lo * es;
+            const uint64_t tps = std::max<uint64_t>(1, ceil_div(len, tile_elems(dtype, kVptReduce)));
+            st = run_rank_kernel(kOneshotTree, off, off, n, len, len, 1, tps, dtype, op, same_phase(off, n), stream);
+        }
+        if (st != RR_OK) return st;
+        ++launches;
+        if ((st = ck(cudaEventRecord(hp->reduced, stream), "event record")) != RR_OK) return st;
+        if ((st = ck(cudaStreamWaitEvent(hp->out, hp->reduced, 0), "stream wait")) != RR_OK) return st;
+        for (int r = 0; r < n; ++r) {
+            cudaError_t e = cudaMemcpyAsync(static_cast<char*>(host_bufs[r]) + lo * es,
+                                            static_cast<const char*>(dev_bufs[r]) + lo * es, len * es,
+                                            cudaMemcpyDeviceToHost, hp->out);
+            if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+        }
     }
+    if ((st = ck(cudaEventRecord(hp->done, hp->out), "event record")) != RR_OK) return st;
+    if ((st = ck(cudaStreamWaitEvent(stream, hp->done, 0), "stream wait")) != RR_OK) return st;
+    stats_begin(a, n, bytes);
+    t_stats.steps = 1;
+    t_stats.launches = launches;
+    t_stats.bytes_sent_max = (uint64_t)(n - 1) * bytes;
+    t_stats.bytes_sent_total = (uint64_t)n * (n - 1) * bytes;
+    t_stats.hbm_bytes = 4ull * n * bytes;  // copies in and out, plus the fold's read and write
+    log_call("allreduce_host", n, count, dtype, op, a);
     return RR_OK;
 }
 
@@ -497,7 +602,7 @@ rr_status_t rr_reduce_scatter(const void* const* send, void* const* recv, int nr
     }
     if ((st = check_spans(spans)) != RR_OK) return st;
     if ((st = check_device_ptrs(send, n)) != RR_OK || (st = check_device_ptrs(recv, n)) != RR_OK) return st;
-    const uint64_t tps = std::max<uint64_t>(1, ceil_div(recvcount, tile_elems(dtype)));
+    const uint64_t tps = std::max<uint64_t>(1, ceil_div(recvcount, tile_elems(dtype, kVptReduce)));
     st = run_rank_kernel(kReduceScatter, send, recv, n, recvcount, (uint64_t)n * recvcount, (uint64_t)n, tps,
                          dtype, op, same_phase(send, n) && same_phase(recv, n), stream);
     t_stats.steps = 1;
@@ -528,7 +633,7 @@ rr_status_t rr_all_gather(const void* const* send, void* const* recv, int nranks
     }
     if ((st = check_spans(spans)) != RR_OK) return st;
     if ((st = check_device_ptrs(send, n)) != RR_OK || (st = check_device_ptrs(recv, n)) != RR_OK) return st;
-    const uint64_t tps = std::max<uint64_t>(1, ceil_div(sendcount, tile_elems(dtype)));
+    const uint64_t tps = std::max<uint64_t>(1, ceil_div(sendcount, tile_elems(dtype, kVptMove)));
     st = run_rank_kernel(kAllGather, send, recv, n, sendcount, (uint64_t)n * sendcount, (uint64_t)n, tps, dtype,
                          RR_SUM, same_phase(send, n) && same_phase(recv, n), stream);
     t_stats.steps = 1;
@@ -557,7 +662,7 @@ rr_status_t rr_all_to_all(const void* const* send, void* const* recv, int nranks
     }
     if ((st = check_spans(spans)) != RR_OK) return st;
     if ((st = check_device_ptrs(send, n)) != RR_OK || (st = check_device_ptrs(recv, n)) != RR_OK) return st;
-    const uint64_t tps = std::max<uint64_t>(1, ceil_div(count_per_peer, tile_elems(dtype)));
+    const uint64_t tps = std::max<uint64_t>(1, ceil_div(count_per_peer, tile_elems(dtype, kVptMove)));
     st = run_rank_kernel(kAllToAll, send, recv, n, count_per_peer, (uint64_t)n * count_per_peer,
                          (uint64_t)n * n, tps, dtype, RR_SUM, true, stream);
     t_stats.steps = 1;
@@ -744,7 +849,7 @@ rr_status_t rr_bucket_allreduce(const rr_bucket_plan_t* plan, int bucket, void* 
         for (int s = 0; s < p->nseg; ++s) maxlen = std::max(maxlen, p->seg[s].len);
         p->n = n;
         p->divisor = (float)n;
-        p->tps = std::max<uint64_t>(1, ceil_div(maxlen, tile_elems(plan->grad_dtype)));
+        p->tps = std::max<uint64_t>(1, ceil_div(maxlen, tile_elems(plan->grad_dtype, kVptReduce)));
         bool v = true;
         for (int t = 0; t < ntens; ++t) v = v && same_phase(&p->grad[t * n], n);
         p->vec_ok = v;

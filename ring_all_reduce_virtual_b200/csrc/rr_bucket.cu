@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(kThreads) bucket_fold_kernel(const __grid_cons
             return static_cast<const T*>(p.grad[base + r]) + sg.off;
         };
         auto out = [&](int o) { return static_cast<T*>(p.grad[base + o]) + sg.off; };
-        fold_tile<G, OP>(in, n, out, n, sg.len, tile, p.vec_ok, p.divisor);
+        fold_tile<G, OP, kVptReduce, kGroup>(in, n, out, n, sg.len, tile, p.vec_ok, p.divisor);
     }
 }
 

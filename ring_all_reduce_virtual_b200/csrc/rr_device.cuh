@@ -24,7 +24,7 @@ namespace rr {
 
 constexpr int kMaxRanks = 64;
 constexpr int kThreads = 256;  // threads per CTA of every kernel
-constexpr int kGroup = 8;      // input ranks whose loads are issued together
+constexpr int kGroup = 8;      // input ranks whose loads are issued together (N-input folds)
 
 enum OpCode : int { kSum = 0, kAvg = 1, kMax = 2, kMin = 3, kProd = 4 };
 
@@ -166,14 +166,11 @@ __device__ __forceinline__ void fold_one(const InF& in, int nin, const OutF& out
     for (int o = 0; o < nout; ++o) Ty::st1(out(o) + e, acc);
 }
 
-// Vectors per tile per thread.
-template <class Ty>
-struct Vpt {
-    static constexpr int value = 2;
-};
-
 // Fold (nin > 1) or copy (nin == 1) tile `tile` of a segment of `len`
-// elements.  in(j) / out(o) return the segment's base pointers.  vec_ok says
+// elements.  VPT is the number of 16-byte vectors per thread per tile, G the
+// number of further input ranks whose loads are issued before they are
+// folded: every thread keeps up to VPT * (G + 1) loads in flight.  in(j) /
+// out(o) return the segment's base pointers.  vec_ok says
 // that every in(j) has the same address modulo 16 as in(0), and every out(o)
 // the same as out(0) (checked by the host); when in(0) and out(0) also agree,
 // the segment splits into a scalar head up to the first 16-byte boundary, a
@@ -181,14 +178,13 @@ struct Vpt {
 // scalar.  Tile t covers body vectors [t*TV, (t+1)*TV), TV = kThreads*VPT, or
 // the same number of elements on the scalar path; tile 0 also does the head
 // and tail.
-template <class Ty, int OP, class InF, class OutF>
+template <class Ty, int OP, int VPT, int G, class InF, class OutF>
 __device__ __forceinline__ void fold_tile(const InF& in, int nin, const OutF& out, int nout, uint64_t len,
                                           uint64_t tile, bool vec_ok, float divisor)
 {
     using T = typename Ty::T;
     using Acc = typename Ty::Acc;
     constexpr int L = Ty::L;
-    constexpr int VPT = Vpt<Ty>::value;
     constexpr uint64_t TV = (uint64_t)kThreads * VPT;
     const int tid = threadIdx.x;
     const int pin = phase_of(in(0), L);
@@ -242,10 +238,10 @@ __device__ __forceinline__ void fold_tile(const InF& in, int nin, const OutF& ou
         for (int u = 0; u < VPT; ++u)
             if (ok[u]) Ty::unpack(ldv(p + off[u]), a[u]);
     }
-    for (int g = 1; g < nin; g += kGroup) {
-        uint4 raw[kGroup][VPT];
+    for (int g = 1; g < nin; g += G) {
+        uint4 raw[G][VPT];
 #pragma unroll
-        for (int k = 0; k < kGroup; ++k) {
+        for (int k = 0; k < G; ++k) {
             if (g + k < nin) {
                 const T* p = in(g + k);
 #pragma unroll
@@ -254,7 +250,7 @@ __device__ __forceinline__ void fold_tile(const InF& in, int nin, const OutF& ou
             }
         }
 #pragma unroll
-        for (int k = 0; k < kGroup; ++k) {
+        for (int k = 0; k < G; ++k) {
             if (g + k < nin) {
 #pragma unroll
                 for (int u = 0; u < VPT; ++u) {

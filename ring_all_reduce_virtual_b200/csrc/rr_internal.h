@@ -24,6 +24,8 @@ struct RankParams {
     uint64_t count; // elements per rank buffer (all-reduce)
     uint64_t nseg;  // segments
     uint64_t tps;   // tiles per segment
+    uint64_t lo;    // one-shot all-reduce: element range [lo, hi) of every
+    uint64_t hi;    //   rank processed by this launch
 };
 
 // One segment of a table-driven step (a ring step, a tree level): fold
@@ -86,9 +88,15 @@ struct BucketFoldParams {
 enum DType : int { kF32 = 0, kBF16 = 1, kI32 = 2 };
 enum Kind : int { kOneshotRing = 0, kOneshotTree = 1, kReduceScatter = 2, kAllGather = 3, kAllToAll = 4 };
 
+// Vectors per thread per tile: kernels that fold N inputs keep N loads per
+// vector in flight and use few vectors; kernels with one or two inputs use
+// more vectors to keep as many loads in flight.
+constexpr int kVptReduce = 2;
+constexpr int kVptMove = 4;
+
 // Elements one fold tile covers (for sizing tiles per segment on the host),
 // and one bucket pack/unpack tile.
-uint64_t tile_elems(int dtype);
+uint64_t tile_elems(int dtype, int vpt);
 uint64_t bucket_tile_elems(int grad_dtype);
 
 // Resident CTAs per SM of a kernel at kThreads threads (cached per kernel).

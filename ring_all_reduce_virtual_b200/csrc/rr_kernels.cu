@@ -21,7 +21,7 @@ namespace rr {
 namespace {
 
 template <class Ty>
-constexpr uint64_t kTileElems = (uint64_t)kThreads * Vpt<Ty>::value * Ty::L;
+constexpr uint64_t kTileElems = (uint64_t)kThreads * kVptReduce * Ty::L;  // tree one-shot tiles
 
 // ------------------------------------------------ one-shot, ring order
 // Segment c = chunk c of every rank buffer; its fold starts on rank c and
@@ -34,9 +34,12 @@ __global__ void __launch_bounds__(kThreads) oneshot_ring_kernel(const __grid_con
     const uint64_t total = p.nseg * p.tps;
     for (uint64_t w = blockIdx.x; w < total; w += gridDim.x) {
         const uint64_t c = w / p.tps, tile = w - c * p.tps;
-        const uint64_t lo = c * p.C;
-        if (lo >= p.count) continue;
-        const uint64_t len = p.count - lo < p.C ? p.count - lo : p.C;
+        // chunk c clipped to this launch's element range
+        const uint64_t c_lo = c * p.C, c_hi = c_lo + p.C < p.count ? c_lo + p.C : p.count;
+        const uint64_t lo = c_lo > p.lo ? c_lo : p.lo;
+        const uint64_t hi = c_hi < p.hi ? c_hi : p.hi;
+        if (lo >= hi) continue;
+        const uint64_t len = hi - lo;
         const int start = (int)c;
         auto in = [&](int j) {
             int r = start + j;
@@ -44,7 +47,7 @@ __global__ void __launch_bounds__(kThreads) oneshot_ring_kernel(const __grid_con
             return static_cast<const T*>(p.in[r]) + lo;
         };
         auto out = [&](int o) { return static_cast<T*>(p.out[o]) + lo; };
-        fold_tile<Ty, OP>(in, p.n, out, p.n, len, tile, p.vec_ok, p.divisor);
+        fold_tile<Ty, OP, kVptReduce, kGroup>(in, p.n, out, p.n, len, tile, p.vec_ok, p.divisor);
     }
 }
 
@@ -66,7 +69,7 @@ __global__ void __launch_bounds__(kThreads) reduce_scatter_kernel(const __grid_c
             return static_cast<const T*>(p.in[q]) + lo;
         };
         auto out = [&](int) { return static_cast<T*>(p.out[start]); };
-        fold_tile<Ty, OP>(in, p.n, out, 1, p.C, tile, p.vec_ok, p.divisor);
+        fold_tile<Ty, OP, kVptReduce, kGroup>(in, p.n, out, 1, p.C, tile, p.vec_ok, p.divisor);
     }
 }
 
@@ -82,7 +85,7 @@ __global__ void __launch_bounds__(kThreads) all_gather_kernel(const __grid_const
         const uint64_t q = w / p.tps, tile = w - q * p.tps;
         auto in = [&](int) { return static_cast<const T*>(p.in[q]); };
         auto out = [&](int o) { return static_cast<T*>(p.out[o]) + q * p.C; };
-        fold_tile<Ty, kSum>(in, 1, out, p.n, p.C, tile, p.vec_ok, 1.0f);
+        fold_tile<Ty, kSum, kVptMove, 1>(in, 1, out, p.n, p.C, tile, p.vec_ok, 1.0f);
     }
 }
 
@@ -98,7 +101,7 @@ __global__ void __launch_bounds__(kThreads) all_to_all_kernel(const __grid_const
         const uint64_t r = s / (uint64_t)p.n, q = s - r * (uint64_t)p.n;
         auto in = [&](int) { return static_cast<const T*>(p.in[q]) + r * p.C; };
         auto out = [&](int) { return static_cast<T*>(p.out[r]) + q * p.C; };
-        fold_tile<Ty, kSum>(in, 1, out, 1, p.C, tile, 1, 1.0f);
+        fold_tile<Ty, kSum, kVptMove, 1>(in, 1, out, 1, p.C, tile, 1, 1.0f);
     }
 }
 
@@ -208,7 +211,7 @@ __global__ void __launch_bounds__(kThreads) oneshot_tree_kernel(const __grid_con
             const uint64_t e = (uint64_t)tid < head ? (uint64_t)tid : tail_lo + ((uint64_t)tid - head);
             tree_fold_lanes<Ty, OP, 1>(p, e, false);
         }
-        for (int u = 0; u < Vpt<Ty>::value; ++u) {
+        for (int u = 0; u < kVptReduce; ++u) {
             const uint64_t v = tile * (TE / L) + (uint64_t)u * kThreads + tid;
             if (v < nv) tree_fold_lanes<Ty, OP, L>(p, head + v * L, true);
         }
@@ -229,7 +232,7 @@ __global__ void __launch_bounds__(kThreads) step_kernel(const __grid_constant__ 
         if (sg.len == 0) continue;
         auto in = [&](int j) { return static_cast<const T*>(j == 0 ? sg.in0 : sg.in1); };
         auto out = [&](int) { return static_cast<T*>(sg.out); };
-        fold_tile<Ty, OP>(in, p.nin, out, 1, sg.len, tile, p.vec_ok, p.divisor);
+        fold_tile<Ty, OP, kVptMove, 1>(in, p.nin, out, 1, sg.len, tile, p.vec_ok, p.divisor);
     }
 }
 
@@ -306,13 +309,9 @@ cudaError_t resident_ctas(const void* kernel, int* out)
     return cudaSuccess;
 }
 
-uint64_t tile_elems(int dtype)
+uint64_t tile_elems(int dtype, int vpt)
 {
-    switch (dtype) {
-    case kF32: return kTileElems<F32T>;
-    case kBF16: return kTileElems<BF16T>;
-    default: return kTileElems<I32T>;
-    }
+    return (uint64_t)kThreads * (uint64_t)vpt * (dtype == kBF16 ? 8u : 4u);
 }
 
 cudaError_t launch_rank_kernel(int kind, int dtype, int op, const RankParams& p, cudaStream_t s)

@@ -27,7 +27,8 @@ ORACLE = {
     "tree": oracle.tree_schedule,
     "tree_oneshot": oracle.tree_fold,
 }
-TILE = {"f32": 2048, "bf16": 4096, "i32": 2048}  # elements per tile of the fold kernels
+TILE = {"f32": 2048, "bf16": 4096, "i32": 2048}  # elements per tile of the N-input fold kernels
+TILE_MOVE = {"f32": 4096, "bf16": 8192, "i32": 4096}  # per tile of the 1- and 2-input kernels
 
 
 def _dist(op, dtype):
@@ -172,7 +173,7 @@ def test_max_signed_zero_ties_follow_the_fold():
 def test_ring_steps_track_the_oracle_state(n, dtype, op):
     # after every one of the 2(N-1) steps the device buffers equal the
     # oracle's per-rank chunk arrays bit for bit
-    count = 2 * TILE[dtype] * n + 13
+    count = 3 * TILE_MOVE[dtype] * n + 13
     x = synth.ranks(6, n, count, "uniform", dtype)
     d = to_dev(x)
     host = [a.copy() for a in x]
@@ -203,7 +204,7 @@ def test_ring_stats_match_the_schedule():
 @pytest.mark.parametrize("n", [1, 2, 3, 4, 8, 64])
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "i32"])
 def test_reduce_scatter_all_gather_all_to_all(n, dtype):
-    per = 2 * TILE[dtype] + 9
+    per = 2 * TILE_MOVE[dtype] + 9
     x = synth.ranks(8, n, n * per, "int" if dtype == "i32" else "uniform", dtype)
     d = to_dev(x)
     for op in ("sum", "max") if dtype != "bf16" else ("sum", "avg"):
@@ -294,3 +295,25 @@ def test_bucket_fused_misaligned_tensors():
         plan.all_reduce(b, grads, "avg")
     for r in range(n):
         assert_bits_equal(to_host(grads[r]), want[r], f"rank {r}")
+
+
+# ------------------------------------------------------ host buffers --
+
+@pytest.mark.parametrize("algo", ["auto", "oneshot", "tree_oneshot", "ring"])
+@pytest.mark.parametrize("count", [1000, (8 << 20) // 4 * 3 + 17])  # below and above one 8 MiB slice
+def test_allreduce_host_buffers(algo, count):
+    # host -> device -> reduce -> host, pipelined in slices for the one-shot
+    # algorithms; ordered on a side stream; host and device both hold the result
+    n = 4
+    x = synth.ranks(12, n, count, "uniform")
+    want = [a.copy() for a in x]
+    ORACLE[algo](want, "avg")
+    host = [torch.from_numpy(a.copy()).pin_memory() for a in x]
+    dev = [torch.full((count,), float("nan"), device="cuda") for _ in range(n)]
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        rrv.all_reduce_host(host, dev, "avg", algo, side)
+    side.synchronize()
+    assert_bits_equal([h.numpy() for h in host], want, "host")
+    assert_bits_equal(to_host(dev), want, "device")
