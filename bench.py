@@ -511,21 +511,23 @@ def run_gpt_buckets(args):
     grads = [[(torch.randn(m, device=dev, generator=gen) * 1e-3).to(torch.bfloat16) for m in numels]
              for _ in range(n)]
     plan = rrv.BucketPlan(numels, "bf16", synth.BUCKET_CAP_BYTES)
+    gset = rrv.GradSet(grads)  # pointers marshalled once, as a DDP step would
     nb = plan.num_buckets
     biggest = max(plan.info(b)[2] for b in range(nb))
     buckets = [torch.empty(biggest, dtype=torch.float32, device=dev) for _ in range(n)]
     peak, _ = hbm_peak()
 
+    views = [[t[:plan.info(b)[2]] for t in buckets] for b in range(nb)]
+
     def fused():
         for b in range(nb):
-            plan.all_reduce(b, grads, "avg", stream)
+            plan.all_reduce(b, gset, "avg", stream)
 
     def staged():
         for b in range(nb):
-            numel = plan.info(b)[2]
-            plan.pack(b, grads, buckets, stream)
-            rrv.all_reduce([t[:numel] for t in buckets], "sum", "auto", stream)
-            plan.unpack(b, buckets, grads, "avg", stream)
+            plan.pack(b, gset, buckets, stream)
+            rrv.all_reduce(views[b], "sum", "auto", stream)
+            plan.unpack(b, buckets, gset, "avg", stream)
 
     for name, fn, bpp in (("fused", fused, 4), ("staged", staged, 20)):
         for _ in range(max(args.warmup, 3)):

@@ -21,7 +21,7 @@ from ._lib import MAX_RANKS, Cost, RingEvent, RRError, Stats, check, lib
 
 __all__ = [
     "all_reduce", "all_reduce_host", "ring_step", "ring_schedule", "reduce_scatter", "all_gather", "all_to_all",
-    "BucketPlan", "cost_model", "pick_algo", "set_picker_params", "last_stats", "RRError",
+    "BucketPlan", "GradSet", "cost_model", "pick_algo", "set_picker_params", "last_stats", "RRError",
     "OPS", "ALGOS", "MAX_RANKS",
 ]
 
@@ -152,6 +152,23 @@ def all_to_all(send: Sequence, recv: Sequence, stream=None) -> None:
           "all_to_all")
 
 
+class GradSet:
+    """The gradient tensors of all ranks (``grads[r][t]``), with their device
+    pointers marshalled once.  Bucket calls accept either this or the nested
+    lists; a DDP step reuses the same gradient buffers every step, so building
+    the pointer array once keeps the per-bucket host cost to a few
+    microseconds."""
+
+    def __init__(self, grads: Sequence[Sequence]):
+        flat = [g for rank in grads for g in rank]
+        if not flat:
+            raise ValueError("GradSet: no gradients")
+        self.nranks = len(grads)
+        self.device = flat[0].device
+        self.ptrs = _ptr_array(flat)
+        self._keep = [list(rank) for rank in grads]  # the tensors must outlive the pointers
+
+
 class BucketPlan:
     """DDP-style bucket plan over a list of gradient sizes (``rr_bucket_plan``)."""
 
@@ -187,9 +204,11 @@ class BucketPlan:
         return b.value, o.value
 
     @staticmethod
-    def _grads(grads: Sequence[Sequence]):
-        flat = [g for rank in grads for g in rank]
-        return _ptr_array(flat), len(grads), flat[0].device
+    def _grads(grads):
+        if isinstance(grads, GradSet):
+            return grads.ptrs, grads.nranks, grads.device
+        gs = GradSet(grads)
+        return gs.ptrs, gs.nranks, gs.device
 
     def pack(self, bucket: int, grads: Sequence[Sequence], buckets: Sequence, stream=None) -> None:
         """``grads[r][t]`` -> fp32 ``buckets[r]`` for the bucket's tensors."""

@@ -414,7 +414,7 @@ rr_status_t rr_allreduce(void* const* bufs, int nranks, size_t count, rr_dtype_t
         break;
     case RR_ALGO_ONESHOT: {
         const uint64_t C = ceil_div(count, (uint64_t)n);
-        const uint64_t tps = std::max<uint64_t>(1, ceil_div(C, tile_elems(dtype, kVptReduce)));
+        const uint64_t tps = std::max<uint64_t>(1, ceil_div(C, tile_elems(dtype, reduce_vpt(n))));
         st = run_rank_kernel(kOneshotRing, bufs, bufs, n, C, count, (uint64_t)n, tps, dtype, op,
                              same_phase(bufs, n), stream);
         t_stats.steps = 1;
@@ -496,7 +496,8 @@ rr_status_t rr_allreduce_host(void* const* host_bufs, void* const* dev_bufs, int
         if ((st = ck(cudaEventRecord(hp->arrived, hp->in), "event record")) != RR_OK) return st;
         if ((st = ck(cudaStreamWaitEvent(stream, hp->arrived, 0), "stream wait")) != RR_OK) return st;
         if (a == RR_ALGO_ONESHOT) {
-            const uint64_t tps = std::max<uint64_t>(1, ceil_div(std::min(C, len), tile_elems(dtype, kVptReduce)));
+            const uint64_t tps =
+                std::max<uint64_t>(1, ceil_div(std::min(C, len), tile_elems(dtype, reduce_vpt(n))));
             st = run_rank_kernel(kOneshotRing, dev_bufs, dev_bufs, n, C, count, (uint64_t)n, tps, dtype, op, vec,
                                  stream, lo, hi);
         } else {
@@ -602,7 +603,7 @@ rr_status_t rr_reduce_scatter(const void* const* send, void* const* recv, int nr
     }
     if ((st = check_spans(spans)) != RR_OK) return st;
     if ((st = check_device_ptrs(send, n)) != RR_OK || (st = check_device_ptrs(recv, n)) != RR_OK) return st;
-    const uint64_t tps = std::max<uint64_t>(1, ceil_div(recvcount, tile_elems(dtype, kVptReduce)));
+    const uint64_t tps = std::max<uint64_t>(1, ceil_div(recvcount, tile_elems(dtype, reduce_vpt(n))));
     st = run_rank_kernel(kReduceScatter, send, recv, n, recvcount, (uint64_t)n * recvcount, (uint64_t)n, tps,
                          dtype, op, same_phase(send, n) && same_phase(recv, n), stream);
     t_stats.steps = 1;
@@ -849,7 +850,7 @@ rr_status_t rr_bucket_allreduce(const rr_bucket_plan_t* plan, int bucket, void* 
         for (int s = 0; s < p->nseg; ++s) maxlen = std::max(maxlen, p->seg[s].len);
         p->n = n;
         p->divisor = (float)n;
-        p->tps = std::max<uint64_t>(1, ceil_div(maxlen, tile_elems(plan->grad_dtype, kVptReduce)));
+        p->tps = std::max<uint64_t>(1, ceil_div(maxlen, tile_elems(plan->grad_dtype, reduce_vpt(n))));
         bool v = true;
         for (int t = 0; t < ntens; ++t) v = v && same_phase(&p->grad[t * n], n);
         p->vec_ok = v;

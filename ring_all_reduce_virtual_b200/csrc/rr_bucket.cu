@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(kThreads) bucket_unpack_kernel(const __grid_co
 // bucket's flat index; every rank's copy is read once, folded in fp32 in ring
 // order from rank c, divided (AVG), rounded once and written back to every
 // rank.  Same bits as pack -> one-shot all-reduce (SUM) -> unpack.
-template <class G, int OP>
+template <class G, int OP, int VPT, int GR>
 __global__ void __launch_bounds__(kThreads) bucket_fold_kernel(const __grid_constant__ BucketFoldParams p)
 {
     using T = typename G::T;
@@ -125,32 +125,26 @@ __global__ void __launch_bounds__(kThreads) bucket_fold_kernel(const __grid_cons
             return static_cast<const T*>(p.grad[base + r]) + sg.off;
         };
         auto out = [&](int o) { return static_cast<T*>(p.grad[base + o]) + sg.off; };
-        fold_tile<G, OP, kVptReduce, kGroup>(in, n, out, n, sg.len, tile, p.vec_ok, p.divisor);
+        fold_tile<G, OP, VPT, GR>(in, n, out, n, sg.len, tile, p.vec_ok, p.divisor);
     }
 }
 
-int sm_count_b()
-{
-    static int sms = [] {
-        int dev = 0, v = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-        return v > 0 ? v : 148;
-    }();
-    return sms;
-}
-
 template <class P>
-cudaError_t launch_wave_b(void (*kernel)(P), const P& p, uint64_t work, cudaStream_t s)
+cudaError_t launch_all_b(void (*kernel)(P), const P& p, uint64_t work, cudaStream_t s)
 {
     if (work == 0) return cudaSuccess;
-    int occ = 0;
-    cudaError_t e = resident_ctas(reinterpret_cast<const void*>(kernel), &occ);
-    if (e != cudaSuccess) return e;
-    uint64_t grid = (uint64_t)sm_count_b() * (uint64_t)occ;
-    if (grid > work) grid = work;
+    const uint64_t grid = work < kMaxGrid ? work : kMaxGrid;
     kernel<<<(unsigned)grid, kThreads, 0, s>>>(p);
     return cudaGetLastError();
+}
+
+template <class G, int OP>
+cudaError_t launch_fold(const BucketFoldParams& p, uint64_t work, cudaStream_t s)
+{
+    const int vpt = reduce_vpt(p.n);
+    if (vpt == 8) return launch_all_b(bucket_fold_kernel<G, OP, 8, 1>, p, work, s);
+    if (vpt == 4) return launch_all_b(bucket_fold_kernel<G, OP, 4, 3>, p, work, s);
+    return launch_all_b(bucket_fold_kernel<G, OP, kVptReduce, kGroup>, p, work, s);
 }
 
 }  // namespace
@@ -165,8 +159,8 @@ uint64_t bucket_tile_elems(int grad_dtype)
 cudaError_t launch_bucket_pack(int grad_dtype, const BucketCopyParams& p, cudaStream_t s)
 {
     const uint64_t work = (uint64_t)p.nt * (uint64_t)p.n * p.tps;
-    if (grad_dtype == kBF16) return launch_wave_b(bucket_pack_kernel<BF16T>, p, work, s);
-    if (grad_dtype == kF32) return launch_wave_b(bucket_pack_kernel<F32T>, p, work, s);
+    if (grad_dtype == kBF16) return launch_all_b(bucket_pack_kernel<BF16T>, p, work, s);
+    if (grad_dtype == kF32) return launch_all_b(bucket_pack_kernel<F32T>, p, work, s);
     return cudaErrorInvalidValue;
 }
 
@@ -175,11 +169,11 @@ cudaError_t launch_bucket_unpack(int grad_dtype, int op, const BucketCopyParams&
     const uint64_t work = (uint64_t)p.nt * (uint64_t)p.n * p.tps;
     const bool avg = op == kAvg;
     if (grad_dtype == kBF16)
-        return avg ? launch_wave_b(bucket_unpack_kernel<BF16T, kAvg>, p, work, s)
-                   : launch_wave_b(bucket_unpack_kernel<BF16T, kSum>, p, work, s);
+        return avg ? launch_all_b(bucket_unpack_kernel<BF16T, kAvg>, p, work, s)
+                   : launch_all_b(bucket_unpack_kernel<BF16T, kSum>, p, work, s);
     if (grad_dtype == kF32)
-        return avg ? launch_wave_b(bucket_unpack_kernel<F32T, kAvg>, p, work, s)
-                   : launch_wave_b(bucket_unpack_kernel<F32T, kSum>, p, work, s);
+        return avg ? launch_all_b(bucket_unpack_kernel<F32T, kAvg>, p, work, s)
+                   : launch_all_b(bucket_unpack_kernel<F32T, kSum>, p, work, s);
     return cudaErrorInvalidValue;
 }
 
@@ -187,12 +181,8 @@ cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p
 {
     const uint64_t work = (uint64_t)p.nseg * p.tps;
     const bool avg = op == kAvg;
-    if (grad_dtype == kBF16)
-        return avg ? launch_wave_b(bucket_fold_kernel<BF16T, kAvg>, p, work, s)
-                   : launch_wave_b(bucket_fold_kernel<BF16T, kSum>, p, work, s);
-    if (grad_dtype == kF32)
-        return avg ? launch_wave_b(bucket_fold_kernel<F32T, kAvg>, p, work, s)
-                   : launch_wave_b(bucket_fold_kernel<F32T, kSum>, p, work, s);
+    if (grad_dtype == kBF16) return avg ? launch_fold<BF16T, kAvg>(p, work, s) : launch_fold<BF16T, kSum>(p, work, s);
+    if (grad_dtype == kF32) return avg ? launch_fold<F32T, kAvg>(p, work, s) : launch_fold<F32T, kSum>(p, work, s);
     return cudaErrorInvalidValue;
 }
 

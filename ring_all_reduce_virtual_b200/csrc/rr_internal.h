@@ -94,13 +94,19 @@ enum Kind : int { kOneshotRing = 0, kOneshotTree = 1, kReduceScatter = 2, kAllGa
 constexpr int kVptReduce = 2;
 constexpr int kVptMove = 4;
 
+// Vectors per thread of the N-input folds (one-shot all-reduce, reduce-scatter,
+// fused bucket sync) by rank count: few ranks give few loads per vector, so
+// each thread takes more vectors (N * VPT loads in flight).
+inline int reduce_vpt(int n) { return n <= 2 ? 8 : (n <= 4 ? 4 : kVptReduce); }
+
 // Elements one fold tile covers (for sizing tiles per segment on the host),
 // and one bucket pack/unpack tile.
 uint64_t tile_elems(int dtype, int vpt);
 uint64_t bucket_tile_elems(int grad_dtype);
 
-// Resident CTAs per SM of a kernel at kThreads threads (cached per kernel).
-cudaError_t resident_ctas(const void* kernel, int* out);
+// Launch configuration: one CTA per work item (a tile of a segment), up to
+// the grid limit; kernels loop over the rest.
+constexpr uint64_t kMaxGrid = 0x7fffffffull;
 
 // Launchers: return the launch's cudaError_t.  `op` is an rr_op_t value.
 cudaError_t launch_rank_kernel(int kind, int dtype, int op, const RankParams& p, cudaStream_t s);
