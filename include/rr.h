@@ -87,15 +87,21 @@ typedef enum rr_op { RR_SUM = 0, RR_AVG = 1, RR_MAX = 2, RR_MIN = 3, RR_PROD = 4
  *   TREE         the tree schedule: ceil(log2 N) pairwise reduce levels,
  *                then as many broadcast levels ([P3] s6)
  *   TREE_ONESHOT one launch that folds in the tree's pairwise order
- *   AUTO         the picker's choice between RING and ONESHOT (never a tree
- *                order, whose bits differ); env RR_ALGO=ring|oneshot|tree|
- *                tree_oneshot overrides it. */
+ *   TWO_SHOT     two launches: a reduce-scatter by direct reads (chunk c
+ *                folded in ring order into its owner, rank c), then an
+ *                all-gather by direct reads ([P4] "alpha-beta model": the
+ *                two-shot all-reduce); the ring's bits and its 2(N-1)/N S
+ *                bytes per rank, in 2 steps instead of 2(N-1)
+ *   AUTO         the picker's choice among RING, ONESHOT and TWO_SHOT
+ *                (never a tree order, whose bits differ); env
+ *                RR_ALGO=ring|oneshot|tree|tree_oneshot|two_shot overrides it. */
 typedef enum rr_algo {
     RR_ALGO_AUTO = 0,
     RR_ALGO_RING = 1,
     RR_ALGO_ONESHOT = 2,
     RR_ALGO_TREE = 3,
-    RR_ALGO_TREE_ONESHOT = 4
+    RR_ALGO_TREE_ONESHOT = 4,
+    RR_ALGO_TWO_SHOT = 5
 } rr_algo_t;
 
 /* The two phases of the ring ([P3] s3; [P4]). */

@@ -26,7 +26,7 @@ __all__ = [
 ]
 
 OPS = {"sum": 0, "avg": 1, "max": 2, "min": 3, "prod": 4}
-ALGOS = {"auto": 0, "ring": 1, "oneshot": 2, "tree": 3, "tree_oneshot": 4}
+ALGOS = {"auto": 0, "ring": 1, "oneshot": 2, "tree": 3, "tree_oneshot": 4, "two_shot": 5}
 ALGO_NAMES = {v: k for k, v in ALGOS.items()}
 PHASES = {"reduce_scatter": 0, "all_gather": 1}
 _DTYPE_NAMES = {"f32": 0, "bf16": 1, "i32": 2}
@@ -209,6 +209,28 @@ class BucketPlan:
             return grads.ptrs, grads.nranks, grads.device
         gs = GradSet(grads)
         return gs.ptrs, gs.nranks, gs.device
+
+    def flat_buffers(self, nranks: int, device=None, dtype=None):
+        """Gradients laid out as views into one flat buffer per bucket and
+        rank (DDP's ``gradient_as_bucket_view``): returns ``(flats, grads)``
+        with ``flats[b][r]`` the bucket's buffer on rank r and ``grads[r][t]``
+        a view of tensor t inside it.  A bucket sync on this layout is
+        ``all_reduce(flats[b], op, "oneshot")``, with the same bits as
+        ``all_reduce(b, grads, op)`` and no gather or scatter at all.  (The
+        buffers are allocated by PyTorch here, not by the library.)"""
+        import torch
+
+        dtype = dtype or torch.bfloat16
+        flats, grads = [], [[None] * len(self.numels) for _ in range(nranks)]
+        for b in range(self.num_buckets):
+            first, cnt, numel = self.info(b)
+            row = [torch.zeros(numel, dtype=dtype, device=device) for _ in range(nranks)]
+            flats.append(row)
+            for t in range(first, first + cnt):
+                off = self.tensor(t)[1]
+                for r in range(nranks):
+                    grads[r][t] = row[r][off:off + self.numels[t]]
+        return flats, grads
 
     def pack(self, bucket: int, grads: Sequence[Sequence], buckets: Sequence, stream=None) -> None:
         """``grads[r][t]`` -> fp32 ``buckets[r]`` for the bucket's tensors."""

@@ -74,6 +74,7 @@ const char* algo_name(int a)
     case RR_ALGO_ONESHOT: return "oneshot";
     case RR_ALGO_TREE: return "tree";
     case RR_ALGO_TREE_ONESHOT: return "tree_oneshot";
+    case RR_ALGO_TWO_SHOT: return "two_shot";
     }
     return "?";
 }
@@ -280,7 +281,7 @@ rr_status_t run_tree(void* const* bufs, int n, size_t count, rr_dtype_t dtype, r
 
 rr_status_t run_rank_kernel(int kind, const void* const* in, void* const* out, int n, uint64_t C,
                             uint64_t count, uint64_t nseg, uint64_t tps, rr_dtype_t dtype, int op, bool vec,
-                            cudaStream_t stream, uint64_t lo = 0, uint64_t hi = UINT64_MAX)
+                            cudaStream_t stream, uint64_t lo = 0, uint64_t hi = UINT64_MAX, bool owner_only = false)
 {
     RankParams p{};
     for (int r = 0; r < n; ++r) {
@@ -296,6 +297,7 @@ rr_status_t run_rank_kernel(int kind, const void* const* in, void* const* out, i
     p.tps = tps;
     p.lo = lo;
     p.hi = hi;
+    p.owner_only = owner_only ? 1 : 0;
     cudaError_t e = launch_rank_kernel(kind, dtype, op, p, stream);
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     t_stats.launches += 1;
@@ -312,6 +314,7 @@ rr_algo_t resolve_algo(rr_algo_t algo, int n, size_t count, rr_dtype_t dtype)
         if (!std::strcmp(v, "oneshot")) return (int)RR_ALGO_ONESHOT;
         if (!std::strcmp(v, "tree")) return (int)RR_ALGO_TREE;
         if (!std::strcmp(v, "tree_oneshot")) return (int)RR_ALGO_TREE_ONESHOT;
+        if (!std::strcmp(v, "two_shot")) return (int)RR_ALGO_TWO_SHOT;
         return -1;
     }();
     if (forced >= 0) return (rr_algo_t)forced;
@@ -391,7 +394,7 @@ rr_status_t rr_allreduce(void* const* bufs, int nranks, size_t count, rr_dtype_t
 {
     rr_status_t st = check_basic(nranks, dtype, op);
     if (st != RR_OK) return st;
-    if (algo < RR_ALGO_AUTO || algo > RR_ALGO_TREE_ONESHOT) return fail(RR_ERR_INVALID_ARG, "unknown algo");
+    if (algo < RR_ALGO_AUTO || algo > RR_ALGO_TWO_SHOT) return fail(RR_ERR_INVALID_ARG, "unknown algo");
     if (!bufs) return fail(RR_ERR_INVALID_ARG, "NULL bufs array");
     const int n = nranks;
     const size_t es = esize(dtype);
@@ -423,6 +426,28 @@ rr_status_t rr_allreduce(void* const* bufs, int nranks, size_t count, rr_dtype_t
         t_stats.hbm_bytes = 2ull * n * S;
         break;
     }
+    case RR_ALGO_TWO_SHOT: {
+        // shot 1: chunk c folded in ring order into rank c only; shot 2: every
+        // rank copies the chunks it does not own from their owners
+        const uint64_t C = ceil_div(count, (uint64_t)n);
+        const bool vec = same_phase(bufs, n);
+        uint64_t tps = std::max<uint64_t>(1, ceil_div(C, tile_elems(dtype, reduce_vpt(n))));
+        st = run_rank_kernel(kOneshotRing, bufs, bufs, n, C, count, (uint64_t)n, tps, dtype, op, vec, stream, 0,
+                             UINT64_MAX, true);
+        if (st != RR_OK) break;
+        tps = std::max<uint64_t>(1, ceil_div(C, tile_elems(dtype, kVptMove)));
+        st = run_rank_kernel(kChunkBroadcast, bufs, bufs, n, C, count, (uint64_t)n, tps, dtype, RR_SUM, vec, stream);
+        t_stats.steps = 2;
+        t_stats.bytes_sent_max = 0;
+        for (int r = 0; r < n; ++r) {  // r sends its copy of every other chunk, then its own chunk N-1 times
+            const uint64_t own = chunk_len(count, n, r) * es;
+            const uint64_t b = (S - own) + (uint64_t)(n - 1) * own;
+            t_stats.bytes_sent_max = std::max(t_stats.bytes_sent_max, b);
+            t_stats.bytes_sent_total += b;
+        }
+        t_stats.hbm_bytes = (2ull * n + 1) * S;  // shot 1: N S read, S written; shot 2: S read, (N-1) S written
+        break;
+    }
     case RR_ALGO_TREE_ONESHOT: {
         const uint64_t tps = std::max<uint64_t>(1, ceil_div(count, tile_elems(dtype, kVptReduce)));
         st = run_rank_kernel(kOneshotTree, bufs, bufs, n, count, count, 1, tps, dtype, op, same_phase(bufs, n),
@@ -445,7 +470,7 @@ rr_status_t rr_allreduce_host(void* const* host_bufs, void* const* dev_bufs, int
 {
     rr_status_t st = check_basic(nranks, dtype, op);
     if (st != RR_OK) return st;
-    if (algo < RR_ALGO_AUTO || algo > RR_ALGO_TREE_ONESHOT) return fail(RR_ERR_INVALID_ARG, "unknown algo");
+    if (algo < RR_ALGO_AUTO || algo > RR_ALGO_TWO_SHOT) return fail(RR_ERR_INVALID_ARG, "unknown algo");
     if (!host_bufs || !dev_bufs) return fail(RR_ERR_INVALID_ARG, "NULL pointer array");
     const int n = nranks;
     const size_t es = esize(dtype), bytes = count * es;
@@ -912,6 +937,10 @@ rr_status_t rr_cost_model(rr_algo_t algo, int nranks, double bytes, double alpha
         c.steps = nranks > 1 ? 1 : 0;
         c.bytes_sent = (n - 1) * bytes;
         break;
+    case RR_ALGO_TWO_SHOT:  // [P4]: reduce-scatter then all-gather by direct reads
+        c.steps = nranks > 1 ? 2 : 0;
+        c.bytes_sent = 2 * (n - 1) / n * bytes;
+        break;
     default:
         return fail(RR_ERR_INVALID_ARG, "unknown algo");
     }
@@ -941,7 +970,9 @@ rr_algo_t rr_pick_algo(int nranks, size_t count, rr_dtype_t dtype)
     const double n = nranks, S = (double)count * (double)esize(dtype);
     const double ring = 2 * (n - 1) * g_launch_s + 5 * (n - 1) * S / g_hbm_bps;
     const double one = g_launch_s + 2 * n * S / g_hbm_bps;
-    return ring < one ? RR_ALGO_RING : RR_ALGO_ONESHOT;
+    const double two = 2 * g_launch_s + (2 * n + 1) * S / g_hbm_bps;
+    if (ring < one && ring < two) return RR_ALGO_RING;
+    return two < one ? RR_ALGO_TWO_SHOT : RR_ALGO_ONESHOT;
 }
 
 }  // extern "C"

@@ -16,7 +16,7 @@ namespace rr {
 
 namespace {
 
-constexpr int kUnitsPerThread = 2;
+constexpr int kUnitsPerThread = 4;
 
 // Convert one tile of a segment from In's element type to Out's, dividing by
 // `divisor` first when OP is AVG.  A unit is U elements, one 16-byte vector
@@ -49,16 +49,28 @@ __device__ __forceinline__ void convert_tile(const typename In::T* src, typename
     const uint64_t tail = len - head - nu * U;
     if (tile == 0 && (uint64_t)tid < head + tail)
         one((uint64_t)tid < head ? (uint64_t)tid : head + nu * U + ((uint64_t)tid - head));
+    // all of this thread's loads first (kUnitsPerThread * NI in flight), then
+    // the conversions and stores
+    uint4 raw[kUnitsPerThread][NI];
+    uint64_t e[kUnitsPerThread];
+    bool ok[kUnitsPerThread];
 #pragma unroll
     for (int k = 0; k < kUnitsPerThread; ++k) {
         const uint64_t u = tile * TU + (uint64_t)k * kThreads + tid;
-        if (u >= nu) continue;
-        const uint64_t e = head + u * U;
+        ok[k] = u < nu;
+        e[k] = head + u * U;
+#pragma unroll
+        for (int i = 0; i < NI; ++i)
+            if (ok[k]) raw[k][i] = ldv(src + e[k] + (uint64_t)i * In::L);
+    }
+#pragma unroll
+    for (int k = 0; k < kUnitsPerThread; ++k) {
+        if (!ok[k]) continue;
         float a[U];
 #pragma unroll
         for (int i = 0; i < NI; ++i) {
             typename In::Acc t[In::L];
-            In::unpack(ldv(src + e + (uint64_t)i * In::L), t);
+            In::unpack(raw[k][i], t);
 #pragma unroll
             for (int l = 0; l < In::L; ++l) a[i * In::L + l] = finish<OP>((float)t[l], divisor);
         }
@@ -67,7 +79,7 @@ __device__ __forceinline__ void convert_tile(const typename In::T* src, typename
             typename Out::Acc t[Out::L];
 #pragma unroll
             for (int l = 0; l < Out::L; ++l) t[l] = a[i * Out::L + l];
-            stv(dst + e + (uint64_t)i * Out::L, Out::pack(t));
+            stv(dst + e[k] + (uint64_t)i * Out::L, Out::pack(t));
         }
     }
 }

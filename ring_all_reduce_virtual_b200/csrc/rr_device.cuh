@@ -128,11 +128,24 @@ __device__ __forceinline__ int32_t apply(int32_t a, int32_t b)
 }
 
 // AVG's last step: one IEEE division of the full fold by the rank count.
+// When the count is a power of two its reciprocal is exact, and a * (1/N) is
+// then the same correctly rounded value of the same real quotient as a / N,
+// so the cheaper multiply gives identical bits.
+__device__ __forceinline__ bool is_pow2(float d)
+{
+    const uint32_t u = __float_as_uint(d);
+    return (u & 0x007fffffu) == 0u && d >= 1.0f;  // positive, normal, zero mantissa
+}
+
 template <int OP>
 __device__ __forceinline__ float finish(float a, float divisor)
 {
-    if constexpr (OP == kAvg) return __fdiv_rn(a, divisor);
-    else return a;
+    if constexpr (OP == kAvg) {
+        if (is_pow2(divisor)) return __fmul_rn(a, __frcp_rn(divisor));
+        return __fdiv_rn(a, divisor);
+    } else {
+        return a;
+    }
 }
 
 template <int OP>

@@ -26,6 +26,8 @@ struct RankParams {
     uint64_t tps;   // tiles per segment
     uint64_t lo;    // one-shot all-reduce: element range [lo, hi) of every
     uint64_t hi;    //   rank processed by this launch
+    int owner_only; // one-shot all-reduce: write chunk c only to rank c (two-shot's first shot)
+    int pad2_;
 };
 
 // One segment of a table-driven step (a ring step, a tree level): fold
@@ -86,7 +88,14 @@ struct BucketFoldParams {
 };
 
 enum DType : int { kF32 = 0, kBF16 = 1, kI32 = 2 };
-enum Kind : int { kOneshotRing = 0, kOneshotTree = 1, kReduceScatter = 2, kAllGather = 3, kAllToAll = 4 };
+enum Kind : int {
+    kOneshotRing = 0,
+    kOneshotTree = 1,
+    kReduceScatter = 2,
+    kAllGather = 3,
+    kAllToAll = 4,
+    kChunkBroadcast = 5  // chunk c of rank c copied to chunk c of every other rank
+};
 
 // Vectors per thread per tile: kernels that fold N inputs keep N loads per
 // vector in flight and use few vectors; kernels with one or two inputs use

@@ -44,8 +44,28 @@ __global__ void __launch_bounds__(kThreads) oneshot_ring_kernel(const __grid_con
             if (r >= p.n) r -= p.n;
             return static_cast<const T*>(p.in[r]) + lo;
         };
-        auto out = [&](int o) { return static_cast<T*>(p.out[o]) + lo; };
-        fold_tile<Ty, OP, VPT, G>(in, p.n, out, p.n, len, tile, p.vec_ok, p.divisor);
+        auto out = [&](int o) { return static_cast<T*>(p.out[p.owner_only ? start : o]) + lo; };
+        fold_tile<Ty, OP, VPT, G>(in, p.n, out, p.owner_only ? 1 : p.n, len, tile, p.vec_ok, p.divisor);
+    }
+}
+
+// ------------------------------------------------- chunk broadcast
+// Two-shot's second shot: segment c = chunk c, read once from its owner
+// (rank c) and written to chunk c of the N-1 other ranks.
+template <class Ty>
+__global__ void __launch_bounds__(kThreads) chunk_bcast_kernel(const __grid_constant__ RankParams p)
+{
+    using T = typename Ty::T;
+    const uint64_t total = p.nseg * p.tps;
+    for (uint64_t w = blockIdx.x; w < total; w += gridDim.x) {
+        const uint64_t c = w / p.tps, tile = w - c * p.tps;
+        const uint64_t lo = c * p.C;
+        if (lo >= p.count) continue;
+        const uint64_t len = p.count - lo < p.C ? p.count - lo : p.C;
+        const int owner = (int)c;
+        auto in = [&](int) { return static_cast<const T*>(p.in[owner]) + lo; };
+        auto out = [&](int o) { return static_cast<T*>(p.out[o < owner ? o : o + 1]) + lo; };
+        fold_tile<Ty, kSum, kVptMove, 1>(in, 1, out, p.n - 1, len, tile, p.vec_ok, 1.0f);
     }
 }
 
@@ -281,7 +301,7 @@ uint64_t tile_elems(int dtype, int vpt)
 cudaError_t launch_rank_kernel(int kind, int dtype, int op, const RankParams& p, cudaStream_t s)
 {
     const uint64_t work = kind == kOneshotTree ? p.tps : p.nseg * p.tps;
-    if (kind == kAllGather || kind == kAllToAll) op = kSum;
+    if (kind == kAllGather || kind == kAllToAll || kind == kChunkBroadcast) op = kSum;
     const int vpt = reduce_vpt(p.n);
     return with_type(dtype, op, [&]<class Ty, int OP>() -> cudaError_t {
         switch (kind) {
@@ -296,6 +316,7 @@ cudaError_t launch_rank_kernel(int kind, int dtype, int op, const RankParams& p,
         case kOneshotTree: return launch_all(oneshot_tree_kernel<Ty, OP>, p, work, s);
         case kAllGather: return launch_all(all_gather_kernel<Ty>, p, work, s);
         case kAllToAll: return launch_all(all_to_all_kernel<Ty>, p, work, s);
+        case kChunkBroadcast: return launch_all(chunk_bcast_kernel<Ty>, p, work, s);
         }
         return cudaErrorInvalidValue;
     });

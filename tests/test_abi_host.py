@@ -141,13 +141,16 @@ def test_cost_model_tree_and_oneshot_steps():
         assert rrv.cost_model("tree", n, 1.0, 1.0, 1.0)["steps"] == 2 * np.log2(n)
         assert rrv.cost_model("ring", n, 1.0, 1.0, 1.0)["steps"] == 2 * (n - 1)
         assert rrv.cost_model("oneshot", n, 1.0, 1.0, 1.0)["steps"] == 1
+        # two-shot: the ring's per-rank volume in two steps
+        two = rrv.cost_model("two_shot", n, 1.0, 1.0, 1.0)
+        assert two["steps"] == 2 and two["bytes_sent"] == rrv.cost_model("ring", n, 1.0, 1.0, 1.0)["bytes_sent"]
 
 
 def test_picker_is_size_aware_and_exact():
     # AUTO only ever picks schedules with the ring's bits
     for n in (2, 4, 8, 16, 64):
         for count in (1, 256, 1 << 20, 1 << 28):
-            assert rrv.pick_algo(n, count, "f32") in ("ring", "oneshot")
+            assert rrv.pick_algo(n, count, "f32") in ("ring", "oneshot", "two_shot")
             assert rrv.pick_algo(n, count, "bf16") == "oneshot"
     # with launches free and bandwidth the only cost, fewer bytes win
     rrv.set_picker_params(0.0, 1e12)
@@ -172,6 +175,7 @@ def test_argument_errors_return_before_any_launch():
     assert lib.rr_allreduce(_fake(4), 4, 16, 7, 0, 0, s) == _lib.RR_ERR_INVALID_ARG
     assert lib.rr_allreduce(_fake(4), 4, 16, 0, 9, 0, s) == _lib.RR_ERR_INVALID_ARG
     assert lib.rr_allreduce(_fake(4), 4, 16, 0, 0, 9, s) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_allreduce(_fake(4), 4, 16, 0, 0, 6, s) == _lib.RR_ERR_INVALID_ARG
     assert lib.rr_allreduce(_fake(4), 4, 16, 2, 1, 0, s) == _lib.RR_ERR_UNSUPPORTED  # int32 AVG
     assert lib.rr_allreduce(None, 4, 16, 0, 0, 0, s) == _lib.RR_ERR_INVALID_ARG
     overlapping = _fake(4, stride=32)  # 16 fp32 = 64 bytes apart by 32

@@ -19,8 +19,9 @@ from ring_all_reduce_virtual_b200 import synth
 
 pytestmark = pytest.mark.gpu
 
-ALGOS = ["ring", "oneshot", "tree", "tree_oneshot", "auto"]
+ALGOS = ["ring", "oneshot", "tree", "tree_oneshot", "two_shot", "auto"]
 ORACLE = {
+    "two_shot": oracle.fold_ring_order,
     "ring": oracle.ring_allreduce,
     "oneshot": oracle.fold_ring_order,
     "auto": oracle.fold_ring_order,
@@ -317,3 +318,23 @@ def test_allreduce_host_buffers(algo, count):
     side.synchronize()
     assert_bits_equal([h.numpy() for h in host], want, "host")
     assert_bits_equal(to_host(dev), want, "device")
+
+
+def test_bucket_views_layout_equals_fused_bucket_sync():
+    # gradients as views into one flat bf16 buffer per bucket and rank: a
+    # plain one-shot all-reduce of the flat buffer gives the fused bucket
+    # sync's bits (same chunking over the bucket's flat index, same fold)
+    n = 8
+    numels = [5, 3000, 64, 1, 9000, 77, 20000, 333, 4096]
+    host = _grad_set(13, n, numels)
+    want = [[g.copy() for g in rank] for rank in host]
+    oracle.bucket_sync(want, 4 * 4096 * 2, "avg")
+    plan = rrv.BucketPlan(numels, "bf16", 4 * 4096 * 2)
+    flats, views = plan.flat_buffers(n, "cuda")
+    for r in range(n):
+        for t, g in enumerate(host[r]):
+            views[r][t].copy_(torch.from_numpy(g.view(np.int16)).cuda().view(torch.bfloat16))
+    for b in range(plan.num_buckets):
+        rrv.all_reduce(flats[b], "avg", "oneshot")
+    for r in range(n):
+        assert_bits_equal(to_host(views[r]), want[r], f"rank {r}")
