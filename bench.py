@@ -41,7 +41,7 @@ FALLBACK_HBM_GBS = 6650.0
 # from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), with the
 # hash of the kernel sources it was taken on.  The summary with its command is
 # in profiles/oneshot_ring_kernel_allreduce-8x64MiB-f32.md.
-NCU_TRAFFIC = {"per_algorithmic_byte": None, "sources_sha1": None}
+NCU_TRAFFIC = {"per_algorithmic_byte": (536951296 + 479357952) / 1073741824, "sources_sha1": "9e541d55bed5d43b1a26e20616c156b3b2af75e3"}
 
 
 def sources_sha1() -> str:
@@ -65,9 +65,12 @@ def parse_args():
     ap.add_argument("--no-extra", action="store_true", help="skip the per-algorithm extra timings")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end host-buffer timing")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
-    ap.add_argument("--workload", choices=[WORKLOAD, "sweep", "gpt-buckets", "64x256MiB"], default=WORKLOAD,
+    ap.add_argument("--workload", choices=[WORKLOAD, "sweep", "gpt-buckets", "64x256MiB", "kernels"],
+                    default=WORKLOAD,
                     help="the headline workload (default), the message-size sweep, or the bucketed "
                          "gradient sync of a GPT-like model; the last two print one JSON line per point")
+    ap.add_argument("--nranks", type=int, default=NRANKS, help="virtual ranks of --workload kernels")
+    ap.add_argument("--reps", type=int, default=5, help="timed calls per kernel family of --workload kernels")
     ap.add_argument("--count", type=int, default=COUNT,
                     help="fp32 elements per virtual rank (default 2^26 = 256 MiB); smaller for profiling")
     return ap.parse_args()
@@ -604,6 +607,61 @@ def run_64_ranks(args):
     emit("all_to_all", *timed(lambda: rrv.all_to_all(x, out, stream)))
 
 
+def run_kernels(args):
+    """Every kernel family once per call at a chosen size (--nranks, --count
+    fp32 elements per rank): one-shot, two-shot, ring, tree and tree-order
+    all-reduce, reduce-scatter, all-gather, all-to-all, and the bucket pack,
+    unpack and fused sync on bf16 gradients of the same total size.  One JSON
+    line per call with its time and HBM fraction; small sizes make this the
+    target for per-kernel ncu captures."""
+    import torch
+
+    import ring_all_reduce_virtual_b200 as rrv
+    from ring_all_reduce_virtual_b200.build import build
+
+    build()
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    n, count = args.nranks, args.count - args.count % args.nranks
+    S = count * ELEM
+    peak, _ = hbm_peak()
+    gen = torch.Generator(device=dev).manual_seed(SEED)
+    x = [torch.randn(count, device=dev, generator=gen) * 1e-3 for _ in range(n)]
+    per = count // n
+    rs = [torch.empty(per, device=dev) for _ in range(n)]
+    out = [torch.empty(count, device=dev) for _ in range(n)]
+    numels = [per // 3, per // 3, count - 2 * (per // 3)]  # three tensors: two small, one large
+    grads = rrv.GradSet([[(torch.randn(m, device=dev, generator=gen) * 1e-3).to(torch.bfloat16) for m in numels]
+                         for _ in range(n)])
+    plan = rrv.BucketPlan(numels, "bf16", 2 * count)  # one bucket
+    buckets = [torch.empty(count, device=dev) for _ in range(n)]
+
+    def emit(what, fn):
+        fn()
+        st = rrv.last_stats()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        t = a.elapsed_time(b) / max(args.reps, 1) / 1e3
+        print(json.dumps({"workload": f"kernels-{n}x{count}-f32", "call": what, "ms": round(t * 1e3, 4),
+                          "hbm_gbs": round(st["hbm_bytes"] / t / 1e9, 1),
+                          "hbm_frac": round(st["hbm_bytes"] / t / 1e9 / peak, 4), "launches": st["launches"]}),
+              flush=True)
+
+    for algo in ("oneshot", "two_shot", "ring", "tree", "tree_oneshot"):
+        emit(f"all_reduce {algo}", lambda: rrv.all_reduce(x, "sum", algo, stream))
+    emit("reduce_scatter", lambda: rrv.reduce_scatter(x, rs, "sum", "auto", stream))
+    emit("all_gather", lambda: rrv.all_gather(rs, out, "auto", stream))
+    emit("all_to_all", lambda: rrv.all_to_all(x, out, stream))
+    emit("bucket_pack", lambda: plan.pack(0, grads, buckets, stream))
+    emit("bucket_unpack", lambda: plan.unpack(0, buckets, grads, "avg", stream))
+    emit("bucket_allreduce", lambda: plan.all_reduce(0, grads, "avg", stream))
+
+
 def main():
     args = parse_args()
     d = Dist()
@@ -618,6 +676,9 @@ def main():
         return
     if args.workload == "64x256MiB":
         run_64_ranks(args)
+        return
+    if args.workload == "kernels":
+        run_kernels(args)
         return
     run_ours(args, d)
 

@@ -198,6 +198,9 @@ def test_ring_stats_match_the_schedule():
     rrv.all_reduce(d, "sum", "oneshot")
     st = rrv.last_stats()
     assert st["launches"] == 1 and st["hbm_bytes"] == 2 * 4 * 4096
+    rrv.all_reduce(d, "sum", "two_shot")  # the ring's per-rank volume in 2 steps
+    st = rrv.last_stats()
+    assert st["launches"] == 2 and st["steps"] == 2 and st["bytes_sent_max"] == 6144
 
 
 # --------------------------------------------- reduce-scatter, all-gather --
