@@ -65,12 +65,13 @@ def parse_args():
     ap.add_argument("--no-extra", action="store_true", help="skip the per-algorithm extra timings")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end host-buffer timing")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
-    ap.add_argument("--workload", choices=[WORKLOAD, "sweep", "gpt-buckets", "64x256MiB", "kernels"],
+    ap.add_argument("--workload", choices=[WORKLOAD, "sweep", "gpt-buckets", "64x256MiB", "kernels", "overlap"],
                     default=WORKLOAD,
                     help="the headline workload (default), the message-size sweep, or the bucketed "
                          "gradient sync of a GPT-like model; the last two print one JSON line per point")
     ap.add_argument("--nranks", type=int, default=NRANKS, help="virtual ranks of --workload kernels")
     ap.add_argument("--reps", type=int, default=5, help="timed calls per kernel family of --workload kernels")
+    ap.add_argument("--tokens", type=int, default=1024, help="tokens of the synthetic backward of --workload overlap")
     ap.add_argument("--count", type=int, default=COUNT,
                     help="fp32 elements per virtual rank (default 2^26 = 256 MiB); smaller for profiling")
     return ap.parse_args()
@@ -662,6 +663,90 @@ def run_kernels(args):
     emit("bucket_allreduce", lambda: plan.all_reduce(0, grads, "avg", stream))
 
 
+def run_overlap(args):
+    """Bucket syncs overlapped with a synthetic backward (GPT-like model, 8
+    virtual ranks, 25 MiB buckets, AVG).  The backward produces every rank's
+    gradient of each tensor, in gradient-ready order, with one batched bf16
+    GEMM per tensor (weight gradient = X^T dY over --tokens tokens; vectors
+    as a GEMM with a ones row).  Timed: backward alone, syncs alone, backward
+    then syncs, backward with the reducer launching each bucket's sync on a
+    second stream as soon as it is ready, and that overlapped step captured
+    in one CUDA graph."""
+    import torch
+
+    import ring_all_reduce_virtual_b200 as rrv
+    from ring_all_reduce_virtual_b200 import synth
+    from ring_all_reduce_virtual_b200.build import build
+
+    build()
+    dev = torch.device("cuda", 0)
+    n, T = 8, args.tokens
+    tensors = synth.grad_ready_order(synth.gpt_grad_tensors())
+    d = 2048
+    shapes = []
+    for name, m in tensors:  # (rows, cols) of each gradient as a GEMM output
+        rows = d if m % d == 0 and m // d > 1 else 1
+        shapes.append((rows, m // rows))
+    bufs = [torch.empty((n, r, c), dtype=torch.bfloat16, device=dev) for r, c in shapes]
+    grads = rrv.GradSet([[bufs[t][r].view(-1) for t in range(len(tensors))] for r in range(n)])
+    gen = torch.Generator(device=dev).manual_seed(SEED)
+    act = {}
+    for r, c in shapes:  # one activation / output-gradient pair per shape, shared by the ranks
+        for k in (r, c):
+            if k not in act:
+                act[k] = (torch.randn((1, T, k), device=dev, generator=gen) * 1e-2).to(torch.bfloat16)
+    ones = torch.ones((1, 1, T), dtype=torch.bfloat16, device=dev)
+    lhs = [(ones if r == 1 else act[r].transpose(1, 2)).expand(n, r, T) for r, c in shapes]
+    rhs = [act[c].expand(n, T, c) for r, c in shapes]
+    plan = rrv.BucketPlan([m for _, m in tensors], "bf16", synth.BUCKET_CAP_BYTES)
+    compute = torch.cuda.Stream(dev)
+    red = rrv.Reducer(plan, grads, "avg")
+
+    def backward(mark):
+        for t in range(len(tensors)):
+            torch.bmm(lhs[t], rhs[t], out=bufs[t])
+            if mark:
+                red.ready(t, compute)
+        if mark:
+            red.finish(compute)
+
+    def syncs():
+        for b in range(plan.num_buckets):
+            plan.all_reduce(b, grads, "avg", compute)
+
+    def timed(fn, reps=5):
+        with torch.cuda.stream(compute):
+            fn()
+            compute.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(compute)
+            for _ in range(reps):
+                fn()
+            b.record(compute)
+            b.synchronize()
+        return a.elapsed_time(b) / reps
+
+    t_b = timed(lambda: backward(False))
+    t_s = timed(syncs)
+    t_serial = timed(lambda: (backward(False), syncs()))
+    t_over = timed(lambda: backward(True))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(compute):
+        backward(True)
+        compute.synchronize()
+    with torch.cuda.graph(g, stream=compute):
+        backward(True)
+    t_graph = timed(g.replay)
+    flops = 2.0 * T * sum(m for _, m in tensors) * n
+    print(json.dumps({
+        "workload": "gpt-24x2048-overlap-bf16-avg", "nranks_virtual": n, "tokens": T, "buckets": plan.num_buckets,
+        "backward_ms": round(t_b, 3), "backward_tflops": round(flops / t_b / 1e9, 1), "syncs_ms": round(t_s, 3),
+        "serial_ms": round(t_serial, 3), "overlapped_ms": round(t_over, 3), "overlapped_graph_ms": round(t_graph, 3),
+        "exposed_sync_ms": round(t_over - t_b, 3), "exposed_sync_graph_ms": round(t_graph - t_b, 3),
+        "hidden_fraction": round(1 - (t_over - t_b) / t_s, 3) if t_s > 0 else None}), flush=True)
+    del g
+
+
 def main():
     args = parse_args()
     d = Dist()
@@ -679,6 +764,9 @@ def main():
         return
     if args.workload == "kernels":
         run_kernels(args)
+        return
+    if args.workload == "overlap":
+        run_overlap(args)
         return
     run_ours(args, d)
 

@@ -252,6 +252,39 @@ rr_status_t rr_bucket_unpack(const rr_bucket_plan_t* plan, int bucket, const voi
 rr_status_t rr_bucket_allreduce(const rr_bucket_plan_t* plan, int bucket, void* const* grads,
                                 int nranks, rr_op_t op, cudaStream_t stream);
 
+/* ------------------------------------------------ overlapped bucket sync -- */
+
+/* Opaque reducer (host memory and CUDA events owned by the library). */
+typedef struct rr_reducer rr_reducer_t;
+
+/* A DDP-style reducer: buckets are synced while backward still runs
+ * ([P3] s5: backward produces gradients from the last layer to the first and
+ * each bucket's all-reduce starts as soon as the bucket is ready, so the
+ * communication hides behind the remaining backward; [P2] s3.3: each full
+ * bucket triggers its all-reduce; [P1] s4.2).  Binds a plan (which must
+ * outlive the reducer) to the gradients of all ranks -- grads holds
+ * nranks*ntensors device pointers, rank-major, copied -- and to a
+ * communication stream `comm`.  op: SUM or AVG.  Creates one CUDA event per
+ * bucket plus one; allocates no device memory. */
+rr_status_t rr_reducer_create(const rr_bucket_plan_t* plan, void* const* grads, int nranks, rr_op_t op,
+                              cudaStream_t comm, rr_reducer_t** out);
+
+/* Marks tensor `tensor` (on every rank) as final once the work already
+ * enqueued on `producer` has run.  When this completes its bucket, an event
+ * is recorded on `producer`, `comm` waits for it and the bucket's fused sync
+ * (rr_bucket_allreduce) is enqueued on `comm`.  The bucket's other tensors
+ * must have been produced on `producer` too, or be ordered before it by the
+ * caller.  RR_ERR_INVALID_ARG if the tensor was already marked in this
+ * step. */
+rr_status_t rr_reducer_ready(rr_reducer_t* red, int tensor, cudaStream_t producer);
+
+/* Ends a step: `stream` waits for every bucket sync of the step, and the
+ * marks are cleared for the next step.  RR_ERR_INVALID_ARG (and nothing
+ * enqueued) if some tensor was not marked, i.e. its bucket was never
+ * synced -- the situation in which DDP would hang. */
+rr_status_t rr_reducer_finish(rr_reducer_t* red, cudaStream_t stream);
+void rr_reducer_free(rr_reducer_t* red);
+
 /* ----------------------------------------------------- picker and model -- */
 
 /* The alpha-beta model of one algorithm for N ranks and M bytes per rank

@@ -21,7 +21,7 @@ from ._lib import MAX_RANKS, Cost, RingEvent, RRError, Stats, check, lib
 
 __all__ = [
     "all_reduce", "all_reduce_host", "ring_step", "ring_schedule", "reduce_scatter", "all_gather", "all_to_all",
-    "BucketPlan", "GradSet", "cost_model", "pick_algo", "set_picker_params", "last_stats", "RRError",
+    "BucketPlan", "GradSet", "Reducer", "cost_model", "pick_algo", "set_picker_params", "last_stats", "RRError",
     "OPS", "ALGOS", "MAX_RANKS",
 ]
 
@@ -249,6 +249,37 @@ class BucketPlan:
         g, n, dev = self._grads(grads)
         check(lib().rr_bucket_allreduce(self._h, bucket, g, n, _op(op), _stream(stream, dev)),
               "bucket_allreduce")
+
+
+class Reducer:
+    """DDP-style overlapped bucket sync (``rr_reducer_*``): mark each
+    gradient ready on the stream that produced it; every bucket's fused sync
+    starts on ``comm`` as soon as its last gradient is ready; ``finish``
+    joins the step.  Keep ``plan`` and the gradients alive while in use."""
+
+    def __init__(self, plan: BucketPlan, grads, op="avg", comm=None):
+        import torch
+
+        g = grads if isinstance(grads, GradSet) else GradSet(grads)
+        self.comm = comm if comm is not None else torch.cuda.Stream(g.device)
+        self._plan, self._grads = plan, g
+        handle = ctypes.c_void_p()
+        check(lib().rr_reducer_create(plan._h, g.ptrs, g.nranks, _op(op), _stream(self.comm, g.device),
+                                      ctypes.byref(handle)), "reducer_create")
+        self._h = handle
+        self._device = g.device
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            lib().rr_reducer_free(h)
+            self._h = None
+
+    def ready(self, tensor: int, stream=None) -> None:
+        check(lib().rr_reducer_ready(self._h, tensor, _stream(stream, self._device)), "reducer_ready")
+
+    def finish(self, stream=None) -> None:
+        check(lib().rr_reducer_finish(self._h, _stream(stream, self._device)), "reducer_finish")
 
 
 def cost_model(algo, nranks: int, bytes_per_rank: float, alpha_s: float, beta_bytes_per_s: float) -> dict:

@@ -69,6 +69,10 @@ def _declare(lib: ctypes.CDLL) -> None:
         "rr_bucket_pack": (st, [P, i, PP, PP, i, P]),
         "rr_bucket_unpack": (st, [P, i, PP, PP, i, i, P]),
         "rr_bucket_allreduce": (st, [P, i, PP, i, i, P]),
+        "rr_reducer_create": (st, [P, PP, i, i, P, ctypes.POINTER(P)]),
+        "rr_reducer_ready": (st, [P, i, P]),
+        "rr_reducer_finish": (st, [P, P]),
+        "rr_reducer_free": (None, [P]),
         "rr_cost_model": (st, [i, i, d, d, d, ctypes.POINTER(Cost)]),
         "rr_pick_algo": (i, [i, sz, i]),
         "rr_set_picker_params": (st, [d, d]),

@@ -813,17 +813,19 @@ static rr_status_t bucket_copy(const rr_bucket_plan_t* plan, int bucket, const v
         p->divisor = (float)n;
         uint64_t maxlen = 0;
         bool v = vec;
+        const uint64_t te = bucket_tile_elems(plan->grad_dtype);
+        p->tile0[0] = 0;
         for (int t = g0; t < g1; ++t) {
             const int gt = t0 + t;
             for (int r = 0; r < n; ++r) p->grad[(t - g0) * n + r] = grads[(size_t)r * plan->ntensors + gt];
             v = v && same_phase(&p->grad[(t - g0) * n], n);
             p->toff[t - g0] = plan->offset[gt];
             p->tlen[t - g0] = plan->numel[gt];
+            p->tile0[t - g0 + 1] = p->tile0[t - g0] + (uint64_t)n * ceil_div(plan->numel[gt], te);
             maxlen = std::max<uint64_t>(maxlen, plan->numel[gt]);
         }
         for (int r = 0; r < n; ++r) p->bucket[r] = buckets[r];
         p->vec_ok = v;
-        p->tps = std::max<uint64_t>(1, ceil_div(maxlen, bucket_tile_elems(plan->grad_dtype)));
         if (maxlen == 0) continue;
         cudaError_t e = pack ? launch_bucket_pack(plan->grad_dtype, *p, stream)
                              : launch_bucket_unpack(plan->grad_dtype, op, *p, stream);
@@ -871,11 +873,11 @@ rr_status_t rr_bucket_allreduce(const rr_bucket_plan_t* plan, int bucket, void* 
     auto* p = new BucketFoldParams();
     auto flush = [&](int ntens) -> rr_status_t {
         if (p->nseg == 0) return RR_OK;
-        uint64_t maxlen = 0;
-        for (int s = 0; s < p->nseg; ++s) maxlen = std::max(maxlen, p->seg[s].len);
+        const uint64_t te = tile_elems(plan->grad_dtype, reduce_vpt(n));
+        p->tile0[0] = 0;
+        for (int s = 0; s < p->nseg; ++s) p->tile0[s + 1] = p->tile0[s] + ceil_div(p->seg[s].len, te);
         p->n = n;
         p->divisor = (float)n;
-        p->tps = std::max<uint64_t>(1, ceil_div(maxlen, tile_elems(plan->grad_dtype, reduce_vpt(n))));
         bool v = true;
         for (int t = 0; t < ntens; ++t) v = v && same_phase(&p->grad[t * n], n);
         p->vec_ok = v;
@@ -911,6 +913,99 @@ rr_status_t rr_bucket_allreduce(const rr_bucket_plan_t* plan, int bucket, void* 
     log_call("bucket_allreduce", n, total, (rr_dtype_t)plan->grad_dtype, op, RR_ALGO_ONESHOT);
     return st;
 }
+
+// -------------------------------------------------------------- reducer --
+
+}  // extern "C"
+
+struct rr_reducer {
+    const rr_bucket_plan_t* plan = nullptr;
+    int n = 0;
+    rr_op_t op = RR_AVG;
+    cudaStream_t comm = nullptr;
+    std::vector<void*> grads;         // nranks * ntensors, rank-major
+    std::vector<int> pending;         // per bucket: tensors not yet marked in this step
+    std::vector<char> marked;         // per tensor
+    std::vector<cudaEvent_t> ready;   // per bucket: recorded on the producer when it completes
+    cudaEvent_t done = nullptr;       // recorded on comm at the end of a step
+
+    void reset()
+    {
+        for (size_t b = 0; b < pending.size(); ++b) pending[b] = plan->count[b];
+        std::fill(marked.begin(), marked.end(), 0);
+    }
+    ~rr_reducer()
+    {
+        for (cudaEvent_t e : ready)
+            if (e) cudaEventDestroy(e);
+        if (done) cudaEventDestroy(done);
+    }
+};
+
+extern "C" {
+
+rr_status_t rr_reducer_create(const rr_bucket_plan_t* plan, void* const* grads, int nranks, rr_op_t op,
+                              cudaStream_t comm, rr_reducer_t** out)
+{
+    if (!out) return fail(RR_ERR_INVALID_ARG, "NULL reducer output");
+    *out = nullptr;
+    if (!plan || !grads) return fail(RR_ERR_INVALID_ARG, "NULL plan or gradient array");
+    if (nranks < 1 || nranks > RR_MAX_RANKS) return fail(RR_ERR_INVALID_ARG, "nranks must be in 1..64");
+    if (op != RR_SUM && op != RR_AVG) return fail(RR_ERR_UNSUPPORTED, "the reducer takes SUM or AVG");
+    auto* red = new rr_reducer();
+    red->plan = plan;
+    red->n = nranks;
+    red->op = op;
+    red->comm = comm;
+    red->grads.assign(grads, grads + (size_t)nranks * plan->ntensors);
+    const int nb = (int)plan->first.size();
+    red->pending.assign(nb, 0);
+    red->marked.assign(plan->ntensors, 0);
+    red->ready.assign(nb, nullptr);
+    for (int b = 0; b < nb; ++b) {
+        cudaError_t e = cudaEventCreateWithFlags(&red->ready[b], cudaEventDisableTiming);
+        if (e != cudaSuccess) {
+            delete red;
+            return cuda_fail(e, "creating the reducer's events");
+        }
+    }
+    cudaError_t e = cudaEventCreateWithFlags(&red->done, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+        delete red;
+        return cuda_fail(e, "creating the reducer's events");
+    }
+    red->reset();
+    *out = red;
+    return RR_OK;
+}
+
+rr_status_t rr_reducer_ready(rr_reducer_t* red, int tensor, cudaStream_t producer)
+{
+    if (!red) return fail(RR_ERR_INVALID_ARG, "NULL reducer");
+    if (tensor < 0 || tensor >= red->plan->ntensors) return fail(RR_ERR_INVALID_ARG, "bad tensor");
+    if (red->marked[tensor]) return fail(RR_ERR_INVALID_ARG, "tensor marked ready twice in one step");
+    red->marked[tensor] = 1;
+    const int b = red->plan->bucket_of[tensor];
+    if (--red->pending[b] > 0) return RR_OK;
+    cudaError_t e = cudaEventRecord(red->ready[b], producer);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(red->comm, red->ready[b], 0);
+    if (e != cudaSuccess) return cuda_fail(e, "ordering the bucket sync after its gradients");
+    return rr_bucket_allreduce(red->plan, b, red->grads.data(), red->n, red->op, red->comm);
+}
+
+rr_status_t rr_reducer_finish(rr_reducer_t* red, cudaStream_t stream)
+{
+    if (!red) return fail(RR_ERR_INVALID_ARG, "NULL reducer");
+    for (size_t b = 0; b < red->pending.size(); ++b)
+        if (red->pending[b] > 0) return fail(RR_ERR_INVALID_ARG, "a bucket still waits for gradients");
+    cudaError_t e = cudaEventRecord(red->done, red->comm);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, red->done, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "joining the communication stream");
+    red->reset();
+    return RR_OK;
+}
+
+void rr_reducer_free(rr_reducer_t* red) { delete red; }
 
 // ------------------------------------------------------ model, picker --
 

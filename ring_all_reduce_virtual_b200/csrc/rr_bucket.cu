@@ -84,16 +84,40 @@ __device__ __forceinline__ void convert_tile(const typename In::T* src, typename
     }
 }
 
+// The segment owning work item w: the last s with prefix[s] <= w (segments
+// without tiles have prefix[s] == prefix[s + 1] and are never returned).
+__device__ __forceinline__ int find_segment(const uint64_t* prefix, int nseg, uint64_t w)
+{
+    int lo = 0, hi = nseg;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (prefix[mid] <= w) lo = mid;
+        else hi = mid;
+    }
+    return lo;
+}
+
+// Work item w of a pack/unpack launch -> (tensor t, rank r, tile).
+__device__ __forceinline__ void copy_item(const BucketCopyParams& p, uint64_t w, uint64_t& t, uint64_t& r,
+                                          uint64_t& tile)
+{
+    t = (uint64_t)find_segment(p.tile0, p.nt, w);
+    const uint64_t local = w - p.tile0[t];
+    const uint64_t tiles = (p.tile0[t + 1] - p.tile0[t]) / (uint64_t)p.n;
+    r = local / tiles;
+    tile = local - r * tiles;
+}
+
 // Pack: segment (t, r) copies rank r's tensor t into rank r's fp32 bucket at
 // the tensor's offset (exact widening).
 template <class G>
 __global__ void __launch_bounds__(kThreads) bucket_pack_kernel(const __grid_constant__ BucketCopyParams p)
 {
-    const uint64_t nseg = (uint64_t)p.nt * (uint64_t)p.n;
-    const uint64_t total = nseg * p.tps;
+    const uint64_t total = p.tile0[p.nt];
     for (uint64_t w = blockIdx.x; w < total; w += gridDim.x) {
-        const uint64_t s = w / p.tps, tile = w - s * p.tps;
-        const uint64_t t = s / (uint64_t)p.n, r = s - t * (uint64_t)p.n;
+        uint64_t t, r, tile;
+        copy_item(p, w, t, r, tile);
+        const uint64_t s = t * (uint64_t)p.n + r;
         const auto* src = static_cast<const typename G::T*>(p.grad[s]);
         float* dst = static_cast<float*>(p.bucket[r]) + p.toff[t];
         convert_tile<G, F32T, kSum>(src, dst, p.tlen[t], tile, p.vec_ok, 1.0f);
@@ -105,11 +129,11 @@ __global__ void __launch_bounds__(kThreads) bucket_pack_kernel(const __grid_cons
 template <class G, int OP>
 __global__ void __launch_bounds__(kThreads) bucket_unpack_kernel(const __grid_constant__ BucketCopyParams p)
 {
-    const uint64_t nseg = (uint64_t)p.nt * (uint64_t)p.n;
-    const uint64_t total = nseg * p.tps;
+    const uint64_t total = p.tile0[p.nt];
     for (uint64_t w = blockIdx.x; w < total; w += gridDim.x) {
-        const uint64_t s = w / p.tps, tile = w - s * p.tps;
-        const uint64_t t = s / (uint64_t)p.n, r = s - t * (uint64_t)p.n;
+        uint64_t t, r, tile;
+        copy_item(p, w, t, r, tile);
+        const uint64_t s = t * (uint64_t)p.n + r;
         const float* src = static_cast<const float*>(p.bucket[r]) + p.toff[t];
         auto* dst = static_cast<typename G::T*>(const_cast<void*>(p.grad[s]));
         convert_tile<F32T, G, OP>(src, dst, p.tlen[t], tile, p.vec_ok, p.divisor);
@@ -124,9 +148,10 @@ template <class G, int OP, int VPT, int GR>
 __global__ void __launch_bounds__(kThreads) bucket_fold_kernel(const __grid_constant__ BucketFoldParams p)
 {
     using T = typename G::T;
-    const uint64_t total = (uint64_t)p.nseg * p.tps;
+    const uint64_t total = p.tile0[p.nseg];
     for (uint64_t w = blockIdx.x; w < total; w += gridDim.x) {
-        const uint64_t s = w / p.tps, tile = w - s * p.tps;
+        const int s = find_segment(p.tile0, p.nseg, w);
+        const uint64_t tile = w - p.tile0[s];
         const BucketSeg& sg = p.seg[s];
         const int n = p.n;
         const int base = (int)sg.t * n;
@@ -170,7 +195,7 @@ uint64_t bucket_tile_elems(int grad_dtype)
 
 cudaError_t launch_bucket_pack(int grad_dtype, const BucketCopyParams& p, cudaStream_t s)
 {
-    const uint64_t work = (uint64_t)p.nt * (uint64_t)p.n * p.tps;
+    const uint64_t work = p.tile0[p.nt];
     if (grad_dtype == kBF16) return launch_all_b(bucket_pack_kernel<BF16T>, p, work, s);
     if (grad_dtype == kF32) return launch_all_b(bucket_pack_kernel<F32T>, p, work, s);
     return cudaErrorInvalidValue;
@@ -178,7 +203,7 @@ cudaError_t launch_bucket_pack(int grad_dtype, const BucketCopyParams& p, cudaSt
 
 cudaError_t launch_bucket_unpack(int grad_dtype, int op, const BucketCopyParams& p, cudaStream_t s)
 {
-    const uint64_t work = (uint64_t)p.nt * (uint64_t)p.n * p.tps;
+    const uint64_t work = p.tile0[p.nt];
     const bool avg = op == kAvg;
     if (grad_dtype == kBF16)
         return avg ? launch_all_b(bucket_unpack_kernel<BF16T, kAvg>, p, work, s)
@@ -191,7 +216,7 @@ cudaError_t launch_bucket_unpack(int grad_dtype, int op, const BucketCopyParams&
 
 cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p, cudaStream_t s)
 {
-    const uint64_t work = (uint64_t)p.nseg * p.tps;
+    const uint64_t work = p.tile0[p.nseg];
     const bool avg = op == kAvg;
     if (grad_dtype == kBF16) return avg ? launch_fold<BF16T, kAvg>(p, work, s) : launch_fold<BF16T, kSum>(p, work, s);
     if (grad_dtype == kF32) return avg ? launch_fold<F32T, kAvg>(p, work, s) : launch_fold<F32T, kSum>(p, work, s);

@@ -56,16 +56,20 @@ constexpr int kMaxBucketPtrs = 2048;
 constexpr int kMaxBucketTensors = 384;
 constexpr int kMaxBucketSegs = kMaxBucketTensors + kMaxRanksH;
 
+// Work items of the bucket kernels are numbered through per-segment prefix
+// sums of their tile counts, so segments of very different lengths launch no
+// empty CTAs: work item w belongs to the segment s with
+// tile0[s] <= w < tile0[s + 1].
 struct BucketCopyParams {
-    const void* grad[kMaxBucketPtrs];  // pack: sources; unpack: destinations
-    void* bucket[kMaxRanksH];          // fp32 bucket of each rank
-    uint64_t toff[kMaxBucketTensors];  // element offset of tensor t in the bucket
-    uint64_t tlen[kMaxBucketTensors];  // elements of tensor t
+    const void* grad[kMaxBucketPtrs];      // pack: sources; unpack: destinations
+    void* bucket[kMaxRanksH];              // fp32 bucket of each rank
+    uint64_t toff[kMaxBucketTensors];      // element offset of tensor t in the bucket
+    uint64_t tlen[kMaxBucketTensors];      // elements of tensor t
+    uint64_t tile0[kMaxBucketTensors + 1]; // first work item of tensor t (n ranks x its tiles)
     int n;
     int nt;
     int vec_ok;
     float divisor;
-    uint64_t tps;
 };
 
 // A fused bucket segment: elements [off, off + len) of launch tensor t, all
@@ -80,11 +84,11 @@ struct BucketSeg {
 struct BucketFoldParams {
     void* grad[kMaxBucketPtrs];
     BucketSeg seg[kMaxBucketSegs];
+    uint64_t tile0[kMaxBucketSegs + 1];  // first work item (tile) of segment s
     int n;
     int nseg;
     int vec_ok;
     float divisor;
-    uint64_t tps;
 };
 
 enum DType : int { kF32 = 0, kBF16 = 1, kI32 = 2 };
@@ -124,4 +128,12 @@ cudaError_t launch_bucket_pack(int grad_dtype, const BucketCopyParams& p, cudaSt
 cudaError_t launch_bucket_unpack(int grad_dtype, int op, const BucketCopyParams& p, cudaStream_t s);
 cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p, cudaStream_t s);
 
+}  // namespace rr
+
+namespace rr {
+// Kernel parameter blocks must fit the 32,764-byte kernel parameter limit.
+static_assert(sizeof(RankParams) <= 32764, "RankParams too large");
+static_assert(sizeof(StepParams) <= 32764, "StepParams too large");
+static_assert(sizeof(BucketCopyParams) <= 32764, "BucketCopyParams too large");
+static_assert(sizeof(BucketFoldParams) <= 32764, "BucketFoldParams too large");
 }  // namespace rr

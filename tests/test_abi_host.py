@@ -194,6 +194,17 @@ def test_argument_errors_return_before_any_launch():
     assert lib.rr_reduce_scatter(_fake(2), _fake(2, base=1 << 41), 2, 4, 0, 0, 1, s) == _lib.RR_ERR_UNSUPPORTED
 
 
+def test_reducer_argument_errors():
+    lib = _lib.lib()
+    out = ctypes.c_void_p()
+    assert lib.rr_reducer_create(None, _fake(2), 2, 1, None, ctypes.byref(out)) == _lib.RR_ERR_INVALID_ARG
+    plan = rrv.BucketPlan([10, 20], "bf16", 100)
+    assert lib.rr_reducer_create(plan._h, _fake(4), 2, 2, None, ctypes.byref(out)) == _lib.RR_ERR_UNSUPPORTED
+    assert lib.rr_reducer_create(plan._h, _fake(4), 0, 1, None, ctypes.byref(out)) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_reducer_ready(None, 0, None) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_reducer_finish(None, None) == _lib.RR_ERR_INVALID_ARG
+
+
 def test_trivial_calls_enqueue_nothing():
     lib = _lib.lib()
     s = ctypes.c_void_p(0)

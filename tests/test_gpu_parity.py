@@ -341,3 +341,80 @@ def test_bucket_views_layout_equals_fused_bucket_sync():
         rrv.all_reduce(flats[b], "avg", "oneshot")
     for r in range(n):
         assert_bits_equal(to_host(views[r]), want[r], f"rank {r}")
+
+
+# ------------------------------------------------- overlapped bucket sync --
+
+def _reducer_setup(n, numels, cap, seed):
+    host = _grad_set(seed, n, numels)
+    want = [[g.copy() for g in rank] for rank in host]
+    oracle.bucket_sync(want, cap, "avg")
+    src = [to_dev(rank) for rank in host]  # the "backward" copies these into the gradients
+    grads = [[torch.zeros_like(t) for t in rank] for rank in src]
+    plan = rrv.BucketPlan(numels, "bf16", cap)
+    return host, want, src, grads, plan
+
+
+def _backward_step(red, src, grads, stream):
+    # a synthetic backward on `stream`: gradients become final one tensor at a
+    # time, in the plan's order; each is marked ready right after
+    for t in range(len(grads[0])):
+        for r in range(len(grads)):
+            grads[r][t].copy_(src[r][t])
+        red.ready(t, stream)
+    red.finish(stream)
+
+
+def test_reducer_overlaps_bucket_syncs_with_backward():
+    n = 8
+    numels = [4096, 5, 30000, 64, 9000, 1, 12000, 333]
+    host, want, src, grads, plan = _reducer_setup(n, numels, 8192, 20)
+    assert plan.num_buckets > 2
+    compute = torch.cuda.Stream()
+    compute.wait_stream(torch.cuda.current_stream())
+    red = rrv.Reducer(plan, grads, "avg")
+    with torch.cuda.stream(compute):
+        _backward_step(red, src, grads, compute)
+        _backward_step(red, src, grads, compute)  # a second step reuses the reducer
+    compute.synchronize()
+    for r in range(n):
+        assert_bits_equal(to_host(grads[r]), want[r], f"rank {r}")
+
+
+def test_reducer_step_captured_in_a_cuda_graph():
+    n = 4
+    numels = [2048, 7, 20000, 100, 5000]
+    host, want, src, grads, plan = _reducer_setup(n, numels, 4096, 21)
+    red = rrv.Reducer(plan, grads, "avg")
+    compute = torch.cuda.Stream()
+    compute.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(compute):
+        _backward_step(red, src, grads, compute)  # warm-up outside the graph
+    compute.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=compute):
+        _backward_step(red, src, grads, compute)
+    for _ in range(2):
+        for rank in grads:
+            for t in rank:
+                t.zero_()
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        for r in range(n):
+            assert_bits_equal(to_host(grads[r]), want[r], f"rank {r}")
+
+
+def test_reducer_refuses_an_incomplete_step():
+    n = 2
+    numels = [100, 200, 300]
+    host, want, src, grads, plan = _reducer_setup(n, numels, 500, 22)
+    red = rrv.Reducer(plan, grads, "avg")
+    red.ready(0)
+    with pytest.raises(rrv.RRError):
+        red.ready(0)  # twice in one step
+    with pytest.raises(rrv.RRError):
+        red.finish()  # tensors 1 and 2 never marked
+    red.ready(1)
+    red.ready(2)
+    red.finish()
