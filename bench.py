@@ -653,7 +653,7 @@ def run_kernels(args):
                           "hbm_frac": round(st["hbm_bytes"] / t / 1e9 / peak, 4), "launches": st["launches"]}),
               flush=True)
 
-    for algo in ("oneshot", "two_shot", "ring", "tree", "tree_oneshot"):
+    for algo in ("oneshot", "two_shot", "ring", "double_ring", "tree", "tree_oneshot"):
         emit(f"all_reduce {algo}", lambda: rrv.all_reduce(x, "sum", algo, stream))
     emit("reduce_scatter", lambda: rrv.reduce_scatter(x, rs, "sum", "auto", stream))
     emit("all_gather", lambda: rrv.all_gather(rs, out, "auto", stream))
@@ -700,7 +700,7 @@ def run_overlap(args):
     rhs = [act[c].expand(n, T, c) for r, c in shapes]
     plan = rrv.BucketPlan([m for _, m in tensors], "bf16", synth.BUCKET_CAP_BYTES)
     compute = torch.cuda.Stream(dev)
-    red = rrv.Reducer(plan, grads, "avg")
+    red = None
 
     def backward(mark):
         for t in range(len(tensors)):
@@ -729,22 +729,26 @@ def run_overlap(args):
     t_b = timed(lambda: backward(False))
     t_s = timed(syncs)
     t_serial = timed(lambda: (backward(False), syncs()))
-    t_over = timed(lambda: backward(True))
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(compute):
-        backward(True)
-        compute.synchronize()
-    with torch.cuda.graph(g, stream=compute):
-        backward(True)
-    t_graph = timed(g.replay)
     flops = 2.0 * T * sum(m for _, m in tensors) * n
-    print(json.dumps({
-        "workload": "gpt-24x2048-overlap-bf16-avg", "nranks_virtual": n, "tokens": T, "buckets": plan.num_buckets,
-        "backward_ms": round(t_b, 3), "backward_tflops": round(flops / t_b / 1e9, 1), "syncs_ms": round(t_s, 3),
-        "serial_ms": round(t_serial, 3), "overlapped_ms": round(t_over, 3), "overlapped_graph_ms": round(t_graph, 3),
-        "exposed_sync_ms": round(t_over - t_b, 3), "exposed_sync_graph_ms": round(t_graph - t_b, 3),
-        "hidden_fraction": round(1 - (t_over - t_b) / t_s, 3) if t_s > 0 else None}), flush=True)
-    del g
+    for ctas in (0, 32, 64, 128, 256):
+        # each bucket sync on a high-priority stream, with at most `ctas` CTAs
+        red = rrv.Reducer(plan, grads, "avg", max_ctas=ctas)
+        t_over = timed(lambda: backward(True))
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(compute):
+            backward(True)
+            compute.synchronize()
+        with torch.cuda.graph(g, stream=compute):
+            backward(True)
+        t_graph = timed(g.replay)
+        del g
+        print(json.dumps({
+            "workload": "gpt-24x2048-overlap-bf16-avg", "nranks_virtual": n, "tokens": T, "buckets": plan.num_buckets,
+            "sync_ctas": ctas or "one per tile", "backward_ms": round(t_b, 3),
+            "backward_tflops": round(flops / t_b / 1e9, 1), "syncs_ms": round(t_s, 3),
+            "serial_ms": round(t_serial, 3), "overlapped_ms": round(t_over, 3), "overlapped_graph_ms": round(t_graph, 3),
+            "exposed_sync_ms": round(t_over - t_b, 3), "exposed_sync_graph_ms": round(t_graph - t_b, 3),
+            "hidden_fraction_graph": round(1 - (t_graph - t_b) / t_s, 3) if t_s > 0 else None}), flush=True)
 
 
 def main():

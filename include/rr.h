@@ -92,16 +92,24 @@ typedef enum rr_op { RR_SUM = 0, RR_AVG = 1, RR_MAX = 2, RR_MIN = 3, RR_PROD = 4
  *                all-gather by direct reads ([P4] "alpha-beta model": the
  *                two-shot all-reduce); the ring's bits and its 2(N-1)/N S
  *                bytes per rank, in 2 steps instead of 2(N-1)
+ *   DOUBLE_RING  two rings in opposite directions at once ([P3] s6: the
+ *                double ring): the first half of every buffer (H =
+ *                ceil(count/2) elements) runs the RING schedule, the second
+ *                half the mirror-image ring whose ranks send to the left, so
+ *                a second-half chunk c folds downwards (c, c-1, ...); 2(N-1)
+ *                launches, each rank sending half its bytes each way
  *   AUTO         the picker's choice among RING, ONESHOT and TWO_SHOT
- *                (never a tree order, whose bits differ); env
- *                RR_ALGO=ring|oneshot|tree|tree_oneshot|two_shot overrides it. */
+ *                (never a tree order or the double ring, whose bits differ);
+ *                env RR_ALGO=ring|oneshot|tree|tree_oneshot|two_shot|
+ *                double_ring overrides it. */
 typedef enum rr_algo {
     RR_ALGO_AUTO = 0,
     RR_ALGO_RING = 1,
     RR_ALGO_ONESHOT = 2,
     RR_ALGO_TREE = 3,
     RR_ALGO_TREE_ONESHOT = 4,
-    RR_ALGO_TWO_SHOT = 5
+    RR_ALGO_TWO_SHOT = 5,
+    RR_ALGO_DOUBLE_RING = 6
 } rr_algo_t;
 
 /* The two phases of the ring ([P3] s3; [P4]). */
@@ -146,10 +154,12 @@ typedef struct rr_cost {
 
 /* All-reduce in place over bufs[0..nranks): afterwards every buffer holds the
  * reduction of all inputs, element by element ([P4] "The five primitives";
- * [P1] s2.1).  count elements per rank.  Bits: RING, ONESHOT and AUTO give
- * the ring order for fp32 and int32; for bf16, ONESHOT rounds once and RING
- * rounds per hop.  TREE and TREE_ONESHOT give the tree order.  Buffers must
- * not overlap.  nranks == 1 enqueues nothing. */
+ * [P1] s2.1).  count elements per rank.  Bits: RING, ONESHOT, TWO_SHOT and
+ * AUTO give the ring order for fp32 and int32; for bf16, ONESHOT and
+ * TWO_SHOT round once and RING rounds per hop.  TREE and TREE_ONESHOT give
+ * the tree order; DOUBLE_RING the ring order in the first half and the
+ * downward order in the second (rounding per hop for bf16).  Buffers must not
+ * overlap.  nranks == 1 enqueues nothing. */
 rr_status_t rr_allreduce(void* const* bufs, int nranks, size_t count, rr_dtype_t dtype, rr_op_t op,
                          rr_algo_t algo, cudaStream_t stream);
 
@@ -264,10 +274,13 @@ typedef struct rr_reducer rr_reducer_t;
  * bucket triggers its all-reduce; [P1] s4.2).  Binds a plan (which must
  * outlive the reducer) to the gradients of all ranks -- grads holds
  * nranks*ntensors device pointers, rank-major, copied -- and to a
- * communication stream `comm`.  op: SUM or AVG.  Creates one CUDA event per
- * bucket plus one; allocates no device memory. */
+ * communication stream `comm`.  op: SUM or AVG.  max_ctas > 0 caps the CTAs
+ * of each bucket sync (they then loop over the bucket's tiles), leaving the
+ * other SMs to the kernels that produce the gradients, as a communication
+ * library runs its collectives on a few channels; 0 launches one CTA per tile.
+ * Creates one CUDA event per bucket plus one; allocates no device memory. */
 rr_status_t rr_reducer_create(const rr_bucket_plan_t* plan, void* const* grads, int nranks, rr_op_t op,
-                              cudaStream_t comm, rr_reducer_t** out);
+                              cudaStream_t comm, int max_ctas, rr_reducer_t** out);
 
 /* Marks tensor `tensor` (on every rank) as final once the work already
  * enqueued on `producer` has run.  When this completes its bucket, an event
@@ -289,8 +302,9 @@ void rr_reducer_free(rr_reducer_t* red);
 
 /* The alpha-beta model of one algorithm for N ranks and M bytes per rank
  * ([P3] s4-s6; [P4] "alpha-beta model"): RING 2(N-1) steps moving 2(N-1)/N M
- * per rank; TREE 2 ceil(log2 N) steps each moving M; ONESHOT 1 step in which
- * each rank reads (N-1) M.  alpha in seconds, beta in bytes/second. */
+ * per rank; DOUBLE_RING 2(N-1) steps moving (N-1)/N M on each of a rank's two
+ * links; TREE 2 ceil(log2 N) steps each moving M; ONESHOT 1 step in which
+ * each rank reads (N-1) M; TWO_SHOT 2 steps moving 2(N-1)/N M.  alpha in seconds, beta in bytes/second. */
 rr_status_t rr_cost_model(rr_algo_t algo, int nranks, double bytes_per_rank, double alpha_s,
                           double beta_bytes_per_s, rr_cost_t* out);
 

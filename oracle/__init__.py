@@ -70,6 +70,9 @@ def _load(mutant: bool = False) -> ctypes.CDLL:
         lib.orc_ring_allreduce.argtypes = [PP, i32, sz, i32, i32, ctypes.POINTER(Event), P]
         lib.orc_ring_allreduce_omp.argtypes = [PP, i32, sz, i32, i32, i32]
         lib.orc_fold_ring_order.argtypes = [PP, i32, sz, i32, i32]
+        lib.orc_double_ring_step.argtypes = [PP, i32, sz, i32, i32, i32, i32, P]
+        lib.orc_double_ring_allreduce.argtypes = [PP, i32, sz, i32, i32, P]
+        lib.orc_fold_double_ring.argtypes = [PP, i32, sz, i32, i32]
         lib.orc_fold_samples.argtypes = [P, i32, sz, P, i32, i32, P]
         lib.orc_naive_allreduce.argtypes = [PP, i32, sz, i32, i32, P]
         lib.orc_tree_schedule.argtypes = [PP, i32, sz, i32, i32, P]
@@ -213,6 +216,34 @@ def ring_allreduce_omp(bufs, op="sum", nthreads: int = 0) -> None:
     timed CPU baseline); same arithmetic as ``ring_allreduce``."""
     d, count = _same(bufs)
     _check(_lib().orc_ring_allreduce_omp(_ptrs(bufs), len(bufs), count, d, _op(op), nthreads), "ring_omp")
+
+
+def double_ring_allreduce(bufs, op="sum"):
+    """The double ring ([P3] section 6): half A on the clockwise ring, half B
+    on the counter-clockwise ring, in place; returns the bytes each rank
+    sent."""
+    d, count = _same(bufs)
+    n = len(bufs)
+    sent = np.zeros(n, dtype=np.uint64)
+    _check(_lib().orc_double_ring_allreduce(_ptrs(bufs), n, count, d, _op(op), sent.ctypes.data), "double ring")
+    return sent
+
+
+def double_ring_step(bufs, op, phase: int, step: int):
+    """One step of both rings, in place; returns the bytes each rank sent."""
+    d, count = _same(bufs)
+    n = len(bufs)
+    sent = np.zeros(n, dtype=np.uint64)
+    _check(_lib().orc_double_ring_step(_ptrs(bufs), n, count, d, _op(op), phase, step, sent.ctypes.data),
+           "double ring step")
+    return sent
+
+
+def fold_double_ring(bufs, op="sum") -> None:
+    """The double ring's result by definition (half B folds downwards),
+    folded in fp32 and rounded once, in place."""
+    d, count = _same(bufs)
+    _check(_lib().orc_fold_double_ring(_ptrs(bufs), len(bufs), count, d, _op(op)), "fold double ring")
 
 
 def fold_ring_order(bufs, op="sum") -> None:

@@ -348,6 +348,116 @@ int orc_ring_allreduce_omp(void** bufs, int n, size_t count, int dtype, int op, 
     return ORC_OK;
 }
 
+/* ---------------------------------------------------------- double ring -- */
+
+/* The double ring ([P3] section 6: two rings running in opposite directions
+ * at once).  Each rank's tensor is cut in two halves, A = [0, H) and
+ * B = [H, count) with H = ceil(count / 2); half A is all-reduced by the
+ * clockwise ring above (each half chunked on its own: C = ceil(len / N)),
+ * half B by the mirror-image ring in which every rank sends to its LEFT
+ * neighbour: reduce-scatter step s sends chunk (r + s) to rank r - 1 and
+ * receives chunk (r + s + 1) from rank r + 1, so chunk c's partial starts on
+ * rank c and gains one rank per hop downwards (c, c-1, c-2, ...), complete
+ * on rank c + 1; all-gather step s sends chunk (r - 1 + s) to rank r - 1 and
+ * receives chunk (r + s) from rank r + 1.  One step of both rings: */
+static int ccw_send_chunk(int phase, int r, int s, int n)
+{
+    if (phase == ORC_PHASE_RS) return mod(r + s, n);
+    return mod(r - 1 + s + (MUTANT(10) ? 1 : 0), n);
+}
+
+int orc_double_ring_step(void** bufs, int n, size_t count, int dtype, int op, int phase, int step,
+                         uint64_t* sent)
+{
+    if (!valid(n, dtype, op) || (phase != ORC_PHASE_RS && phase != ORC_PHASE_AG)) return ORC_EINVAL;
+    if (step < 0 || step > n - 2) return ORC_EINVAL;
+    size_t H = (count + 1) / 2, es = esize(dtype);
+    /* half A: the clockwise ring on views of the first H elements */
+    int rc = orc_ring_step(bufs, n, H, dtype, op, phase, step, NULL);
+    if (rc != ORC_OK) return rc;
+    for (int r = 0; r < n && sent; ++r)
+        sent[r] += (uint64_t)orc_chunk_len(H, n, send_chunk(phase, r, step, n)) * es;
+    /* half B: the counter-clockwise ring */
+    size_t cb = count - H, C = orc_chunk_size(cb, n);
+    unsigned char** msg = (unsigned char**)calloc((size_t)n, sizeof *msg);
+    if (!msg) return ORC_ENOMEM;
+    rc = ORC_OK;
+    for (int r = 0; r < n; ++r) { /* every rank posts its send to the left */
+        int k = ccw_send_chunk(phase, r, step, n);
+        size_t len = orc_chunk_len(cb, n, k);
+        msg[r] = (unsigned char*)malloc(len * es + 1);
+        if (!msg[r]) { rc = ORC_ENOMEM; goto done; }
+        memcpy(msg[r], (unsigned char*)bufs[r] + (H + (size_t)k * C) * es, len * es);
+        if (sent) sent[r] += (uint64_t)(len * es);
+    }
+    for (int r = 0; r < n; ++r) { /* every rank receives from its right */
+        int right = mod(r + 1, n);
+        int k = ccw_send_chunk(phase, right, step, n);
+        size_t len = orc_chunk_len(cb, n, k), off = H + (size_t)k * C;
+        if (phase == ORC_PHASE_AG) {
+            memcpy((unsigned char*)bufs[r] + off * es, msg[right], len * es);
+            continue;
+        }
+        int last = (step == n - 2);
+        for (size_t j = 0; j < len; ++j) {
+            if (dtype == ORC_I32) {
+                int32_t* own = (int32_t*)bufs[r] + off + j;
+                *own = op_i32(op, ((int32_t*)msg[right])[j], *own);
+            } else {
+                float v = op_f32(op, ld_f(msg[right], dtype, j), ld_f(bufs[r], dtype, off + j));
+                if (last) v = finish_f32(op, v, n);
+                st_f(bufs[r], dtype, off + j, v);
+            }
+        }
+    }
+done:
+    for (int r = 0; r < n; ++r) free(msg[r]);
+    free(msg);
+    return rc;
+}
+
+/* The whole double ring: N-1 reduce-scatter steps, then N-1 all-gather steps
+ * of both rings together; sent (optional) receives the bytes each rank sent
+ * (to both neighbours). */
+int orc_double_ring_allreduce(void** bufs, int n, size_t count, int dtype, int op, uint64_t* sent)
+{
+    if (!valid(n, dtype, op)) return ORC_EINVAL;
+    if (sent) memset(sent, 0, (size_t)n * sizeof *sent);
+    for (int phase = ORC_PHASE_RS; phase <= ORC_PHASE_AG; ++phase)
+        for (int s = 0; s < n - 1; ++s) {
+            int rc = orc_double_ring_step(bufs, n, count, dtype, op, phase, s, sent);
+            if (rc != ORC_OK) return rc;
+        }
+    return ORC_OK;
+}
+
+/* The double ring's result as a plain definition: an element of half A in
+ * its half's chunk c folds in ring order c, c+1, ...; an element of half B in
+ * chunk c folds downwards c, c-1, c-2, ...; folded in fp32 for every
+ * floating dtype and rounded once (its fused one-shot form). */
+int orc_fold_double_ring(void** bufs, int n, size_t count, int dtype, int op)
+{
+    if (!valid(n, dtype, op)) return ORC_EINVAL;
+    size_t H = (count + 1) / 2;
+    size_t CA = orc_chunk_size(H, n), CB = orc_chunk_size(count - H, n);
+    for (size_t i = 0; i < count; ++i) {
+        int c, dir;
+        if (i < H) { c = (int)(i / CA); dir = 1; }
+        else { c = (int)((i - H) / CB); dir = -1; }
+        if (dtype == ORC_I32) {
+            int32_t acc = ((int32_t*)bufs[c])[i];
+            for (int j = 1; j < n; ++j) acc = op_i32(op, acc, ((int32_t*)bufs[mod(c + dir * j, n)])[i]);
+            for (int r = 0; r < n; ++r) ((int32_t*)bufs[r])[i] = acc;
+        } else {
+            float acc = ld_f(bufs[c], dtype, i);
+            for (int j = 1; j < n; ++j) acc = op_f32(op, acc, ld_f(bufs[mod(c + dir * j, n)], dtype, i));
+            acc = finish_f32(op, acc, n);
+            for (int r = 0; r < n; ++r) st_f(bufs[r], dtype, i, acc);
+        }
+    }
+    return ORC_OK;
+}
+
 /* ------------------------------------------- one-shot (ring-order fold) -- */
 
 /* The ring's result written as a plain definition.  Following the ring

@@ -26,7 +26,7 @@ __all__ = [
 ]
 
 OPS = {"sum": 0, "avg": 1, "max": 2, "min": 3, "prod": 4}
-ALGOS = {"auto": 0, "ring": 1, "oneshot": 2, "tree": 3, "tree_oneshot": 4, "two_shot": 5}
+ALGOS = {"auto": 0, "ring": 1, "oneshot": 2, "tree": 3, "tree_oneshot": 4, "two_shot": 5, "double_ring": 6}
 ALGO_NAMES = {v: k for k, v in ALGOS.items()}
 PHASES = {"reduce_scatter": 0, "all_gather": 1}
 _DTYPE_NAMES = {"f32": 0, "bf16": 1, "i32": 2}
@@ -257,15 +257,16 @@ class Reducer:
     starts on ``comm`` as soon as its last gradient is ready; ``finish``
     joins the step.  Keep ``plan`` and the gradients alive while in use."""
 
-    def __init__(self, plan: BucketPlan, grads, op="avg", comm=None):
+    def __init__(self, plan: BucketPlan, grads, op="avg", comm=None, max_ctas: int = 0):
         import torch
 
         g = grads if isinstance(grads, GradSet) else GradSet(grads)
-        self.comm = comm if comm is not None else torch.cuda.Stream(g.device)
+        # a high-priority stream lets bucket syncs start as soon as SMs free up
+        self.comm = comm if comm is not None else torch.cuda.Stream(g.device, priority=-1)
         self._plan, self._grads = plan, g
         handle = ctypes.c_void_p()
         check(lib().rr_reducer_create(plan._h, g.ptrs, g.nranks, _op(op), _stream(self.comm, g.device),
-                                      ctypes.byref(handle)), "reducer_create")
+                                      int(max_ctas), ctypes.byref(handle)), "reducer_create")
         self._h = handle
         self._device = g.device
 

@@ -75,6 +75,7 @@ const char* algo_name(int a)
     case RR_ALGO_TREE: return "tree";
     case RR_ALGO_TREE_ONESHOT: return "tree_oneshot";
     case RR_ALGO_TWO_SHOT: return "two_shot";
+    case RR_ALGO_DOUBLE_RING: return "double_ring";
     }
     return "?";
 }
@@ -152,6 +153,16 @@ int ring_send_chunk(int phase, int r, int s, int n)
     return phase == RR_PHASE_REDUCE_SCATTER ? imod(r - s, n) : imod(r + 1 - s, n);
 }
 
+// The mirror-image ring of the double ring ([P3] section 6): every rank sends
+// to its left neighbour.  Reduce-scatter step s sends chunk (r + s) and
+// receives chunk (r + s + 1) from the right; all-gather step s sends chunk
+// (r - 1 + s) and receives (r + s).  Chunk c's partial starts on rank c and
+// gains one rank per hop downwards; it is complete on rank c + 1.
+int ccw_send_chunk(int phase, int r, int s, int n)
+{
+    return phase == RR_PHASE_REDUCE_SCATTER ? imod(r + s, n) : imod(r - 1 + s, n);
+}
+
 void log_call(const char* what, int n, size_t count, rr_dtype_t dtype, int op, int algo)
 {
     static const bool on = env_flag("RR_LOG");
@@ -219,6 +230,65 @@ rr_status_t run_ring(void* const* bufs, int n, size_t count, rr_dtype_t dtype, r
     // each reduce-scatter step reads 2 and writes 1 chunk per rank, each
     // all-gather step reads and writes 1: 5 (N-1) S in all
     t_stats.hbm_bytes = 5ull * (uint64_t)(n - 1) * count * es;
+    return RR_OK;
+}
+
+// One step of both rings of the double ring, one launch: segments 0..N-1 are
+// the clockwise ring on the first half [0, H), segments N..2N-1 the
+// counter-clockwise ring on the second half [H, count).
+rr_status_t double_ring_step_launch(void* const* bufs, int n, size_t count, rr_dtype_t dtype, rr_op_t op,
+                                    int phase, int step, cudaStream_t stream, std::vector<uint64_t>& sent)
+{
+    const size_t es = esize(dtype);
+    const uint64_t H = (count + 1) / 2, cb = count - H;
+    const uint64_t CA = ceil_div(H, (uint64_t)n), CB = ceil_div(cb, (uint64_t)n);
+    StepParams p{};
+    p.nseg = 2 * n;
+    p.nin = phase == RR_PHASE_REDUCE_SCATTER ? 2 : 1;
+    p.vec_ok = same_phase(bufs, n);
+    p.divisor = (float)n;
+    uint64_t maxlen = 0;
+    for (int r = 0; r < n; ++r) {
+        const int left = imod(r - 1, n), right = imod(r + 1, n);
+        const int ka = ring_send_chunk(phase, left, step, n);  // half A, from the left
+        const uint64_t la = (uint64_t)ka * CA, na = chunk_len(H, n, ka);
+        p.seg[r] = {static_cast<const char*>(bufs[left]) + la * es,
+                    p.nin == 2 ? static_cast<const char*>(bufs[r]) + la * es : nullptr,
+                    static_cast<char*>(bufs[r]) + la * es, na};
+        const int kb = ccw_send_chunk(phase, right, step, n);  // half B, from the right
+        const uint64_t lb = H + (uint64_t)kb * CB, nb = chunk_len(cb, n, kb);
+        p.seg[n + r] = {static_cast<const char*>(bufs[right]) + lb * es,
+                        p.nin == 2 ? static_cast<const char*>(bufs[r]) + lb * es : nullptr,
+                        static_cast<char*>(bufs[r]) + lb * es, nb};
+        maxlen = std::max(maxlen, std::max(na, nb));
+        sent[r] += (chunk_len(H, n, ring_send_chunk(phase, r, step, n)) +
+                    chunk_len(cb, n, ccw_send_chunk(phase, r, step, n))) * es;
+    }
+    p.tps = std::max<uint64_t>(1, ceil_div(maxlen, tile_elems(dtype, kVptMove)));
+    int op_eff = op;
+    if (op == RR_AVG && !(phase == RR_PHASE_REDUCE_SCATTER && step == n - 2)) op_eff = RR_SUM;
+    if (maxlen == 0) return RR_OK;
+    cudaError_t e = launch_step(dtype, op_eff, p, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "double ring step launch");
+    t_stats.launches += 1;
+    return RR_OK;
+}
+
+rr_status_t run_double_ring(void* const* bufs, int n, size_t count, rr_dtype_t dtype, rr_op_t op,
+                            cudaStream_t stream)
+{
+    std::vector<uint64_t> sent(n, 0);
+    for (int phase = RR_PHASE_REDUCE_SCATTER; phase <= RR_PHASE_ALL_GATHER; ++phase)
+        for (int s = 0; s < n - 1; ++s) {
+            rr_status_t st = double_ring_step_launch(bufs, n, count, dtype, op, phase, s, stream, sent);
+            if (st != RR_OK) return st;
+        }
+    t_stats.steps = 2 * (n - 1);
+    for (int r = 0; r < n; ++r) {
+        t_stats.bytes_sent_max = std::max<uint64_t>(t_stats.bytes_sent_max, sent[r]);
+        t_stats.bytes_sent_total += sent[r];
+    }
+    t_stats.hbm_bytes = 5ull * (uint64_t)(n - 1) * count * esize(dtype);
     return RR_OK;
 }
 
@@ -315,6 +385,7 @@ rr_algo_t resolve_algo(rr_algo_t algo, int n, size_t count, rr_dtype_t dtype)
         if (!std::strcmp(v, "tree")) return (int)RR_ALGO_TREE;
         if (!std::strcmp(v, "tree_oneshot")) return (int)RR_ALGO_TREE_ONESHOT;
         if (!std::strcmp(v, "two_shot")) return (int)RR_ALGO_TWO_SHOT;
+        if (!std::strcmp(v, "double_ring")) return (int)RR_ALGO_DOUBLE_RING;
         return -1;
     }();
     if (forced >= 0) return (rr_algo_t)forced;
@@ -394,7 +465,7 @@ rr_status_t rr_allreduce(void* const* bufs, int nranks, size_t count, rr_dtype_t
 {
     rr_status_t st = check_basic(nranks, dtype, op);
     if (st != RR_OK) return st;
-    if (algo < RR_ALGO_AUTO || algo > RR_ALGO_TWO_SHOT) return fail(RR_ERR_INVALID_ARG, "unknown algo");
+    if (algo < RR_ALGO_AUTO || algo > RR_ALGO_DOUBLE_RING) return fail(RR_ERR_INVALID_ARG, "unknown algo");
     if (!bufs) return fail(RR_ERR_INVALID_ARG, "NULL bufs array");
     const int n = nranks;
     const size_t es = esize(dtype);
@@ -414,6 +485,9 @@ rr_status_t rr_allreduce(void* const* bufs, int nranks, size_t count, rr_dtype_t
         break;
     case RR_ALGO_TREE:
         st = run_tree(bufs, n, count, dtype, op, stream);
+        break;
+    case RR_ALGO_DOUBLE_RING:
+        st = run_double_ring(bufs, n, count, dtype, op, stream);
         break;
     case RR_ALGO_ONESHOT: {
         const uint64_t C = ceil_div(count, (uint64_t)n);
@@ -470,7 +544,7 @@ rr_status_t rr_allreduce_host(void* const* host_bufs, void* const* dev_bufs, int
 {
     rr_status_t st = check_basic(nranks, dtype, op);
     if (st != RR_OK) return st;
-    if (algo < RR_ALGO_AUTO || algo > RR_ALGO_TWO_SHOT) return fail(RR_ERR_INVALID_ARG, "unknown algo");
+    if (algo < RR_ALGO_AUTO || algo > RR_ALGO_DOUBLE_RING) return fail(RR_ERR_INVALID_ARG, "unknown algo");
     if (!host_bufs || !dev_bufs) return fail(RR_ERR_INVALID_ARG, "NULL pointer array");
     const int n = nranks;
     const size_t es = esize(dtype), bytes = count * es;
@@ -857,8 +931,19 @@ rr_status_t rr_bucket_unpack(const rr_bucket_plan_t* plan, int bucket, const voi
     return bucket_copy(plan, bucket, grads, const_cast<void* const*>(buckets), nranks, op, false, stream);
 }
 
+static rr_status_t bucket_allreduce_capped(const rr_bucket_plan_t* plan, int bucket, void* const* grads,
+                                           int nranks, rr_op_t op, cudaStream_t stream, uint64_t max_grid);
+
 rr_status_t rr_bucket_allreduce(const rr_bucket_plan_t* plan, int bucket, void* const* grads, int nranks,
                                 rr_op_t op, cudaStream_t stream)
+{
+    return bucket_allreduce_capped(plan, bucket, grads, nranks, op, stream, kMaxGrid);
+}
+
+}  // extern "C"
+
+static rr_status_t bucket_allreduce_capped(const rr_bucket_plan_t* plan, int bucket, void* const* grads,
+                                           int nranks, rr_op_t op, cudaStream_t stream, uint64_t max_grid)
 {
     if (op != RR_SUM && op != RR_AVG) return fail(RR_ERR_UNSUPPORTED, "bucket all-reduce takes SUM or AVG");
     int t0 = 0, nt = 0;
@@ -881,7 +966,7 @@ rr_status_t rr_bucket_allreduce(const rr_bucket_plan_t* plan, int bucket, void* 
         bool v = true;
         for (int t = 0; t < ntens; ++t) v = v && same_phase(&p->grad[t * n], n);
         p->vec_ok = v;
-        cudaError_t e = launch_bucket_fold(plan->grad_dtype, op, *p, stream);
+        cudaError_t e = launch_bucket_fold(plan->grad_dtype, op, *p, stream, max_grid);
         if (e != cudaSuccess) return cuda_fail(e, "bucket all-reduce launch");
         t_stats.launches += 1;
         return RR_OK;
@@ -914,6 +999,8 @@ rr_status_t rr_bucket_allreduce(const rr_bucket_plan_t* plan, int bucket, void* 
     return st;
 }
 
+extern "C" {
+
 // -------------------------------------------------------------- reducer --
 
 }  // extern "C"
@@ -923,6 +1010,7 @@ struct rr_reducer {
     int n = 0;
     rr_op_t op = RR_AVG;
     cudaStream_t comm = nullptr;
+    uint64_t max_grid = kMaxGrid;     // CTAs of each bucket sync
     std::vector<void*> grads;         // nranks * ntensors, rank-major
     std::vector<int> pending;         // per bucket: tensors not yet marked in this step
     std::vector<char> marked;         // per tensor
@@ -945,7 +1033,7 @@ struct rr_reducer {
 extern "C" {
 
 rr_status_t rr_reducer_create(const rr_bucket_plan_t* plan, void* const* grads, int nranks, rr_op_t op,
-                              cudaStream_t comm, rr_reducer_t** out)
+                              cudaStream_t comm, int max_ctas, rr_reducer_t** out)
 {
     if (!out) return fail(RR_ERR_INVALID_ARG, "NULL reducer output");
     *out = nullptr;
@@ -957,6 +1045,7 @@ rr_status_t rr_reducer_create(const rr_bucket_plan_t* plan, void* const* grads, 
     red->n = nranks;
     red->op = op;
     red->comm = comm;
+    red->max_grid = max_ctas > 0 ? (uint64_t)max_ctas : kMaxGrid;
     red->grads.assign(grads, grads + (size_t)nranks * plan->ntensors);
     const int nb = (int)plan->first.size();
     red->pending.assign(nb, 0);
@@ -990,7 +1079,7 @@ rr_status_t rr_reducer_ready(rr_reducer_t* red, int tensor, cudaStream_t produce
     cudaError_t e = cudaEventRecord(red->ready[b], producer);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(red->comm, red->ready[b], 0);
     if (e != cudaSuccess) return cuda_fail(e, "ordering the bucket sync after its gradients");
-    return rr_bucket_allreduce(red->plan, b, red->grads.data(), red->n, red->op, red->comm);
+    return bucket_allreduce_capped(red->plan, b, red->grads.data(), red->n, red->op, red->comm, red->max_grid);
 }
 
 rr_status_t rr_reducer_finish(rr_reducer_t* red, cudaStream_t stream)
@@ -1035,6 +1124,10 @@ rr_status_t rr_cost_model(rr_algo_t algo, int nranks, double bytes, double alpha
     case RR_ALGO_TWO_SHOT:  // [P4]: reduce-scatter then all-gather by direct reads
         c.steps = nranks > 1 ? 2 : 0;
         c.bytes_sent = 2 * (n - 1) / n * bytes;
+        break;
+    case RR_ALGO_DOUBLE_RING:  // [P3] section 6: half the bytes on each of two links
+        c.steps = 2 * (n - 1);
+        c.bytes_sent = (n - 1) / n * bytes;
         break;
     default:
         return fail(RR_ERR_INVALID_ARG, "unknown algo");

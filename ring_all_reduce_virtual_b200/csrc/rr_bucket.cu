@@ -167,21 +167,21 @@ __global__ void __launch_bounds__(kThreads) bucket_fold_kernel(const __grid_cons
 }
 
 template <class P>
-cudaError_t launch_all_b(void (*kernel)(P), const P& p, uint64_t work, cudaStream_t s)
+cudaError_t launch_all_b(void (*kernel)(P), const P& p, uint64_t work, cudaStream_t s, uint64_t max_grid = kMaxGrid)
 {
     if (work == 0) return cudaSuccess;
-    const uint64_t grid = work < kMaxGrid ? work : kMaxGrid;
+    const uint64_t grid = work < max_grid ? work : max_grid;
     kernel<<<(unsigned)grid, kThreads, 0, s>>>(p);
     return cudaGetLastError();
 }
 
 template <class G, int OP>
-cudaError_t launch_fold(const BucketFoldParams& p, uint64_t work, cudaStream_t s)
+cudaError_t launch_fold(const BucketFoldParams& p, uint64_t work, cudaStream_t s, uint64_t max_grid)
 {
     const int vpt = reduce_vpt(p.n);
-    if (vpt == 8) return launch_all_b(bucket_fold_kernel<G, OP, 8, 1>, p, work, s);
-    if (vpt == 4) return launch_all_b(bucket_fold_kernel<G, OP, 4, 3>, p, work, s);
-    return launch_all_b(bucket_fold_kernel<G, OP, kVptReduce, kGroup>, p, work, s);
+    if (vpt == 8) return launch_all_b(bucket_fold_kernel<G, OP, 8, 1>, p, work, s, max_grid);
+    if (vpt == 4) return launch_all_b(bucket_fold_kernel<G, OP, 4, 3>, p, work, s, max_grid);
+    return launch_all_b(bucket_fold_kernel<G, OP, kVptReduce, kGroup>, p, work, s, max_grid);
 }
 
 }  // namespace
@@ -214,12 +214,14 @@ cudaError_t launch_bucket_unpack(int grad_dtype, int op, const BucketCopyParams&
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p, cudaStream_t s)
+cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p, cudaStream_t s, uint64_t max_grid)
 {
     const uint64_t work = p.tile0[p.nseg];
     const bool avg = op == kAvg;
-    if (grad_dtype == kBF16) return avg ? launch_fold<BF16T, kAvg>(p, work, s) : launch_fold<BF16T, kSum>(p, work, s);
-    if (grad_dtype == kF32) return avg ? launch_fold<F32T, kAvg>(p, work, s) : launch_fold<F32T, kSum>(p, work, s);
+    if (grad_dtype == kBF16)
+        return avg ? launch_fold<BF16T, kAvg>(p, work, s, max_grid) : launch_fold<BF16T, kSum>(p, work, s, max_grid);
+    if (grad_dtype == kF32)
+        return avg ? launch_fold<F32T, kAvg>(p, work, s, max_grid) : launch_fold<F32T, kSum>(p, work, s, max_grid);
     return cudaErrorInvalidValue;
 }
 

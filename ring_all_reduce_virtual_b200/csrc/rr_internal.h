@@ -41,7 +41,7 @@ struct StepSeg {
 };
 
 struct StepParams {
-    StepSeg seg[kMaxRanksH];
+    StepSeg seg[2 * kMaxRanksH];  // one per rank, or two (the double ring's two directions)
     int nseg;
     int nin;        // 2: fold, 1: copy
     int vec_ok;     // every segment's pointers agree modulo 16 bytes
@@ -126,7 +126,8 @@ cudaError_t launch_rank_kernel(int kind, int dtype, int op, const RankParams& p,
 cudaError_t launch_step(int dtype, int op, const StepParams& p, cudaStream_t s);
 cudaError_t launch_bucket_pack(int grad_dtype, const BucketCopyParams& p, cudaStream_t s);
 cudaError_t launch_bucket_unpack(int grad_dtype, int op, const BucketCopyParams& p, cudaStream_t s);
-cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p, cudaStream_t s);
+cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p, cudaStream_t s,
+                               uint64_t max_grid = kMaxGrid);
 
 }  // namespace rr
 

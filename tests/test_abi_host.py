@@ -144,6 +144,10 @@ def test_cost_model_tree_and_oneshot_steps():
         # two-shot: the ring's per-rank volume in two steps
         two = rrv.cost_model("two_shot", n, 1.0, 1.0, 1.0)
         assert two["steps"] == 2 and two["bytes_sent"] == rrv.cost_model("ring", n, 1.0, 1.0, 1.0)["bytes_sent"]
+        # [P3] section 6: the double ring halves the bytes on each link
+        dbl = rrv.cost_model("double_ring", n, 1.0, 1.0, 1.0)
+        assert dbl["steps"] == 2 * (n - 1)
+        assert dbl["bytes_sent"] == rrv.cost_model("ring", n, 1.0, 1.0, 1.0)["bytes_sent"] / 2
 
 
 def test_picker_is_size_aware_and_exact():
@@ -175,7 +179,7 @@ def test_argument_errors_return_before_any_launch():
     assert lib.rr_allreduce(_fake(4), 4, 16, 7, 0, 0, s) == _lib.RR_ERR_INVALID_ARG
     assert lib.rr_allreduce(_fake(4), 4, 16, 0, 9, 0, s) == _lib.RR_ERR_INVALID_ARG
     assert lib.rr_allreduce(_fake(4), 4, 16, 0, 0, 9, s) == _lib.RR_ERR_INVALID_ARG
-    assert lib.rr_allreduce(_fake(4), 4, 16, 0, 0, 6, s) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_allreduce(_fake(4), 4, 16, 0, 0, 7, s) == _lib.RR_ERR_INVALID_ARG
     assert lib.rr_allreduce(_fake(4), 4, 16, 2, 1, 0, s) == _lib.RR_ERR_UNSUPPORTED  # int32 AVG
     assert lib.rr_allreduce(None, 4, 16, 0, 0, 0, s) == _lib.RR_ERR_INVALID_ARG
     overlapping = _fake(4, stride=32)  # 16 fp32 = 64 bytes apart by 32
@@ -197,10 +201,10 @@ def test_argument_errors_return_before_any_launch():
 def test_reducer_argument_errors():
     lib = _lib.lib()
     out = ctypes.c_void_p()
-    assert lib.rr_reducer_create(None, _fake(2), 2, 1, None, ctypes.byref(out)) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_reducer_create(None, _fake(2), 2, 1, None, 0, ctypes.byref(out)) == _lib.RR_ERR_INVALID_ARG
     plan = rrv.BucketPlan([10, 20], "bf16", 100)
-    assert lib.rr_reducer_create(plan._h, _fake(4), 2, 2, None, ctypes.byref(out)) == _lib.RR_ERR_UNSUPPORTED
-    assert lib.rr_reducer_create(plan._h, _fake(4), 0, 1, None, ctypes.byref(out)) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_reducer_create(plan._h, _fake(4), 2, 2, None, 0, ctypes.byref(out)) == _lib.RR_ERR_UNSUPPORTED
+    assert lib.rr_reducer_create(plan._h, _fake(4), 0, 1, None, 0, ctypes.byref(out)) == _lib.RR_ERR_INVALID_ARG
     assert lib.rr_reducer_ready(None, 0, None) == _lib.RR_ERR_INVALID_ARG
     assert lib.rr_reducer_finish(None, None) == _lib.RR_ERR_INVALID_ARG
 

@@ -19,8 +19,9 @@ from ring_all_reduce_virtual_b200 import synth
 
 pytestmark = pytest.mark.gpu
 
-ALGOS = ["ring", "oneshot", "tree", "tree_oneshot", "two_shot", "auto"]
+ALGOS = ["ring", "oneshot", "tree", "tree_oneshot", "two_shot", "double_ring", "auto"]
 ORACLE = {
+    "double_ring": oracle.double_ring_allreduce,
     "two_shot": oracle.fold_ring_order,
     "ring": oracle.ring_allreduce,
     "oneshot": oracle.fold_ring_order,
@@ -201,6 +202,10 @@ def test_ring_stats_match_the_schedule():
     rrv.all_reduce(d, "sum", "two_shot")  # the ring's per-rank volume in 2 steps
     st = rrv.last_stats()
     assert st["launches"] == 2 and st["steps"] == 2 and st["bytes_sent_max"] == 6144
+    rrv.all_reduce(d, "sum", "double_ring")  # the same volume, half to each neighbour
+    st = rrv.last_stats()
+    want = oracle.double_ring_allreduce(synth.ranks(7, n, count, "uniform"))
+    assert st["launches"] == 6 and st["bytes_sent_max"] == int(want.max()) == 6144
 
 
 # --------------------------------------------- reduce-scatter, all-gather --

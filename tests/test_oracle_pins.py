@@ -516,3 +516,61 @@ def test_mutants_are_caught(kind):
     assert failed > 0, f"mutant {kind} passed every pin"
     for pin in _pins():  # and the real oracle passes them all
         pin()
+
+
+# ------------------------------------------------------------ double ring --
+
+def _double_fixture():
+    n = 4
+    big = np.float32(2.0 ** 24)
+    pattern = [np.float32(1), big, np.float32(1), -big]
+    x = [np.zeros(8, dtype=np.float32) for _ in range(n)]
+    for i in range(n):
+        for k, v in enumerate(pattern):
+            x[(i + k) % n][i] = v          # half A: upwards from rank i
+            x[(i - k) % n][4 + i] = v      # half B: downwards from rank i
+    return x
+
+
+def test_double_ring_fold_order_golden():
+    g = {ln.split(":")[0]: _vals(ln) for ln in golden_lines("double_ring_fold_order.txt")}
+    for f in (oracle.double_ring_allreduce, oracle.fold_double_ring):
+        x = _double_fixture()
+        f(x, "sum")
+        for r in range(4):
+            assert x[r].tolist() == g["double_ring"]
+    # half B folded upwards from its own chunk index instead
+    x = _double_fixture()
+    vals = np.stack([v[4:] for v in x])
+    assert oracle.fold_samples(vals, np.arange(4)).tolist() == g["half_b_folded_upwards"][4:]
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 4, 5, 8])
+@pytest.mark.parametrize("op", ["sum", "max", "min", "prod"])
+def test_double_ring_brute_force_integer_data(n, op):
+    for count in [0, 1, 2 * n - 1, 4 * n + 3]:
+        lo, hi = (-3, 4) if op == "prod" else (-100, 100)
+        rng = np.random.default_rng([n, count, 7])
+        x = [synth.cast(rng.integers(lo, hi, size=count), "f32") for _ in range(n)]
+        want = _np_reduce(x, op)
+        oracle.double_ring_allreduce(x, op)
+        for r in range(n):
+            assert np.array_equal(x[r], want)
+
+
+@pytest.mark.parametrize("n", [2, 3, 4, 8, 16])
+def test_double_ring_bytes(n):
+    # each step sends one chunk of each half to each neighbour: in all
+    # 2(N-1) S, and 2(N-1)/N S per rank when 2N divides the count
+    for per in (1, 5):
+        count = 2 * n * per
+        sent = oracle.double_ring_allreduce(synth.ranks(3, n, count, "uniform"))
+        assert sent.tolist() == [2 * (n - 1) * count * 4 // n] * n
+    sent = oracle.double_ring_allreduce(synth.ranks(3, n, 2 * n + 3, "uniform"))
+    assert int(sent.sum()) == 2 * (n - 1) * (2 * n + 3) * 4
+
+
+def test_double_ring_mutant_is_caught():
+    with oracle.mutant(10):
+        with pytest.raises(AssertionError):
+            test_double_ring_brute_force_integer_data(4, "sum")
