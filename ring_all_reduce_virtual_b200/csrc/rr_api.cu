@@ -523,7 +523,7 @@ rr_status_t rr_allreduce(void* const* bufs, int nranks, size_t count, rr_dtype_t
         break;
     }
     case RR_ALGO_TREE_ONESHOT: {
-        const uint64_t tps = std::max<uint64_t>(1, ceil_div(count, tile_elems(dtype, kVptReduce)));
+        const uint64_t tps = std::max<uint64_t>(1, ceil_div(count, tile_elems(dtype, reduce_vpt(n))));
         st = run_rank_kernel(kOneshotTree, bufs, bufs, n, count, count, 1, tps, dtype, op, same_phase(bufs, n),
                              stream);
         t_stats.steps = 1;
@@ -602,7 +602,7 @@ rr_status_t rr_allreduce_host(void* const* host_bufs, void* const* dev_bufs, int
         } else {
             void* off[RR_MAX_RANKS];
             for (int r = 0; r < n; ++r) off[r] = static_cast<char*>(dev_bufs[r]) + lo * es;
-            const uint64_t tps = std::max<uint64_t>(1, ceil_div(len, tile_elems(dtype, kVptReduce)));
+            const uint64_t tps = std::max<uint64_t>(1, ceil_div(len, tile_elems(dtype, reduce_vpt(n))));
             st = run_rank_kernel(kOneshotTree, off, off, n, len, len, 1, tps, dtype, op, same_phase(off, n), stream);
         }
         if (st != RR_OK) return st;

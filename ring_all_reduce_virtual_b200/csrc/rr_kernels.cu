@@ -18,8 +18,6 @@ namespace rr {
 
 namespace {
 
-template <class Ty>
-constexpr uint64_t kTileElems = (uint64_t)kThreads * kVptReduce * Ty::L;  // tree one-shot tiles
 
 // ------------------------------------------------ one-shot, ring order
 // Segment c = chunk c of every rank buffer; its fold starts on rank c and
@@ -203,11 +201,81 @@ __device__ __forceinline__ void tree_fold_lanes(const RankParams& p, uint64_t e0
     for (int o = 0; o < n; ++o) Ty::st1(static_cast<T*>(p.out[o]) + e0, cur[0]);
 }
 
-template <class Ty, int OP>
+// For N <= NMAX <= 8: every rank's vectors for VPT vectors are loaded first
+// (N * VPT loads in flight per thread), then each vector is folded in tree
+// order with the same stack as tree_fold_lanes, levels fixed at compile time.
+template <class Ty, int OP, int NMAX, int VPT>
+__device__ __forceinline__ void tree_vectors(const RankParams& p, uint64_t v0, uint64_t nv, uint64_t head)
+{
+    using T = typename Ty::T;
+    using Acc = typename Ty::Acc;
+    constexpr int L = Ty::L;
+    constexpr int LV = NMAX <= 2 ? 2 : (NMAX <= 4 ? 3 : 4);  // log2(NMAX) + 1 stack levels
+    const int n = p.n;
+    uint64_t off[VPT];
+    bool ok[VPT];
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) {
+        const uint64_t v = v0 + (uint64_t)u * kThreads + threadIdx.x;
+        ok[u] = v < nv;
+        off[u] = head + v * L;
+    }
+    uint4 raw[NMAX][VPT];
+#pragma unroll
+    for (int j = 0; j < NMAX; ++j)
+        if (j < n) {
+            const T* src = static_cast<const T*>(p.in[j]);
+#pragma unroll
+            for (int u = 0; u < VPT; ++u)
+                if (ok[u]) raw[j][u] = ldv(src + off[u]);
+        }
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) {
+        if (!ok[u]) continue;
+        Acc slot[LV][L];
+        Acc cur[L];
+#pragma unroll
+        for (int j = 0; j < NMAX; ++j) {
+            if (j < n) {
+                Ty::unpack(raw[j][u], cur);
+                int lvl = 0;
+#pragma unroll
+                for (int b = 0; b < LV - 1; ++b) {
+                    if (((j >> b) & 1) && lvl == b) {
+#pragma unroll
+                        for (int l = 0; l < L; ++l) cur[l] = apply<OP>(slot[b][l], cur[l]);
+                        lvl = b + 1;
+                    }
+                }
+#pragma unroll
+                for (int b = 0; b < LV; ++b)
+                    if (b == lvl)
+#pragma unroll
+                        for (int l = 0; l < L; ++l) slot[b][l] = cur[l];
+            }
+        }
+        bool have = false;
+#pragma unroll
+        for (int b = 0; b < LV; ++b) {
+            if ((n >> b) & 1) {
+#pragma unroll
+                for (int l = 0; l < L; ++l) cur[l] = have ? apply<OP>(slot[b][l], cur[l]) : slot[b][l];
+                have = true;
+            }
+        }
+#pragma unroll
+        for (int l = 0; l < L; ++l) cur[l] = finish<OP>(cur[l], p.divisor);
+        const uint4 r = Ty::pack(cur);
+#pragma unroll 4
+        for (int o = 0; o < n; ++o) stv(static_cast<T*>(p.out[o]) + off[u], r);
+    }
+}
+
+template <class Ty, int OP, int NMAX, int VPT>
 __global__ void __launch_bounds__(kThreads) oneshot_tree_kernel(const __grid_constant__ RankParams p)
 {
     constexpr int L = Ty::L;
-    constexpr uint64_t TE = kTileElems<Ty>;
+    constexpr uint64_t TE = (uint64_t)kThreads * VPT * L;
     const int tid = threadIdx.x;
     const int ph = p.vec_ok ? phase_of(static_cast<const typename Ty::T*>(p.in[0]), L) : -1;
     uint64_t head = 0, nv = 0;
@@ -229,9 +297,13 @@ __global__ void __launch_bounds__(kThreads) oneshot_tree_kernel(const __grid_con
             const uint64_t e = (uint64_t)tid < head ? (uint64_t)tid : tail_lo + ((uint64_t)tid - head);
             tree_fold_lanes<Ty, OP, 1>(p, e, false);
         }
-        for (int u = 0; u < kVptReduce; ++u) {
-            const uint64_t v = tile * (TE / L) + (uint64_t)u * kThreads + tid;
-            if (v < nv) tree_fold_lanes<Ty, OP, L>(p, head + v * L, true);
+        if constexpr (NMAX <= 8) {
+            tree_vectors<Ty, OP, NMAX, VPT>(p, tile * (TE / L), nv, head);
+        } else {
+            for (int u = 0; u < VPT; ++u) {
+                const uint64_t v = tile * (TE / L) + (uint64_t)u * kThreads + tid;
+                if (v < nv) tree_fold_lanes<Ty, OP, L>(p, head + v * L, true);
+            }
         }
     }
 }
@@ -313,7 +385,11 @@ cudaError_t launch_rank_kernel(int kind, int dtype, int op, const RankParams& p,
             if (vpt == 8) return launch_all(reduce_scatter_kernel<Ty, OP, 8, 1>, p, work, s);
             if (vpt == 4) return launch_all(reduce_scatter_kernel<Ty, OP, 4, 3>, p, work, s);
             return launch_all(reduce_scatter_kernel<Ty, OP, kVptReduce, kGroup>, p, work, s);
-        case kOneshotTree: return launch_all(oneshot_tree_kernel<Ty, OP>, p, work, s);
+        case kOneshotTree:
+            if (p.n <= 2) return launch_all(oneshot_tree_kernel<Ty, OP, 2, 8>, p, work, s);
+            if (p.n <= 4) return launch_all(oneshot_tree_kernel<Ty, OP, 4, 4>, p, work, s);
+            if (p.n <= 8) return launch_all(oneshot_tree_kernel<Ty, OP, 8, kVptReduce>, p, work, s);
+            return launch_all(oneshot_tree_kernel<Ty, OP, kMaxRanks, kVptReduce>, p, work, s);
         case kAllGather: return launch_all(all_gather_kernel<Ty>, p, work, s);
         case kAllToAll: return launch_all(all_to_all_kernel<Ty>, p, work, s);
         case kChunkBroadcast: return launch_all(chunk_bcast_kernel<Ty>, p, work, s);
