@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kThreads) bucket_unpack_kernel(const __grid_co
 // bucket's flat index; every rank's copy is read once, folded in fp32 in ring
 // order from rank c, divided (AVG), rounded once and written back to every
 // rank.  Same bits as pack -> one-shot all-reduce (SUM) -> unpack.
-template <class G, int OP, int VPT, int GR>
+template <class G, int OP, int VPT, int GR, int NS>
 __global__ void __launch_bounds__(kThreads) bucket_fold_kernel(const __grid_constant__ BucketFoldParams p)
 {
     using T = typename G::T;
@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(kThreads) bucket_fold_kernel(const __grid_cons
         const int s = find_segment(p.tile0, p.nseg, w);
         const uint64_t tile = w - p.tile0[s];
         const BucketSeg& sg = p.seg[s];
-        const int n = p.n;
+        const int n = NS > 0 ? NS : p.n;
         const int base = (int)sg.t * n;
         const int start = (int)sg.c;
         auto in = [&](int j) {
@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(kThreads) bucket_fold_kernel(const __grid_cons
             return static_cast<const T*>(p.grad[base + r]) + sg.off;
         };
         auto out = [&](int o) { return static_cast<T*>(p.grad[base + o]) + sg.off; };
-        fold_tile<G, OP, VPT, GR>(in, n, out, n, sg.len, tile, p.vec_ok, p.divisor);
+        fold_tile<G, OP, VPT, GR, NS>(in, n, out, n, sg.len, tile, p.vec_ok, p.divisor);
     }
 }
 
@@ -178,10 +178,13 @@ cudaError_t launch_all_b(void (*kernel)(P), const P& p, uint64_t work, cudaStrea
 template <class G, int OP>
 cudaError_t launch_fold(const BucketFoldParams& p, uint64_t work, cudaStream_t s, uint64_t max_grid)
 {
-    const int vpt = reduce_vpt(p.n);
-    if (vpt == 8) return launch_all_b(bucket_fold_kernel<G, OP, 8, 1>, p, work, s, max_grid);
-    if (vpt == 4) return launch_all_b(bucket_fold_kernel<G, OP, 4, 3>, p, work, s, max_grid);
-    return launch_all_b(bucket_fold_kernel<G, OP, kVptReduce, kGroup>, p, work, s, max_grid);
+    constexpr int V = kVptReduce;
+    switch (p.n) {
+    case 2: return launch_all_b(bucket_fold_kernel<G, OP, V, 1, 2>, p, work, s, max_grid);
+    case 4: return launch_all_b(bucket_fold_kernel<G, OP, V, 3, 4>, p, work, s, max_grid);
+    case 8: return launch_all_b(bucket_fold_kernel<G, OP, V, 7, 8>, p, work, s, max_grid);
+    }
+    return launch_all_b(bucket_fold_kernel<G, OP, V, kGroup, 0>, p, work, s, max_grid);
 }
 
 }  // namespace

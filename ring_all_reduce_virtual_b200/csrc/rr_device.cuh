@@ -151,6 +151,18 @@ __device__ __forceinline__ float finish(float a, float divisor)
 template <int OP>
 __device__ __forceinline__ int32_t finish(int32_t a, float) { return a; }
 
+// finish() for a rank count NS fixed at compile time (0: use the runtime
+// divisor): a power-of-two NS multiplies by its exact reciprocal, a constant.
+template <int OP, int NS>
+__device__ __forceinline__ float finish_n(float a, float divisor)
+{
+    if constexpr (OP == kAvg && NS > 0 && (NS & (NS - 1)) == 0) return __fmul_rn(a, 1.0f / (float)NS);
+    else return finish<OP>(a, divisor);
+}
+
+template <int OP, int NS>
+__device__ __forceinline__ int32_t finish_n(int32_t a, float) { return a; }
+
 // ------------------------------------------------------------------ memory
 
 // 128-bit streaming access: every byte is touched once per call, so hint the
@@ -182,7 +194,8 @@ __device__ __forceinline__ void fold_one(const InF& in, int nin, const OutF& out
 // Fold (nin > 1) or copy (nin == 1) tile `tile` of a segment of `len`
 // elements.  VPT is the number of 16-byte vectors per thread per tile, G the
 // number of further input ranks whose loads are issued before they are
-// folded: every thread keeps up to VPT * (G + 1) loads in flight.  in(j) /
+// folded: every thread keeps up to VPT * (G + 1) loads in flight.  NS > 0 is
+// the rank count (AVG's divisor) when it is fixed at compile time.  in(j) /
 // out(o) return the segment's base pointers.  vec_ok says
 // that every in(j) has the same address modulo 16 as in(0), and every out(o)
 // the same as out(0) (checked by the host); when in(0) and out(0) also agree,
@@ -191,7 +204,7 @@ __device__ __forceinline__ void fold_one(const InF& in, int nin, const OutF& out
 // scalar.  Tile t covers body vectors [t*TV, (t+1)*TV), TV = kThreads*VPT, or
 // the same number of elements on the scalar path; tile 0 also does the head
 // and tail.
-template <class Ty, int OP, int VPT, int G, class InF, class OutF>
+template <class Ty, int OP, int VPT, int G, int NS = 0, class InF, class OutF>
 __device__ __forceinline__ void fold_tile(const InF& in, int nin, const OutF& out, int nout, uint64_t len,
                                           uint64_t tile, bool vec_ok, float divisor)
 {
@@ -279,7 +292,7 @@ __device__ __forceinline__ void fold_tile(const InF& in, int nin, const OutF& ou
 #pragma unroll
     for (int u = 0; u < VPT; ++u) {
 #pragma unroll
-        for (int l = 0; l < L; ++l) a[u][l] = finish<OP>(a[u][l], divisor);
+        for (int l = 0; l < L; ++l) a[u][l] = finish_n<OP, NS>(a[u][l], divisor);
         res[u] = Ty::pack(a[u]);
     }
 #pragma unroll 4

@@ -108,9 +108,12 @@ constexpr int kVptReduce = 2;
 constexpr int kVptMove = 4;
 
 // Vectors per thread of the N-input folds (one-shot all-reduce, reduce-scatter,
-// fused bucket sync) by rank count: few ranks give few loads per vector, so
-// each thread takes more vectors (N * VPT loads in flight).
-inline int reduce_vpt(int n) { return n <= 2 ? 8 : (n <= 4 ? 4 : kVptReduce); }
+// fused bucket sync, tree-order one-shot).  These kernels are also compiled for
+// fixed rank counts (2, 3, 4, 8, 16; the bucket kernel 2, 4, 8): with the
+// count known the compiler unrolls every rank loop, needs few registers and
+// keeps N * 2 loads per thread in flight at high occupancy.  Other counts run
+// a variant with a runtime rank count.
+inline int reduce_vpt(int) { return kVptReduce; }
 
 // Elements one fold tile covers (for sizing tiles per segment on the host),
 // and one bucket pack/unpack tile.

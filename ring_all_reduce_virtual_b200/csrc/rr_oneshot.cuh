@@ -1,0 +1,38 @@
+// rr_oneshot.cuh -- launchers of the one-shot kernels (ring order and tree
+// order), compiled in their own files (rr_oneshot.cu, rr_tree.cu) and
+// instantiated there for every (element type, op) pair.
+#pragma once
+
+#include "rr_launch.cuh"
+
+namespace rr {
+
+template <class Ty, int OP>
+cudaError_t launch_oneshot_ring(const RankParams& p, uint64_t work, cudaStream_t s);
+template <class Ty, int OP>
+cudaError_t launch_oneshot_tree(const RankParams& p, uint64_t work, cudaStream_t s);
+
+#define RR_FOR_EACH_TYPE_OP(X)                                                                   \
+    X(F32T, kSum) X(F32T, kAvg) X(F32T, kMax) X(F32T, kMin) X(F32T, kProd) X(BF16T, kSum)         \
+    X(BF16T, kAvg) X(BF16T, kMax) X(BF16T, kMin) X(BF16T, kProd) X(I32T, kSum) X(I32T, kMax)     \
+    X(I32T, kMin) X(I32T, kProd)
+
+#define RR_DECLARE_ONESHOT(TY, OP)                                                               \
+    extern template cudaError_t launch_oneshot_ring<TY, OP>(const RankParams&, uint64_t, cudaStream_t); \
+    extern template cudaError_t launch_oneshot_tree<TY, OP>(const RankParams&, uint64_t, cudaStream_t);
+RR_FOR_EACH_TYPE_OP(RR_DECLARE_ONESHOT)
+#undef RR_DECLARE_ONESHOT
+
+// I32T has no AVG; these are never launched (the host rejects AVG on int32).
+template <>
+inline cudaError_t launch_oneshot_ring<I32T, kAvg>(const RankParams&, uint64_t, cudaStream_t)
+{
+    return cudaErrorInvalidValue;
+}
+template <>
+inline cudaError_t launch_oneshot_tree<I32T, kAvg>(const RankParams&, uint64_t, cudaStream_t)
+{
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace rr
