@@ -41,7 +41,7 @@ FALLBACK_HBM_GBS = 6650.0
 # from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), with the
 # hash of the kernel sources it was taken on.  The summary with its command is
 # in profiles/oneshot_ring_kernel_allreduce-8x64MiB-f32.md.
-NCU_TRAFFIC = {"per_algorithmic_byte": (536951296 + 479357952) / 1073741824, "sources_sha1": "9e541d55bed5d43b1a26e20616c156b3b2af75e3"}
+NCU_TRAFFIC = {"per_algorithmic_byte": (536897536 + 479857152) / 1073741824, "sources_sha1": "55f841d8773d0e298817017275745aae91002d67"}
 
 
 def sources_sha1() -> str:
@@ -367,7 +367,7 @@ def run_ours(args, d: Dist):
             "hbm_gbs": round(achieved, 1), "hbm_frac": round(achieved / peak, 4),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,
-                         "kernel": "oneshot_ring_kernel<F32T, AVG>",
+                         "kernel": "oneshot_ring_kernel<F32T, AVG, VPT 2, G 7, N 8>",
                          "algorithmic_bytes_per_launch": alg_bytes, "peak_kind": peak_kind + " (burst copy)"},
             "cpu_baseline": cpu,
             "e2e": e2e,
