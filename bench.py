@@ -39,15 +39,19 @@ FALLBACK_HBM_GBS = 6650.0
 
 # DRAM traffic of one launch of the dominant kernel per algorithmic byte,
 # from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), with the
-# hash of the kernel sources it was taken on.  The summary with its command is
+# hash of the dominant kernel's source files it was taken on.  The summary with its command is
 # in profiles/oneshot_ring_kernel_allreduce-8x64MiB-f32.md.
-NCU_TRAFFIC = {"per_algorithmic_byte": (536897536 + 479857152) / 1073741824, "sources_sha1": "55f841d8773d0e298817017275745aae91002d67"}
+NCU_TRAFFIC = {"per_algorithmic_byte": (536897536 + 479857152) / 1073741824, "sources_sha1": "6479c4fa7bafa2b72ac0443d7e663b319536b012"}
+
+
+# The files that define the dominant kernel (oneshot_ring_kernel).
+KERNEL_SOURCES = ("rr_device.cuh", "rr_internal.h", "rr_launch.cuh", "rr_oneshot.cuh", "rr_oneshot.cu")
 
 
 def sources_sha1() -> str:
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "ring_all_reduce_virtual_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()

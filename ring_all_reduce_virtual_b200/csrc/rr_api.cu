@@ -392,8 +392,17 @@ rr_algo_t resolve_algo(rr_algo_t algo, int n, size_t count, rr_dtype_t dtype)
     return rr_pick_algo(n, count, dtype);
 }
 
-// Slice size of the pipelined host-buffer all-reduce, per rank.
-constexpr uint64_t kHostSliceBytes = 8ull << 20;
+// Slice size of the pipelined host-buffer all-reduce, per rank: 8 MiB, or
+// RR_HOST_SLICE_MB (1..256) from the environment.
+uint64_t host_slice_bytes()
+{
+    static const uint64_t v = [] {
+        const char* e = std::getenv("RR_HOST_SLICE_MB");
+        const long mb = e ? std::strtol(e, nullptr, 10) : 8;
+        return (uint64_t)(mb >= 1 && mb <= 256 ? mb : 8) << 20;
+    }();
+    return v;
+}
 
 // Two copy streams and the events that order them against the caller's
 // stream; created once per device and kept until exit.
@@ -556,7 +565,7 @@ rr_status_t rr_allreduce_host(void* const* host_bufs, void* const* dev_bufs, int
     if ((st = check_spans(spans)) != RR_OK) return st;
     const rr_algo_t a = resolve_algo(algo, n, count, dtype);
     if (count == 0) return rr_allreduce(dev_bufs, n, 0, dtype, op, a, stream);
-    const bool sliced = n > 1 && (a == RR_ALGO_ONESHOT || a == RR_ALGO_TREE_ONESHOT) && bytes > kHostSliceBytes;
+    const bool sliced = n > 1 && (a == RR_ALGO_ONESHOT || a == RR_ALGO_TREE_ONESHOT) && bytes > host_slice_bytes();
     if (!sliced) {  // copy in, reduce, copy out, all on the caller's stream
         for (int r = 0; r < n; ++r) {
             cudaError_t e = cudaMemcpyAsync(dev_bufs[r], host_bufs[r], bytes, cudaMemcpyHostToDevice, stream);
@@ -580,7 +589,7 @@ rr_status_t rr_allreduce_host(void* const* host_bufs, void* const* dev_bufs, int
     if ((st = ck(cudaEventRecord(hp->start, stream), "event record")) != RR_OK) return st;
     if ((st = ck(cudaStreamWaitEvent(hp->in, hp->start, 0), "stream wait")) != RR_OK) return st;
     if ((st = ck(cudaStreamWaitEvent(hp->out, hp->start, 0), "stream wait")) != RR_OK) return st;
-    const uint64_t slice = std::max<uint64_t>(1, kHostSliceBytes / es);
+    const uint64_t slice = std::max<uint64_t>(1, host_slice_bytes() / es);
     const uint64_t C = ceil_div(count, (uint64_t)n);
     const bool vec = same_phase(dev_bufs, n);
     int launches = 0;

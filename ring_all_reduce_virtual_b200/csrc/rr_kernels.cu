@@ -95,7 +95,9 @@ __global__ void __launch_bounds__(kThreads) all_to_all_kernel(const __grid_const
 // ------------------------------------------------------- table steps
 // One ring step or one tree level: every segment folds in0 op in1 into out
 // (nin == 2) or copies in0 to out (nin == 1).
-template <class Ty, int OP>
+// NIN: 2 folds (a reduce-scatter step or reduce level), 1 copies (an
+// all-gather step or broadcast level); fixed at compile time.
+template <class Ty, int OP, int NIN>
 __global__ void __launch_bounds__(kThreads) step_kernel(const __grid_constant__ StepParams p)
 {
     using T = typename Ty::T;
@@ -106,7 +108,7 @@ __global__ void __launch_bounds__(kThreads) step_kernel(const __grid_constant__ 
         if (sg.len == 0) continue;
         auto in = [&](int j) { return static_cast<const T*>(j == 0 ? sg.in0 : sg.in1); };
         auto out = [&](int) { return static_cast<T*>(sg.out); };
-        fold_tile<Ty, OP, kVptMove, 1>(in, p.nin, out, 1, sg.len, tile, p.vec_ok, p.divisor);
+        fold_tile<Ty, OP, kVptMove, 1>(in, NIN, out, 1, sg.len, tile, p.vec_ok, p.divisor);
     }
 }
 
@@ -148,8 +150,10 @@ cudaError_t launch_step(int dtype, int op, const StepParams& p, cudaStream_t s)
 {
     const uint64_t work = (uint64_t)p.nseg * p.tps;
     if (p.nin == 1) op = kSum;
-    return with_type(dtype, op,
-                     [&]<class Ty, int OP>() { return launch_all(step_kernel<Ty, OP>, p, work, s); });
+    return with_type(dtype, op, [&]<class Ty, int OP>() {
+        return p.nin == 2 ? launch_all(step_kernel<Ty, OP, 2>, p, work, s)
+                          : launch_all(step_kernel<Ty, kSum, 1>, p, work, s);
+    });
 }
 
 }  // namespace rr
