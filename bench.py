@@ -303,12 +303,12 @@ def run_ours(args, d: Dist):
     import ring_all_reduce_virtual_b200 as rrv
     from ring_all_reduce_virtual_b200.build import build
 
-    if d.rank == 0:
-        build()
-    d.barrier()
     torch.cuda.set_device(d.local_rank)
     dev = torch.device("cuda", d.local_rank)
     d.init("nccl")
+    if d.rank == 0:
+        build()  # no-op when the library is up to date
+    d.barrier()  # the other ranks load the library only once it is built
     stream = torch.cuda.current_stream(dev)
 
     count = args.count
@@ -676,6 +676,8 @@ def run_kernels(args):
 
     for algo in ("oneshot", "two_shot", "ring", "double_ring", "tree", "tree_oneshot"):
         emit(f"all_reduce {algo}", lambda: rrv.all_reduce(x, "sum", algo, stream))
+    for algo in ("oneshot", "ring"):
+        emit(f"all_reduce_wire bf16 {algo}", lambda: rrv.all_reduce_wire(x, "avg", "bf16", algo, stream))
     emit("reduce_scatter", lambda: rrv.reduce_scatter(x, rs, "sum", "auto", stream))
     emit("all_gather", lambda: rrv.all_gather(rs, out, "auto", stream))
     emit("all_to_all", lambda: rrv.all_to_all(x, out, stream))

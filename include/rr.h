@@ -163,6 +163,22 @@ typedef struct rr_cost {
 rr_status_t rr_allreduce(void* const* bufs, int nranks, size_t count, rr_dtype_t dtype, rr_op_t op,
                          rr_algo_t algo, cudaStream_t stream);
 
+/* All-reduce of fp32 buffers with a low-precision wire ([P1] s7.3: represent
+ * gradients in low precision to cut the communication volume): every value
+ * that crosses a link -- each partial a reduce-scatter step sends, and each
+ * finished chunk the all-gather sends -- is rounded to `wire` (RR_BF16, round
+ * to nearest even), while every rank folds in fp32.  Element i of chunk c
+ * gives acc = x_c; acc = bf16(acc) op x_{c+j} for j = 1..N-1; result =
+ * bf16(acc, divided by N for AVG), the same value on every rank.  op: SUM or
+ * AVG.  algo: RING (the 2(N-1)-step schedule with bf16 transfers) or
+ * ONESHOT / AUTO (one launch, the same bits).  Error against the exact
+ * reduction: at most about N * 2^-8 * sum |x|.  On one GPU the buffers stay
+ * fp32 in HBM, so the HBM traffic is that of the fp32 call; the bytes counted
+ * as sent (rr_get_stats) are the bf16 ones.  nranks == 1 sends nothing and
+ * leaves the buffer unchanged. */
+rr_status_t rr_allreduce_wire(void* const* bufs, int nranks, size_t count, rr_op_t op, rr_dtype_t wire,
+                              rr_algo_t algo, cudaStream_t stream);
+
 /* All-reduce of HOST buffers through caller-provided device buffers: copies
  * host_bufs[r] -> dev_bufs[r], reduces dev_bufs as rr_allreduce does, and
  * copies the result back into every host_bufs[r]; dev_bufs hold the result

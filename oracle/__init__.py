@@ -70,6 +70,8 @@ def _load(mutant: bool = False) -> ctypes.CDLL:
         lib.orc_ring_allreduce.argtypes = [PP, i32, sz, i32, i32, ctypes.POINTER(Event), P]
         lib.orc_ring_allreduce_omp.argtypes = [PP, i32, sz, i32, i32, i32]
         lib.orc_fold_ring_order.argtypes = [PP, i32, sz, i32, i32]
+        lib.orc_ring_allreduce_wire.argtypes = [PP, i32, sz, i32]
+        lib.orc_fold_wire.argtypes = [PP, i32, sz, i32]
         lib.orc_double_ring_step.argtypes = [PP, i32, sz, i32, i32, i32, i32, P]
         lib.orc_double_ring_allreduce.argtypes = [PP, i32, sz, i32, i32, P]
         lib.orc_fold_double_ring.argtypes = [PP, i32, sz, i32, i32]
@@ -216,6 +218,24 @@ def ring_allreduce_omp(bufs, op="sum", nthreads: int = 0) -> None:
     timed CPU baseline); same arithmetic as ``ring_allreduce``."""
     d, count = _same(bufs)
     _check(_lib().orc_ring_allreduce_omp(_ptrs(bufs), len(bufs), count, d, _op(op), nthreads), "ring_omp")
+
+
+def ring_allreduce_wire(bufs, op="sum") -> None:
+    """The ring all-reduce of fp32 buffers with every transfer rounded to
+    bf16 and fp32 folds, in place ([P1] s7.3: low-precision gradients on the
+    wire)."""
+    d, count = _same(bufs)
+    if d != F32:
+        raise TypeError("the bf16 wire carries fp32 buffers")
+    _check(_lib().orc_ring_allreduce_wire(_ptrs(bufs), len(bufs), count, _op(op)), "ring wire")
+
+
+def fold_wire(bufs, op="sum") -> None:
+    """The bf16-wire all-reduce by definition (its fused one-shot form)."""
+    d, count = _same(bufs)
+    if d != F32:
+        raise TypeError("the bf16 wire carries fp32 buffers")
+    _check(_lib().orc_fold_wire(_ptrs(bufs), len(bufs), count, _op(op)), "fold wire")
 
 
 def double_ring_allreduce(bufs, op="sum"):

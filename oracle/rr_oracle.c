@@ -348,6 +348,81 @@ int orc_ring_allreduce_omp(void** bufs, int n, size_t count, int dtype, int op, 
     return ORC_OK;
 }
 
+/* ------------------------------------------------ bf16 wire (compressed) -- */
+
+/* A wire value: what arrives after a transfer in the bf16 wire format. */
+static float wire_bf16(float v)
+{
+    if (MUTANT(11)) return v;
+    return orc_bf16_to_f32(orc_f32_to_bf16(v));
+}
+
+/* The ring all-reduce of fp32 buffers with a low-precision wire ([P1] s7.3:
+ * represent gradients in low precision to cut the communication volume):
+ * every chunk that crosses a link is rounded to bf16, while each rank folds in
+ * fp32.  Reduce-scatter step s: rank r folds the bf16 image of the partial it
+ * receives into its own fp32 copy (received partial on the left); in the last
+ * step the owner applies AVG's division and keeps the bf16 image of the
+ * result, which is what the all-gather then sends, so every rank ends with
+ * the same values.  fp32 buffers, SUM or AVG. */
+int orc_ring_allreduce_wire(void** bufs, int n, size_t count, int op)
+{
+    if (n < 1 || (op != ORC_SUM && op != ORC_AVG)) return ORC_EINVAL;
+    size_t C = orc_chunk_size(count, n);
+    float* msg = (float*)malloc((size_t)n * (C ? C : 1) * sizeof(float));
+    if (!msg) return ORC_ENOMEM;
+    for (int phase = ORC_PHASE_RS; phase <= ORC_PHASE_AG; ++phase) {
+        for (int s = 0; s < n - 1; ++s) {
+            for (int r = 0; r < n; ++r) { /* every rank sends one chunk through the wire */
+                int k = send_chunk(phase, r, s, n);
+                size_t len = orc_chunk_len(count, n, k);
+                for (size_t j = 0; j < len; ++j) {
+                    float v = ((float*)bufs[r])[(size_t)k * C + j];
+                    msg[(size_t)r * C + j] = phase == ORC_PHASE_RS ? wire_bf16(v) : v;
+                }
+            }
+            for (int r = 0; r < n; ++r) {
+                int left = mod(r - 1, n);
+                int k = send_chunk(phase, left, s, n);
+                size_t len = orc_chunk_len(count, n, k);
+                float* own = (float*)bufs[r] + (size_t)k * C;
+                for (size_t j = 0; j < len; ++j) {
+                    float got = msg[(size_t)left * C + j];
+                    if (phase == ORC_PHASE_AG) {
+                        own[j] = got; /* already a bf16 image */
+                    } else {
+                        float v = op_f32(op, got, own[j]);
+                        if (s == n - 2) v = wire_bf16(finish_f32(op, v, n));
+                        own[j] = v;
+                    }
+                }
+            }
+        }
+    }
+    free(msg);
+    return ORC_OK;
+}
+
+/* Its result as a definition: element i of chunk c folds
+ * acc = x_c; acc = bf16(acc) op x_{c+j} for j = 1..N-1 (the partial is
+ * rounded as it is sent, the local value is not), then AVG's division and one
+ * last bf16 rounding for the value the all-gather sends.  N = 1 sends
+ * nothing and leaves the buffer unchanged. */
+int orc_fold_wire(void** bufs, int n, size_t count, int op)
+{
+    if (n < 1 || (op != ORC_SUM && op != ORC_AVG)) return ORC_EINVAL;
+    if (n == 1) return ORC_OK;
+    size_t C = orc_chunk_size(count, n);
+    for (size_t i = 0; i < count; ++i) {
+        int c = (int)(i / C);
+        float acc = ((float*)bufs[c])[i];
+        for (int j = 1; j < n; ++j) acc = op_f32(op, wire_bf16(acc), ((float*)bufs[mod(c + j, n)])[i]);
+        acc = wire_bf16(finish_f32(op, acc, n));
+        for (int r = 0; r < n; ++r) ((float*)bufs[r])[i] = acc;
+    }
+    return ORC_OK;
+}
+
 /* ---------------------------------------------------------- double ring -- */
 
 /* The double ring ([P3] section 6: two rings running in opposite directions

@@ -20,7 +20,7 @@ from typing import Sequence
 from ._lib import MAX_RANKS, Cost, RingEvent, RRError, Stats, check, lib
 
 __all__ = [
-    "all_reduce", "all_reduce_host", "ring_step", "ring_schedule", "reduce_scatter", "all_gather", "all_to_all",
+    "all_reduce", "all_reduce_wire", "all_reduce_host", "ring_step", "ring_schedule", "reduce_scatter", "all_gather", "all_to_all",
     "BucketPlan", "GradSet", "Reducer", "cost_model", "pick_algo", "set_picker_params", "last_stats", "RRError",
     "OPS", "ALGOS", "MAX_RANKS",
 ]
@@ -86,6 +86,14 @@ def all_reduce(tensors: Sequence, op="sum", algo="auto", stream=None) -> None:
     count, d, dev = _ranks(tensors, "all_reduce")
     check(lib().rr_allreduce(_ptr_array(tensors), len(tensors), count, d, _op(op), _algo(algo),
                              _stream(stream, dev)), "all_reduce")
+
+
+def all_reduce_wire(tensors: Sequence, op="sum", wire="bf16", algo="auto", stream=None) -> None:
+    """In-place all-reduce of fp32 rank tensors whose transfers are rounded
+    to the bf16 wire format while the folds stay fp32 (``rr_allreduce_wire``)."""
+    count, d, dev = _ranks(tensors, "all_reduce_wire")
+    check(lib().rr_allreduce_wire(_ptr_array(tensors), len(tensors), count, _op(op), _dtype_code(wire),
+                                  _algo(algo), _stream(stream, dev)), "all_reduce_wire")
 
 
 def all_reduce_host(host: Sequence, device: Sequence, op="sum", algo="auto", stream=None) -> None:

@@ -181,7 +181,7 @@ void stats_begin(int algo, int n, uint64_t S)
 
 // Build and launch one ring step (all ranks at once).
 rr_status_t ring_step_launch(void* const* bufs, int n, size_t count, rr_dtype_t dtype, rr_op_t op, int phase,
-                             int step, cudaStream_t stream)
+                             int step, cudaStream_t stream, bool wire = false)
 {
     const size_t es = esize(dtype);
     const uint64_t C = ceil_div(count, (uint64_t)n);
@@ -206,7 +206,11 @@ rr_status_t ring_step_launch(void* const* bufs, int n, size_t count, rr_dtype_t 
     int op_eff = op;
     if (op == RR_AVG && !(phase == RR_PHASE_REDUCE_SCATTER && step == n - 2)) op_eff = RR_SUM;
     if (maxlen == 0) return RR_OK;
-    cudaError_t e = launch_step(dtype, op_eff, p, stream);
+    cudaError_t e;
+    if (wire && p.nin == 2)  // a bf16-wire reduce-scatter step; the all-gather copies wire values
+        e = launch_step_wire(op_eff, step == n - 2 ? 1 : 2, p, stream);
+    else
+        e = launch_step(dtype, op_eff, p, stream);
     if (e != cudaSuccess) return cuda_fail(e, "ring step launch");
     t_stats.launches += 1;
     return RR_OK;
@@ -546,6 +550,57 @@ rr_status_t rr_allreduce(void* const* bufs, int nranks, size_t count, rr_dtype_t
     }
     log_call("allreduce", n, count, dtype, op, a);
     return st;
+}
+
+rr_status_t rr_allreduce_wire(void* const* bufs, int nranks, size_t count, rr_op_t op, rr_dtype_t wire,
+                              rr_algo_t algo, cudaStream_t stream)
+{
+    rr_status_t st = check_basic(nranks, RR_F32, op);
+    if (st != RR_OK) return st;
+    if (op != RR_SUM && op != RR_AVG) return fail(RR_ERR_UNSUPPORTED, "the wire format carries SUM or AVG");
+    if (wire != RR_BF16) return fail(RR_ERR_UNSUPPORTED, "the wire format is bf16");
+    if (algo != RR_ALGO_AUTO && algo != RR_ALGO_ONESHOT && algo != RR_ALGO_RING)
+        return fail(RR_ERR_UNSUPPORTED, "the bf16 wire runs AUTO, ONESHOT or RING");
+    if (!bufs) return fail(RR_ERR_INVALID_ARG, "NULL bufs array");
+    const int n = nranks;
+    const rr_algo_t a = algo == RR_ALGO_RING ? RR_ALGO_RING : RR_ALGO_ONESHOT;
+    const uint64_t S = (uint64_t)count * 4;
+    stats_begin(a, n, S);
+    if (count == 0) return RR_OK;
+    std::vector<Span> spans;
+    for (int r = 0; r < n; ++r) spans.push_back({(uintptr_t)bufs[r], (uintptr_t)bufs[r] + S, true});
+    if ((st = check_spans(spans)) != RR_OK) return st;
+    if ((st = check_device_ptrs(bufs, n)) != RR_OK) return st;
+    if (n == 1) return RR_OK;  // nothing crosses a wire
+    if (a == RR_ALGO_RING) {
+        for (int phase = RR_PHASE_REDUCE_SCATTER; phase <= RR_PHASE_ALL_GATHER; ++phase)
+            for (int s = 0; s < n - 1; ++s)
+                if ((st = ring_step_launch(bufs, n, count, RR_F32, op, phase, s, stream, true)) != RR_OK) return st;
+        t_stats.steps = 2 * (n - 1);
+        t_stats.bytes_sent_max = 2ull * (n - 1) * ceil_div(count, (uint64_t)n) * 2;  // bf16 on the wire
+        t_stats.hbm_bytes = 5ull * (uint64_t)(n - 1) * S;
+    } else {
+        RankParams p{};
+        for (int r = 0; r < n; ++r) p.in[r] = p.out[r] = bufs[r];
+        p.n = n;
+        p.vec_ok = same_phase(bufs, n);
+        p.divisor = (float)n;
+        p.C = ceil_div(count, (uint64_t)n);
+        p.count = count;
+        p.nseg = (uint64_t)n;
+        p.tps = std::max<uint64_t>(1, ceil_div(p.C, tile_elems(RR_F32, kVptReduce)));
+        p.lo = 0;
+        p.hi = UINT64_MAX;
+        cudaError_t e = launch_oneshot_wire(op, p, p.nseg * p.tps, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "wire one-shot launch");
+        t_stats.launches = 1;
+        t_stats.steps = 1;
+        t_stats.bytes_sent_max = (uint64_t)(n - 1) * count * 2;  // each rank's values go out as bf16
+        t_stats.hbm_bytes = 2ull * n * S;
+    }
+    t_stats.bytes_sent_total = (uint64_t)n * t_stats.bytes_sent_max;
+    log_call("allreduce_wire", n, count, RR_F32, op, a);
+    return RR_OK;
 }
 
 rr_status_t rr_allreduce_host(void* const* host_bufs, void* const* dev_bufs, int nranks, size_t count,

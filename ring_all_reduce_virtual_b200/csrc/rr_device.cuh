@@ -163,6 +163,37 @@ __device__ __forceinline__ float finish_n(float a, float divisor)
 template <int OP, int NS>
 __device__ __forceinline__ int32_t finish_n(int32_t a, float) { return a; }
 
+// The bf16 wire format: a value as it arrives after crossing a link that
+// carries bf16 (round to nearest even, back to fp32 exactly).
+__device__ __forceinline__ float wire_q(float v)
+{
+    return __uint_as_float((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v)) << 16);
+}
+
+// WIRE modes of the folds: 0 exact transfers; 1 the partial is rounded to the
+// wire format before each fold step and the result before it is stored (it is
+// what the all-gather sends); 2 partials only (a reduce-scatter step that does
+// not complete its chunk).
+template <int WIRE>
+__device__ __forceinline__ float wire_in(float a)
+{
+    if constexpr (WIRE != 0) return wire_q(a);
+    else return a;
+}
+
+template <int WIRE>
+__device__ __forceinline__ int32_t wire_in(int32_t a) { return a; }
+
+template <int WIRE>
+__device__ __forceinline__ float wire_out(float a)
+{
+    if constexpr (WIRE == 1) return wire_q(a);
+    else return a;
+}
+
+template <int WIRE>
+__device__ __forceinline__ int32_t wire_out(int32_t a) { return a; }
+
 // ------------------------------------------------------------------ memory
 
 // 128-bit streaming access: every byte is touched once per call, so hint the
@@ -180,14 +211,14 @@ __device__ __forceinline__ int phase_of(const T* p, int L)
 // --------------------------------------------------------------- the tile
 
 // Scalar fold of element e of a segment.
-template <class Ty, int OP, class InF, class OutF>
+template <class Ty, int OP, int WIRE, class InF, class OutF>
 __device__ __forceinline__ void fold_one(const InF& in, int nin, const OutF& out, int nout, uint64_t e,
                                          float divisor)
 {
     using Acc = typename Ty::Acc;
     Acc acc = Ty::ld1(in(0) + e);
-    for (int j = 1; j < nin; ++j) acc = apply<OP>(acc, Ty::ld1(in(j) + e));
-    if (nin > 1) acc = finish<OP>(acc, divisor);
+    for (int j = 1; j < nin; ++j) acc = apply<OP>(wire_in<WIRE>(acc), Ty::ld1(in(j) + e));
+    if (nin > 1) acc = wire_out<WIRE>(finish<OP>(acc, divisor));
     for (int o = 0; o < nout; ++o) Ty::st1(out(o) + e, acc);
 }
 
@@ -195,7 +226,8 @@ __device__ __forceinline__ void fold_one(const InF& in, int nin, const OutF& out
 // elements.  VPT is the number of 16-byte vectors per thread per tile, G the
 // number of further input ranks whose loads are issued before they are
 // folded: every thread keeps up to VPT * (G + 1) loads in flight.  NS > 0 is
-// the rank count (AVG's divisor) when it is fixed at compile time.  in(j) /
+// the rank count (AVG's divisor) when it is fixed at compile time; WIRE
+// selects the bf16 wire format (see wire_in / wire_out).  in(j) /
 // out(o) return the segment's base pointers.  vec_ok says
 // that every in(j) has the same address modulo 16 as in(0), and every out(o)
 // the same as out(0) (checked by the host); when in(0) and out(0) also agree,
@@ -204,7 +236,7 @@ __device__ __forceinline__ void fold_one(const InF& in, int nin, const OutF& out
 // scalar.  Tile t covers body vectors [t*TV, (t+1)*TV), TV = kThreads*VPT, or
 // the same number of elements on the scalar path; tile 0 also does the head
 // and tail.
-template <class Ty, int OP, int VPT, int G, int NS = 0, class InF, class OutF>
+template <class Ty, int OP, int VPT, int G, int NS = 0, int WIRE = 0, class InF, class OutF>
 __device__ __forceinline__ void fold_tile(const InF& in, int nin, const OutF& out, int nout, uint64_t len,
                                           uint64_t tile, bool vec_ok, float divisor)
 {
@@ -220,7 +252,7 @@ __device__ __forceinline__ void fold_tile(const InF& in, int nin, const OutF& ou
 #pragma unroll 4
         for (int k = 0; k < VPT * L; ++k) {
             uint64_t e = e0 + (uint64_t)k * kThreads + tid;
-            if (e < len) fold_one<Ty, OP>(in, nin, out, nout, e, divisor);
+            if (e < len) fold_one<Ty, OP, WIRE>(in, nin, out, nout, e, divisor);
         }
         return;
     }
@@ -230,7 +262,7 @@ __device__ __forceinline__ void fold_tile(const InF& in, int nin, const OutF& ou
     const uint64_t tail = len - head - nv * L;
     if (tile == 0 && (uint64_t)tid < head + tail) {
         uint64_t e = (uint64_t)tid < head ? (uint64_t)tid : head + nv * L + ((uint64_t)tid - head);
-        fold_one<Ty, OP>(in, nin, out, nout, e, divisor);
+        fold_one<Ty, OP, WIRE>(in, nin, out, nout, e, divisor);
     }
     const uint64_t v0 = tile * TV;
     if (v0 >= nv) return;
@@ -283,7 +315,7 @@ __device__ __forceinline__ void fold_tile(const InF& in, int nin, const OutF& ou
                     Acc b[L];
                     Ty::unpack(raw[k][u], b);
 #pragma unroll
-                    for (int l = 0; l < L; ++l) a[u][l] = apply<OP>(a[u][l], b[l]);
+                    for (int l = 0; l < L; ++l) a[u][l] = apply<OP>(wire_in<WIRE>(a[u][l]), b[l]);
                 }
             }
         }
@@ -292,7 +324,7 @@ __device__ __forceinline__ void fold_tile(const InF& in, int nin, const OutF& ou
 #pragma unroll
     for (int u = 0; u < VPT; ++u) {
 #pragma unroll
-        for (int l = 0; l < L; ++l) a[u][l] = finish_n<OP, NS>(a[u][l], divisor);
+        for (int l = 0; l < L; ++l) a[u][l] = wire_out<WIRE>(finish_n<OP, NS>(a[u][l], divisor));
         res[u] = Ty::pack(a[u]);
     }
 #pragma unroll 4

@@ -127,6 +127,10 @@ constexpr uint64_t kMaxGrid = 0x7fffffffull;
 // Launchers: return the launch's cudaError_t.  `op` is an rr_op_t value.
 cudaError_t launch_rank_kernel(int kind, int dtype, int op, const RankParams& p, cudaStream_t s);
 cudaError_t launch_step(int dtype, int op, const StepParams& p, cudaStream_t s);
+// bf16 wire (fp32 buffers, SUM or AVG): the fused one-shot, and a reduce-scatter
+// step (wire 1: the step completes its chunks; 2: it does not).
+cudaError_t launch_oneshot_wire(int op, const RankParams& p, uint64_t work, cudaStream_t s);
+cudaError_t launch_step_wire(int op, int wire, const StepParams& p, cudaStream_t s);
 cudaError_t launch_bucket_pack(int grad_dtype, const BucketCopyParams& p, cudaStream_t s);
 cudaError_t launch_bucket_unpack(int grad_dtype, int op, const BucketCopyParams& p, cudaStream_t s);
 cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p, cudaStream_t s,

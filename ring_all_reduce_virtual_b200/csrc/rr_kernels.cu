@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(kThreads) all_to_all_kernel(const __grid_const
 // (nin == 2) or copies in0 to out (nin == 1).
 // NIN: 2 folds (a reduce-scatter step or reduce level), 1 copies (an
 // all-gather step or broadcast level); fixed at compile time.
-template <class Ty, int OP, int NIN>
+template <class Ty, int OP, int NIN, int WIRE = 0>
 __global__ void __launch_bounds__(kThreads) step_kernel(const __grid_constant__ StepParams p)
 {
     using T = typename Ty::T;
@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(kThreads) step_kernel(const __grid_constant__ 
         if (sg.len == 0) continue;
         auto in = [&](int j) { return static_cast<const T*>(j == 0 ? sg.in0 : sg.in1); };
         auto out = [&](int) { return static_cast<T*>(sg.out); };
-        fold_tile<Ty, OP, kVptMove, 1>(in, NIN, out, 1, sg.len, tile, p.vec_ok, p.divisor);
+        fold_tile<Ty, OP, kVptMove, 1, 0, WIRE>(in, NIN, out, 1, sg.len, tile, p.vec_ok, p.divisor);
     }
 }
 
@@ -144,6 +144,16 @@ cudaError_t launch_rank_kernel(int kind, int dtype, int op, const RankParams& p,
         }
         return cudaErrorInvalidValue;
     });
+}
+
+cudaError_t launch_step_wire(int op, int wire, const StepParams& p, cudaStream_t s)
+{
+    const uint64_t work = (uint64_t)p.nseg * p.tps;
+    if (wire == 1)
+        return op == kAvg ? launch_all(step_kernel<F32T, kAvg, 2, 1>, p, work, s)
+                          : launch_all(step_kernel<F32T, kSum, 2, 1>, p, work, s);
+    return op == kAvg ? launch_all(step_kernel<F32T, kAvg, 2, 2>, p, work, s)
+                      : launch_all(step_kernel<F32T, kSum, 2, 2>, p, work, s);
 }
 
 cudaError_t launch_step(int dtype, int op, const StepParams& p, cudaStream_t s)

@@ -15,7 +15,7 @@ namespace {
 // walks the ring (c, c+1, ..., c+N-1 mod N); the result goes to all N
 // buffers.  One launch replaces the ring's 2(N-1) steps with the same bits.
 // NS > 0: the rank count, fixed at compile time (p.n == NS); 0: runtime.
-template <class Ty, int OP, int VPT, int G, int NS>
+template <class Ty, int OP, int VPT, int G, int NS, int WIRE = 0>
 __global__ void __launch_bounds__(kThreads) oneshot_ring_kernel(const __grid_constant__ RankParams p)
 {
     using T = typename Ty::T;
@@ -36,7 +36,7 @@ __global__ void __launch_bounds__(kThreads) oneshot_ring_kernel(const __grid_con
             return static_cast<const T*>(p.in[r]) + lo;
         };
         auto out = [&](int o) { return static_cast<T*>(p.out[p.owner_only ? start : o]) + lo; };
-        fold_tile<Ty, OP, VPT, G, NS>(in, n, out, p.owner_only ? 1 : n, len, tile, p.vec_ok, p.divisor);
+        fold_tile<Ty, OP, VPT, G, NS, WIRE>(in, n, out, p.owner_only ? 1 : n, len, tile, p.vec_ok, p.divisor);
     }
 }
 
@@ -55,6 +55,13 @@ cudaError_t launch_oneshot_ring(const RankParams& p, uint64_t work, cudaStream_t
     case 16: return launch_all(oneshot_ring_kernel<Ty, OP, V, kGroup, 16>, p, work, s);
     }
     return launch_all(oneshot_ring_kernel<Ty, OP, V, kGroup, 0>, p, work, s);
+}
+
+// The bf16-wire one-shot (fp32 buffers, SUM or AVG, any rank count).
+cudaError_t launch_oneshot_wire(int op, const RankParams& p, uint64_t work, cudaStream_t s)
+{
+    if (op == kAvg) return launch_all(oneshot_ring_kernel<F32T, kAvg, kVptReduce, kGroup, 0, 1>, p, work, s);
+    return launch_all(oneshot_ring_kernel<F32T, kSum, kVptReduce, kGroup, 0, 1>, p, work, s);
 }
 
 #define RR_INSTANTIATE(TY, OP) \

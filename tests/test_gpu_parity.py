@@ -433,3 +433,27 @@ def test_reducer_refuses_an_incomplete_step():
     red.ready(1)
     red.ready(2)
     red.finish()
+
+
+# ------------------------------------------------------------- bf16 wire --
+
+@pytest.mark.parametrize("algo", ["ring", "oneshot", "auto"])
+@pytest.mark.parametrize("n", [1, 2, 3, 4, 5, 8, 16])
+@pytest.mark.parametrize("op", ["sum", "avg"])
+def test_allreduce_bf16_wire(algo, n, op):
+    for count in (1, 7, 3 * TILE["f32"] * n + 37):
+        x = synth.ranks(14, n, count, "uniform")
+        want = [a.copy() for a in x]
+        (oracle.ring_allreduce_wire if algo == "ring" else oracle.fold_wire)(want, op)
+        d = to_dev(x)
+        rrv.all_reduce_wire(d, op, "bf16", algo)
+        assert_bits_equal(to_host(d), want, f"wire {algo} n={n} count={count}")
+
+
+def test_bf16_wire_golden_on_gpu():
+    g = {ln.split(":")[0]: [float(v) for v in ln.split(":")[1].split()] for ln in golden_lines("bf16_wire.txt")}
+    for algo in ("ring", "oneshot"):
+        d = to_dev([np.array(g["inputs_rank0"], np.float32), np.array(g["inputs_rank1"], np.float32)])
+        rrv.all_reduce_wire(d, "sum", "bf16", algo)
+        for t in to_host(d):
+            assert t.tolist() == g["bf16_wire"]

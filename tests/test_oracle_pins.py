@@ -574,3 +574,60 @@ def test_double_ring_mutant_is_caught():
     with oracle.mutant(10):
         with pytest.raises(AssertionError):
             test_double_ring_brute_force_integer_data(4, "sum")
+
+
+# ------------------------------------------------------------- bf16 wire --
+
+def _wire_fixture():
+    g = {ln.split(":")[0]: _vals(ln) for ln in golden_lines("bf16_wire.txt")}
+    x = [np.array(g["inputs_rank0"], dtype=np.float32), np.array(g["inputs_rank1"], dtype=np.float32)]
+    return g, x
+
+
+def test_bf16_wire_golden():
+    g, x = _wire_fixture()
+    assert x[0][0] == 1 + 2.0 ** -10 and x[1][1] == 1 + 3 * 2.0 ** -9  # the fixture's values are exact
+    for f in (oracle.ring_allreduce_wire, oracle.fold_wire):
+        _, y = _wire_fixture()
+        f(y, "sum")
+        for r in range(2):
+            assert y[r].tolist() == g["bf16_wire"]
+    _, y = _wire_fixture()
+    oracle.ring_allreduce(y, "sum")  # the exact fp32 ring for contrast
+    assert y[0].tolist() == g["fp32_wire"]
+
+
+@pytest.mark.parametrize("n", [2, 3, 4, 8])
+def test_bf16_wire_is_lossless_on_small_integers(n):
+    # every partial is an integer below 256 in magnitude: exactly
+    # representable in bf16, so the wire changes nothing
+    rng = np.random.default_rng([n, 11])
+    x = [synth.cast(rng.integers(-20, 20, size=5 * n + 3), "f32") for _ in range(n)]
+    y = [a.copy() for a in x]
+    oracle.ring_allreduce_wire(x, "sum")
+    oracle.ring_allreduce(y, "sum")
+    for r in range(n):
+        assert np.array_equal(x[r], y[r])
+
+
+@pytest.mark.parametrize("n", [2, 4, 8, 16])
+@pytest.mark.parametrize("op", ["sum", "avg"])
+def test_bf16_wire_error_bound(n, op):
+    # N-1 partials and the result are each rounded once to bf16 (relative
+    # error <= 2^-8 each), every value bounded by sum |x|: the wire's error
+    # against the fp64 reduction is at most about N * 2^-8 * sum |x|
+    x = synth.ranks(12, n, 4000, "uniform")
+    a = np.stack(x).astype(np.float64)
+    exact, mag = a.sum(0), np.abs(a).sum(0)
+    if op == "avg":
+        exact, mag = exact / n, mag / n
+    oracle.ring_allreduce_wire(x, op)
+    err = np.abs(x[0].astype(np.float64) - exact)
+    assert np.all(err <= n * 2.0 ** -8 * mag * (1 + 1e-3) + 1e-30)
+    assert err.max() > 0  # and it is lossy on random data
+
+
+def test_bf16_wire_mutant_is_caught():
+    with oracle.mutant(11):
+        with pytest.raises(AssertionError):
+            test_bf16_wire_golden()
