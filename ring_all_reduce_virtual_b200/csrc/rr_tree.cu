@@ -18,21 +18,22 @@ namespace {
 // for the set bits of N are combined from the smallest upwards, each larger
 // (earlier) block on the left: exactly the level schedule in which a rank
 // without a partner carries its value up.
-template <class Ty, int OP, int W>
+template <class Ty, int OP, int W, int NMAX>
 __device__ __forceinline__ void tree_fold_lanes(const RankParams& p, uint64_t e0, bool vec)
 {
     using T = typename Ty::T;
     using Acc = typename Ty::Acc;
-    Acc slot[7][W];
+    constexpr int LV = NMAX <= 2 ? 2 : (NMAX <= 4 ? 3 : (NMAX <= 8 ? 4 : 7));  // log2(NMAX) + 1
+    Acc slot[LV][W];
     Acc cur[W];
     const int n = p.n;
 #pragma unroll
-    for (int g = 0; g < kMaxRanks; g += kGroup) {
+    for (int g = 0; g < NMAX; g += kGroup) {
         if (g < n) {
             Acc v[kGroup][W];
 #pragma unroll
             for (int k = 0; k < kGroup; ++k) {
-                if (g + k < n) {
+                if (g + k < n && g + k < NMAX) {
                     const T* src = static_cast<const T*>(p.in[g + k]) + e0;
                     if constexpr (W == Ty::L) {
                         if (vec) {
@@ -46,12 +47,12 @@ __device__ __forceinline__ void tree_fold_lanes(const RankParams& p, uint64_t e0
 #pragma unroll
             for (int k = 0; k < kGroup; ++k) {
                 const int j = g + k;
-                if (j < n) {
+                if (j < n && j < NMAX) {
 #pragma unroll
                     for (int l = 0; l < W; ++l) cur[l] = v[k][l];
                     int lvl = 0;
 #pragma unroll
-                    for (int b = 0; b < 6; ++b) {
+                    for (int b = 0; b < LV - 1; ++b) {
                         if (((j >> b) & 1) && lvl == b) {
 #pragma unroll
                             for (int l = 0; l < W; ++l) cur[l] = apply<OP>(slot[b][l], cur[l]);
@@ -59,7 +60,7 @@ __device__ __forceinline__ void tree_fold_lanes(const RankParams& p, uint64_t e0
                         }
                     }
 #pragma unroll
-                    for (int b = 0; b < 7; ++b)
+                    for (int b = 0; b < LV; ++b)
                         if (b == lvl)
 #pragma unroll
                             for (int l = 0; l < W; ++l) slot[b][l] = cur[l];
@@ -69,7 +70,7 @@ __device__ __forceinline__ void tree_fold_lanes(const RankParams& p, uint64_t e0
     }
     bool have = false;
 #pragma unroll
-    for (int b = 0; b < 7; ++b) {
+    for (int b = 0; b < LV; ++b) {
         if ((n >> b) & 1) {
 #pragma unroll
             for (int l = 0; l < W; ++l) cur[l] = have ? apply<OP>(slot[b][l], cur[l]) : slot[b][l];
@@ -177,20 +178,20 @@ __global__ void __launch_bounds__(kThreads) oneshot_tree_kernel(const __grid_con
         if (ph < 0) {
             for (int k = 0; k < (int)(TE / kThreads); ++k) {
                 const uint64_t e = tile * TE + (uint64_t)k * kThreads + tid;
-                if (e < p.count) tree_fold_lanes<Ty, OP, 1>(p, e, false);
+                if (e < p.count) tree_fold_lanes<Ty, OP, 1, NMAX>(p, e, false);
             }
             continue;
         }
         if (tile == 0 && (uint64_t)tid < head + (p.count - tail_lo)) {
             const uint64_t e = (uint64_t)tid < head ? (uint64_t)tid : tail_lo + ((uint64_t)tid - head);
-            tree_fold_lanes<Ty, OP, 1>(p, e, false);
+            tree_fold_lanes<Ty, OP, 1, NMAX>(p, e, false);
         }
         if constexpr (NMAX <= 8) {
             tree_vectors<Ty, OP, NMAX, VPT, EXACT>(p, tile * (TE / L), nv, head);
         } else {
             for (int u = 0; u < VPT; ++u) {
                 const uint64_t v = tile * (TE / L) + (uint64_t)u * kThreads + tid;
-                if (v < nv) tree_fold_lanes<Ty, OP, L>(p, head + v * L, true);
+                if (v < nv) tree_fold_lanes<Ty, OP, L, NMAX>(p, head + v * L, true);
             }
         }
     }
