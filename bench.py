@@ -616,10 +616,8 @@ def run_64_ranks(args):
 
     for op in ("sum", "max", "min"):
         emit(f"all_reduce {op}", *timed(lambda: rrv.all_reduce(x, op, "auto", stream)))
-    prod = [torch.rand(count, device=dev, generator=gen) * 0.02 + 0.99 for _ in range(4)]
-    for i in range(4):  # PROD inputs for the first ranks; the rest stay uniform[-1, 1)
-        x[i].copy_(prod[i])
-    del prod
+    for t in x:  # PROD inputs: uniform[0.99, 1.01) on every rank
+        t.uniform_(0.99, 1.01, generator=gen)
     emit("all_reduce prod", *timed(lambda: rrv.all_reduce(x, "prod", "auto", stream)))
     per = count // n
     rs = [torch.empty(per, device=dev) for _ in range(n)]
