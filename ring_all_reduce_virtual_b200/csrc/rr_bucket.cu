@@ -18,69 +18,89 @@ namespace {
 
 constexpr int kUnitsPerThread = 4;
 
+// Four elements of a gradient or bucket type as raw bits: one 16-byte vector
+// of fp32, or 8 bytes of bf16.  Pack and unpack move quads, so both sides of
+// a conversion are read and written with whole, contiguous warp accesses
+// (lane i touches quad i of the warp's run).
+template <class X>
+struct Quad;
+
+template <>
+struct Quad<F32T> {
+    using R = uint4;
+    __device__ static __forceinline__ R ld(const float* p) { return ldv(p); }
+    __device__ static __forceinline__ void st(float* p, const R& r) { stv(p, r); }
+    __device__ static __forceinline__ void to_f(const R& r, float (&a)[4]) { F32T::unpack(r, a); }
+    __device__ static __forceinline__ R from_f(const float (&a)[4]) { return F32T::pack(a); }
+};
+
+template <>
+struct Quad<BF16T> {
+    using R = uint2;
+    __device__ static __forceinline__ R ld(const uint16_t* p) { return __ldcs(reinterpret_cast<const uint2*>(p)); }
+    __device__ static __forceinline__ void st(uint16_t* p, const R& r) { __stcs(reinterpret_cast<uint2*>(p), r); }
+    __device__ static __forceinline__ void to_f(const R& r, float (&a)[4])
+    {
+        BF16T::unpack2(r.x, a[0], a[1]);
+        BF16T::unpack2(r.y, a[2], a[3]);
+    }
+    __device__ static __forceinline__ R from_f(const float (&a)[4])
+    {
+        return make_uint2(BF16T::pack2(a[0], a[1]), BF16T::pack2(a[2], a[3]));
+    }
+};
+
 // Convert one tile of a segment from In's element type to Out's, dividing by
-// `divisor` first when OP is AVG.  A unit is U elements, one 16-byte vector
-// of the narrower type; both sides must reach a 16-byte boundary after the
-// same scalar head, otherwise the whole segment is scalar.
+// `divisor` first when OP is AVG.  A tile is kThreads * Q quads, Q chosen so
+// that it covers kThreads * kUnitsPerThread 16-byte vectors of the narrower
+// type (bucket_tile_elems).  When src and dst reach a quad boundary after the
+// same scalar head, the body moves quads and tile 0 also does the head and
+// the tail (< 4 elements each); otherwise every element is scalar.
 template <class In, class Out, int OP>
 __device__ __forceinline__ void convert_tile(const typename In::T* src, typename Out::T* dst, uint64_t len,
                                              uint64_t tile, bool vec_ok, float divisor)
 {
-    constexpr int U = In::L > Out::L ? In::L : Out::L;
-    constexpr int NI = U / In::L, NO = U / Out::L;
-    constexpr uint64_t TU = (uint64_t)kThreads * kUnitsPerThread;
+    constexpr int LMAX = In::L > Out::L ? In::L : Out::L;
+    constexpr int Q = kUnitsPerThread * LMAX / 4;  // quads per thread per tile
+    constexpr uint64_t TQ = (uint64_t)kThreads * Q;
     const int tid = threadIdx.x;
-    const int ps = phase_of(src, In::L), pd = phase_of(dst, Out::L);
-    int h = In::L == U ? (U - ps) % U : (U - pd) % U;
-    const bool vec = vec_ok && ((ps + h) % In::L == 0) && ((pd + h) % Out::L == 0);
+    const int ps = phase_of(src, 4), pd = phase_of(dst, 4);
     auto one = [&](uint64_t e) { Out::st1(dst + e, finish<OP>((float)In::ld1(src + e), divisor)); };
-    if (!vec) {
-        const uint64_t e0 = tile * TU * U;
+    if (!(vec_ok && ps == pd)) {
+        const uint64_t e0 = tile * TQ * 4;
 #pragma unroll 4
-        for (int k = 0; k < kUnitsPerThread * U; ++k) {
+        for (int k = 0; k < Q * 4; ++k) {
             const uint64_t e = e0 + (uint64_t)k * kThreads + tid;
             if (e < len) one(e);
         }
         return;
     }
-    uint64_t head = (uint64_t)h;
+    uint64_t head = (uint64_t)((4 - ps) & 3);
     if (head > len) head = len;
-    const uint64_t nu = (len - head) / U;
-    const uint64_t tail = len - head - nu * U;
+    const uint64_t nq = (len - head) / 4;
+    const uint64_t tail = len - head - nq * 4;
     if (tile == 0 && (uint64_t)tid < head + tail)
-        one((uint64_t)tid < head ? (uint64_t)tid : head + nu * U + ((uint64_t)tid - head));
-    // all of this thread's loads first (kUnitsPerThread * NI in flight), then
-    // the conversions and stores
-    uint4 raw[kUnitsPerThread][NI];
-    uint64_t e[kUnitsPerThread];
-    bool ok[kUnitsPerThread];
+        one((uint64_t)tid < head ? (uint64_t)tid : head + nq * 4 + ((uint64_t)tid - head));
+    // all of this thread's loads first (Q in flight), then the conversions
+    // and stores
+    typename Quad<In>::R raw[Q];
+    uint64_t e[Q];
+    bool ok[Q];
 #pragma unroll
-    for (int k = 0; k < kUnitsPerThread; ++k) {
-        const uint64_t u = tile * TU + (uint64_t)k * kThreads + tid;
-        ok[k] = u < nu;
-        e[k] = head + u * U;
-#pragma unroll
-        for (int i = 0; i < NI; ++i)
-            if (ok[k]) raw[k][i] = ldv(src + e[k] + (uint64_t)i * In::L);
+    for (int k = 0; k < Q; ++k) {
+        const uint64_t q = tile * TQ + (uint64_t)k * kThreads + tid;
+        ok[k] = q < nq;
+        e[k] = head + q * 4;
+        if (ok[k]) raw[k] = Quad<In>::ld(src + e[k]);
     }
 #pragma unroll
-    for (int k = 0; k < kUnitsPerThread; ++k) {
+    for (int k = 0; k < Q; ++k) {
         if (!ok[k]) continue;
-        float a[U];
+        float a[4];
+        Quad<In>::to_f(raw[k], a);
 #pragma unroll
-        for (int i = 0; i < NI; ++i) {
-            typename In::Acc t[In::L];
-            In::unpack(raw[k][i], t);
-#pragma unroll
-            for (int l = 0; l < In::L; ++l) a[i * In::L + l] = finish<OP>((float)t[l], divisor);
-        }
-#pragma unroll
-        for (int i = 0; i < NO; ++i) {
-            typename Out::Acc t[Out::L];
-#pragma unroll
-            for (int l = 0; l < Out::L; ++l) t[l] = a[i * Out::L + l];
-            stv(dst + e[k] + (uint64_t)i * Out::L, Out::pack(t));
-        }
+        for (int l = 0; l < 4; ++l) a[l] = finish<OP>(a[l], divisor);
+        Quad<Out>::st(dst + e[k], Quad<Out>::from_f(a));
     }
 }
 
@@ -189,8 +209,8 @@ cudaError_t launch_fold(const BucketFoldParams& p, uint64_t work, cudaStream_t s
 
 }  // namespace
 
-// Elements one pack/unpack tile covers: kThreads * kUnitsPerThread units of
-// U elements (U = 8 for bf16 gradients, 4 for fp32).
+// Elements one pack/unpack tile covers: kThreads * kUnitsPerThread 16-byte
+// vectors of the gradient type (8 elements each for bf16, 4 for fp32).
 uint64_t bucket_tile_elems(int grad_dtype)
 {
     return (uint64_t)kThreads * kUnitsPerThread * (grad_dtype == kBF16 ? 8u : 4u);
