@@ -455,8 +455,9 @@ def time_extra(dev, stream, host, S, peak):
 def run_sweep(args):
     """Message-size sweep: 1 KiB .. 1 GiB per rank, N in {2, 4, 8, 16}, fp32
     SUM, every algorithm.  Per point: median per-call device time over 20
-    calls after 5 warm-ups, and for sizes up to 1 MiB the per-call time of a
-    CUDA graph holding 100 calls.  Points whose 2 N S bytes fit in L2 are
+    calls after 5 warm-ups, and for sizes up to 1 MiB the same through a
+    RankSet (pointers marshalled once) and the per-call time of a CUDA graph
+    holding 100 calls.  Points whose 2 N S bytes fit in L2 are
     flagged."""
     import torch
 
@@ -486,8 +487,19 @@ def run_sweep(args):
                         times.append((a, b))
                     stream.synchronize()
                     t = statistics.median(x.elapsed_time(y) for x, y in times) / 1e3
-                    graph_us = None
+                    graph_us = rankset_us = None
                     if nbytes <= 1 << 20:
+                        # the same per-call timing through a RankSet (marshalled once)
+                        rs = rrv.RankSet(bufs)
+                        times = []
+                        for _ in range(20):
+                            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                            a.record(stream)
+                            rrv.all_reduce(rs, "sum", algo, stream)
+                            b.record(stream)
+                            times.append((a, b))
+                        stream.synchronize()
+                        rankset_us = statistics.median(x.elapsed_time(y) for x, y in times) * 1e3
                         g = torch.cuda.CUDAGraph()
                         with torch.cuda.graph(g, stream=stream):
                             for _ in range(100):
@@ -505,7 +517,9 @@ def run_sweep(args):
                 algbw = nbytes / t / 1e9
                 print(json.dumps({
                     "workload": "size-sweep-f32-sum", "nranks_virtual": n, "bytes_per_rank": nbytes, "algo": algo,
-                    "latency_us": round(t * 1e6, 3), "graph_latency_us": None if graph_us is None else round(graph_us, 3),
+                    "latency_us": round(t * 1e6, 3),
+                    "rankset_latency_us": None if rankset_us is None else round(rankset_us, 3),
+                    "graph_latency_us": None if graph_us is None else round(graph_us, 3),
                     "algbw_gbs": round(algbw, 3), "busbw_gbs": round(algbw * 2 * (n - 1) / n, 3),
                     "hbm_gbs": round(st["hbm_bytes"] / t / 1e9, 1), "hbm_frac": round(st["hbm_bytes"] / t / 1e9 / peak, 4),
                     "launches": st["launches"], "l2_resident": 2 * n * nbytes <= 126 * 10**6}), flush=True)

@@ -21,7 +21,7 @@ from ._lib import MAX_RANKS, Cost, RingEvent, RRError, Stats, check, lib
 
 __all__ = [
     "all_reduce", "all_reduce_wire", "all_reduce_host", "ring_step", "ring_schedule", "reduce_scatter", "all_gather", "all_to_all",
-    "BucketPlan", "GradSet", "Reducer", "cost_model", "pick_algo", "set_picker_params", "last_stats", "RRError",
+    "RankSet", "BucketPlan", "GradSet", "Reducer", "cost_model", "pick_algo", "set_picker_params", "last_stats", "RRError",
     "OPS", "ALGOS", "MAX_RANKS",
 ]
 
@@ -65,6 +65,35 @@ def _ranks(tensors: Sequence, what: str):
     return t0.numel(), _dtype_code(t0.dtype), t0.device
 
 
+class RankSet:
+    """The N rank tensors of an all-reduce, checked and marshalled once.
+
+    ``all_reduce``, ``all_reduce_wire`` and ``ring_step`` accept either this
+    or a list of tensors.  A list is checked (CUDA, contiguous, same dtype,
+    size and device) and its pointers copied into a ctypes array on every
+    call, which costs several microseconds for 8 ranks -- as much as the
+    kernel of a small message.  A RankSet does that once: it keeps the tensors
+    alive and stays valid while they keep their storage (in-place updates are
+    fine; ``resize_`` or ``set_`` on a member is not)."""
+
+    def __init__(self, tensors: Sequence):
+        self.count, self.dtype, self.device = _ranks(tensors, "RankSet")
+        self.nranks = len(tensors)
+        self.ptrs = _ptr_array(tensors)
+        self.tensors = list(tensors)
+
+    def __len__(self) -> int:
+        return self.nranks
+
+
+def _rank_args(tensors, what: str):
+    """(pointer array, nranks, count, dtype code, device) of a list or a RankSet."""
+    if isinstance(tensors, RankSet):
+        return tensors.ptrs, tensors.nranks, tensors.count, tensors.dtype, tensors.device
+    count, d, dev = _ranks(tensors, what)
+    return _ptr_array(tensors), len(tensors), count, d, dev
+
+
 def _stream(stream, device):
     import torch
 
@@ -81,19 +110,21 @@ def _algo(algo) -> int:
     return ALGOS[algo] if isinstance(algo, str) else int(algo)
 
 
-def all_reduce(tensors: Sequence, op="sum", algo="auto", stream=None) -> None:
-    """In-place all-reduce over the rank tensors (``rr_allreduce``)."""
-    count, d, dev = _ranks(tensors, "all_reduce")
-    check(lib().rr_allreduce(_ptr_array(tensors), len(tensors), count, d, _op(op), _algo(algo),
-                             _stream(stream, dev)), "all_reduce")
+def all_reduce(tensors, op="sum", algo="auto", stream=None) -> None:
+    """In-place all-reduce over the rank tensors, a list or a ``RankSet``
+    (``rr_allreduce``)."""
+    ptrs, n, count, d, dev = _rank_args(tensors, "all_reduce")
+    check(lib().rr_allreduce(ptrs, n, count, d, _op(op), _algo(algo), _stream(stream, dev)), "all_reduce")
 
 
-def all_reduce_wire(tensors: Sequence, op="sum", wire="bf16", algo="auto", stream=None) -> None:
+def all_reduce_wire(tensors, op="sum", wire="bf16", algo="auto", stream=None) -> None:
     """In-place all-reduce of fp32 rank tensors whose transfers are rounded
     to the bf16 wire format while the folds stay fp32 (``rr_allreduce_wire``)."""
-    count, d, dev = _ranks(tensors, "all_reduce_wire")
-    check(lib().rr_allreduce_wire(_ptr_array(tensors), len(tensors), count, _op(op), _dtype_code(wire),
-                                  _algo(algo), _stream(stream, dev)), "all_reduce_wire")
+    ptrs, n, count, d, dev = _rank_args(tensors, "all_reduce_wire")
+    if d != _DTYPE_NAMES["f32"]:
+        raise TypeError("all_reduce_wire: the rank tensors must be float32 (the wire format is bf16)")
+    check(lib().rr_allreduce_wire(ptrs, n, count, _op(op), _dtype_code(wire), _algo(algo), _stream(stream, dev)),
+          "all_reduce_wire")
 
 
 def all_reduce_host(host: Sequence, device: Sequence, op="sum", algo="auto", stream=None) -> None:
@@ -111,12 +142,11 @@ def all_reduce_host(host: Sequence, device: Sequence, op="sum", algo="auto", str
                                   _algo(algo), _stream(stream, dev)), "all_reduce_host")
 
 
-def ring_step(tensors: Sequence, op, phase, step: int, stream=None) -> None:
+def ring_step(tensors, op, phase, step: int, stream=None) -> None:
     """One ring step for all ranks at once (``rr_ring_step``)."""
-    count, d, dev = _ranks(tensors, "ring_step")
+    ptrs, n, count, d, dev = _rank_args(tensors, "ring_step")
     ph = PHASES[phase] if isinstance(phase, str) else int(phase)
-    check(lib().rr_ring_step(_ptr_array(tensors), len(tensors), count, d, _op(op), ph, step,
-                             _stream(stream, dev)), "ring_step")
+    check(lib().rr_ring_step(ptrs, n, count, d, _op(op), ph, step, _stream(stream, dev)), "ring_step")
 
 
 def ring_schedule(nranks: int, count: int, dtype="f32") -> list[dict]:

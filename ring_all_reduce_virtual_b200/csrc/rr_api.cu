@@ -120,7 +120,8 @@ bool same_phase(const void* const* p, int n)
 // or managed memory, before any launch.
 rr_status_t check_device_ptrs(const void* const* p, int n)
 {
-    if (!env_flag("RR_DEBUG")) return RR_OK;
+    static const bool debug = env_flag("RR_DEBUG");  // read once: getenv scans the environment
+    if (!debug) return RR_OK;
     for (int i = 0; i < n; ++i) {
         cudaPointerAttributes a{};
         if (cudaPointerGetAttributes(&a, p[i]) != cudaSuccess ||

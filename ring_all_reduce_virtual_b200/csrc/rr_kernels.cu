@@ -17,23 +17,37 @@ namespace rr {
 namespace {
 
 
+// The one-to-many copies below give each CTA one tile of one output (16 KB
+// in, 16 KB out): such short-lived CTAs keep enough bytes in flight only at
+// full occupancy, so they are held to the registers of 8 CTAs per SM
+// (measured on the 64-rank all-gather: 6 CTAs per SM ran at 0.86 of the copy
+// peak, 8 at 1.03).  The all-to-all reads a separate tile per CTA and ran
+// slightly slower with the cap, so it keeps its registers.
+constexpr int kSmallCtasPerSm = 8;
+
 // ------------------------------------------------- chunk broadcast
-// Two-shot's second shot: segment c = chunk c, read once from its owner
-// (rank c) and written to chunk c of the N-1 other ranks.
+// Two-shot's second shot: segment c = chunk c, read from its owner (rank c)
+// and written to chunk c of the N-1 other ranks.  One output per work item:
+// item w = (c * tps + tile) * (N-1) + k writes rank k (k < c) or k+1, so the
+// N-1 CTAs of a tile run side by side and all but the first read the owner's
+// tile from L2 (HBM reads it once).
 template <class Ty>
-__global__ void __launch_bounds__(kThreads) chunk_bcast_kernel(const __grid_constant__ RankParams p)
+__global__ void __launch_bounds__(kThreads, kSmallCtasPerSm) chunk_bcast_kernel(const __grid_constant__ RankParams p)
 {
     using T = typename Ty::T;
-    const uint64_t total = p.nseg * p.tps;
+    const uint64_t m = (uint64_t)p.n - 1;
+    const uint64_t total = p.nseg * p.tps * m;
     for (uint64_t w = blockIdx.x; w < total; w += gridDim.x) {
-        const uint64_t c = w / p.tps, tile = w - c * p.tps;
+        const uint64_t st = w / m, k = w - st * m;
+        const uint64_t c = st / p.tps, tile = st - c * p.tps;
         const uint64_t lo = c * p.C;
         if (lo >= p.count) continue;
         const uint64_t len = p.count - lo < p.C ? p.count - lo : p.C;
         const int owner = (int)c;
+        const int dst = (int)k < owner ? (int)k : (int)k + 1;
         auto in = [&](int) { return static_cast<const T*>(p.in[owner]) + lo; };
-        auto out = [&](int o) { return static_cast<T*>(p.out[o < owner ? o : o + 1]) + lo; };
-        fold_tile<Ty, kSum, kVptMove, 1>(in, 1, out, p.n - 1, len, tile, p.vec_ok, 1.0f);
+        auto out = [&](int) { return static_cast<T*>(p.out[dst]) + lo; };
+        fold_tile<Ty, kSum, kVptMove, 1>(in, 1, out, 1, len, tile, p.vec_ok, 1.0f);
     }
 }
 
@@ -61,18 +75,23 @@ __global__ void __launch_bounds__(kThreads) reduce_scatter_kernel(const __grid_c
 }
 
 // ------------------------------------------------------ all-gather
-// Segment q = rank q's part: read once, written to offset q*C of every
-// output.
+// Segment q = rank q's part, written to offset q*C of every output.  One
+// output per work item: item w = (q * tps + tile) * N + o, so the N CTAs of
+// a tile run side by side and HBM reads the source tile once (the others hit
+// L2).  Writing all N outputs from one CTA measured 0.94 of the copy peak at
+// 8 ranks x 256 MiB, this map 0.99.
 template <class Ty>
-__global__ void __launch_bounds__(kThreads) all_gather_kernel(const __grid_constant__ RankParams p)
+__global__ void __launch_bounds__(kThreads, kSmallCtasPerSm) all_gather_kernel(const __grid_constant__ RankParams p)
 {
     using T = typename Ty::T;
-    const uint64_t total = p.nseg * p.tps;
+    const uint64_t n = (uint64_t)p.n;
+    const uint64_t total = p.nseg * p.tps * n;
     for (uint64_t w = blockIdx.x; w < total; w += gridDim.x) {
-        const uint64_t q = w / p.tps, tile = w - q * p.tps;
+        const uint64_t st = w / n, o = w - st * n;
+        const uint64_t q = st / p.tps, tile = st - q * p.tps;
         auto in = [&](int) { return static_cast<const T*>(p.in[q]); };
-        auto out = [&](int o) { return static_cast<T*>(p.out[o]) + q * p.C; };
-        fold_tile<Ty, kSum, kVptMove, 1>(in, 1, out, p.n, p.C, tile, p.vec_ok, 1.0f);
+        auto out = [&](int) { return static_cast<T*>(p.out[o]) + q * p.C; };
+        fold_tile<Ty, kSum, kVptMove, 1>(in, 1, out, 1, p.C, tile, p.vec_ok, 1.0f);
     }
 }
 
@@ -123,7 +142,9 @@ uint64_t tile_elems(int dtype, int vpt)
 
 cudaError_t launch_rank_kernel(int kind, int dtype, int op, const RankParams& p, cudaStream_t s)
 {
-    const uint64_t work = kind == kOneshotTree ? p.tps : p.nseg * p.tps;
+    uint64_t work = kind == kOneshotTree ? p.tps : p.nseg * p.tps;
+    if (kind == kAllGather) work *= (uint64_t)p.n;  // one output per work item
+    if (kind == kChunkBroadcast) work *= (uint64_t)(p.n - 1);
     if (kind == kAllGather || kind == kAllToAll || kind == kChunkBroadcast) op = kSum;
     const int n = p.n;
     constexpr int V = kVptReduce;

@@ -221,3 +221,15 @@ def test_trivial_calls_enqueue_nothing():
 def test_bucket_plan_rejects_bad_dtype():
     with pytest.raises(rrv.RRError):
         rrv.BucketPlan([1, 2, 3], "i32", 100)
+
+
+def test_rank_set_checks_its_tensors_once():
+    """RankSet applies the same checks as the list form, at construction."""
+    import torch
+
+    with pytest.raises(ValueError):
+        rrv.RankSet([])
+    with pytest.raises(ValueError):
+        rrv.RankSet([torch.zeros(4), torch.zeros(4)])  # not CUDA tensors
+    with pytest.raises(ValueError):
+        rrv.RankSet([torch.zeros(4)] * (rrv.MAX_RANKS + 1))

@@ -457,3 +457,52 @@ def test_bf16_wire_golden_on_gpu():
         rrv.all_reduce_wire(d, "sum", "bf16", algo)
         for t in to_host(d):
             assert t.tolist() == g["bf16_wire"]
+
+
+# ----------------------------------------------------- registered rank sets --
+
+@pytest.mark.parametrize("algo", ["oneshot", "ring", "tree_oneshot", "auto"])
+def test_rank_set_matches_the_oracle_across_reuse(algo):
+    """A RankSet is marshalled once and reused: each call still reduces the
+    tensors' current contents."""
+    n, count = 8, 3 * TILE["f32"] * 8 + 11
+    x = synth.ranks(21, n, count, "uniform")
+    d = to_dev(x)
+    rs = rrv.RankSet(d)
+    want = [a.copy() for a in x]
+    ORACLE[algo](want, "sum")
+    rrv.all_reduce(rs, "sum", algo)
+    assert_bits_equal(to_host(d), want, f"rank set {algo} first call")
+    y = synth.ranks(22, n, count, "uniform")
+    for t, a in zip(d, y):  # in place: same storage, new values
+        t.copy_(torch.from_numpy(a))
+    want = [a.copy() for a in y]
+    ORACLE[algo](want, "avg")
+    rrv.all_reduce(rs, "avg", algo)
+    assert_bits_equal(to_host(d), want, f"rank set {algo} reused")
+
+
+def test_rank_set_ring_steps_and_wire():
+    n, count = 4, 5000
+    x = synth.ranks(23, n, count, "uniform")
+    d = to_dev(x)
+    rs = rrv.RankSet(d)
+    for phase in ("reduce_scatter", "all_gather"):
+        for s in range(n - 1):
+            rrv.ring_step(rs, "sum", phase, s)
+    want = [a.copy() for a in x]
+    oracle.ring_allreduce(want, "sum")
+    assert_bits_equal(to_host(d), want, "rank set ring steps")
+    d = to_dev(x)
+    rrv.all_reduce_wire(rrv.RankSet(d), "sum", "bf16", "oneshot")
+    want = [a.copy() for a in x]
+    oracle.fold_wire(want, "sum")
+    assert_bits_equal(to_host(d), want, "rank set wire")
+
+
+def test_wire_refuses_non_fp32_tensors():
+    d = [torch.zeros(16, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    with pytest.raises(TypeError):
+        rrv.all_reduce_wire(d, "sum", "bf16", "oneshot")
+    with pytest.raises(TypeError):
+        rrv.all_reduce_wire(rrv.RankSet(d), "sum", "bf16", "oneshot")
