@@ -57,11 +57,24 @@ cudaError_t launch_oneshot_ring(const RankParams& p, uint64_t work, cudaStream_t
     return launch_all(oneshot_ring_kernel<Ty, OP, V, kGroup, 0>, p, work, s);
 }
 
-// The bf16-wire one-shot (fp32 buffers, SUM or AVG, any rank count).
+// The bf16-wire one-shot (fp32 buffers, SUM or AVG, any rank count; the
+// counts 2, 4, 8 and 16 fixed at compile time, as for the plain one-shot).
+template <int OP>
+cudaError_t launch_oneshot_wire_op(const RankParams& p, uint64_t work, cudaStream_t s)
+{
+    constexpr int V = kVptReduce;
+    switch (p.n) {
+    case 2: return launch_all(oneshot_ring_kernel<F32T, OP, V, 1, 2, 1>, p, work, s);
+    case 4: return launch_all(oneshot_ring_kernel<F32T, OP, V, 3, 4, 1>, p, work, s);
+    case 8: return launch_all(oneshot_ring_kernel<F32T, OP, V, 7, 8, 1>, p, work, s);
+    case 16: return launch_all(oneshot_ring_kernel<F32T, OP, V, kGroup, 16, 1>, p, work, s);
+    }
+    return launch_all(oneshot_ring_kernel<F32T, OP, V, kGroup, 0, 1>, p, work, s);
+}
+
 cudaError_t launch_oneshot_wire(int op, const RankParams& p, uint64_t work, cudaStream_t s)
 {
-    if (op == kAvg) return launch_all(oneshot_ring_kernel<F32T, kAvg, kVptReduce, kGroup, 0, 1>, p, work, s);
-    return launch_all(oneshot_ring_kernel<F32T, kSum, kVptReduce, kGroup, 0, 1>, p, work, s);
+    return op == kAvg ? launch_oneshot_wire_op<kAvg>(p, work, s) : launch_oneshot_wire_op<kSum>(p, work, s);
 }
 
 #define RR_INSTANTIATE(TY, OP) \
