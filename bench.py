@@ -531,8 +531,8 @@ def run_gpt_buckets(args):
     """Bucketed gradient sync of a GPT-like model (24 layers, d_model 2048,
     4x MLP, 32k vocab: 293 bf16 tensors, 1.34 B parameters per rank) over 8
     virtual ranks with 25 MiB buckets and AVG: the fused path (4 bytes per
-    parameter per rank) and the staged pack -> all-reduce -> unpack path (20
-    bytes).  Gradients are normal(0, 1e-3) drawn on the device (timing does
+    parameter per rank) one bucket per call and all buckets in one range call,
+    and the staged pack -> all-reduce -> unpack path (20 bytes).  Gradients are normal(0, 1e-3) drawn on the device (timing does
     not depend on the values)."""
     import torch
 
@@ -558,18 +558,27 @@ def run_gpt_buckets(args):
 
     views = [[t[:plan.info(b)[2]] for t in buckets] for b in range(nb)]
 
-    def fused():
-        for b in range(nb):
-            plan.all_reduce(b, gset, "avg", stream)
+    def launches(call):  # run one library call and return how many kernels it launched
+        call()
+        return rrv.last_stats()["launches"]
+
+    def fused():  # one fused sync per bucket, as each bucket becomes ready
+        return sum(launches(lambda: plan.all_reduce(b, gset, "avg", stream)) for b in range(nb))
+
+    def fused_range():  # every bucket at once: the buckets share launches
+        return launches(lambda: plan.all_reduce_range(0, nb, gset, "avg", stream))
 
     def staged():
+        k = 0
         for b in range(nb):
-            plan.pack(b, gset, buckets, stream)
-            rrv.all_reduce(views[b], "sum", "auto", stream)
-            plan.unpack(b, buckets, gset, "avg", stream)
+            k += launches(lambda: plan.pack(b, gset, buckets, stream))
+            k += launches(lambda: rrv.all_reduce(views[b], "sum", "auto", stream))
+            k += launches(lambda: plan.unpack(b, buckets, gset, "avg", stream))
+        return k
 
-    for name, fn, bpp in (("fused", fused, 4), ("staged", staged, 20)):
-        for _ in range(max(args.warmup, 3)):
+    for name, fn, bpp in (("fused", fused, 4), ("fused_range", fused_range, 4), ("staged", staged, 20)):
+        nl = fn()
+        for _ in range(max(args.warmup, 3) - 1):
             fn()
         torch.cuda.synchronize(dev)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -587,7 +596,7 @@ def run_gpt_buckets(args):
             "ms_per_sync": round(t * 1e3, 3), "grad_bytes_per_rank": params * 2,
             "algbw_gbs": round(params * 2 / t / 1e9, 2), "hbm_bytes_per_param_per_rank": bpp,
             "hbm_gbs": round(hbm / t / 1e9, 1), "hbm_frac": round(hbm / t / 1e9 / peak, 4),
-            "launches_per_sync": nb * (1 if name == "fused" else 3)}), flush=True)
+            "launches_per_sync": nl}), flush=True)
 
 
 def run_64_ranks(args):

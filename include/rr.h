@@ -278,6 +278,19 @@ rr_status_t rr_bucket_unpack(const rr_bucket_plan_t* plan, int bucket, const voi
 rr_status_t rr_bucket_allreduce(const rr_bucket_plan_t* plan, int bucket, void* const* grads,
                                 int nranks, rr_op_t op, cudaStream_t stream);
 
+/* Fused sync of buckets first_bucket .. first_bucket + nbuckets - 1 (a
+ * gradient sync when every bucket is ready at once, e.g. without overlap):
+ * the same bits as rr_bucket_allreduce on each bucket in turn -- every bucket
+ * is still chunked over its own flat index -- but the buckets share launches
+ * until a kernel parameter block is full (up to 384 tensors, 2048 gradient
+ * pointers and 448 segments per launch), so the range costs a few launches
+ * instead of one per bucket.  Same arguments and errors as
+ * rr_bucket_allreduce; the range must lie inside the plan (RR_ERR_INVALID_ARG
+ * otherwise) and every gradient it covers must be disjoint from the others.
+ * Statistics cover the whole range. */
+rr_status_t rr_bucket_allreduce_range(const rr_bucket_plan_t* plan, int first_bucket, int nbuckets,
+                                      void* const* grads, int nranks, rr_op_t op, cudaStream_t stream);
+
 /* ------------------------------------------------ overlapped bucket sync -- */
 
 /* Opaque reducer (host memory and CUDA events owned by the library). */

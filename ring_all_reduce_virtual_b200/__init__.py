@@ -288,6 +288,14 @@ class BucketPlan:
         check(lib().rr_bucket_allreduce(self._h, bucket, g, n, _op(op), _stream(stream, dev)),
               "bucket_allreduce")
 
+    def all_reduce_range(self, first: int, count: int, grads: Sequence[Sequence], op="avg", stream=None) -> None:
+        """Fused sync of buckets ``first .. first + count - 1`` in a few shared
+        launches, with the bits of ``all_reduce`` on each of them
+        (``rr_bucket_allreduce_range``)."""
+        g, n, dev = self._grads(grads)
+        check(lib().rr_bucket_allreduce_range(self._h, first, count, g, n, _op(op), _stream(stream, dev)),
+              "bucket_allreduce_range")
+
 
 class Reducer:
     """DDP-style overlapped bucket sync (``rr_reducer_*``): mark each

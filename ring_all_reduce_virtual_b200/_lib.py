@@ -70,6 +70,7 @@ def _declare(lib: ctypes.CDLL) -> None:
         "rr_bucket_pack": (st, [P, i, PP, PP, i, P]),
         "rr_bucket_unpack": (st, [P, i, PP, PP, i, i, P]),
         "rr_bucket_allreduce": (st, [P, i, PP, i, i, P]),
+        "rr_bucket_allreduce_range": (st, [P, i, i, PP, i, i, P]),
         "rr_reducer_create": (st, [P, PP, i, i, P, i, ctypes.POINTER(P)]),
         "rr_reducer_ready": (st, [P, i, P]),
         "rr_reducer_finish": (st, [P, P]),

@@ -905,15 +905,19 @@ rr_status_t rr_bucket_tensor(const rr_bucket_plan_t* plan, int tensor, int* buck
 namespace {
 
 // Checks shared by the bucket calls; fills the bucket's tensor range.
-rr_status_t bucket_check(const rr_bucket_plan_t* plan, int bucket, const void* const* grads, int nranks, int* t0,
-                         int* nt)
+// Checks buckets [b0, b0 + nb) of a plan and the gradients they cover (every
+// rank's copy of every tensor in the range, pairwise disjoint); *t0 and *nt
+// are the range's first tensor and tensor count.
+rr_status_t bucket_range_check(const rr_bucket_plan_t* plan, int b0, int nb, const void* const* grads, int nranks,
+                               int* t0, int* nt)
 {
     if (!plan) return fail(RR_ERR_INVALID_ARG, "NULL plan");
     if (nranks < 1 || nranks > RR_MAX_RANKS) return fail(RR_ERR_INVALID_ARG, "nranks must be in 1..64");
-    if (bucket < 0 || bucket >= (int)plan->first.size()) return fail(RR_ERR_INVALID_ARG, "bad bucket");
+    const int nbk = (int)plan->first.size();
+    if (b0 < 0 || nb < 1 || b0 >= nbk || nb > nbk - b0) return fail(RR_ERR_INVALID_ARG, "bad bucket");
     if (!grads) return fail(RR_ERR_INVALID_ARG, "NULL gradient array");
-    *t0 = plan->first[bucket];
-    *nt = plan->count[bucket];
+    *t0 = plan->first[b0];
+    *nt = plan->first[b0 + nb - 1] + plan->count[b0 + nb - 1] - *t0;
     const uint64_t es = esize((rr_dtype_t)plan->grad_dtype);
     std::vector<Span> spans;
     for (int r = 0; r < nranks; ++r)
@@ -923,6 +927,12 @@ rr_status_t bucket_check(const rr_bucket_plan_t* plan, int bucket, const void* c
             spans.push_back({(uintptr_t)g, (uintptr_t)g + plan->numel[t] * es, true});
         }
     return check_spans(spans);
+}
+
+rr_status_t bucket_check(const rr_bucket_plan_t* plan, int bucket, const void* const* grads, int nranks, int* t0,
+                         int* nt)
+{
+    return bucket_range_check(plan, bucket, 1, grads, nranks, t0, nt);
 }
 
 }  // namespace
@@ -996,30 +1006,42 @@ rr_status_t rr_bucket_unpack(const rr_bucket_plan_t* plan, int bucket, const voi
     return bucket_copy(plan, bucket, grads, const_cast<void* const*>(buckets), nranks, op, false, stream);
 }
 
-static rr_status_t bucket_allreduce_capped(const rr_bucket_plan_t* plan, int bucket, void* const* grads,
-                                           int nranks, rr_op_t op, cudaStream_t stream, uint64_t max_grid);
+static rr_status_t bucket_fold_range(const rr_bucket_plan_t* plan, int b0, int nb, void* const* grads, int nranks,
+                                     rr_op_t op, cudaStream_t stream, uint64_t max_grid);
 
 rr_status_t rr_bucket_allreduce(const rr_bucket_plan_t* plan, int bucket, void* const* grads, int nranks,
                                 rr_op_t op, cudaStream_t stream)
 {
-    return bucket_allreduce_capped(plan, bucket, grads, nranks, op, stream, kMaxGrid);
+    return bucket_fold_range(plan, bucket, 1, grads, nranks, op, stream, kMaxGrid);
+}
+
+rr_status_t rr_bucket_allreduce_range(const rr_bucket_plan_t* plan, int first_bucket, int nbuckets, void* const* grads,
+                                      int nranks, rr_op_t op, cudaStream_t stream)
+{
+    return bucket_fold_range(plan, first_bucket, nbuckets, grads, nranks, op, stream, kMaxGrid);
 }
 
 }  // extern "C"
 
-static rr_status_t bucket_allreduce_capped(const rr_bucket_plan_t* plan, int bucket, void* const* grads,
-                                           int nranks, rr_op_t op, cudaStream_t stream, uint64_t max_grid)
+// The fused sync of buckets [b0, b0 + nb): every bucket is chunked over its
+// own flat index (chunk size ceil(bucket numel / N)) exactly as a sync of
+// that bucket alone, and its tensors are split at its chunk boundaries into
+// segments (tensor, chunk); segments of consecutive buckets share a launch
+// until the parameter block is full, so a range costs a few launches instead
+// of one per bucket, with the same bits.
+static rr_status_t bucket_fold_range(const rr_bucket_plan_t* plan, int b0, int nb, void* const* grads, int nranks,
+                                     rr_op_t op, cudaStream_t stream, uint64_t max_grid)
 {
     if (op != RR_SUM && op != RR_AVG) return fail(RR_ERR_UNSUPPORTED, "bucket all-reduce takes SUM or AVG");
     int t0 = 0, nt = 0;
-    rr_status_t st = bucket_check(plan, bucket, grads, nranks, &t0, &nt);
+    rr_status_t st = bucket_range_check(plan, b0, nb, grads, nranks, &t0, &nt);
     if (st != RR_OK) return st;
     const int n = nranks;
     const uint64_t es = esize((rr_dtype_t)plan->grad_dtype);
-    const uint64_t total = plan->bnumel[bucket];
+    uint64_t total = 0;
+    for (int b = b0; b < b0 + nb; ++b) total += plan->bnumel[b];
     stats_begin(RR_ALGO_ONESHOT, n, total * es);
     if (n == 1 || total == 0) return RR_OK;
-    const uint64_t C = ceil_div(total, (uint64_t)n);  // the bucket's chunk size
     auto* p = new BucketFoldParams();
     auto flush = [&](int ntens) -> rr_status_t {
         if (p->nseg == 0) return RR_OK;
@@ -1038,21 +1060,24 @@ static rr_status_t bucket_allreduce_capped(const rr_bucket_plan_t* plan, int buc
     };
     int lt = 0;  // tensors in the current launch
     *p = BucketFoldParams{};
-    for (int t = t0; t < t0 + nt && st == RR_OK; ++t) {
-        const uint64_t lo = plan->offset[t], hi = lo + plan->numel[t];
-        const int nsegs_t = hi > lo ? (int)((hi - 1) / C - lo / C + 1) : 0;
-        if (lt + 1 > kMaxBucketTensors || (lt + 1) * n > kMaxBucketPtrs || p->nseg + nsegs_t > kMaxBucketSegs) {
-            st = flush(lt);
-            *p = BucketFoldParams{};
-            lt = 0;
+    for (int b = b0; b < b0 + nb && st == RR_OK; ++b) {
+        const uint64_t C = ceil_div(plan->bnumel[b], (uint64_t)n);  // this bucket's chunk size
+        for (int t = plan->first[b]; t < plan->first[b] + plan->count[b] && st == RR_OK; ++t) {
+            const uint64_t lo = plan->offset[t], hi = lo + plan->numel[t];  // offsets are bucket-relative
+            const int nsegs_t = hi > lo ? (int)((hi - 1) / C - lo / C + 1) : 0;
+            if (lt + 1 > kMaxBucketTensors || (lt + 1) * n > kMaxBucketPtrs || p->nseg + nsegs_t > kMaxBucketSegs) {
+                st = flush(lt);
+                *p = BucketFoldParams{};
+                lt = 0;
+            }
+            for (int r = 0; r < n; ++r) p->grad[lt * n + r] = grads[(size_t)r * plan->ntensors + t];
+            for (uint64_t pos = lo; pos < hi;) {  // split the tensor at the bucket's chunk boundaries
+                const uint64_t c = pos / C, end = std::min(hi, (c + 1) * C);
+                p->seg[p->nseg++] = BucketSeg{(uint32_t)lt, (uint32_t)c, pos - lo, end - pos};
+                pos = end;
+            }
+            ++lt;
         }
-        for (int r = 0; r < n; ++r) p->grad[lt * n + r] = grads[(size_t)r * plan->ntensors + t];
-        for (uint64_t pos = lo; pos < hi;) {  // split the tensor at the bucket's chunk boundaries
-            const uint64_t c = pos / C, end = std::min(hi, (c + 1) * C);
-            p->seg[p->nseg++] = BucketSeg{(uint32_t)lt, (uint32_t)c, pos - lo, end - pos};
-            pos = end;
-        }
-        ++lt;
     }
     if (st == RR_OK) st = flush(lt);
     delete p;
@@ -1144,7 +1169,7 @@ rr_status_t rr_reducer_ready(rr_reducer_t* red, int tensor, cudaStream_t produce
     cudaError_t e = cudaEventRecord(red->ready[b], producer);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(red->comm, red->ready[b], 0);
     if (e != cudaSuccess) return cuda_fail(e, "ordering the bucket sync after its gradients");
-    return bucket_allreduce_capped(red->plan, b, red->grads.data(), red->n, red->op, red->comm, red->max_grid);
+    return bucket_fold_range(red->plan, b, 1, red->grads.data(), red->n, red->op, red->comm, red->max_grid);
 }
 
 rr_status_t rr_reducer_finish(rr_reducer_t* red, cudaStream_t stream)

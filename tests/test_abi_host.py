@@ -233,3 +233,22 @@ def test_rank_set_checks_its_tensors_once():
         rrv.RankSet([torch.zeros(4), torch.zeros(4)])  # not CUDA tensors
     with pytest.raises(ValueError):
         rrv.RankSet([torch.zeros(4)] * (rrv.MAX_RANKS + 1))
+
+
+def test_bucket_range_argument_errors():
+    """rr_bucket_allreduce_range checks the range and the gradients before any
+    launch; a single rank or empty buckets enqueue nothing."""
+    lib = _lib.lib()
+    s = ctypes.c_void_p(0)
+    plan = rrv.BucketPlan([10, 20, 30, 40], "bf16", 60)  # buckets [10, 20] (60 B), [30], [40]
+    assert plan.num_buckets == 3
+    grads = _fake(8, stride=1 << 20)  # 2 ranks x 4 tensors, disjoint
+    for first, count in ((-1, 1), (0, 0), (0, 4), (3, 1), (2, 2)):
+        assert lib.rr_bucket_allreduce_range(plan._h, first, count, grads, 2, 1, s) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_bucket_allreduce_range(plan._h, 0, 3, grads, 2, 2, s) == _lib.RR_ERR_UNSUPPORTED  # MAX
+    assert lib.rr_bucket_allreduce_range(None, 0, 1, grads, 2, 1, s) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_bucket_allreduce_range(plan._h, 0, 2, None, 2, 1, s) == _lib.RR_ERR_INVALID_ARG
+    repeated = _fake(8, stride=0)
+    assert lib.rr_bucket_allreduce_range(plan._h, 0, 3, repeated, 2, 1, s) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_bucket_allreduce_range(plan._h, 0, 3, grads, 1, 1, s) == 0  # one rank: identity
+    assert rrv.last_stats()["launches"] == 0

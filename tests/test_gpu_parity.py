@@ -292,6 +292,42 @@ def test_bucket_staged_and_fused_match_the_oracle(dtype, op):
         assert_bits_equal(to_host(grads[r]), want[r], f"fused rank {r}")
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("op", ["avg", "sum"])
+def test_bucket_range_matches_per_bucket_syncs(dtype, op):
+    """A bucket range shares launches but keeps every bucket's own chunking:
+    the whole plan at once, and a sub-range that leaves the other buckets
+    alone.  300 tensors x 8 ranks (2400 gradient pointers) need more than one
+    launch."""
+    n = 8
+    rng = np.random.default_rng(31)
+    numels = [int(v) for v in rng.integers(0, 3000, size=300)]
+    numels[7] = 70001  # one tensor larger than the cap: a bucket of its own
+    cap = 3000 * (2 if dtype == "bf16" else 4)
+    host = _grad_set(12, n, numels, dtype)
+    want = [[g.copy() for g in rank] for rank in host]
+    oracle.bucket_sync(want, cap, op)
+    plan = rrv.BucketPlan(numels, dtype, cap)
+    nb = plan.num_buckets
+    assert nb > 50
+    grads = [to_dev(rank) for rank in host]
+    plan.all_reduce_range(0, nb, grads, op)
+    st = rrv.last_stats()
+    assert 1 < st["launches"] < nb
+    for r in range(n):
+        assert_bits_equal(to_host(grads[r]), want[r], f"range rank {r}")
+    # buckets 3 .. nb-4 only: their tensors reduced, the rest untouched
+    first, last = 3, nb - 4
+    t_lo = plan.info(first)[0]
+    t_hi = plan.info(last)[0] + plan.info(last)[1]
+    grads = [to_dev(rank) for rank in host]
+    plan.all_reduce_range(first, last - first + 1, grads, op)
+    for r in range(n):
+        got = to_host(grads[r])
+        exp = [want[r][t] if t_lo <= t < t_hi else host[r][t] for t in range(len(numels))]
+        assert_bits_equal(got, exp, f"sub-range rank {r}")
+
+
 def test_bucket_fused_misaligned_tensors():
     # tensors carved out of one flat allocation at odd element offsets
     n = 4
