@@ -129,7 +129,7 @@ def _bucket_expect(host, numels, plan, b, pos, n):
     return oracle.f32_to_bf16(f), tens, starts
 
 
-@pytest.mark.parametrize("path", ["fused", "staged"])
+@pytest.mark.parametrize("path", ["fused", "fused_range", "staged"])
 def test_gpt_like_bucketed_sync(gpt_grads, path):
     """293 bf16 gradient tensors (1.34 B parameters per rank), 8 ranks, 25 MiB
     buckets in gradient-ready order, AVG with fp32 accumulation: sampled
@@ -142,6 +142,9 @@ def test_gpt_like_bucketed_sync(gpt_grads, path):
     if path == "fused":
         for b in range(plan.num_buckets):
             plan.all_reduce(b, grads, "avg")
+    elif path == "fused_range":
+        plan.all_reduce_range(0, plan.num_buckets, grads, "avg")
+        assert rrv.last_stats()["launches"] < plan.num_buckets
     else:
         biggest = max(plan.info(b)[2] for b in range(plan.num_buckets))
         buckets = [torch.empty(biggest, dtype=torch.float32, device="cuda") for _ in range(n)]
