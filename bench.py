@@ -673,7 +673,11 @@ def run_kernels(args):
     per = count // n
     rs = [torch.empty(per, device=dev) for _ in range(n)]
     out = [torch.empty(count, device=dev) for _ in range(n)]
-    numels = [per // 3, per // 3, count - 2 * (per // 3)]  # three tensors: two small, one large
+    # three tensors, two small and one large, sized in multiples of 8 elements so
+    # every tensor's offset in the fp32 bucket has its gradient's 16-byte phase
+    # (a model's tensors usually do; mismatched phases take the scalar path)
+    small = (per // 3) & ~7
+    numels = [small, small, count - 2 * small]
     grads = rrv.GradSet([[(torch.randn(m, device=dev, generator=gen) * 1e-3).to(torch.bfloat16) for m in numels]
                          for _ in range(n)])
     plan = rrv.BucketPlan(numels, "bf16", 2 * count)  # one bucket

@@ -56,13 +56,11 @@ struct Quad<BF16T> {
 // type (bucket_tile_elems).  When src and dst reach a quad boundary after the
 // same scalar head, the body moves quads and tile 0 also does the head and
 // the tail (< 4 elements each); otherwise every element is scalar.
-template <class In, class Out, int OP>
+template <class In, class Out, int OP, int Q = kUnitsPerThread * (In::L > Out::L ? In::L : Out::L) / 4>
 __device__ __forceinline__ void convert_tile(const typename In::T* src, typename Out::T* dst, uint64_t len,
                                              uint64_t tile, bool vec_ok, float divisor)
 {
-    constexpr int LMAX = In::L > Out::L ? In::L : Out::L;
-    constexpr int Q = kUnitsPerThread * LMAX / 4;  // quads per thread per tile
-    constexpr uint64_t TQ = (uint64_t)kThreads * Q;
+    constexpr uint64_t TQ = (uint64_t)kThreads * Q;  // Q: quads per thread per tile
     const int tid = threadIdx.x;
     const int ps = phase_of(src, 4), pd = phase_of(dst, 4);
     auto one = [&](uint64_t e) { Out::st1(dst + e, finish<OP>((float)In::ld1(src + e), divisor)); };
