@@ -5,10 +5,11 @@ and the CPU-baseline leg of ``bench.py`` may import this package.  It shares
 no code with the CUDA library and never imports it.
 
 Buffers are numpy arrays, one per virtual rank: ``float32`` for fp32,
-``uint16`` bit patterns for bf16, ``int32`` for int32.  Functions that the C
-file defines "in place" modify the arrays given to them.  Each function's
-docstring names the passage of the pages it follows; the C file has the full
-statements and the readings taken where the pages are silent.
+``uint16`` bit patterns for bf16, ``float16`` for fp16, ``int32`` for int32.
+Functions that the C file defines "in place" modify the arrays given to them.
+Each function's docstring names the passage of the pages it follows; the C
+file has the full statements and the readings taken where the pages are
+silent.
 """
 from __future__ import annotations
 
@@ -21,7 +22,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
-F32, BF16, I32 = 0, 1, 2
+F32, BF16, I32, F16 = 0, 1, 2, 3
 SUM, AVG, MAX, MIN, PROD = 0, 1, 2, 3, 4
 PHASE_RS, PHASE_AG = 0, 1
 OPS = {"sum": SUM, "avg": AVG, "max": MAX, "min": MIN, "prod": PROD}
@@ -87,6 +88,8 @@ def _load(mutant: bool = False) -> ctypes.CDLL:
         lib.orc_bucket_unpack.argtypes = [PP, P, P, P, i32, i32, i32, P, i32, i32]
         lib.orc_f32_to_bf16_array.argtypes = [P, P, sz]
         lib.orc_bf16_to_f32_array.argtypes = [P, P, sz]
+        lib.orc_f32_to_f16_array.argtypes = [P, P, sz]
+        lib.orc_f16_to_f32_array.argtypes = [P, P, sz]
         lib.orc_chunk_size.argtypes = [sz, i32]
         lib.orc_chunk_size.restype = sz
         lib.orc_chunk_len.argtypes = [sz, i32, i32]
@@ -139,7 +142,9 @@ def dtype_code(a: np.ndarray) -> int:
         return BF16
     if a.dtype == np.int32:
         return I32
-    raise TypeError(f"oracle buffers are float32, uint16 (bf16 bits) or int32, not {a.dtype}")
+    if a.dtype == np.float16:
+        return F16
+    raise TypeError(f"oracle buffers are float32, uint16 (bf16 bits), float16 or int32, not {a.dtype}")
 
 
 def _op(op) -> int:
@@ -413,4 +418,25 @@ def bf16_to_f32(h: np.ndarray) -> np.ndarray:
     h = np.ascontiguousarray(h, dtype=np.uint16)
     out = np.empty(h.shape, dtype=np.float32)
     _lib().orc_bf16_to_f32_array(h.ctypes.data, out.ctypes.data, h.size)
+    return out
+
+
+# ------------------------------------------------------------------ fp16 --
+# fp16 rank buffers are numpy float16 arrays; the oracle reads and writes
+# their bit patterns with its own conversions (IEEE 754 binary16, round to
+# nearest even), not numpy's.
+
+def f32_to_f16(x: np.ndarray) -> np.ndarray:
+    """fp32 -> fp16 (as float16 whose bits the oracle computed), round to nearest even."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, dtype=np.uint16)
+    _lib().orc_f32_to_f16_array(x.ctypes.data, out.ctypes.data, x.size)
+    return out.view(np.float16)
+
+
+def f16_to_f32(h: np.ndarray) -> np.ndarray:
+    """fp16 -> fp32 (exact), by the oracle's own widening of the bit patterns."""
+    h = np.ascontiguousarray(h).view(np.uint16)
+    out = np.empty(h.shape, dtype=np.float32)
+    _lib().orc_f16_to_f32_array(h.ctypes.data, out.ctypes.data, h.size)
     return out

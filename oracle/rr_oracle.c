@@ -22,7 +22,7 @@
  * low-precision gradients as fp32 ([P1] s5.3); fp32 buffers are reduced in
  * fp32.  So every floating-point fold here is an fp32 fold, evaluated one
  * IEEE binary32 operation at a time (FLT_EVAL_METHOD == 0, no contraction, no
- * fast-math).  bf16 values are carried as their 16-bit patterns.
+ * fast-math).  bf16 and fp16 values are carried as their 16-bit patterns.
  *
  * Readings where the pages are silent (stated once, used everywhere):
  *   - chunk size C = ceil(count / N); chunk k is [k*C, min((k+1)*C, count)),
@@ -34,9 +34,10 @@
  *     (including +0 / -0) the left operand is kept.
  *   - AVG = the full fold, then one IEEE division by N ([P1] s2.1 "add, then
  *     divide by N"; [P3] section 3 "sum, then divide by 4").
- *   - bf16 buffers moved by the ring or tree schedules are rounded back to
- *     bf16 (round to nearest, ties to even) after every hop; the one-shot
- *     definitions fold the widened values in fp32 and round once at the end.
+ *   - bf16 (and fp16) buffers moved by the ring or tree schedules are rounded
+ *     back to their type (round to nearest, ties to even) after every hop;
+ *     the one-shot definitions fold the widened values in fp32 and round once
+ *     at the end.
  *   - int32 SUM and PROD wrap modulo 2^32; AVG is not defined for int32.
  */
 #include <float.h>
@@ -52,7 +53,7 @@
 #error "the oracle needs single-precision evaluation of float expressions"
 #endif
 
-enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_I32 = 2 };
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_I32 = 2, ORC_F16 = 3 };
 enum { ORC_SUM = 0, ORC_AVG = 1, ORC_MAX = 2, ORC_MIN = 3, ORC_PROD = 4 };
 enum { ORC_PHASE_RS = 0, ORC_PHASE_AG = 1 };
 enum { ORC_OK = 0, ORC_EINVAL = 1, ORC_ENOMEM = 2 };
@@ -118,14 +119,84 @@ void orc_bf16_to_f32_array(const uint16_t* in, float* out, size_t n)
     for (size_t i = 0; i < n; ++i) out[i] = orc_bf16_to_f32(in[i]);
 }
 
+/* ---------------------------------------------------------------- fp16 -- */
+
+/* IEEE 754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction
+ * bits.  Exponent field 0 holds zeros and subnormals (fraction * 2^-24), 31
+ * holds infinities and NaNs; every other field e is a normal number
+ * (1 + fraction / 2^10) * 2^(e - 15).  Every binary16 value is a binary32
+ * value, so widening is exact. */
+float orc_f16_to_f32(uint16_t h)
+{
+    const uint32_t sign = (uint32_t)(h >> 15) << 31;
+    const uint32_t e = (h >> 10) & 0x1fu, m = h & 0x3ffu;
+    uint32_t u;
+    if (e == 0) {  /* zero or subnormal: m * 2^-24, exact in binary32 */
+        float f = (float)m * 5.9604644775390625e-08f;
+        memcpy(&u, &f, sizeof u);
+        u |= sign;
+    } else if (e == 31) {
+        u = sign | 0x7f800000u | (m << 13) | (m ? 0x00400000u : 0u);  /* inf, or a quiet NaN */
+    } else {
+        u = sign | ((e - 15u + 127u) << 23) | (m << 13);
+    }
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* Round n / 2^shift to the nearest integer, ties to even (shift >= 1). */
+static uint32_t rne_shift(uint32_t n, int shift)
+{
+    if (shift > 31) return 0;
+    const uint32_t q = n >> shift, rem = n & ((1u << shift) - 1u), half = 1u << (shift - 1);
+    if (rem > half || (rem == half && (MUTANT(12) || (q & 1u)))) return q + 1u;
+    return q;
+}
+
+/* Narrow binary32 -> binary16 by round-to-nearest, ties-to-even.  A normal
+ * binary32 with unbiased exponent E >= -14 keeps the top 10 of its 23
+ * fraction bits, rounded on the 13 dropped ones; a carry out of the fraction
+ * moves into the exponent, and exponents past 15 (or a carry into 16) give
+ * infinity.  Below 2^-14 the result is the subnormal round(|f| / 2^-24);
+ * 1024 there is the smallest normal, 0x0400.  NaN stays a quiet NaN with its
+ * sign. */
+uint16_t orc_f32_to_f16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    const uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+    const uint32_t e32 = (u >> 23) & 0xffu, m32 = u & 0x7fffffu;
+    if (e32 == 0xffu) return (uint16_t)(sign | 0x7c00u | (m32 ? 0x0200u | (m32 >> 13) : 0u));
+    if (e32 == 0) return sign;  /* binary32 zero or subnormal: below half of 2^-24 */
+    const int E = (int)e32 - 127;
+    if (E > 15) return (uint16_t)(sign | 0x7c00u);
+    const uint32_t sig = m32 | 0x800000u;  /* 24-bit significand: |f| = sig * 2^(E - 23) */
+    if (E < -14)                           /* subnormal result: sig * 2^(E - 23) / 2^-24 */
+        return (uint16_t)(sign | rne_shift(sig, -1 - E));
+    uint32_t bits = ((uint32_t)(E + 15) << 10) + rne_shift(sig, 13) - 0x400u;  /* drop the hidden bit */
+    if (bits >= 0x7c00u) bits = 0x7c00u;
+    return (uint16_t)(sign | bits);
+}
+
+void orc_f32_to_f16_array(const float* in, uint16_t* out, size_t n)
+{
+    for (size_t i = 0; i < n; ++i) out[i] = orc_f32_to_f16(in[i]);
+}
+
+void orc_f16_to_f32_array(const uint16_t* in, float* out, size_t n)
+{
+    for (size_t i = 0; i < n; ++i) out[i] = orc_f16_to_f32(in[i]);
+}
+
 /* ------------------------------------------------------------- helpers -- */
 
-static size_t esize(int dtype) { return dtype == ORC_BF16 ? 2u : 4u; }
+static size_t esize(int dtype) { return dtype == ORC_BF16 || dtype == ORC_F16 ? 2u : 4u; }
 
 static int valid(int n, int dtype, int op)
 {
     if (n < 1) return 0;
-    if (dtype != ORC_F32 && dtype != ORC_BF16 && dtype != ORC_I32) return 0;
+    if (dtype != ORC_F32 && dtype != ORC_BF16 && dtype != ORC_I32 && dtype != ORC_F16) return 0;
     if (op < ORC_SUM || op > ORC_PROD) return 0;
     if (dtype == ORC_I32 && op == ORC_AVG) return 0;
     return 1;
@@ -175,6 +246,7 @@ static int32_t op_i32(int op, int32_t a, int32_t b)
 static float ld_f(const void* p, int dtype, size_t i)
 {
     if (dtype == ORC_BF16) return orc_bf16_to_f32(((const uint16_t*)p)[i]);
+    if (dtype == ORC_F16) return orc_f16_to_f32(((const uint16_t*)p)[i]);
     return ((const float*)p)[i];
 }
 
@@ -182,6 +254,8 @@ static void st_f(void* p, int dtype, size_t i, float v)
 {
     if (dtype == ORC_BF16)
         ((uint16_t*)p)[i] = orc_f32_to_bf16(v);
+    else if (dtype == ORC_F16)
+        ((uint16_t*)p)[i] = orc_f32_to_f16(v);
     else
         ((float*)p)[i] = v;
 }

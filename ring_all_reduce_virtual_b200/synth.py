@@ -33,7 +33,8 @@ def rank_values(seed: int, rank: int, count: int, dist: str = "uniform", dtype: 
         few ranks
       - ``arange``: ``arange(count) + 10 * rank`` (the 4-rank worked example)
       - ``pow2``: ``2 ** rank`` everywhere (shows which ranks were summed)
-    dtype: ``f32``, ``bf16`` (returned as uint16 bits) or ``i32``.
+    dtype: ``f32``, ``bf16`` (returned as uint16 bits), ``f16`` (float16) or
+      ``i32``.
     """
     key = [seed, rank] if stream is None else [seed, rank, stream]
     rng = np.random.default_rng(key)
@@ -55,7 +56,8 @@ def rank_values(seed: int, rank: int, count: int, dist: str = "uniform", dtype: 
 
 
 def cast(v: np.ndarray, dtype: str) -> np.ndarray:
-    """Cast drawn values to the buffer dtype (bf16 as uint16 bit patterns)."""
+    """Cast drawn values to the buffer dtype (bf16 as uint16 bit patterns,
+    fp16 as float16), rounding with PyTorch's CPU conversion."""
     if dtype == "f32":
         return np.ascontiguousarray(v, dtype=np.float32)
     if dtype == "i32":
@@ -65,6 +67,10 @@ def cast(v: np.ndarray, dtype: str) -> np.ndarray:
 
         t = torch.from_numpy(np.ascontiguousarray(v, dtype=np.float32)).to(torch.bfloat16)
         return t.view(torch.int16).numpy().view(np.uint16).copy()
+    if dtype == "f16":
+        import torch
+
+        return torch.from_numpy(np.ascontiguousarray(v, dtype=np.float32)).to(torch.float16).numpy().copy()
     raise ValueError(f"unknown dtype {dtype!r}")
 
 

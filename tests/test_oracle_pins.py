@@ -37,7 +37,7 @@ def _p4_expect():
     return t
 
 
-@pytest.mark.parametrize("dtype", ["f32", "i32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "i32", "bf16", "f16"])
 @pytest.mark.parametrize("path", ["ring", "fold", "naive", "tree", "tree_fold"])
 def test_worked_example_allreduce(path, dtype):
     exp = _p4_expect()
@@ -631,3 +631,112 @@ def test_bf16_wire_mutant_is_caught():
     with oracle.mutant(11):
         with pytest.raises(AssertionError):
             test_bf16_wire_golden()
+
+
+# ------------------------------------------------------------------ fp16 --
+# The oracle converts fp16 with its own code from the IEEE 754 binary16
+# definition; numpy's float16 conversion is an independent implementation of
+# the same rounding, so it pins it on the cases that decide it.
+
+def _f16_rounding_cases():
+    rng = np.random.default_rng(41)
+    finite = np.arange(0, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float64)
+    mid = ((finite[:-1] + finite[1:]) / 2).astype(np.float32)  # every tie, exact in fp32
+    mid = np.concatenate([mid, [np.float32(65520.0)]])         # the tie above the largest finite
+    x = np.concatenate([
+        mid, np.nextafter(mid, np.float32(np.inf)), np.nextafter(mid, np.float32(0)),
+        rng.standard_normal(200000).astype(np.float32) * np.float32(300),
+        (rng.standard_normal(50000) * 1e-6).astype(np.float32),
+        np.array([0.0, 65504, 65519.996, 65536, 1e30, 3.4e38, 2.0 ** -24, 2.0 ** -25, 2.0 ** -26, 1e-40,
+                  np.inf], dtype=np.float32)])
+    return np.concatenate([x, -x])
+
+
+def test_f16_widening_matches_numpy_exhaustively():
+    h = np.arange(65536, dtype=np.uint16).view(np.float16)
+    got, want = oracle.f16_to_f32(h), h.astype(np.float32)
+    nan = np.isnan(want)
+    assert np.array_equal(got[~nan].view(np.uint32), want[~nan].view(np.uint32))
+    assert np.isnan(got[nan]).all()
+
+
+def test_f16_rounding_matches_numpy():
+    x = _f16_rounding_cases()
+    with np.errstate(over="ignore"):
+        want = x.astype(np.float16)
+    assert np.array_equal(oracle.f32_to_f16(x).view(np.uint16), want.view(np.uint16))
+    nan = oracle.f32_to_f16(np.array([np.nan, -np.nan], np.float32))
+    assert np.isnan(nan.astype(np.float32)).all()
+
+
+def test_f16_rounding_hand_cases():
+    # 1 + 2^-11 lies halfway between 1 and 1 + 2^-10: ties to even -> 1
+    # 1 + 3 * 2^-11 lies halfway between 1 + 2^-10 and 1 + 2^-9: even -> 1 + 2^-9
+    # 65520 lies halfway between 65504 (odd significand) and 2^16: -> infinity
+    # 2^-25 lies halfway between 0 and 2^-24 (odd): -> 0; 3 * 2^-25 -> 2^-23
+    x = np.array([1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11, 65519.0, 65520.0, 2.0 ** -25, 3 * 2.0 ** -25],
+                 dtype=np.float32)
+    got = oracle.f16_to_f32(oracle.f32_to_f16(x)).tolist()
+    assert got == [1.0, 1 + 2.0 ** -9, 65504.0, float("inf"), 0.0, 2.0 ** -23]
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 4, 5, 8])
+@pytest.mark.parametrize("op", ["sum", "max", "min", "prod"])
+def test_f16_brute_force_integer_data(n, op):
+    # integers whose every partial fold is below 2^11 are exact in fp16, so
+    # every path equals numpy's float64 reduction
+    lo, hi = {"sum": (-100, 100), "prod": (-2, 3)}.get(op, (-1000, 1000))
+    for count in [0, 1, 2 * n + 3, 37]:
+        rng = np.random.default_rng([n, count, 16])
+        raw = [rng.integers(lo, hi, size=count) for _ in range(n)]
+        x0 = [synth.cast(v, "f16") for v in raw]
+        want = _np_reduce(x0, op)
+        for path in (oracle.ring_allreduce, oracle.fold_ring_order, oracle.naive_allreduce,
+                     oracle.tree_schedule, oracle.tree_fold, oracle.double_ring_allreduce):
+            x = [v.copy() for v in x0]
+            path(x, op)
+            for r in range(n):
+                assert np.array_equal(x[r].astype(np.float64), want), (path.__name__, r)
+
+
+@pytest.mark.parametrize("n", [2, 4, 8, 16])
+def test_f16_one_shot_rounds_once_and_ring_stays_within_bound(n):
+    # one-shot: the fp32 ring-order fold of the widened values, rounded once
+    # (numpy's rounding of the oracle's own fp32 fold); ring schedule: per-hop
+    # rounding, within gamma_{N-1} * sum|x| of the fp64 sum, u = 2^-11
+    x = synth.ranks(42, n, 5000, "uniform", "f16")
+    wide = [v.astype(np.float32) for v in x]
+    oracle.fold_ring_order(wide, "sum")
+    one = [v.copy() for v in x]
+    oracle.fold_ring_order(one, "sum")
+    assert np.array_equal(one[0].view(np.uint16), wide[0].astype(np.float16).view(np.uint16))
+    ring = [v.copy() for v in x]
+    oracle.ring_allreduce(ring, "sum")
+    exact = np.sum([v.astype(np.float64) for v in x], axis=0)
+    u = 2.0 ** -11
+    gamma = (n - 1) * u / (1 - (n - 1) * u)
+    bound = gamma * np.sum([np.abs(v.astype(np.float64)) for v in x], axis=0) + u * np.abs(exact)
+    assert (np.abs(ring[0].astype(np.float64) - exact) <= bound).all()
+
+
+def test_f16_bucket_sync_of_small_integers_is_exact():
+    n = 4
+    numels = [10, 33, 7, 120]
+    rng = np.random.default_rng(43)
+    raw = [[rng.integers(-8, 8, size=m) for m in numels] for _ in range(n)]
+    grads = [[synth.cast(v, "f16") for v in rr] for rr in raw]
+    oracle.bucket_sync(grads, cap_bytes=64, op="sum")
+    for t in range(len(numels)):
+        want = sum(raw[r][t] for r in range(n)).astype(np.float16)
+        for r in range(n):
+            assert np.array_equal(grads[r][t], want)
+
+
+def test_f16_rounding_mutant_is_caught():
+    # kind 12: ties round away from zero instead of to even
+    with oracle.mutant(12):
+        with pytest.raises(AssertionError):
+            test_f16_rounding_matches_numpy()
+        with pytest.raises(AssertionError):
+            test_f16_rounding_hand_cases()
+    test_f16_rounding_matches_numpy()
