@@ -432,23 +432,24 @@ def time_extra(dev, stream, host, S, peak):
                        "hbm_gbs": round(st["hbm_bytes"] / tm / 1e9, 1),
                        "hbm_frac": round(st["hbm_bytes"] / tm / 1e9 / peak, 4), "launches": st["launches"]}
         del fresh
-    # bf16 gradients (fp32 accumulation, one rounding): the same 256 MiB per rank
+    # bf16 and fp16 gradients (fp32 accumulation, one rounding): the same 256 MiB per rank
     gen = torch.Generator(device=dev).manual_seed(SEED)
-    bf = [(torch.randn(2 * len(h), device=dev, generator=gen) * 1e-3).to(torch.bfloat16) for h in host]
-    rrv.all_reduce(bf, "avg", "auto", stream)
-    st = rrv.last_stats()
-    torch.cuda.synchronize(dev)
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a0.record(stream)
-    for _ in range(20):
-        rrv.all_reduce(bf, "avg", "auto", stream)
-    a1.record(stream)
-    torch.cuda.synchronize(dev)
-    tm = a0.elapsed_time(a1) / 20 / 1e3
-    extra["oneshot_bf16_avg"] = {"ms": round(tm * 1e3, 4), "algbw_gbs": round(S / tm / 1e9, 2),
-                                 "hbm_gbs": round(st["hbm_bytes"] / tm / 1e9, 1),
-                                 "hbm_frac": round(st["hbm_bytes"] / tm / 1e9 / peak, 4), "launches": st["launches"]}
-    del bf
+    for name, dt in (("oneshot_bf16_avg", torch.bfloat16), ("oneshot_f16_avg", torch.float16)):
+        g16 = [(torch.randn(2 * len(h), device=dev, generator=gen) * 1e-3).to(dt) for h in host]
+        rrv.all_reduce(g16, "avg", "auto", stream)
+        st = rrv.last_stats()
+        torch.cuda.synchronize(dev)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(20):
+            rrv.all_reduce(g16, "avg", "auto", stream)
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        tm = a0.elapsed_time(a1) / 20 / 1e3
+        extra[name] = {"ms": round(tm * 1e3, 4), "algbw_gbs": round(S / tm / 1e9, 2),
+                       "hbm_gbs": round(st["hbm_bytes"] / tm / 1e9, 1),
+                       "hbm_frac": round(st["hbm_bytes"] / tm / 1e9 / peak, 4), "launches": st["launches"]}
+        del g16
     return extra
 
 

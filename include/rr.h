@@ -43,11 +43,11 @@
  *     schedule folds chunk c (its partial starts on rank c and gains one rank
  *     per hop).  AVG is that SUM divided once by N.  MAX keeps the left
  *     operand unless it is smaller, MIN unless it is larger.
- *   - Precision: fp32 and bf16 reduce in fp32 ([P1] s5.3: reduce
- *     low-precision gradients in fp32); bf16 results are rounded once to
- *     nearest-even, except in the RING and TREE schedules, whose partials
- *     live in the bf16 buffers between steps and are rounded at every hop.
- *     int32 SUM and PROD wrap modulo 2^32.
+ *   - Precision: fp32, bf16 and fp16 reduce in fp32 ([P1] s5.3: reduce
+ *     low-precision gradients in fp32); bf16 and fp16 results are rounded
+ *     once to nearest-even, except in the RING, TREE and DOUBLE_RING
+ *     schedules, whose partials live in the 16-bit buffers between steps and
+ *     are rounded at every hop.  int32 SUM and PROD wrap modulo 2^32.
  */
 #ifndef RR_H_
 #define RR_H_
@@ -72,8 +72,9 @@ typedef enum rr_status {
     RR_ERR_TIMEOUT = 4 /* reserved: no kernel of this library waits on another */
 } rr_status_t;
 
-/* Element types of the rank buffers. */
-typedef enum rr_dtype { RR_F32 = 0, RR_BF16 = 1, RR_I32 = 2 } rr_dtype_t;
+/* Element types of the rank buffers: IEEE binary32, bfloat16 (the upper half
+ * of a binary32), int32, IEEE binary16. */
+typedef enum rr_dtype { RR_F32 = 0, RR_BF16 = 1, RR_I32 = 2, RR_F16 = 3 } rr_dtype_t;
 
 /* Reductions of [P1] s2.1: SUM, AVG (sum then divide by N), MAX, MIN, PROD. */
 typedef enum rr_op { RR_SUM = 0, RR_AVG = 1, RR_MAX = 2, RR_MIN = 3, RR_PROD = 4 } rr_op_t;
@@ -155,10 +156,11 @@ typedef struct rr_cost {
 /* All-reduce in place over bufs[0..nranks): afterwards every buffer holds the
  * reduction of all inputs, element by element ([P4] "The five primitives";
  * [P1] s2.1).  count elements per rank.  Bits: RING, ONESHOT, TWO_SHOT and
- * AUTO give the ring order for fp32 and int32; for bf16, ONESHOT and
- * TWO_SHOT round once and RING rounds per hop.  TREE and TREE_ONESHOT give
- * the tree order; DOUBLE_RING the ring order in the first half and the
- * downward order in the second (rounding per hop for bf16).  Buffers must not
+ * AUTO give the ring order for fp32 and int32; for bf16 and fp16, ONESHOT,
+ * TWO_SHOT and AUTO round once and RING rounds per hop.  TREE and
+ * TREE_ONESHOT give the tree order; DOUBLE_RING the ring order in the first
+ * half and the downward order in the second (rounding per hop for bf16 and
+ * fp16).  Buffers must not
  * overlap.  nranks == 1 enqueues nothing. */
 rr_status_t rr_allreduce(void* const* bufs, int nranks, size_t count, rr_dtype_t dtype, rr_op_t op,
                          rr_algo_t algo, cudaStream_t stream);
@@ -242,7 +244,7 @@ typedef struct rr_bucket_plan rr_bucket_plan_t;
  * bucket_cap_mb, default 25).  Greedy over numels[0..ntensors) in the order
  * given, never splitting a tensor: each tensor joins the open bucket, which
  * closes as soon as its bytes (in grad_dtype) reach cap_bytes.  grad_dtype is
- * RR_BF16 or RR_F32; buckets are fp32.  Host only; free with
+ * RR_BF16, RR_F16 or RR_F32; buckets are fp32.  Host only; free with
  * rr_bucket_plan_free. */
 rr_status_t rr_bucket_plan(const size_t* numels, int ntensors, rr_dtype_t grad_dtype, size_t cap_bytes,
                            rr_bucket_plan_t** out);

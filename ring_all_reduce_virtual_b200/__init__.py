@@ -29,17 +29,17 @@ OPS = {"sum": 0, "avg": 1, "max": 2, "min": 3, "prod": 4}
 ALGOS = {"auto": 0, "ring": 1, "oneshot": 2, "tree": 3, "tree_oneshot": 4, "two_shot": 5, "double_ring": 6}
 ALGO_NAMES = {v: k for k, v in ALGOS.items()}
 PHASES = {"reduce_scatter": 0, "all_gather": 1}
-_DTYPE_NAMES = {"f32": 0, "bf16": 1, "i32": 2}
+_DTYPE_NAMES = {"f32": 0, "bf16": 1, "i32": 2, "f16": 3}
 
 
 def _dtype_code(dtype) -> int:
     import torch
 
-    codes = {torch.float32: 0, torch.bfloat16: 1, torch.int32: 2}
+    codes = {torch.float32: 0, torch.bfloat16: 1, torch.int32: 2, torch.float16: 3}
     if isinstance(dtype, str):
         return _DTYPE_NAMES[dtype]
     if dtype not in codes:
-        raise TypeError(f"unsupported dtype {dtype}; use float32, bfloat16 or int32")
+        raise TypeError(f"unsupported dtype {dtype}; use float32, bfloat16, float16 or int32")
     return codes[dtype]
 
 

@@ -61,9 +61,9 @@ bool env_flag(const char* name)
     return v && *v && std::strcmp(v, "0") != 0;
 }
 
-size_t esize(rr_dtype_t d) { return d == RR_BF16 ? 2u : 4u; }
+size_t esize(rr_dtype_t d) { return d == RR_BF16 || d == RR_F16 ? 2u : 4u; }
 
-bool dtype_ok(rr_dtype_t d) { return d == RR_F32 || d == RR_BF16 || d == RR_I32; }
+bool dtype_ok(rr_dtype_t d) { return d == RR_F32 || d == RR_BF16 || d == RR_I32 || d == RR_F16; }
 bool op_ok(rr_op_t o) { return o >= RR_SUM && o <= RR_PROD; }
 
 const char* algo_name(int a)
@@ -846,8 +846,8 @@ rr_status_t rr_bucket_plan(const size_t* numels, int ntensors, rr_dtype_t grad_d
     if (!out) return fail(RR_ERR_INVALID_ARG, "NULL plan output");
     *out = nullptr;
     if (ntensors < 0 || (ntensors > 0 && !numels)) return fail(RR_ERR_INVALID_ARG, "bad tensor list");
-    if (grad_dtype != RR_BF16 && grad_dtype != RR_F32)
-        return fail(RR_ERR_UNSUPPORTED, "gradients must be bf16 or fp32");
+    if (grad_dtype != RR_BF16 && grad_dtype != RR_F16 && grad_dtype != RR_F32)
+        return fail(RR_ERR_UNSUPPORTED, "gradients must be bf16, fp16 or fp32");
     auto* p = new rr_bucket_plan_t();
     p->ntensors = ntensors;
     p->grad_dtype = grad_dtype;
@@ -1239,12 +1239,12 @@ rr_status_t rr_set_picker_params(double launch_s, double hbm_bytes_per_s)
 
 // On one GPU every "link" is HBM: a step costs one launch, and its bytes are
 // the HBM bytes it reads and writes (ring 5(N-1) S over 2(N-1) launches,
-// one-shot 2 N S in one).  bf16 always takes ONESHOT: the ring rounds its
-// bf16 partials at every hop, the fp32-accumulating one-shot does not
+// one-shot 2 N S in one).  bf16 and fp16 always take ONESHOT: the ring rounds
+// its 16-bit partials at every hop, the fp32-accumulating one-shot does not
 // ([P1] s5.3).
 rr_algo_t rr_pick_algo(int nranks, size_t count, rr_dtype_t dtype)
 {
-    if (dtype == RR_BF16 || nranks <= 1) return RR_ALGO_ONESHOT;
+    if (dtype == RR_BF16 || dtype == RR_F16 || nranks <= 1) return RR_ALGO_ONESHOT;
     const double n = nranks, S = (double)count * (double)esize(dtype);
     const double ring = 2 * (n - 1) * g_launch_s + 5 * (n - 1) * S / g_hbm_bps;
     const double one = g_launch_s + 2 * n * S / g_hbm_bps;

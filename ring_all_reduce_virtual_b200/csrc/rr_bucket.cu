@@ -34,21 +34,28 @@ struct Quad<F32T> {
     __device__ static __forceinline__ R from_f(const float (&a)[4]) { return F32T::pack(a); }
 };
 
-template <>
-struct Quad<BF16T> {
+// The 16-bit types (bf16, fp16): a quad is 8 bytes, two packed pairs.
+template <class X>
+struct Quad16 {
     using R = uint2;
     __device__ static __forceinline__ R ld(const uint16_t* p) { return __ldcs(reinterpret_cast<const uint2*>(p)); }
     __device__ static __forceinline__ void st(uint16_t* p, const R& r) { __stcs(reinterpret_cast<uint2*>(p), r); }
     __device__ static __forceinline__ void to_f(const R& r, float (&a)[4])
     {
-        BF16T::unpack2(r.x, a[0], a[1]);
-        BF16T::unpack2(r.y, a[2], a[3]);
+        X::unpack2(r.x, a[0], a[1]);
+        X::unpack2(r.y, a[2], a[3]);
     }
     __device__ static __forceinline__ R from_f(const float (&a)[4])
     {
-        return make_uint2(BF16T::pack2(a[0], a[1]), BF16T::pack2(a[2], a[3]));
+        return make_uint2(X::pack2(a[0], a[1]), X::pack2(a[2], a[3]));
     }
 };
+
+template <>
+struct Quad<BF16T> : Quad16<BF16T> {};
+
+template <>
+struct Quad<F16T> : Quad16<F16T> {};
 
 // Convert one tile of a segment from In's element type to Out's, dividing by
 // `divisor` first when OP is AVG.  A tile is kThreads * Q quads, Q chosen so
@@ -208,16 +215,17 @@ cudaError_t launch_fold(const BucketFoldParams& p, uint64_t work, cudaStream_t s
 }  // namespace
 
 // Elements one pack/unpack tile covers: kThreads * kUnitsPerThread 16-byte
-// vectors of the gradient type (8 elements each for bf16, 4 for fp32).
+// vectors of the gradient type (8 elements each for bf16 and fp16, 4 for fp32).
 uint64_t bucket_tile_elems(int grad_dtype)
 {
-    return (uint64_t)kThreads * kUnitsPerThread * (grad_dtype == kBF16 ? 8u : 4u);
+    return (uint64_t)kThreads * kUnitsPerThread * (grad_dtype == kBF16 || grad_dtype == kF16 ? 8u : 4u);
 }
 
 cudaError_t launch_bucket_pack(int grad_dtype, const BucketCopyParams& p, cudaStream_t s)
 {
     const uint64_t work = p.tile0[p.nt];
     if (grad_dtype == kBF16) return launch_all_b(bucket_pack_kernel<BF16T>, p, work, s);
+    if (grad_dtype == kF16) return launch_all_b(bucket_pack_kernel<F16T>, p, work, s);
     if (grad_dtype == kF32) return launch_all_b(bucket_pack_kernel<F32T>, p, work, s);
     return cudaErrorInvalidValue;
 }
@@ -229,6 +237,9 @@ cudaError_t launch_bucket_unpack(int grad_dtype, int op, const BucketCopyParams&
     if (grad_dtype == kBF16)
         return avg ? launch_all_b(bucket_unpack_kernel<BF16T, kAvg>, p, work, s)
                    : launch_all_b(bucket_unpack_kernel<BF16T, kSum>, p, work, s);
+    if (grad_dtype == kF16)
+        return avg ? launch_all_b(bucket_unpack_kernel<F16T, kAvg>, p, work, s)
+                   : launch_all_b(bucket_unpack_kernel<F16T, kSum>, p, work, s);
     if (grad_dtype == kF32)
         return avg ? launch_all_b(bucket_unpack_kernel<F32T, kAvg>, p, work, s)
                    : launch_all_b(bucket_unpack_kernel<F32T, kSum>, p, work, s);
@@ -241,6 +252,8 @@ cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p
     const bool avg = op == kAvg;
     if (grad_dtype == kBF16)
         return avg ? launch_fold<BF16T, kAvg>(p, work, s, max_grid) : launch_fold<BF16T, kSum>(p, work, s, max_grid);
+    if (grad_dtype == kF16)
+        return avg ? launch_fold<F16T, kAvg>(p, work, s, max_grid) : launch_fold<F16T, kSum>(p, work, s, max_grid);
     if (grad_dtype == kF32)
         return avg ? launch_fold<F32T, kAvg>(p, work, s, max_grid) : launch_fold<F32T, kSum>(p, work, s, max_grid);
     return cudaErrorInvalidValue;

@@ -18,6 +18,7 @@
 #include <cstdint>
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 namespace rr {
@@ -70,6 +71,38 @@ struct BF16T {
     __device__ static __forceinline__ uint32_t pack2(Acc lo, Acc hi)
     {
         __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half), .y = hi
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+    __device__ static __forceinline__ void unpack(const uint4& r, Acc (&a)[L])
+    {
+        unpack2(r.x, a[0], a[1]);
+        unpack2(r.y, a[2], a[3]);
+        unpack2(r.z, a[4], a[5]);
+        unpack2(r.w, a[6], a[7]);
+    }
+    __device__ static __forceinline__ uint4 pack(const Acc (&a)[L])
+    {
+        return make_uint4(pack2(a[0], a[1]), pack2(a[2], a[3]), pack2(a[4], a[5]), pack2(a[6], a[7]));
+    }
+};
+
+// fp16 buffers (raw IEEE binary16 patterns), fp32 arithmetic; widening is
+// exact, narrowing rounds to nearest even (overflow to infinity).
+struct F16T {
+    using T = uint16_t;
+    using Acc = float;
+    static constexpr int L = 8;
+    __device__ static __forceinline__ Acc ld1(const T* p) { return __half2float(__ushort_as_half(*p)); }
+    __device__ static __forceinline__ void st1(T* p, Acc v) { *p = __half_as_ushort(__float2half_rn(v)); }
+    __device__ static __forceinline__ void unpack2(uint32_t w, Acc& lo, Acc& hi)
+    {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));  // .x = low half
+        lo = f.x;
+        hi = f.y;
+    }
+    __device__ static __forceinline__ uint32_t pack2(Acc lo, Acc hi)
+    {
+        __half2 h = __floats2half2_rn(lo, hi);  // .x = lo (low half), .y = hi
         return *reinterpret_cast<uint32_t*>(&h);
     }
     __device__ static __forceinline__ void unpack(const uint4& r, Acc (&a)[L])

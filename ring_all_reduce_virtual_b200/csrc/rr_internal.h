@@ -91,7 +91,7 @@ struct BucketFoldParams {
     float divisor;
 };
 
-enum DType : int { kF32 = 0, kBF16 = 1, kI32 = 2 };
+enum DType : int { kF32 = 0, kBF16 = 1, kI32 = 2, kF16 = 3 };
 enum Kind : int {
     kOneshotRing = 0,
     kOneshotTree = 1,

@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(kThreads) step_kernel(const __grid_constant__ 
 
 uint64_t tile_elems(int dtype, int vpt)
 {
-    return (uint64_t)kThreads * (uint64_t)vpt * (dtype == kBF16 ? 8u : 4u);
+    return (uint64_t)kThreads * (uint64_t)vpt * (dtype == kBF16 || dtype == kF16 ? 8u : 4u);
 }
 
 cudaError_t launch_rank_kernel(int kind, int dtype, int op, const RankParams& p, cudaStream_t s)

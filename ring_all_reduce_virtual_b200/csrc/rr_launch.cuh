@@ -39,6 +39,7 @@ inline cudaError_t with_type(int dtype, int op, F&& f)
     switch (dtype) {
     case kF32: return by_op.template operator()<F32T>();
     case kBF16: return by_op.template operator()<BF16T>();
+    case kF16: return by_op.template operator()<F16T>();
     case kI32: return by_op.template operator()<I32T>();
     }
     return cudaErrorInvalidValue;

@@ -15,7 +15,8 @@ cudaError_t launch_oneshot_tree(const RankParams& p, uint64_t work, cudaStream_t
 #define RR_FOR_EACH_TYPE_OP(X)                                                                   \
     X(F32T, kSum) X(F32T, kAvg) X(F32T, kMax) X(F32T, kMin) X(F32T, kProd) X(BF16T, kSum)         \
     X(BF16T, kAvg) X(BF16T, kMax) X(BF16T, kMin) X(BF16T, kProd) X(I32T, kSum) X(I32T, kMax)     \
-    X(I32T, kMin) X(I32T, kProd)
+    X(I32T, kMin) X(I32T, kProd) X(F16T, kSum) X(F16T, kAvg) X(F16T, kMax) X(F16T, kMin)         \
+    X(F16T, kProd)
 
 #define RR_DECLARE_ONESHOT(TY, OP)                                                               \
     extern template cudaError_t launch_oneshot_ring<TY, OP>(const RankParams&, uint64_t, cudaStream_t); \

@@ -1,5 +1,6 @@
 """Helpers for the GPU tests: move synthetic host arrays to and from CUDA
-tensors (bf16 travels as its 16-bit patterns) and compare bit patterns."""
+tensors (bf16 travels as its 16-bit patterns, fp16 as numpy float16) and
+compare bit patterns."""
 import numpy as np
 import torch
 
@@ -41,7 +42,7 @@ def to_host(tensors):
 
 def bits(a):
     a = np.ascontiguousarray(a)
-    return a.view(np.uint16) if a.dtype == np.uint16 else a.view(np.uint32)
+    return a.view(np.uint16) if a.dtype in (np.uint16, np.float16) else a.view(np.uint32)
 
 
 def assert_bits_equal(got, want, what=""):
@@ -56,5 +57,5 @@ def assert_bits_equal(got, want, what=""):
 def empty_like_ranks(n, count, dtype):
     if dtype == "bf16":
         return [torch.empty(count, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
-    td = torch.float32 if dtype == "f32" else torch.int32
+    td = {"f32": torch.float32, "f16": torch.float16, "i32": torch.int32}[dtype]
     return [torch.empty(count, dtype=td, device="cuda") for _ in range(n)]

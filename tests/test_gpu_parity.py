@@ -30,8 +30,8 @@ ORACLE = {
     "tree_oneshot": oracle.tree_fold,
 }
 PER_HOP = ("ring", "tree", "double_ring")  # bf16 schedules that round at every hop
-TILE = {"f32": 2048, "bf16": 4096, "i32": 2048}  # elements per tile of the N-input fold kernels
-TILE_MOVE = {"f32": 4096, "bf16": 8192, "i32": 4096}  # per tile of the 1- and 2-input kernels
+TILE = {"f32": 2048, "bf16": 4096, "f16": 4096, "i32": 2048}  # elements per tile of the N-input fold kernels
+TILE_MOVE = {"f32": 4096, "bf16": 8192, "f16": 8192, "i32": 4096}  # per tile of the 1- and 2-input kernels
 
 
 def _dist(op, dtype):
@@ -91,7 +91,7 @@ def test_worked_example(algo):
 # ------------------------------------------------------ all-reduce parity --
 
 @pytest.mark.parametrize("algo", ALGOS)
-@pytest.mark.parametrize("dtype", ["f32", "bf16", "i32"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16", "i32"])
 @pytest.mark.parametrize("op", ["sum", "avg", "max", "min", "prod"])
 def test_allreduce_every_op_and_dtype(algo, dtype, op):
     if dtype == "i32" and op == "avg":
@@ -99,16 +99,18 @@ def test_allreduce_every_op_and_dtype(algo, dtype, op):
     n = 5
     count = 3 * TILE[dtype] * n + 37  # several tiles per chunk and a ragged tail
     x, got = _run(n, count, dtype, op, algo, seed=1)
-    if dtype == "bf16" and op in ("sum", "avg"):
-        wide = np.stack([oracle.bf16_to_f32(v) for v in x]).astype(np.float64)
+    if dtype in ("bf16", "f16") and op in ("sum", "avg"):
+        widen = oracle.bf16_to_f32 if dtype == "bf16" else oracle.f16_to_f32
+        wide = np.stack([widen(v) for v in x]).astype(np.float64)
         ref, mag = wide.sum(0), np.abs(wide).sum(0)
         if op == "avg":
             ref, mag = ref / n, mag / n
-        g = oracle.bf16_to_f32(got[0]).astype(np.float64)
+        g = widen(got[0]).astype(np.float64)
         if algo in PER_HOP:
-            # partials rounded to bf16 after every hop: recursive summation in
-            # bf16, |error| <= gamma_{N-1} * sum |x| with u = 2^-8 (Higham 4.2)
-            u = 2.0 ** -8
+            # partials rounded to 16 bits after every hop: recursive summation
+            # in bf16 (u = 2^-8) or fp16 (u = 2^-11), |error| <= gamma_{N-1} *
+            # sum |x| (Higham 4.2)
+            u = 2.0 ** -8 if dtype == "bf16" else 2.0 ** -11
             gamma = (n - 1) * u / (1 - (n - 1) * u)
             assert np.all(np.abs(g - ref) <= gamma * mag + 1e-30)
         else:  # fp32 accumulation, one rounding: the stated abs/rel 1e-2
@@ -123,13 +125,13 @@ def test_allreduce_sizes(algo, n, count):
 
 
 @pytest.mark.parametrize("algo", ALGOS)
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 def test_allreduce_64_ranks(algo, dtype):
     _run(64, 64 * 700 + 3, dtype, "sum", algo, seed=3)
 
 
 @pytest.mark.parametrize("algo", ["ring", "oneshot", "tree_oneshot"])
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 def test_allreduce_shared_misalignment(algo, dtype):
     # every base 1 element past a 16-byte boundary: vector path after a head
     n = 4
@@ -137,7 +139,7 @@ def test_allreduce_shared_misalignment(algo, dtype):
 
 
 @pytest.mark.parametrize("algo", ["ring", "oneshot", "tree", "tree_oneshot"])
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 def test_allreduce_mixed_misalignment(algo, dtype):
     # bases disagree modulo 16 bytes: the scalar path
     n = 4
@@ -180,7 +182,7 @@ def test_max_signed_zero_ties_follow_the_fold():
 # ----------------------------------------------------------- ring steps --
 
 @pytest.mark.parametrize("n", [2, 3, 4, 8])
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("op", ["sum", "avg"])
 def test_ring_steps_track_the_oracle_state(n, dtype, op):
     # after every one of the 2(N-1) steps the device buffers equal the
@@ -221,12 +223,12 @@ def test_ring_stats_match_the_schedule():
 # --------------------------------------------- reduce-scatter, all-gather --
 
 @pytest.mark.parametrize("n", [1, 2, 3, 4, 8, 64])
-@pytest.mark.parametrize("dtype", ["f32", "bf16", "i32"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16", "i32"])
 def test_reduce_scatter_all_gather_all_to_all(n, dtype):
     per = 2 * TILE_MOVE[dtype] + 9
     x = synth.ranks(8, n, n * per, "int" if dtype == "i32" else "uniform", dtype)
     d = to_dev(x)
-    for op in ("sum", "max") if dtype != "bf16" else ("sum", "avg"):
+    for op in ("sum", "max") if dtype not in ("bf16", "f16") else ("sum", "avg"):
         rs = empty_like_ranks(n, per, dtype)
         rrv.reduce_scatter(d, rs, op)
         assert_bits_equal(to_host(rs), oracle.reduce_scatter([a.copy() for a in x], op), f"rs {op}")
@@ -257,12 +259,12 @@ def _grad_set(seed, n, numels, dtype="bf16"):
     return [synth.rank_grads(seed, r, numels, "normal", dtype) for r in range(n)]
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
 @pytest.mark.parametrize("op", ["avg", "sum"])
 def test_bucket_staged_and_fused_match_the_oracle(dtype, op):
     n = 8
     numels = [5, 3000, 64, 1, 9000, 77, 0, 20000, 333, 4096]
-    cap = 4 * 4096 * (2 if dtype == "bf16" else 4)
+    cap = 4 * 4096 * (4 if dtype == "f32" else 2)
     host = _grad_set(10, n, numels, dtype)
     want = [[g.copy() for g in rank] for rank in host]
     oracle.bucket_sync(want, cap, op)
@@ -280,7 +282,7 @@ def test_bucket_staged_and_fused_match_the_oracle(dtype, op):
         bo, off = [], []
         first, cnt, _ = plan.info(b)
         for t in range(first, first + cnt):
-            w = oracle.bf16_to_f32(host[0][t]) if dtype == "bf16" else host[0][t]
+            w = {"bf16": oracle.bf16_to_f32, "f16": oracle.f16_to_f32}.get(dtype, np.asarray)(host[0][t])
             assert np.array_equal(packed[0][plan.tensor(t)[1]:plan.tensor(t)[1] + numels[t]], w)
     for r in range(n):
         assert_bits_equal(to_host(grads[r]), want[r], f"staged rank {r}")
@@ -292,7 +294,7 @@ def test_bucket_staged_and_fused_match_the_oracle(dtype, op):
         assert_bits_equal(to_host(grads[r]), want[r], f"fused rank {r}")
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
 @pytest.mark.parametrize("op", ["avg", "sum"])
 def test_bucket_range_matches_per_bucket_syncs(dtype, op):
     """A bucket range shares launches but keeps every bucket's own chunking:
@@ -303,7 +305,7 @@ def test_bucket_range_matches_per_bucket_syncs(dtype, op):
     rng = np.random.default_rng(31)
     numels = [int(v) for v in rng.integers(0, 3000, size=300)]
     numels[7] = 70001  # one tensor larger than the cap: a bucket of its own
-    cap = 3000 * (2 if dtype == "bf16" else 4)
+    cap = 3000 * (4 if dtype == "f32" else 2)
     host = _grad_set(12, n, numels, dtype)
     want = [[g.copy() for g in rank] for rank in host]
     oracle.bucket_sync(want, cap, op)
