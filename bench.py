@@ -41,7 +41,7 @@ FALLBACK_HBM_GBS = 6650.0
 # from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), with the
 # hash of the dominant kernel's source files it was taken on.  The summary with its command is
 # in profiles/oneshot_ring_kernel_allreduce-8x64MiB-f32.md.
-NCU_TRAFFIC = {"per_algorithmic_byte": (536896768 + 479010048) / 1073741824, "sources_sha1": "14e30a8379188f7b032b2c097d40db4c442cfb7d"}
+NCU_TRAFFIC = {"per_algorithmic_byte": (536918272 + 479562496) / 1073741824, "sources_sha1": "6772def93fdf3d0fd41ebe5dea839b5f96e50b1b"}
 
 
 # The files that define the dominant kernel (oneshot_ring_kernel).
