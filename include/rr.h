@@ -27,8 +27,10 @@
  *     returned as RR_ERR_CUDA (detail in rr_last_error()).
  *   - Argument errors are returned before anything is enqueued:
  *     RR_ERR_INVALID_ARG for a NULL or repeated device pointer, nranks
- *     outside 1..RR_MAX_RANKS, overlapping buffers, a bad enum or a count
- *     that the operation cannot split; RR_ERR_UNSUPPORTED for a valid but
+ *     outside 1..RR_MAX_RANKS, overlapping buffers, a bad enum, an element
+ *     count above 2^48 (far past any device memory; it keeps byte ranges
+ *     from wrapping) or a count that the operation cannot split;
+ *     RR_ERR_UNSUPPORTED for a valid but
  *     unsupported combination (AVG on int32).
  *   - count == 0 is RR_OK and enqueues nothing.  Any pointer alignment is
  *     accepted; buffers whose addresses agree modulo 16 bytes take the

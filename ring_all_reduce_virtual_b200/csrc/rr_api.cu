@@ -90,6 +90,16 @@ rr_status_t check_basic(int n, rr_dtype_t dtype, rr_op_t op)
     return RR_OK;
 }
 
+// Element counts above 2^48 (far beyond any device memory) are refused, so
+// count * 64 ranks * 4 bytes stays below 2^56 and no byte range wraps.
+constexpr uint64_t kMaxElems = 1ull << 48;
+
+rr_status_t check_count(uint64_t count)
+{
+    if (count > kMaxElems) return fail(RR_ERR_INVALID_ARG, "element count above 2^48");
+    return RR_OK;
+}
+
 struct Span {
     uintptr_t lo, hi;
     bool out;
@@ -479,6 +489,7 @@ rr_status_t rr_allreduce(void* const* bufs, int nranks, size_t count, rr_dtype_t
 {
     rr_status_t st = check_basic(nranks, dtype, op);
     if (st != RR_OK) return st;
+    if ((st = check_count(count)) != RR_OK) return st;
     if (algo < RR_ALGO_AUTO || algo > RR_ALGO_DOUBLE_RING) return fail(RR_ERR_INVALID_ARG, "unknown algo");
     if (!bufs) return fail(RR_ERR_INVALID_ARG, "NULL bufs array");
     const int n = nranks;
@@ -558,6 +569,7 @@ rr_status_t rr_allreduce_wire(void* const* bufs, int nranks, size_t count, rr_op
 {
     rr_status_t st = check_basic(nranks, RR_F32, op);
     if (st != RR_OK) return st;
+    if ((st = check_count(count)) != RR_OK) return st;
     if (op != RR_SUM && op != RR_AVG) return fail(RR_ERR_UNSUPPORTED, "the wire format carries SUM or AVG");
     if (wire != RR_BF16) return fail(RR_ERR_UNSUPPORTED, "the wire format is bf16");
     if (algo != RR_ALGO_AUTO && algo != RR_ALGO_ONESHOT && algo != RR_ALGO_RING)
@@ -609,6 +621,7 @@ rr_status_t rr_allreduce_host(void* const* host_bufs, void* const* dev_bufs, int
 {
     rr_status_t st = check_basic(nranks, dtype, op);
     if (st != RR_OK) return st;
+    if ((st = check_count(count)) != RR_OK) return st;
     if (algo < RR_ALGO_AUTO || algo > RR_ALGO_DOUBLE_RING) return fail(RR_ERR_INVALID_ARG, "unknown algo");
     if (!host_bufs || !dev_bufs) return fail(RR_ERR_INVALID_ARG, "NULL pointer array");
     const int n = nranks;
@@ -698,6 +711,7 @@ rr_status_t rr_ring_step(void* const* bufs, int nranks, size_t count, rr_dtype_t
 {
     rr_status_t st = check_basic(nranks, dtype, op);
     if (st != RR_OK) return st;
+    if ((st = check_count(count)) != RR_OK) return st;
     if (phase != RR_PHASE_REDUCE_SCATTER && phase != RR_PHASE_ALL_GATHER)
         return fail(RR_ERR_INVALID_ARG, "unknown phase");
     if (step < 0 || step > nranks - 2) return fail(RR_ERR_INVALID_ARG, "step must be in 0..nranks-2");
@@ -752,6 +766,7 @@ rr_status_t rr_reduce_scatter(const void* const* send, void* const* recv, int nr
 {
     rr_status_t st = check_basic(nranks, dtype, op);
     if (st != RR_OK) return st;
+    if ((st = check_count(recvcount)) != RR_OK) return st;
     if (algo != RR_ALGO_AUTO && algo != RR_ALGO_ONESHOT)
         return fail(RR_ERR_UNSUPPORTED, "reduce-scatter runs AUTO or ONESHOT");
     if (!send || !recv) return fail(RR_ERR_INVALID_ARG, "NULL pointer array");
@@ -783,6 +798,7 @@ rr_status_t rr_all_gather(const void* const* send, void* const* recv, int nranks
 {
     rr_status_t st = check_basic(nranks, dtype, RR_SUM);
     if (st != RR_OK) return st;
+    if ((st = check_count(sendcount)) != RR_OK) return st;
     if (algo != RR_ALGO_AUTO && algo != RR_ALGO_ONESHOT)
         return fail(RR_ERR_UNSUPPORTED, "all-gather runs AUTO or ONESHOT");
     if (!send || !recv) return fail(RR_ERR_INVALID_ARG, "NULL pointer array");
@@ -814,6 +830,7 @@ rr_status_t rr_all_to_all(const void* const* send, void* const* recv, int nranks
 {
     rr_status_t st = check_basic(nranks, dtype, RR_SUM);
     if (st != RR_OK) return st;
+    if ((st = check_count(count_per_peer)) != RR_OK) return st;
     if (!send || !recv) return fail(RR_ERR_INVALID_ARG, "NULL pointer array");
     const int n = nranks;
     const size_t es = esize(dtype);
@@ -856,6 +873,10 @@ rr_status_t rr_bucket_plan(const size_t* numels, int ntensors, rr_dtype_t grad_d
     uint64_t off = 0, bytes = 0;
     int b = 0, open = 0;
     for (int t = 0; t < ntensors; ++t) {
+        if (numels[t] > kMaxElems || off + numels[t] > kMaxElems) {
+            delete p;
+            return fail(RR_ERR_INVALID_ARG, "element count above 2^48");
+        }
         if (!open) {
             p->first.push_back(t);
             p->count.push_back(0);

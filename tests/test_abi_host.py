@@ -252,3 +252,18 @@ def test_bucket_range_argument_errors():
     assert lib.rr_bucket_allreduce_range(plan._h, 0, 3, repeated, 2, 1, s) == _lib.RR_ERR_INVALID_ARG
     assert lib.rr_bucket_allreduce_range(plan._h, 0, 3, grads, 1, 1, s) == 0  # one rank: identity
     assert rrv.last_stats()["launches"] == 0
+
+
+def test_element_counts_above_2_pow_48_are_refused():
+    """A count whose byte range could wrap is refused before any launch."""
+    lib = _lib.lib()
+    s = ctypes.c_void_p(0)
+    huge = (1 << 48) + 1
+    assert lib.rr_allreduce(_fake(4), 4, huge, 0, 0, 2, s) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_allreduce(_fake(4), 4, 1 << 62, 0, 0, 2, s) == _lib.RR_ERR_INVALID_ARG
+    assert b"2^48" in lib.rr_last_error()
+    assert lib.rr_reduce_scatter(_fake(2), _fake(2, base=1 << 41), 2, huge, 0, 0, 0, s) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_all_gather(_fake(2), _fake(2, base=1 << 41), 2, huge, 0, 0, s) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_all_to_all(_fake(2), _fake(2, base=1 << 41), 2, huge, 0, s) == _lib.RR_ERR_INVALID_ARG
+    with pytest.raises(rrv.RRError):
+        rrv.BucketPlan([10, huge], "bf16", 100)
