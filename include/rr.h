@@ -30,8 +30,8 @@
  *     outside 1..RR_MAX_RANKS, overlapping buffers, a bad enum, an element
  *     count above 2^48 (far past any device memory; it keeps byte ranges
  *     from wrapping) or a count that the operation cannot split;
- *     RR_ERR_UNSUPPORTED for a valid but
- *     unsupported combination (AVG on int32).
+ *     RR_ERR_UNSUPPORTED for a valid but unsupported combination (AVG on
+ *     int32).
  *   - count == 0 is RR_OK and enqueues nothing.  Any pointer alignment is
  *     accepted; buffers whose addresses agree modulo 16 bytes take the
  *     128-bit vector path, the rest a scalar path.
