@@ -311,6 +311,8 @@ typedef struct rr_reducer rr_reducer_t;
  * of each bucket sync (they then loop over the bucket's tiles), leaving the
  * other SMs to the kernels that produce the gradients, as a communication
  * library runs its collectives on a few channels; 0 launches one CTA per tile.
+ * The gradients are checked here, once (RR_ERR_INVALID_ARG for a NULL or
+ * overlapping one), so a step's syncs meet no argument error.
  * Creates one CUDA event per bucket plus one; allocates no device memory. */
 rr_status_t rr_reducer_create(const rr_bucket_plan_t* plan, void* const* grads, int nranks, rr_op_t op,
                               cudaStream_t comm, int max_ctas, rr_reducer_t** out);

@@ -1151,6 +1151,11 @@ rr_status_t rr_reducer_create(const rr_bucket_plan_t* plan, void* const* grads, 
     if (!plan || !grads) return fail(RR_ERR_INVALID_ARG, "NULL plan or gradient array");
     if (nranks < 1 || nranks > RR_MAX_RANKS) return fail(RR_ERR_INVALID_ARG, "nranks must be in 1..64");
     if (op != RR_SUM && op != RR_AVG) return fail(RR_ERR_UNSUPPORTED, "the reducer takes SUM or AVG");
+    if (!plan->first.empty()) {  // every gradient of every bucket, once, before any step
+        int t0 = 0, nt = 0;
+        rr_status_t st = bucket_range_check(plan, 0, (int)plan->first.size(), grads, nranks, &t0, &nt);
+        if (st != RR_OK) return st;
+    }
     auto* red = new rr_reducer();
     red->plan = plan;
     red->n = nranks;

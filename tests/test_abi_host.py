@@ -205,6 +205,10 @@ def test_reducer_argument_errors():
     plan = rrv.BucketPlan([10, 20], "bf16", 100)
     assert lib.rr_reducer_create(plan._h, _fake(4), 2, 2, None, 0, ctypes.byref(out)) == _lib.RR_ERR_UNSUPPORTED
     assert lib.rr_reducer_create(plan._h, _fake(4), 0, 1, None, 0, ctypes.byref(out)) == _lib.RR_ERR_INVALID_ARG
+    # gradients are checked at creation: a repeated pointer is refused there
+    assert lib.rr_reducer_create(plan._h, _fake(4, stride=0), 2, 1, None, 0, ctypes.byref(out)) == \
+        _lib.RR_ERR_INVALID_ARG
+    assert b"overlap" in lib.rr_last_error()
     assert lib.rr_reducer_ready(None, 0, None) == _lib.RR_ERR_INVALID_ARG
     assert lib.rr_reducer_finish(None, None) == _lib.RR_ERR_INVALID_ARG
 
