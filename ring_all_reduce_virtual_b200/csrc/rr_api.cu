@@ -628,9 +628,11 @@ rr_status_t rr_allreduce_host(void* const* host_bufs, void* const* dev_bufs, int
     const size_t es = esize(dtype), bytes = count * es;
     for (int r = 0; r < n && count; ++r)
         if (!host_bufs[r]) return fail(RR_ERR_INVALID_ARG, "NULL host buffer");
-    std::vector<Span> spans;
-    for (int r = 0; r < n && count; ++r)
+    std::vector<Span> spans;  // host buffers are written back too (one address space with UVA)
+    for (int r = 0; r < n && count; ++r) {
         spans.push_back({(uintptr_t)dev_bufs[r], (uintptr_t)dev_bufs[r] + bytes, true});
+        spans.push_back({(uintptr_t)host_bufs[r], (uintptr_t)host_bufs[r] + bytes, true});
+    }
     if ((st = check_spans(spans)) != RR_OK) return st;
     const rr_algo_t a = resolve_algo(algo, n, count, dtype);
     if (count == 0) return rr_allreduce(dev_bufs, n, 0, dtype, op, a, stream);

@@ -271,3 +271,17 @@ def test_element_counts_above_2_pow_48_are_refused():
     assert lib.rr_all_to_all(_fake(2), _fake(2, base=1 << 41), 2, huge, 0, s) == _lib.RR_ERR_INVALID_ARG
     with pytest.raises(rrv.RRError):
         rrv.BucketPlan([10, huge], "bf16", 100)
+
+
+def test_host_buffer_allreduce_checks_every_buffer():
+    """rr_allreduce_host refuses overlapping device buffers, overlapping host
+    buffers and a host buffer that overlaps a device one, before any copy."""
+    lib = _lib.lib()
+    s = ctypes.c_void_p(0)
+    dev, host = _fake(2), _fake(2, base=1 << 42)
+    assert lib.rr_allreduce_host(host, _fake(2, stride=0), 2, 16, 0, 0, 2, s) == _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_allreduce_host(_fake(2, base=1 << 42, stride=8), dev, 2, 16, 0, 0, 2, s) == \
+        _lib.RR_ERR_INVALID_ARG
+    assert lib.rr_allreduce_host(dev, dev, 2, 16, 0, 0, 2, s) == _lib.RR_ERR_INVALID_ARG
+    nulls = (ctypes.c_void_p * 2)(None, None)
+    assert lib.rr_allreduce_host(nulls, dev, 2, 16, 0, 0, 2, s) == _lib.RR_ERR_INVALID_ARG
