@@ -162,9 +162,9 @@ def ring_schedule(nranks: int, count: int, dtype="f32") -> list[dict]:
 def reduce_scatter(send: Sequence, recv: Sequence, op="sum", algo="auto", stream=None) -> None:
     """``recv[r]`` = part r of the reduction of all ``send`` (``rr_reduce_scatter``)."""
     count, d, dev = _ranks(send, "reduce_scatter")
-    rcount, rd, _ = _ranks(recv, "reduce_scatter")
-    if len(recv) != len(send) or rd != d or rcount * len(send) != count:
-        raise ValueError("reduce_scatter: recv must be N tensors of count/N elements of the same dtype")
+    rcount, rd, rdev = _ranks(recv, "reduce_scatter")
+    if len(recv) != len(send) or rd != d or rdev != dev or rcount * len(send) != count:
+        raise ValueError("reduce_scatter: recv must be N tensors of count/N elements of the same dtype and device")
     check(lib().rr_reduce_scatter(_ptr_array(send), _ptr_array(recv), len(send), rcount, d, _op(op),
                                   _algo(algo), _stream(stream, dev)), "reduce_scatter")
 
@@ -172,9 +172,9 @@ def reduce_scatter(send: Sequence, recv: Sequence, op="sum", algo="auto", stream
 def all_gather(send: Sequence, recv: Sequence, algo="auto", stream=None) -> None:
     """``recv[r]`` = concatenation of all ``send`` parts (``rr_all_gather``)."""
     scount, d, dev = _ranks(send, "all_gather")
-    rcount, rd, _ = _ranks(recv, "all_gather")
-    if len(recv) != len(send) or rd != d or rcount != scount * len(send):
-        raise ValueError("all_gather: recv must be N tensors of N*count elements of the same dtype")
+    rcount, rd, rdev = _ranks(recv, "all_gather")
+    if len(recv) != len(send) or rd != d or rdev != dev or rcount != scount * len(send):
+        raise ValueError("all_gather: recv must be N tensors of N*count elements of the same dtype and device")
     check(lib().rr_all_gather(_ptr_array(send), _ptr_array(recv), len(send), scount, d, _algo(algo),
                               _stream(stream, dev)), "all_gather")
 
@@ -182,29 +182,44 @@ def all_gather(send: Sequence, recv: Sequence, algo="auto", stream=None) -> None
 def all_to_all(send: Sequence, recv: Sequence, stream=None) -> None:
     """Block transpose across ranks (``rr_all_to_all``)."""
     count, d, dev = _ranks(send, "all_to_all")
-    rcount, rd, _ = _ranks(recv, "all_to_all")
+    rcount, rd, rdev = _ranks(recv, "all_to_all")
     n = len(send)
-    if len(recv) != n or rd != d or rcount != count or count % n:
-        raise ValueError("all_to_all: recv must match send, and N must divide the count")
+    if len(recv) != n or rd != d or rdev != dev or rcount != count or count % n:
+        raise ValueError("all_to_all: recv must match send (size, dtype, device), and N must divide the count")
     check(lib().rr_all_to_all(_ptr_array(send), _ptr_array(recv), n, count // n, d, _stream(stream, dev)),
           "all_to_all")
 
 
 class GradSet:
-    """The gradient tensors of all ranks (``grads[r][t]``), with their device
-    pointers marshalled once.  Bucket calls accept either this or the nested
-    lists; a DDP step reuses the same gradient buffers every step, so building
-    the pointer array once keeps the per-bucket host cost to a few
-    microseconds."""
+    """The gradient tensors of all ranks (``grads[r][t]``), checked and with
+    their device pointers marshalled once.  Bucket calls accept either this or
+    the nested lists; a DDP step reuses the same gradient buffers every step,
+    so building the pointer array once keeps the per-bucket host cost to a
+    few microseconds.  Every rank must hold the same tensor sizes, all
+    contiguous CUDA tensors of one dtype on one device."""
 
     def __init__(self, grads: Sequence[Sequence]):
-        flat = [g for rank in grads for g in rank]
-        if not flat:
+        import weakref
+
+        if not grads or not grads[0]:
             raise ValueError("GradSet: no gradients")
+        first = grads[0][0]
+        numels = [int(g.numel()) for g in grads[0]]
+        for rank in grads:
+            if len(rank) != len(numels):
+                raise ValueError("GradSet: every rank needs the same number of tensors")
+            for t, g in enumerate(rank):
+                if not g.is_cuda or not g.is_contiguous() or g.device != first.device or g.dtype != first.dtype:
+                    raise ValueError("GradSet: gradients must be contiguous CUDA tensors of one dtype and device")
+                if g.numel() != numels[t]:
+                    raise ValueError(f"GradSet: tensor {t} has different sizes on different ranks")
         self.nranks = len(grads)
-        self.device = flat[0].device
-        self.ptrs = _ptr_array(flat)
+        self.numels = numels
+        self.dtype = _dtype_code(first.dtype)
+        self.device = first.device
+        self.ptrs = _ptr_array([g for rank in grads for g in rank])
         self._keep = [list(rank) for rank in grads]  # the tensors must outlive the pointers
+        self._plans = weakref.WeakSet()  # plans this set was checked against
 
 
 class BucketPlan:
@@ -217,6 +232,7 @@ class BucketPlan:
                                    ctypes.byref(handle)), "bucket_plan")
         self._h = handle
         self.numels = [int(m) for m in numels]
+        self.grad_dtype = _dtype_code(grad_dtype)
 
     def __del__(self):
         h = getattr(self, "_h", None)
@@ -241,12 +257,26 @@ class BucketPlan:
         check(lib().rr_bucket_tensor(self._h, t, ctypes.byref(b), ctypes.byref(o)), "bucket_tensor")
         return b.value, o.value
 
-    @staticmethod
-    def _grads(grads):
-        if isinstance(grads, GradSet):
-            return grads.ptrs, grads.nranks, grads.device
-        gs = GradSet(grads)
+    def _grads(self, grads):
+        """(pointers, nranks, device) of gradients that match this plan's
+        tensor sizes and dtype (checked once per GradSet and plan)."""
+        gs = grads if isinstance(grads, GradSet) else GradSet(grads)
+        if self not in gs._plans:
+            if gs.numels != self.numels or gs.dtype != self.grad_dtype:
+                raise ValueError("gradients do not match the bucket plan (tensor count, sizes or dtype)")
+            gs._plans.add(self)
         return gs.ptrs, gs.nranks, gs.device
+
+    def _buckets(self, bucket: int, buckets: Sequence, n: int, device):
+        """Pointer array of the fp32 bucket buffers, checked against the bucket's size."""
+        numel = self.info(bucket)[2]
+        if len(buckets) != n:
+            raise ValueError("one fp32 bucket buffer per rank")
+        for t in buckets:
+            if (not t.is_cuda or not t.is_contiguous() or t.device != device or _dtype_code(t.dtype) != 0
+                    or t.numel() < numel):
+                raise ValueError(f"bucket buffers must be contiguous fp32 CUDA tensors of at least {numel} elements")
+        return _ptr_array(buckets)
 
     def flat_buffers(self, nranks: int, device=None, dtype=None):
         """Gradients laid out as views into one flat buffer per bucket and
@@ -273,14 +303,14 @@ class BucketPlan:
     def pack(self, bucket: int, grads: Sequence[Sequence], buckets: Sequence, stream=None) -> None:
         """``grads[r][t]`` -> fp32 ``buckets[r]`` for the bucket's tensors."""
         g, n, dev = self._grads(grads)
-        check(lib().rr_bucket_pack(self._h, bucket, g, _ptr_array(buckets), n, _stream(stream, dev)),
-              "bucket_pack")
+        check(lib().rr_bucket_pack(self._h, bucket, g, self._buckets(bucket, buckets, n, dev), n,
+                                   _stream(stream, dev)), "bucket_pack")
 
     def unpack(self, bucket: int, buckets: Sequence, grads: Sequence[Sequence], op="avg", stream=None) -> None:
         """fp32 ``buckets[r]`` -> ``grads[r][t]`` (AVG divides by N)."""
         g, n, dev = self._grads(grads)
-        check(lib().rr_bucket_unpack(self._h, bucket, _ptr_array(buckets), g, n, _op(op), _stream(stream, dev)),
-              "bucket_unpack")
+        check(lib().rr_bucket_unpack(self._h, bucket, self._buckets(bucket, buckets, n, dev), g, n, _op(op),
+                                     _stream(stream, dev)), "bucket_unpack")
 
     def all_reduce(self, bucket: int, grads: Sequence[Sequence], op="avg", stream=None) -> None:
         """Fused pack + ring-order all-reduce + unpack, in place on ``grads``."""
@@ -307,6 +337,7 @@ class Reducer:
         import torch
 
         g = grads if isinstance(grads, GradSet) else GradSet(grads)
+        plan._grads(g)  # the gradients must match the plan
         # a high-priority stream lets bucket syncs start as soon as SMs free up
         self.comm = comm if comm is not None else torch.cuda.Stream(g.device, priority=-1)
         self._plan, self._grads = plan, g

@@ -285,3 +285,14 @@ def test_host_buffer_allreduce_checks_every_buffer():
     assert lib.rr_allreduce_host(dev, dev, 2, 16, 0, 0, 2, s) == _lib.RR_ERR_INVALID_ARG
     nulls = (ctypes.c_void_p * 2)(None, None)
     assert lib.rr_allreduce_host(nulls, dev, 2, 16, 0, 0, 2, s) == _lib.RR_ERR_INVALID_ARG
+
+
+def test_grad_set_checks_its_tensors():
+    import torch
+
+    with pytest.raises(ValueError):
+        rrv.GradSet([])
+    with pytest.raises(ValueError):
+        rrv.GradSet([[]])
+    with pytest.raises(ValueError):
+        rrv.GradSet([[torch.zeros(4)], [torch.zeros(4)]])  # not CUDA tensors

@@ -544,3 +544,35 @@ def test_wire_refuses_non_fp32_tensors():
         rrv.all_reduce_wire(d, "sum", "bf16", "oneshot")
     with pytest.raises(TypeError):
         rrv.all_reduce_wire(rrv.RankSet(d), "sum", "bf16", "oneshot")
+
+
+def test_bucket_calls_refuse_gradients_that_do_not_match_the_plan():
+    """Sizes, tensor count and dtype of the gradients, and the size of the
+    fp32 bucket buffers, are checked before anything is enqueued."""
+    numels = [100, 300, 50]
+    plan = rrv.BucketPlan(numels, "bf16", 1000)
+    good = [[torch.zeros(m, dtype=torch.bfloat16, device="cuda") for m in numels] for _ in range(2)]
+    plan.all_reduce(0, good, "avg")  # matches
+    short = [[torch.zeros(m - (t == 1), dtype=torch.bfloat16, device="cuda") for t, m in enumerate(numels)]
+             for _ in range(2)]
+    fewer = [[torch.zeros(m, dtype=torch.bfloat16, device="cuda") for m in numels[:2]] for _ in range(2)]
+    fp32 = [[torch.zeros(m, device="cuda") for m in numels] for _ in range(2)]
+    ragged = [good[0], [torch.zeros(m + 1, dtype=torch.bfloat16, device="cuda") for m in numels]]
+    for bad in (short, fewer, fp32):
+        with pytest.raises(ValueError):
+            plan.all_reduce(0, bad, "avg")
+        with pytest.raises(ValueError):
+            plan.all_reduce_range(0, plan.num_buckets, bad, "avg")
+        with pytest.raises(ValueError):
+            rrv.Reducer(plan, bad)
+    with pytest.raises(ValueError):
+        rrv.GradSet(ragged)
+    numel = plan.info(0)[2]
+    small = [torch.zeros(numel - 1, device="cuda") for _ in range(2)]
+    with pytest.raises(ValueError):
+        plan.pack(0, good, small)
+    with pytest.raises(ValueError):
+        plan.unpack(0, small, good, "avg")
+    gs = rrv.GradSet(good)
+    plan.all_reduce(0, gs, "avg")
+    plan.all_reduce(0, gs, "avg")  # checked once, reused
