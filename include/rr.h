@@ -71,7 +71,7 @@ typedef enum rr_status {
     RR_ERR_INVALID_ARG = 1,
     RR_ERR_UNSUPPORTED = 2,
     RR_ERR_CUDA = 3,
-    RR_ERR_TIMEOUT = 4 /* reserved: no kernel of this library waits on another */
+    RR_ERR_TIMEOUT = 4 /* a bounded device wait ran out (rr_check_timeouts) */
 } rr_status_t;
 
 /* Element types of the rank buffers: IEEE binary32, bfloat16 (the upper half
@@ -352,6 +352,17 @@ rr_status_t rr_set_picker_params(double launch_s, double hbm_bytes_per_s);
 /* ------------------------------------------------------------ utilities -- */
 
 rr_status_t rr_get_stats(rr_stats_t* out); /* last call on this host thread */
+
+/* Bounded waits.  The one-shot all-reduce stages its tiles in shared memory
+ * with bulk async copies when the rank count is 2, 4, 8 or 16 and every
+ * buffer and chunk is 16-byte aligned; its threads wait on an mbarrier for
+ * those copies with an iteration limit instead of forever.  A wait that runs
+ * out -- no working device lets it -- skips its tile (that tile's result is
+ * not written) and is counted on the device.  This call synchronises the
+ * device, then returns RR_ERR_TIMEOUT if any wait ran out since the last
+ * call (and clears the count), RR_OK otherwise.  No other kernel of the
+ * library waits on anything. */
+rr_status_t rr_check_timeouts(void);
 const char* rr_status_string(rr_status_t status);
 const char* rr_last_error(void); /* detail of the last failure on this thread */
 int rr_version(void);

@@ -21,7 +21,8 @@ from ._lib import MAX_RANKS, Cost, RingEvent, RRError, Stats, check, lib
 
 __all__ = [
     "all_reduce", "all_reduce_wire", "all_reduce_host", "ring_step", "ring_schedule", "reduce_scatter", "all_gather", "all_to_all",
-    "RankSet", "BucketPlan", "GradSet", "Reducer", "cost_model", "pick_algo", "set_picker_params", "last_stats", "RRError",
+    "RankSet", "BucketPlan", "GradSet", "Reducer", "cost_model", "pick_algo", "set_picker_params", "last_stats",
+    "check_timeouts", "RRError",
     "OPS", "ALGOS", "MAX_RANKS",
 ]
 
@@ -384,3 +385,10 @@ def last_stats() -> dict:
     out = {k: int(getattr(s, k)) for k, _ in Stats._fields_}
     out["algo"] = ALGO_NAMES.get(out["algo"], out["algo"])
     return out
+
+
+def check_timeouts() -> None:
+    """Synchronise the device and raise ``RRError`` (status RR_ERR_TIMEOUT)
+    if any bounded device wait ran out since the last check
+    (``rr_check_timeouts``)."""
+    check(lib().rr_check_timeouts(), "check_timeouts")

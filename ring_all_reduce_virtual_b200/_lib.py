@@ -79,6 +79,7 @@ def _declare(lib: ctypes.CDLL) -> None:
         "rr_pick_algo": (i, [i, sz, i]),
         "rr_set_picker_params": (st, [d, d]),
         "rr_get_stats": (st, [ctypes.POINTER(Stats)]),
+        "rr_check_timeouts": (st, []),
         "rr_status_string": (ctypes.c_char_p, [i]),
         "rr_last_error": (ctypes.c_char_p, []),
         "rr_version": (i, []),

@@ -1200,6 +1200,16 @@ rr_status_t rr_reducer_ready(rr_reducer_t* red, int tensor, cudaStream_t produce
     return bucket_fold_range(red->plan, b, 1, red->grads.data(), red->n, red->op, red->comm, red->max_grid);
 }
 
+rr_status_t rr_check_timeouts(void)
+{
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "synchronising before reading the wait counter");
+    unsigned int count = 0;
+    if ((e = take_bulk_timeouts(&count)) != cudaSuccess) return cuda_fail(e, "reading the wait counter");
+    if (count) return fail(RR_ERR_TIMEOUT, "bounded device waits ran out; their tiles were skipped");
+    return RR_OK;
+}
+
 rr_status_t rr_reducer_finish(rr_reducer_t* red, cudaStream_t stream)
 {
     if (!red) return fail(RR_ERR_INVALID_ARG, "NULL reducer");

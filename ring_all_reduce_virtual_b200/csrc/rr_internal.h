@@ -131,6 +131,9 @@ cudaError_t launch_step(int dtype, int op, const StepParams& p, cudaStream_t s);
 // step (wire 1: the step completes its chunks; 2: it does not).
 cudaError_t launch_oneshot_wire(int op, const RankParams& p, uint64_t work, cudaStream_t s);
 cudaError_t launch_step_wire(int op, int wire, const StepParams& p, cudaStream_t s);
+// Reads and clears the device-side count of bounded waits that ran out
+// (the bulk-copy one-shot's mbarrier waits).  Synchronous.
+cudaError_t take_bulk_timeouts(unsigned int* count);
 cudaError_t launch_bucket_pack(int grad_dtype, const BucketCopyParams& p, cudaStream_t s);
 cudaError_t launch_bucket_unpack(int grad_dtype, int op, const BucketCopyParams& p, cudaStream_t s);
 cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p, cudaStream_t s,

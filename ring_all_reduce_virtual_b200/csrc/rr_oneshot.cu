@@ -45,6 +45,7 @@ __global__ void __launch_bounds__(kThreads) oneshot_ring_kernel(const __grid_con
 template <class Ty, int OP>
 cudaError_t launch_oneshot_ring(const RankParams& p, uint64_t work, cudaStream_t s)
 {
+    if (bulk_eligible(p, (int)sizeof(typename Ty::T))) return launch_oneshot_bulk<Ty, OP>(p, s);
     const int n = p.n;
     constexpr int V = kVptReduce;
     switch (n) {

@@ -576,3 +576,51 @@ def test_bucket_calls_refuse_gradients_that_do_not_match_the_plan():
     gs = rrv.GradSet(good)
     plan.all_reduce(0, gs, "avg")
     plan.all_reduce(0, gs, "avg")  # checked once, reused
+
+
+# ------------------------------------------------- bulk-copy one-shot path --
+
+@pytest.mark.parametrize("n", [2, 4, 8, 16])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16", "i32"])
+@pytest.mark.parametrize("op", ["sum", "avg", "max", "min", "prod"])
+def test_bulk_copy_one_shot(n, dtype, op):
+    """Aligned buffers and chunks of whole 16-byte vectors take the one-shot
+    that stages tiles with bulk async copies.  count = n*C - (n-1) with C a
+    multiple of 8 makes the last chunk end n-1 elements short, inside a
+    vector, so the elements past its last whole vector take plain loads."""
+    if dtype == "i32" and op == "avg":
+        pytest.skip("AVG is not defined for int32")
+    C = 8 * 2000
+    count = n * C - (n - 1)
+    x, _ = _run(n, count, dtype, op, "oneshot", seed=50 + n)
+    rrv.check_timeouts()
+
+
+def test_bulk_copy_timeouts_are_reported_and_the_context_survives():
+    """With RR_DEBUG_BULK_TIMEOUT=1 every barrier expects 16 bytes more than
+    its copies bring, so every bounded wait runs out: the call returns, the
+    count shows up as RR_ERR_TIMEOUT, and the context still works."""
+    import os
+    import subprocess
+    import sys
+
+    script = r'''
+import torch, numpy as np
+import ring_all_reduce_virtual_b200 as rrv
+x = [torch.full((2048,), float(r + 1), device="cuda") for r in range(2)]
+rrv.all_reduce(x, "sum", "oneshot")  # bulk path: aligned, C = 1024 floats
+try:
+    rrv.check_timeouts()
+    print("NO TIMEOUT")
+except rrv.RRError as e:
+    print("TIMEOUT", e.status)
+rrv.check_timeouts()  # cleared
+y = [torch.full((2048,), float(r + 1), device="cuda") for r in range(3)]
+rrv.all_reduce(y, "sum", "ring")  # another path on the same context
+assert torch.all(y[0] == 6.0) and torch.all(y[2] == 6.0)
+print("CONTEXT OK")
+'''
+    env = dict(os.environ, RR_DEBUG_BULK_TIMEOUT="1")
+    out = subprocess.run([sys.executable, "-c", script], env=env, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert "TIMEOUT 4" in out.stdout and "CONTEXT OK" in out.stdout, out.stdout
