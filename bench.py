@@ -40,8 +40,8 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic of one launch of the dominant kernel per algorithmic byte,
 # from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), with the
 # hash of the dominant kernel's source files it was taken on.  The summary with its command is
-# in profiles/oneshot_ring_kernel_allreduce-8x64MiB-f32.md.
-NCU_TRAFFIC = {"per_algorithmic_byte": (536918272 + 479562496) / 1073741824, "sources_sha1": "6772def93fdf3d0fd41ebe5dea839b5f96e50b1b"}
+# in profiles/oneshot_bulk_kernel_allreduce-8x64MiB-f32.md.
+NCU_TRAFFIC = {"per_algorithmic_byte": (536887552 + 480653568) / 1073741824, "sources_sha1": "ccfb259091fe23483f348398df23f3711884604b"}
 
 
 # The files that define the dominant kernel (oneshot_bulk_kernel, dispatched
