@@ -354,7 +354,7 @@ rr_status_t rr_set_picker_params(double launch_s, double hbm_bytes_per_s);
 rr_status_t rr_get_stats(rr_stats_t* out); /* last call on this host thread */
 
 /* Bounded waits.  The one-shot all-reduce stages its tiles in shared memory
- * with bulk async copies when the rank count is 2, 4, 8 or 16 and every
+ * with bulk async copies when the rank count is 2, 4, 8, 16, 32 or 64 and every
  * buffer and chunk is 16-byte aligned; its threads wait on an mbarrier for
  * those copies with an iteration limit instead of forever.  A wait that runs
  * out -- no working device lets it -- skips its tile (that tile's result is

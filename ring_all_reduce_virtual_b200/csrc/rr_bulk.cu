@@ -7,7 +7,7 @@
 // It runs where the tiles are whole 16-byte vectors at 16-byte aligned
 // addresses: every buffer 16-byte aligned, the chunk size a multiple of 16
 // bytes, a plain in-place call, and a rank count fixed at compile time (2, 4,
-// 8, 16).  The few elements past a ragged chunk's last whole vector are
+// 8, 16, 32, 64).  The few elements past a ragged chunk's last whole vector are
 // folded with plain loads.  Same bits as oneshot_ring_kernel.  Measured on
 // 8 x 256 MiB fp32: 1.04-1.05 of the copy peak against 1.03 for the
 // per-thread loads.
@@ -30,7 +30,13 @@ namespace {
 
 __device__ unsigned int g_bulk_timeouts = 0;
 
-constexpr uint32_t kBulkSmem = 16384;  // bytes of input tiles per CTA (N tiles of kBulkSmem / N)
+// Bytes of input tiles per CTA (N tiles of bulk_smem<N>() / N): 16 KB, 32 KB
+// from 32 ranks on so that each rank's tile stays at least 512 bytes.
+template <int NS>
+__host__ __device__ constexpr uint32_t bulk_smem()
+{
+    return NS >= 32 ? 32768u : 16384u;
+}
 
 // Test hook, read once per process: RR_DEBUG_BULK_TIMEOUT=1 makes every
 // barrier expect 16 bytes more than its copies bring and bounds each wait at
@@ -85,7 +91,7 @@ __global__ void __launch_bounds__(kThreads) oneshot_bulk_kernel(const __grid_con
     using T = typename Ty::T;
     using Acc = typename Ty::Acc;
     constexpr int L = Ty::L;                       // elements per 16-byte vector
-    constexpr uint32_t TB = kBulkSmem / NS;        // bytes per rank per tile
+    constexpr uint32_t TB = bulk_smem<NS>() / NS;  // bytes per rank per tile
     constexpr uint32_t TV = TB / 16;               // vectors per tile
     static_assert(TB % 16 == 0 && TV >= 1, "tile of whole vectors");
     const RankParams& p = bp.r;
@@ -164,7 +170,7 @@ __global__ void __launch_bounds__(kThreads) oneshot_bulk_kernel(const __grid_con
 template <class Ty, int OP, int NS>
 cudaError_t launch_bulk(const RankParams& p, cudaStream_t s)
 {
-    constexpr uint64_t TE = (uint64_t)(kBulkSmem / NS / 16) * Ty::L;  // elements per tile
+    constexpr uint64_t TE = (uint64_t)(bulk_smem<NS>() / NS / 16) * Ty::L;  // elements per tile
     BulkParams bp{};
     bp.r = p;
     bp.r.tps = (p.C + TE - 1) / TE;
@@ -173,7 +179,7 @@ cudaError_t launch_bulk(const RankParams& p, cudaStream_t s)
     const uint64_t work = bp.r.nseg * bp.r.tps;
     if (work == 0) return cudaSuccess;
     if (work > kMaxGrid) return cudaErrorInvalidValue;  // never reached: bulk_eligible caps the grid
-    oneshot_bulk_kernel<Ty, OP, NS><<<(unsigned)work, kThreads, kBulkSmem, s>>>(bp);
+    oneshot_bulk_kernel<Ty, OP, NS><<<(unsigned)work, kThreads, bulk_smem<NS>(), s>>>(bp);
     return cudaGetLastError();
 }
 
@@ -181,12 +187,13 @@ cudaError_t launch_bulk(const RankParams& p, cudaStream_t s)
 
 bool bulk_eligible(const RankParams& p, int esize)
 {
-    if (p.n != 2 && p.n != 4 && p.n != 8 && p.n != 16) return false;
+    if (p.n != 2 && p.n != 4 && p.n != 8 && p.n != 16 && p.n != 32 && p.n != 64) return false;
     if (p.owner_only || p.lo != 0 || p.hi < p.count || p.nseg != (uint64_t)p.n) return false;
     if ((p.C * (uint64_t)esize) % 16 != 0) return false;
     for (int r = 0; r < p.n; ++r)
         if ((uintptr_t)p.in[r] % 16 != 0 || (uintptr_t)p.out[r] % 16 != 0) return false;
-    const uint64_t tiles = (p.C * (uint64_t)esize + kBulkSmem / p.n - 1) / (kBulkSmem / p.n);
+    const uint64_t tb = (p.n >= 32 ? 32768u : 16384u) / (uint64_t)p.n;  // bulk_smem<N>() / N
+    const uint64_t tiles = (p.C * (uint64_t)esize + tb - 1) / tb;
     return tiles * (uint64_t)p.n <= kMaxGrid;
 }
 
@@ -198,6 +205,8 @@ cudaError_t launch_oneshot_bulk(const RankParams& p, cudaStream_t s)
     case 4: return launch_bulk<Ty, OP, 4>(p, s);
     case 8: return launch_bulk<Ty, OP, 8>(p, s);
     case 16: return launch_bulk<Ty, OP, 16>(p, s);
+    case 32: return launch_bulk<Ty, OP, 32>(p, s);
+    case 64: return launch_bulk<Ty, OP, 64>(p, s);
     }
     return cudaErrorInvalidValue;
 }

@@ -13,7 +13,7 @@ template <class Ty, int OP>
 cudaError_t launch_oneshot_tree(const RankParams& p, uint64_t work, cudaStream_t s);
 
 // The bulk-copy one-shot (rr_bulk.cu): bulk_eligible says whether a one-shot
-// call can take it (rank count 2, 4, 8 or 16; 16-byte aligned buffers and
+// call can take it (rank count 2, 4, 8, 16, 32 or 64; 16-byte aligned buffers and
 // chunks; a plain call over whole chunks), launch_oneshot_bulk launches it
 // with its own tiling.
 bool bulk_eligible(const RankParams& p, int esize);

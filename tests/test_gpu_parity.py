@@ -580,7 +580,7 @@ def test_bucket_calls_refuse_gradients_that_do_not_match_the_plan():
 
 # ------------------------------------------------- bulk-copy one-shot path --
 
-@pytest.mark.parametrize("n", [2, 4, 8, 16])
+@pytest.mark.parametrize("n", [2, 4, 8, 16, 32, 64])
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16", "i32"])
 @pytest.mark.parametrize("op", ["sum", "avg", "max", "min", "prod"])
 def test_bulk_copy_one_shot(n, dtype, op):
