@@ -44,9 +44,10 @@ FALLBACK_HBM_GBS = 6650.0
 NCU_TRAFFIC = {"per_algorithmic_byte": (536887552 + 480653568) / 1073741824, "sources_sha1": "ccfb259091fe23483f348398df23f3711884604b"}
 
 
-# The files that define the dominant kernel (oneshot_bulk_kernel, dispatched
-# from the one-shot launcher).
-KERNEL_SOURCES = ("rr_device.cuh", "rr_internal.h", "rr_launch.cuh", "rr_oneshot.cuh", "rr_oneshot.cu", "rr_bulk.cu")
+# The files that define the dominant kernel (bulk_fold_kernel in ring order,
+# dispatched from the one-shot launcher).
+KERNEL_SOURCES = ("rr_device.cuh", "rr_internal.h", "rr_launch.cuh", "rr_oneshot.cuh", "rr_oneshot.cu", "rr_bulk.cuh",
+                  "rr_bulk.cu")
 
 
 def sources_sha1() -> str:
@@ -372,7 +373,7 @@ def run_ours(args, d: Dist):
             "hbm_gbs": round(achieved, 1), "hbm_frac": round(achieved / peak, 4),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,
-                         "kernel": "oneshot_bulk_kernel<F32T, AVG, N 8> (bulk-copy tiles, 2 KB per rank)",
+                         "kernel": "bulk_fold_kernel<F32T, AVG, N 8, ring order> (bulk-copy tiles, 2 KB per rank)",
                          "algorithmic_bytes_per_launch": alg_bytes, "peak_kind": peak_kind + " (burst copy)"},
             "cpu_baseline": cpu,
             "e2e": e2e,

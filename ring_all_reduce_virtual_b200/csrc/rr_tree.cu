@@ -202,6 +202,7 @@ __global__ void __launch_bounds__(kThreads) oneshot_tree_kernel(const __grid_con
 template <class Ty, int OP>
 cudaError_t launch_oneshot_tree(const RankParams& p, uint64_t work, cudaStream_t s)
 {
+    if (bulk_tree_eligible(p, (int)sizeof(typename Ty::T))) return launch_tree_bulk<Ty, OP>(p, s);
     const int n = p.n;
     constexpr int V = kVptReduce;
     switch (n) {

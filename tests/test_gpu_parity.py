@@ -624,3 +624,34 @@ print("CONTEXT OK")
     out = subprocess.run([sys.executable, "-c", script], env=env, capture_output=True, text=True, timeout=300)
     assert out.returncode == 0, out.stderr[-2000:]
     assert "TIMEOUT 4" in out.stdout and "CONTEXT OK" in out.stdout, out.stdout
+
+
+@pytest.mark.parametrize("n", [2, 4, 8, 16])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16", "i32"])
+@pytest.mark.parametrize("op", ["sum", "avg", "max", "min", "prod"])
+def test_bulk_copy_reduce_scatter_and_tree_order(n, dtype, op):
+    """Parts (reduce-scatter) and buffers (tree order) of whole 16-byte vectors
+    at aligned addresses take the bulk-copy kernels: same bits as the oracle."""
+    if dtype == "i32" and op == "avg":
+        pytest.skip("AVG is not defined for int32")
+    per = 8 * 1500
+    x = synth.ranks(60 + n, n, n * per, _dist(op, dtype), dtype)
+    rs = empty_like_ranks(n, per, dtype)
+    rrv.reduce_scatter(to_dev(x), rs, op)
+    assert_bits_equal(to_host(rs), oracle.reduce_scatter([a.copy() for a in x], op), f"bulk rs {op}")
+    _run(n, n * per, dtype, op, "tree_oneshot", seed=70 + n)
+    rrv.check_timeouts()
+
+
+@pytest.mark.parametrize("n", [2, 4, 8, 16, 32, 64])
+@pytest.mark.parametrize("op", ["sum", "avg"])
+def test_bulk_copy_bf16_wire(n, op):
+    C = 8 * 2000
+    count = n * C - (n - 1)  # a ragged last chunk: its last elements take plain loads
+    x = synth.ranks(80 + n, n, count, "uniform")
+    want = [a.copy() for a in x]
+    oracle.fold_wire(want, op)
+    d = to_dev(x)
+    rrv.all_reduce_wire(d, op, "bf16", "oneshot")
+    assert_bits_equal(to_host(d), want, f"bulk wire n={n}")
+    rrv.check_timeouts()
