@@ -655,3 +655,20 @@ def test_bulk_copy_bf16_wire(n, op):
     rrv.all_reduce_wire(d, op, "bf16", "oneshot")
     assert_bits_equal(to_host(d), want, f"bulk wire n={n}")
     rrv.check_timeouts()
+
+
+@pytest.mark.parametrize("n", [2, 3, 8, 64])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16", "i32"])
+def test_aligned_all_gather_and_two_shot(n, dtype):
+    """Parts of whole 16-byte vectors at aligned addresses (the vector path
+    with no scalar head or tail) for the all-gather and the two-shot; the
+    two-shot count leaves a short last chunk."""
+    per = 8 * 1500
+    x = synth.ranks(90 + n, n, per, "int" if dtype == "i32" else "uniform", dtype)
+    ag = empty_like_ranks(n, n * per, dtype)
+    rrv.all_gather(to_dev(x), ag)
+    assert_bits_equal(to_host(ag), oracle.all_gather(x), f"bulk ag n={n}")
+    if n <= 8:
+        count = n * per - 8 * (n - 1)  # C = per: the last chunk is 8(N-1) elements short
+        _run(n, count, dtype, "sum", "two_shot", seed=95 + n)
+    rrv.check_timeouts()
