@@ -40,8 +40,8 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic of one launch of the dominant kernel per algorithmic byte,
 # from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), with the
 # hash of the dominant kernel's source files it was taken on.  The summary with its command is
-# in profiles/oneshot_bulk_kernel_allreduce-8x64MiB-f32.md.
-NCU_TRAFFIC = {"per_algorithmic_byte": (536887552 + 480653568) / 1073741824, "sources_sha1": "ccfb259091fe23483f348398df23f3711884604b"}
+# in profiles/bulk_fold_kernel_allreduce-8x64MiB-f32.md.
+NCU_TRAFFIC = {"per_algorithmic_byte": (536887808 + 479330048) / 1073741824, "sources_sha1": "5b3e20e931e6036514d429e7eb80ceb98afeb6f4"}
 
 
 # The files that define the dominant kernel (bulk_fold_kernel in ring order,
