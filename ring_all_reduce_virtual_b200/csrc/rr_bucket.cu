@@ -9,8 +9,7 @@
 // s3.3 (gradients fill buckets in order; a full bucket triggers its
 // all-reduce); [P3] "Training gradient sync and collective communication"
 // (geek-doc.cn), section 5 (bucketing hides the per-message latency).
-#include "rr_device.cuh"
-#include "rr_internal.h"
+#include "rr_bulk.cuh"
 
 namespace rr {
 
@@ -191,6 +190,150 @@ __global__ void __launch_bounds__(kThreads) bucket_fold_kernel(const __grid_cons
     }
 }
 
+// The fused bucket sync with its tiles staged by bulk async copies (the
+// fold of rr_bulk.cuh: one elected thread copies the N ranks' tiles into
+// shared memory behind a bounded mbarrier wait, the CTA folds them in ring
+// order, the thread bulk-stores the result to every rank).  A segment starts
+// at any element, so tile 0 folds the elements before the segment's first
+// 16-byte boundary and after its last whole vector with plain loads, and the
+// bulk copies move the whole vectors between.  Needs every rank's copy of a
+// tensor at the same address modulo 16 (vec_ok) and N = 2, 4, 8 or 16.
+struct BucketBulkParams {
+    BucketFoldParams f;  // tile0 counts bulk tiles (bucket_bulk_tile_elems)
+    unsigned int* timeouts;
+    uint32_t extra_tx;
+    uint32_t spin;
+};
+static_assert(sizeof(BucketBulkParams) <= 32764, "BucketBulkParams too large");
+
+template <class G, int OP, int NS>
+__global__ void __launch_bounds__(kThreads) bucket_bulk_kernel(const __grid_constant__ BucketBulkParams bp)
+{
+    using T = typename G::T;
+    using Acc = typename G::Acc;
+    constexpr int L = G::L;
+    constexpr uint32_t TV = bulk_smem<NS>() / NS / 16;  // vectors per rank per tile
+    const BucketFoldParams& p = bp.f;
+    extern __shared__ __align__(128) uint4 sm[];       // [NS][TV]: slot j holds rank (c + j) mod N
+    __shared__ __align__(8) uint64_t bar;
+
+    const uint64_t w = blockIdx.x;
+    const int s = find_segment(p.tile0, p.nseg, w);
+    const uint64_t tile = w - p.tile0[s];
+    const BucketSeg& sg = p.seg[s];
+    const int base = (int)sg.t * NS;
+    const int start = (int)sg.c;
+    auto in = [&](int j) {
+        int r = start + j;
+        if (r >= NS) r -= NS;
+        return static_cast<const T*>(p.grad[base + r]) + sg.off;
+    };
+    auto out = [&](int o) { return static_cast<T*>(p.grad[base + o]) + sg.off; };
+    const uint64_t len = sg.len;
+    uint64_t head = (uint64_t)((L - phase_of(in(0), L)) & (L - 1));
+    if (head > len) head = len;
+    const uint64_t nv = (len - head) / L;
+    const uint64_t tail = len - head - nv * L;
+    if (tile == 0 && (uint64_t)threadIdx.x < head + tail) {
+        const uint64_t e = (uint64_t)threadIdx.x < head ? (uint64_t)threadIdx.x : head + nv * L + (threadIdx.x - head);
+        fold_one<G, OP, 0>(in, NS, out, NS, e, p.divisor);
+    }
+    const uint64_t v0 = tile * TV;
+    if (v0 >= nv) return;
+    const uint32_t nvt = (uint32_t)(nv - v0 < TV ? nv - v0 : TV);
+    const uint32_t bytes = nvt * 16u;
+    const uint64_t e0 = head + v0 * L;  // 16-byte aligned in every rank's copy
+
+    const uint32_t b = bulk_smem_addr(&bar);
+    if (threadIdx.x == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(b) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
+                     ::"r"(b), "r"(bytes * NS + bp.extra_tx) : "memory");
+#pragma unroll
+        for (int j = 0; j < NS; ++j)
+            asm volatile(
+                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                ::"r"(bulk_smem_addr(sm + j * TV)), "l"(in(j) + e0), "r"(bytes), "r"(b)
+                : "memory");
+    }
+    if (!bulk_bar_wait(b, 0, bp.spin)) {
+        if (threadIdx.x == 0) atomicAdd(bp.timeouts, 1u);
+        bulk_bar_wait(b, 0, bp.spin);  // once more for the copies in flight, then leave the tile
+        return;
+    }
+    for (uint32_t v = threadIdx.x; v < nvt; v += kThreads) {
+        Acc a[L];
+        G::unpack(sm[v], a);
+#pragma unroll
+        for (int j = 1; j < NS; ++j) {
+            Acc x[L];
+            G::unpack(sm[j * TV + v], x);
+#pragma unroll
+            for (int l = 0; l < L; ++l) a[l] = apply<OP>(a[l], x[l]);
+        }
+#pragma unroll
+        for (int l = 0; l < L; ++l) a[l] = finish_n<OP, NS>(a[l], p.divisor);
+        sm[v] = G::pack(a);  // one rounding to the gradient type, into slot 0
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int o = 0; o < NS; ++o)
+            asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                         ::"l"(out(o) + e0), "r"(bulk_smem_addr(sm)), "r"(bytes)
+                         : "memory");
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+    }
+}
+
+// Elements per bulk tile of the bucket sync: the whole vectors of one rank's
+// share of bulk_smem<N>().
+uint64_t bucket_bulk_tile_elems(int grad_dtype, int n)
+{
+    const uint64_t bytes = (n >= 32 ? 32768u : 16384u) / (uint64_t)n;
+    return bytes / 16 * (grad_dtype == kF32 ? 4u : 8u);
+}
+
+template <class G, int OP>
+cudaError_t launch_bucket_bulk(const BucketFoldParams& p, int grad_dtype, cudaStream_t s, bool* launched)
+{
+    *launched = false;
+    const BulkParams wait = bulk_params(RankParams{});
+    if (!wait.timeouts) return cudaSuccess;
+    auto* bp = new BucketBulkParams();
+    bp->f = p;
+    bp->timeouts = wait.timeouts;
+    bp->extra_tx = wait.extra_tx;
+    bp->spin = wait.spin;
+    const uint64_t te = bucket_bulk_tile_elems(grad_dtype, p.n);
+    bp->f.tile0[0] = 0;
+    for (int i = 0; i < p.nseg; ++i)  // every non-empty segment has a tile 0 for its head and tail
+        bp->f.tile0[i + 1] = bp->f.tile0[i] + (p.seg[i].len ? (p.seg[i].len + te - 1) / te : 0);
+    const uint64_t work = bp->f.tile0[p.nseg];
+    cudaError_t e = cudaSuccess;
+    if (work > 0 && work <= kMaxGrid) {
+        *launched = true;
+        switch (p.n) {
+        case 2: bucket_bulk_kernel<G, OP, 2><<<(unsigned)work, kThreads, bulk_smem<2>(), s>>>(*bp); break;
+        case 4: bucket_bulk_kernel<G, OP, 4><<<(unsigned)work, kThreads, bulk_smem<4>(), s>>>(*bp); break;
+        case 8: bucket_bulk_kernel<G, OP, 8><<<(unsigned)work, kThreads, bulk_smem<8>(), s>>>(*bp); break;
+        case 16: bucket_bulk_kernel<G, OP, 16><<<(unsigned)work, kThreads, bulk_smem<16>(), s>>>(*bp); break;
+        default: *launched = false;
+        }
+        if (*launched) e = cudaGetLastError();
+    } else if (work == 0) {
+        *launched = true;
+    }
+    delete bp;
+    return e;
+}
+
 template <class P>
 cudaError_t launch_all_b(void (*kernel)(P), const P& p, uint64_t work, cudaStream_t s, uint64_t max_grid = kMaxGrid)
 {
@@ -250,6 +393,21 @@ cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p
 {
     const uint64_t work = p.tile0[p.nseg];
     const bool avg = op == kAvg;
+    // the bulk-copy fold when it applies (no CTA cap: one CTA per tile)
+    if (max_grid >= kMaxGrid && p.vec_ok && (p.n == 2 || p.n == 4 || p.n == 8 || p.n == 16)) {
+        bool launched = false;
+        cudaError_t e = cudaSuccess;
+        if (grad_dtype == kBF16)
+            e = avg ? launch_bucket_bulk<BF16T, kAvg>(p, grad_dtype, s, &launched)
+                    : launch_bucket_bulk<BF16T, kSum>(p, grad_dtype, s, &launched);
+        else if (grad_dtype == kF16)
+            e = avg ? launch_bucket_bulk<F16T, kAvg>(p, grad_dtype, s, &launched)
+                    : launch_bucket_bulk<F16T, kSum>(p, grad_dtype, s, &launched);
+        else if (grad_dtype == kF32)
+            e = avg ? launch_bucket_bulk<F32T, kAvg>(p, grad_dtype, s, &launched)
+                    : launch_bucket_bulk<F32T, kSum>(p, grad_dtype, s, &launched);
+        if (e != cudaSuccess || launched) return e;
+    }
     if (grad_dtype == kBF16)
         return avg ? launch_fold<BF16T, kAvg>(p, work, s, max_grid) : launch_fold<BF16T, kSum>(p, work, s, max_grid);
     if (grad_dtype == kF16)

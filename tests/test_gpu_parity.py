@@ -672,3 +672,34 @@ def test_aligned_all_gather_and_two_shot(n, dtype):
         count = n * per - 8 * (n - 1)  # C = per: the last chunk is 8(N-1) elements short
         _run(n, count, dtype, "sum", "two_shot", seed=95 + n)
     rrv.check_timeouts()
+
+
+@pytest.mark.parametrize("n", [2, 4, 8, 16])
+@pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
+def test_bucket_sync_bulk_path_with_heads_and_tails(n, dtype):
+    """Tensors at odd element offsets, the same on every rank: the fused
+    bucket sync takes the bulk-copy fold, whose tile 0 folds each segment's
+    elements before its first 16-byte boundary and after its last whole
+    vector with plain loads."""
+    numels = [7, 1001, 3, 2500, 64, 12345, 1]
+    es = 4 if dtype == "f32" else 2
+    host = _grad_set(13, n, numels, dtype)
+    want = [[g.copy() for g in rank] for rank in host]
+    cap = 3000 * es
+    oracle.bucket_sync(want, cap, "avg")
+    plan = rrv.BucketPlan(numels, dtype, cap)
+    td = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[dtype]
+    grads = []
+    for r in range(n):
+        flat = torch.zeros(sum(numels) + 8 * len(numels) + 8, dtype=td, device="cuda")
+        ts, o = [], 1  # every rank: the same odd offsets
+        for g in host[r]:
+            t = flat[o:o + g.size]
+            t.copy_(torch.from_numpy(g.view(np.int16) if dtype == "bf16" else g).cuda().view(td))
+            ts.append(t)
+            o += g.size + 3
+        grads.append(ts)
+    plan.all_reduce_range(0, plan.num_buckets, grads, "avg")
+    for r in range(n):
+        assert_bits_equal(to_host(grads[r]), want[r], f"rank {r}")
+    rrv.check_timeouts()
