@@ -11,6 +11,7 @@
 // sections "Ring all-reduce and communication volume" and "alpha-beta model".
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "rr_bulk.cuh"
 
@@ -43,13 +44,21 @@ const BulkDebug& bulk_debug()
     return d;
 }
 
+// The counter's address on the current device (each device holds its own
+// copy of the module's variables), looked up once per device.
 unsigned int* timeout_counter()
 {
-    static unsigned int* ptr = [] {
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static unsigned int* ptr[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptr[dev]) {
         void* p = nullptr;
-        return cudaGetSymbolAddress(&p, g_bulk_timeouts) == cudaSuccess ? static_cast<unsigned int*>(p) : nullptr;
-    }();
-    return ptr;
+        if (cudaGetSymbolAddress(&p, g_bulk_timeouts) == cudaSuccess) ptr[dev] = static_cast<unsigned int*>(p);
+    }
+    return ptr[dev];
 }
 
 uint64_t bulk_tile_bytes(int n) { return (n >= 32 ? 32768u : 16384u) / (uint64_t)n; }  // bulk_smem<N>() / N
