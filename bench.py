@@ -41,7 +41,7 @@ FALLBACK_HBM_GBS = 6650.0
 # from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), with the
 # hash of the dominant kernel's source files it was taken on.  The summary with its command is
 # in profiles/bulk_fold_kernel_allreduce-8x64MiB-f32.md.
-NCU_TRAFFIC = {"per_algorithmic_byte": (536887808 + 479330048) / 1073741824, "sources_sha1": "5b3e20e931e6036514d429e7eb80ceb98afeb6f4"}
+NCU_TRAFFIC = {"per_algorithmic_byte": (536886784 + 479816704) / 1073741824, "sources_sha1": "a50fff8d140ae15085d173571f96b2498ff29a4d"}
 
 
 # The files that define the dominant kernel (bulk_fold_kernel in ring order,
