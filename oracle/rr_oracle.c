@@ -745,17 +745,29 @@ int orc_tree_fold(void** bufs, int n, size_t count, int dtype, int op)
     if (!valid(n, dtype, op)) return ORC_EINVAL;
     float* v = (float*)malloc((size_t)n * sizeof *v);
     int32_t* w = (int32_t*)malloc((size_t)n * sizeof *w);
-    if (!v || !w) { free(v); free(w); return ORC_ENOMEM; }
+    char* alive = (char*)malloc((size_t)n);
+    if (!v || !w || !alive) { free(v); free(w); free(alive); return ORC_ENOMEM; }
     for (size_t e = 0; e < count; ++e) {
         for (int r = 0; r < n; ++r) {
             if (dtype == ORC_I32) w[r] = ((int32_t*)bufs[r])[e];
             else v[r] = ld_f(bufs[r], dtype, e);
+            alive[r] = 1;
         }
-        for (int h = 1; h < n; h *= 2)
+        for (int h = 1; h < n; h *= 2) {
             for (int i = 0; i + h < n; i += 2 * h) {
+                if (!alive[i + h]) continue;
                 if (dtype == ORC_I32) w[i] = op_i32(op, w[i], w[i + h]);
                 else v[i] = op_f32(op, v[i], v[i + h]);
             }
+            if (MUTANT(13)) {  /* the unpaired rank joins the pair before it at this level */
+                int i = ((n - 1) / (2 * h)) * (2 * h);
+                if (i + h >= n && i > 0 && alive[i]) {
+                    if (dtype == ORC_I32) w[i - 2 * h] = op_i32(op, w[i - 2 * h], w[i]);
+                    else v[i - 2 * h] = op_f32(op, v[i - 2 * h], v[i]);
+                    alive[i] = 0;
+                }
+            }
+        }
         for (int r = 0; r < n; ++r) {
             if (dtype == ORC_I32) ((int32_t*)bufs[r])[e] = w[0];
             else st_f(bufs[r], dtype, e, finish_f32(op, v[0], n));
@@ -763,6 +775,7 @@ int orc_tree_fold(void** bufs, int n, size_t count, int dtype, int op)
     }
     free(v);
     free(w);
+    free(alive);
     return ORC_OK;
 }
 

@@ -367,6 +367,32 @@ def test_tree_pairwise_order_on_rounding_fixture():
     assert np.array_equal(x[2], y[2])
 
 
+def _tree_unpaired_cases():
+    for ln in golden_lines("tree_order_unpaired.txt"):
+        n, xs, want = ln.split(":")
+        yield int(n), [np.float32(float(v)) for v in xs.split()], float(want)
+
+
+def test_tree_order_with_unpaired_ranks_golden():
+    """The hand-derived fixture pins where a rank without a partner joins the
+    pairwise tree (N = 3, 5, 6, 7), for the tree schedule and its fused form."""
+    for n, xs, want in _tree_unpaired_cases():
+        assert len(xs) == n
+        for path in (oracle.tree_schedule, oracle.tree_fold):
+            x = [np.array([v], dtype=np.float32) for v in xs]
+            path(x, "sum")
+            for r in range(n):
+                assert float(x[r][0]) == want, (path.__name__, n, r, float(x[r][0]))
+
+
+def test_tree_unpaired_mutant_is_caught():
+    # kind 13: the unpaired rank joins the pair before it at the same level
+    with oracle.mutant(13):
+        with pytest.raises(AssertionError):
+            test_tree_order_with_unpaired_ranks_golden()
+    test_tree_order_with_unpaired_ranks_golden()
+
+
 # ------------------------------------------------------------------- bf16 --
 
 def test_bf16_rounding_matches_torch():
