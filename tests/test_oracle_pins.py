@@ -448,6 +448,32 @@ def _check_plan(numels, es, cap, b, off, nb):
             assert sum(sizes[:-1]) < cap
 
 
+def test_bucket_plan_invariants_admit_only_the_greedy_partition():
+    """The invariants determine the plan: every other contiguous partition of
+    a small example fails them (bf16, cap 60 bytes: 10 and 20 elements fill
+    the first bucket exactly, 30 and 40 are buckets of their own)."""
+    import itertools
+
+    numels, es, cap = [10, 20, 30, 40], 2, 60
+    b, off, nb = oracle.bucket_plan(numels, es, cap)
+    assert list(b) == [0, 0, 1, 2]
+    passing = []
+    for cuts in itertools.product([0, 1], repeat=len(numels) - 1):  # 1 = a new bucket after tensor t
+        bb = [0]
+        for c in cuts:
+            bb.append(bb[-1] + c)
+        oo, run = [], {}
+        for t, k in enumerate(bb):
+            oo.append(run.get(k, 0))
+            run[k] = run.get(k, 0) + numels[t]
+        try:
+            _check_plan(numels, es, cap, np.array(bb), np.array(oo, dtype=np.uint64), bb[-1] + 1)
+            passing.append(bb)
+        except AssertionError:
+            pass
+    assert passing == [[0, 0, 1, 2]]
+
+
 @pytest.mark.parametrize("cap", [0, 1, 100, 4096, 10 ** 9])
 def test_bucket_plan_invariants_random(cap):
     rng = np.random.default_rng(cap)
