@@ -353,14 +353,15 @@ rr_status_t rr_set_picker_params(double launch_s, double hbm_bytes_per_s);
 
 rr_status_t rr_get_stats(rr_stats_t* out); /* last call on this host thread */
 
-/* Bounded waits.  The one-shot all-reduce stages its tiles in shared memory
- * with bulk async copies when the rank count is 2, 4, 8, 16, 32 or 64 and every
- * buffer and chunk is 16-byte aligned; its threads wait on an mbarrier for
- * those copies with an iteration limit instead of forever.  A wait that runs
- * out -- no working device lets it -- skips its tile (that tile's result is
- * not written) and is counted on the device.  This call synchronises the
- * device, then returns RR_ERR_TIMEOUT if any wait ran out since the last
- * call (and clears the count), RR_OK otherwise.  No other kernel of the
+/* Bounded waits.  The one-shot all-reduce (rank count 2, 4, 8, 16, 32 or 64),
+ * the reduce-scatter, the tree-order one-shot and the fused bucket sync (2-16
+ * ranks) stage their tiles in shared memory with bulk async copies when the
+ * buffers are 16-byte aligned; their threads wait on an mbarrier for those
+ * copies with an iteration limit instead of forever.  A wait that runs out --
+ * no working device lets it -- skips its tile (that tile's result is not
+ * written) and is counted on the device.  This call synchronises the current
+ * device, then returns RR_ERR_TIMEOUT if any wait ran out there since the
+ * last call (and clears the count), RR_OK otherwise.  No other kernel of the
  * library waits on anything. */
 rr_status_t rr_check_timeouts(void);
 const char* rr_status_string(rr_status_t status);
