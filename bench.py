@@ -455,13 +455,34 @@ def time_extra(dev, stream, host, S, peak):
     return extra
 
 
+def fit_alpha_beta(rows):
+    """Least-squares fit of the alpha-beta model to the sweep ([P3] section 4:
+    time = steps * alpha + bytes / beta; on one GPU a step is a launch and the
+    bytes are HBM bytes): per call from Python, and per call inside a CUDA
+    graph (small sizes).  Prints one JSON line; rr_set_picker_params takes
+    such a pair."""
+    import numpy as np
+
+    out = {"workload": "size-sweep-f32-sum", "fit": "alpha-beta, least squares over every point (launches, HBM bytes)"}
+    for key, idx in (("per_call", 2), ("in_graph", 3)):
+        pts = [(r[0], r[1], r[idx]) for r in rows if r[idx] is not None]
+        if len(pts) < 3:
+            continue
+        a = np.array([[p[0], p[1]] for p in pts], dtype=float)
+        y = np.array([p[2] for p in pts], dtype=float)
+        sol = np.linalg.lstsq(a, y, rcond=None)[0]
+        if sol[1] > 0:
+            out[key] = {"alpha_us": round(sol[0] * 1e6, 3), "beta_gbs": round(1 / sol[1] / 1e9, 1), "points": len(pts)}
+    print(json.dumps(out), flush=True)
+
+
 def run_sweep(args):
     """Message-size sweep: 1 KiB .. 1 GiB per rank, N in {2, 4, 8, 16}, fp32
     SUM, every algorithm.  Per point: median per-call device time over 20
     calls after 5 warm-ups, and for sizes up to 1 MiB the same through a
     RankSet (pointers marshalled once) and the per-call time of a CUDA graph
     holding 100 calls.  Points whose 2 N S bytes fit in L2 are
-    flagged."""
+    flagged.  The last line is the alpha-beta fit of these points."""
     import torch
 
     import ring_all_reduce_virtual_b200 as rrv
@@ -471,6 +492,7 @@ def run_sweep(args):
     dev = torch.device("cuda", 0)
     stream = torch.cuda.Stream(dev)
     peak, _ = hbm_peak()
+    fit_rows = []  # (launches, HBM bytes, seconds per call, seconds per call in a graph)
     for n in (2, 4, 8, 16):
         for e in range(10, 31):
             nbytes = 1 << e
@@ -518,6 +540,7 @@ def run_sweep(args):
                         graph_us = a.elapsed_time(b) * 1e3 / 500
                         del g
                 algbw = nbytes / t / 1e9
+                fit_rows.append((st["launches"], st["hbm_bytes"], t, None if graph_us is None else graph_us * 1e-6))
                 print(json.dumps({
                     "workload": "size-sweep-f32-sum", "nranks_virtual": n, "bytes_per_rank": nbytes, "algo": algo,
                     "latency_us": round(t * 1e6, 3),
@@ -528,6 +551,7 @@ def run_sweep(args):
                     "launches": st["launches"], "l2_resident": 2 * n * nbytes <= 126 * 10**6}), flush=True)
             del bufs
             torch.cuda.empty_cache()
+    fit_alpha_beta(fit_rows)
 
 
 def run_gpt_buckets(args):
