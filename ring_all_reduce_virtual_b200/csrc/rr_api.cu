@@ -9,6 +9,7 @@
 //        server to Ring AllReduce" (geek-doc.cn)
 //   [P4] "Collective communication primitives" (ai-infra-handbooks)
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
@@ -40,8 +41,9 @@ namespace {
 thread_local rr_stats_t t_stats{};
 thread_local std::string t_error;
 
-double g_launch_s = 4e-6;         // picker: cost of one launch
-double g_hbm_bps = 6.5e12;        // picker: effective HBM bytes/s
+// Picker parameters, set by rr_set_picker_params from any thread.
+std::atomic<double> g_launch_s{4e-6};    // cost of one launch
+std::atomic<double> g_hbm_bps{6.5e12};   // effective HBM bytes/s
 
 rr_status_t fail(rr_status_t st, const std::string& why)
 {
@@ -1270,8 +1272,8 @@ rr_status_t rr_cost_model(rr_algo_t algo, int nranks, double bytes, double alpha
 rr_status_t rr_set_picker_params(double launch_s, double hbm_bytes_per_s)
 {
     if (!(launch_s >= 0) || !(hbm_bytes_per_s > 0)) return fail(RR_ERR_INVALID_ARG, "bad picker parameters");
-    g_launch_s = launch_s;
-    g_hbm_bps = hbm_bytes_per_s;
+    g_launch_s.store(launch_s);
+    g_hbm_bps.store(hbm_bytes_per_s);
     return RR_OK;
 }
 
@@ -1284,9 +1286,10 @@ rr_algo_t rr_pick_algo(int nranks, size_t count, rr_dtype_t dtype)
 {
     if (dtype == RR_BF16 || dtype == RR_F16 || nranks <= 1) return RR_ALGO_ONESHOT;
     const double n = nranks, S = (double)count * (double)esize(dtype);
-    const double ring = 2 * (n - 1) * g_launch_s + 5 * (n - 1) * S / g_hbm_bps;
-    const double one = g_launch_s + 2 * n * S / g_hbm_bps;
-    const double two = 2 * g_launch_s + (2 * n + 1) * S / g_hbm_bps;
+    const double alpha = g_launch_s.load(), beta = g_hbm_bps.load();
+    const double ring = 2 * (n - 1) * alpha + 5 * (n - 1) * S / beta;
+    const double one = alpha + 2 * n * S / beta;
+    const double two = 2 * alpha + (2 * n + 1) * S / beta;
     if (ring < one && ring < two) return RR_ALGO_RING;
     return two < one ? RR_ALGO_TWO_SHOT : RR_ALGO_ONESHOT;
 }
