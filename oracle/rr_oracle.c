@@ -400,7 +400,7 @@ int orc_ring_allreduce_omp(void** bufs, int n, size_t count, int dtype, int op, 
                 int left = mod(r - 1, n);
                 int k = send_chunk(phase, left, s, n);
                 size_t len = orc_chunk_len(count, n, k), off = (size_t)k * C;
-                unsigned char* m = msgs + (size_t)left * C * es;
+                unsigned char* m = msgs + (size_t)(MUTANT(14) ? r : left) * C * es;
                 if (phase == ORC_PHASE_AG) {
                     memcpy((unsigned char*)bufs[r] + off * es, m, len * es);
                     continue;
@@ -658,7 +658,7 @@ int orc_fold_samples(const void* vals, int n, size_t m, const int32_t* start, in
         } else {
             float acc = ld_f(vals, dtype, (size_t)c * m + j);
             for (int k = 1; k < n; ++k) acc = op_f32(op, acc, ld_f(vals, dtype, (size_t)mod(c + k, n) * m + j));
-            st_f(out, dtype, j, finish_f32(op, acc, n));
+            st_f(out, dtype, j, MUTANT(15) ? acc : finish_f32(op, acc, n));
         }
     }
     return ORC_OK;

@@ -6,6 +6,8 @@ invariant, a library routine on a case that reduces to it, an error bound, or
 brute force on tiny inputs.  ``test_mutants_are_caught`` then shows that each
 planted mistake in the oracle fails at least one of these pins.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -292,6 +294,64 @@ def test_ring_steps_equal_direct_fold_fp32(n, op):
             assert np.array_equal(x[r].view(np.uint32), x[0].view(np.uint32))
 
 
+# ---------------------- the timed ring and the sampled fold vs the pinned ones --
+# ``ring_allreduce_omp`` (the timed CPU baseline) and ``fold_samples`` (the
+# checker of every sampled full-size GPU test) are separate code in the C
+# file.  Each is held here to a pinned path bit for bit: the OpenMP ring to
+# the message-stepping ring, the sampled fold to the whole-buffer fold.
+
+def _draw(seed, n, count, op, dtype):
+    dist = "int" if dtype == "i32" else ("prod" if op == "prod" else "uniform")
+    return synth.ranks(seed, n, count, dist, dtype)
+
+
+def _ops_for(dtype):
+    return ["sum", "max", "min", "prod"] + ([] if dtype == "i32" else ["avg"])
+
+
+def _omp_matches(n, dtype, threads=(1, 4)):
+    for op in _ops_for(dtype):
+        for count in (0, 1, n + 1, 3 * n + 2, 1000):
+            x = _draw(11, n, count, op, dtype)
+            want = [v.copy() for v in x]
+            oracle.ring_allreduce(want, op)
+            for nt in threads:
+                got = [v.copy() for v in x]
+                oracle.ring_allreduce_omp(got, op, nt)
+                for r in range(n):
+                    assert np.array_equal(got[r].view(np.uint8), want[r].view(np.uint8)), (op, count, nt, r)
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 5, 8, 13, 64])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16", "i32"])
+def test_ring_omp_equals_the_pinned_ring(n, dtype):
+    # ragged (n + 1, 3n + 2, 1000) and empty counts, every op, one thread and
+    # several: the parallel transfers of a step give the stepping ring's bits
+    _omp_matches(n, dtype, (1, 4, os.cpu_count() or 1))
+
+
+def _samples_match(n, dtype, m=200):
+    count = 7 * n + 3  # ragged last chunk
+    C = oracle.chunk_size(count, n)
+    rng = np.random.default_rng([n, 12])
+    idx = rng.integers(0, count, size=m)
+    idx[:3] = [0, count - 1, min(C, count - 1)]  # first, last, a chunk boundary
+    for op in _ops_for(dtype):
+        x = _draw(12, n, count, op, dtype)
+        want = [v.copy() for v in x]
+        oracle.fold_ring_order(want, op)
+        vals = np.stack(x)[:, idx]
+        got = oracle.fold_samples(vals, idx // C, op)
+        assert np.array_equal(got.view(np.uint8), want[0][idx].view(np.uint8)), op
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 5, 8, 16, 64])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16", "i32"])
+def test_fold_samples_equals_the_pinned_fold(n, dtype):
+    # random sample positions with their chunk index as the fold's start
+    _samples_match(n, dtype)
+
+
 def test_ring_bf16_per_hop_rounding_stays_near_fp32_fold():
     n, count = 8, 4096
     x = synth.ranks(8, n, count, "normal", "bf16")
@@ -548,16 +608,20 @@ def _pins():
         test_p3_four_gpu_walkthrough,
         test_fold_order_golden,
         test_max_signed_zero_tie_keeps_left_operand,
+        lambda: _omp_matches(5, "f32", (1, 3)),
+        lambda: _samples_match(5, "f32"),
     ]
 
 
-@pytest.mark.parametrize("kind", range(1, 10))
+@pytest.mark.parametrize("kind", list(range(1, 10)) + [14, 15])
 def test_mutants_are_caught(kind):
     # kinds (rr_oracle.c): 1 subtract instead of add, 2 AVG multiplies, 3
     # all-gather index off by one, 4 operands of the fold swapped, 5 last step
     # of each phase dropped, 6 one-shot fold starts one rank late, 7
     # reduce-scatter fold starts one rank late, 8 all-gather takes the wrong
-    # rank's part, 9 all-to-all sends the wrong block
+    # rank's part, 9 all-to-all sends the wrong block, 14 the OpenMP ring
+    # reads its own message slot instead of its left neighbour's, 15 the
+    # sampled fold leaves out AVG's division
     failed = 0
     with oracle.mutant(kind):
         for pin in _pins():
