@@ -358,10 +358,13 @@ rr_status_t rr_get_stats(rr_stats_t* out); /* last call on this host thread */
  * ranks) stage their tiles in shared memory with bulk async copies when the
  * buffers are 16-byte aligned; their threads wait on an mbarrier for those
  * copies with an iteration limit instead of forever.  A wait that runs out --
- * no working device lets it -- skips its tile (that tile's result is not
- * written) and is counted on the device.  This call synchronises the current
- * device, then returns RR_ERR_TIMEOUT if any wait ran out there since the
- * last call (and clears the count), RR_OK otherwise.  No other kernel of the
+ * no working device lets it -- makes the whole CTA skip its tile (nothing of
+ * that tile's result is written) and is counted on the device; one thread
+ * then waits once more, bounded, for the tile's copies to land, and counts
+ * the tile a second time if they were not seen to land.  This call
+ * synchronises the current device, takes both counts (atomically exchanged
+ * for zero on the device) and returns RR_ERR_TIMEOUT if either is not zero
+ * (rr_last_error() gives both), RR_OK otherwise.  No other kernel of the
  * library waits on anything. */
 rr_status_t rr_check_timeouts(void);
 const char* rr_status_string(rr_status_t status);

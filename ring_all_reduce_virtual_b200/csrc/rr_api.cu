@@ -385,6 +385,7 @@ rr_status_t run_rank_kernel(int kind, const void* const* in, void* const* out, i
     p.lo = lo;
     p.hi = hi;
     p.owner_only = owner_only ? 1 : 0;
+    p.waits = bulk_wait_counters();  // looked up once per launch
     cudaError_t e = launch_rank_kernel(kind, dtype, op, p, stream);
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     t_stats.launches += 1;
@@ -606,6 +607,7 @@ rr_status_t rr_allreduce_wire(void* const* bufs, int nranks, size_t count, rr_op
         p.tps = std::max<uint64_t>(1, ceil_div(p.C, tile_elems(RR_F32, kVptReduce)));
         p.lo = 0;
         p.hi = UINT64_MAX;
+        p.waits = bulk_wait_counters();
         cudaError_t e = launch_oneshot_wire(op, p, p.nseg * p.tps, stream);
         if (e != cudaSuccess) return cuda_fail(e, "wire one-shot launch");
         t_stats.launches = 1;
@@ -1205,10 +1207,13 @@ rr_status_t rr_reducer_ready(rr_reducer_t* red, int tensor, cudaStream_t produce
 rr_status_t rr_check_timeouts(void)
 {
     cudaError_t e = cudaDeviceSynchronize();
-    if (e != cudaSuccess) return cuda_fail(e, "synchronising before reading the wait counter");
-    unsigned int count = 0;
-    if ((e = take_bulk_timeouts(&count)) != cudaSuccess) return cuda_fail(e, "reading the wait counter");
-    if (count) return fail(RR_ERR_TIMEOUT, "bounded device waits ran out; their tiles were skipped");
+    if (e != cudaSuccess) return cuda_fail(e, "synchronising before reading the wait counters");
+    unsigned int ran_out = 0, in_flight = 0;
+    if ((e = take_bulk_timeouts(&ran_out, &in_flight)) != cudaSuccess) return cuda_fail(e, "reading the wait counters");
+    if (ran_out || in_flight)
+        return fail(RR_ERR_TIMEOUT, "bounded device waits ran out on " + std::to_string(ran_out) +
+                                        " tiles, which were skipped; copies not seen to land: " +
+                                        std::to_string(in_flight));
     return RR_OK;
 }
 

@@ -200,8 +200,8 @@ __global__ void __launch_bounds__(kThreads) bucket_fold_kernel(const __grid_cons
 // tensor at the same address modulo 16 (vec_ok) and N = 2, 4, 8 or 16.
 struct BucketBulkParams {
     BucketFoldParams f;  // tile0 counts bulk tiles (bucket_bulk_tile_elems)
-    unsigned int* timeouts;
-    uint32_t extra_tx;
+    unsigned int* waits; // as BulkParams (rr_bulk.cuh): the wait counters, the test hook, the bound
+    uint32_t hold;
     uint32_t spin;
 };
 static_assert(sizeof(BucketBulkParams) <= 32764, "BucketBulkParams too large");
@@ -245,14 +245,11 @@ __global__ void __launch_bounds__(kThreads) bucket_bulk_kernel(const __grid_cons
     const uint64_t e0 = head + v0 * L;  // 16-byte aligned in every rank's copy
 
     const uint32_t b = bulk_smem_addr(&bar);
-    if (threadIdx.x == 0) {
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(b) : "memory");
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
+    if (threadIdx.x == 0) bulk_bar_init(b, bp.hold);
     __syncthreads();
     if (threadIdx.x == 0) {
         asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
-                     ::"r"(b), "r"(bytes * NS + bp.extra_tx) : "memory");
+                     ::"r"(b), "r"(bytes * NS) : "memory");
 #pragma unroll
         for (int j = 0; j < NS; ++j)
             asm volatile(
@@ -260,11 +257,7 @@ __global__ void __launch_bounds__(kThreads) bucket_bulk_kernel(const __grid_cons
                 ::"r"(bulk_smem_addr(sm + j * TV)), "l"(in(j) + e0), "r"(bytes), "r"(b)
                 : "memory");
     }
-    if (!bulk_bar_wait(b, 0, bp.spin)) {
-        if (threadIdx.x == 0) atomicAdd(bp.timeouts, 1u);
-        bulk_bar_wait(b, 0, bp.spin);  // once more for the copies in flight, then leave the tile
-        return;
-    }
+    if (!bulk_tile_landed(b, bp.waits, bp.hold, bp.spin)) return;  // the whole CTA skips the tile
     for (uint32_t v = threadIdx.x; v < nvt; v += kThreads) {
         Acc a[L];
         G::unpack(sm[v], a);
@@ -289,6 +282,7 @@ __global__ void __launch_bounds__(kThreads) bucket_bulk_kernel(const __grid_cons
                          : "memory");
         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
         asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        bulk_bar_inval(b);
     }
 }
 
@@ -304,12 +298,14 @@ template <class G, int OP>
 cudaError_t launch_bucket_bulk(const BucketFoldParams& p, int grad_dtype, cudaStream_t s, bool* launched)
 {
     *launched = false;
-    const BulkParams wait = bulk_params(RankParams{});
-    if (!wait.timeouts) return cudaSuccess;
+    RankParams rp{};
+    rp.waits = bulk_wait_counters();  // once per launch
+    if (!rp.waits) return cudaSuccess;
+    const BulkParams wait = bulk_params(rp);
     auto* bp = new BucketBulkParams();
     bp->f = p;
-    bp->timeouts = wait.timeouts;
-    bp->extra_tx = wait.extra_tx;
+    bp->waits = wait.waits;
+    bp->hold = wait.hold;
     bp->spin = wait.spin;
     const uint64_t te = bucket_bulk_tile_elems(grad_dtype, p.n);
     bp->f.tile0[0] = 0;

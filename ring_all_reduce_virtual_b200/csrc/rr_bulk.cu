@@ -11,7 +11,7 @@
 // sections "Ring all-reduce and communication volume" and "alpha-beta model".
 #include <cstdlib>
 #include <cstring>
-#include <mutex>
+#include <atomic>
 
 #include "rr_bulk.cuh"
 
@@ -19,20 +19,31 @@ namespace rr {
 
 namespace {
 
-__device__ unsigned int g_bulk_timeouts = 0;
+// [0] tiles whose bounded wait ran out, [1] of those, tiles whose copies
+// were not seen to land; one pair per device (each device holds its own
+// copy of the module's variables).
+__device__ unsigned int g_bulk_waits[2] = {0u, 0u};
+__device__ unsigned int g_bulk_taken[2] = {0u, 0u};
+
+__global__ void take_waits_kernel()
+{
+    g_bulk_taken[0] = atomicExch(&g_bulk_waits[0], 0u);
+    g_bulk_taken[1] = atomicExch(&g_bulk_waits[1], 0u);
+}
 
 // Test hook, read once per process: RR_DEBUG_BULK_TIMEOUT=1 makes every
-// barrier expect 16 bytes more than its copies bring and bounds each wait at
-// 2^16 rounds, so that every wait runs out (the copies themselves complete,
-// long before the second wait ends).
+// barrier expect one arrival more than the copying thread makes, and bounds
+// each wait at 2^16 rounds, so that every first wait runs out; the missing
+// arrival is then made, and the second wait ends when the tile's copies have
+// landed -- the path a real timeout takes.
 struct BulkDebug {
-    uint32_t extra_tx = 0;
+    uint32_t hold = 0;
     uint32_t spin = 1u << 22;  // try_wait rounds, each of which may suspend the thread briefly
     BulkDebug()
     {
         const char* v = std::getenv("RR_DEBUG_BULK_TIMEOUT");
         if (v && std::strcmp(v, "1") == 0) {
-            extra_tx = 16;
+            hold = 1;
             spin = 1u << 16;
         }
     }
@@ -42,23 +53,6 @@ const BulkDebug& bulk_debug()
 {
     static const BulkDebug d;
     return d;
-}
-
-// The counter's address on the current device (each device holds its own
-// copy of the module's variables), looked up once per device.
-unsigned int* timeout_counter()
-{
-    constexpr int kMaxDevices = 64;
-    static std::mutex mu;
-    static unsigned int* ptr[kMaxDevices] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_bulk_timeouts) == cudaSuccess) ptr[dev] = static_cast<unsigned int*>(p);
-    }
-    return ptr[dev];
 }
 
 uint64_t bulk_tile_bytes(int n) { return (n >= 32 ? 32768u : 16384u) / (uint64_t)n; }  // bulk_smem<N>() / N
@@ -79,12 +73,29 @@ cudaError_t launch_ring(const RankParams& p, cudaStream_t s)
 
 }  // namespace
 
+unsigned int* bulk_wait_counters()
+{
+    constexpr int kMaxDevices = 64;
+    static std::atomic<unsigned int*> ptr[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    unsigned int* p = ptr[dev].load(std::memory_order_acquire);
+    if (p) return p;
+    void* q = nullptr;
+    if (cudaGetSymbolAddress(&q, g_bulk_waits) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    ptr[dev].store(static_cast<unsigned int*>(q), std::memory_order_release);  // a racing lookup stores the same
+    return static_cast<unsigned int*>(q);
+}
+
 BulkParams bulk_params(const RankParams& p)
 {
     BulkParams bp{};
     bp.r = p;
-    bp.timeouts = timeout_counter();
-    bp.extra_tx = bulk_debug().extra_tx;
+    bp.waits = p.waits;
+    bp.hold = bulk_debug().hold;
     bp.spin = bulk_debug().spin;
     return bp;
 }
@@ -92,7 +103,7 @@ BulkParams bulk_params(const RankParams& p)
 bool bulk_ranks_aligned(const RankParams& p, int nmax)
 {
     if (p.n > nmax || (p.n != 2 && p.n != 4 && p.n != 8 && p.n != 16 && p.n != 32 && p.n != 64)) return false;
-    if (!timeout_counter()) return false;
+    if (!p.waits) return false;
     for (int r = 0; r < p.n; ++r)
         if ((uintptr_t)p.in[r] % 16 != 0 || (uintptr_t)p.out[r] % 16 != 0) return false;
     return true;
@@ -134,12 +145,18 @@ cudaError_t launch_oneshot_wire_bulk(int op, const RankParams& p, cudaStream_t s
     return op == kAvg ? launch_ring<F32T, kAvg, 1>(p, s) : launch_ring<F32T, kSum, 1>(p, s);
 }
 
-cudaError_t take_bulk_timeouts(unsigned int* count)
+cudaError_t take_bulk_timeouts(unsigned int* ran_out, unsigned int* in_flight)
 {
-    cudaError_t e = cudaMemcpyFromSymbol(count, g_bulk_timeouts, sizeof(unsigned int));
+    // exchanged on the device, so a count that a kernel adds meanwhile is kept
+    // for the next take; the copy below follows the kernel on the same stream
+    take_waits_kernel<<<1, 1>>>();
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const unsigned int zero = 0;
-    return cudaMemcpyToSymbol(g_bulk_timeouts, &zero, sizeof(unsigned int));
+    unsigned int h[2] = {0u, 0u};
+    if ((e = cudaMemcpyFromSymbol(h, g_bulk_taken, sizeof h)) != cudaSuccess) return e;
+    *ran_out = h[0];
+    *in_flight = h[1];
+    return cudaSuccess;
 }
 
 #define RR_INSTANTIATE(TY, OP) template cudaError_t launch_oneshot_bulk<TY, OP>(const RankParams&, cudaStream_t);

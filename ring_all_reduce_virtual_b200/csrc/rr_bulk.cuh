@@ -18,10 +18,14 @@
 // every other call takes the per-thread-load kernels, with the same bits.
 // The fold itself uses the same apply / finish / wire steps as those kernels.
 //
-// Every mbarrier wait is bounded.  A wait that runs out (no working device
-// lets it) skips its tile, counts itself in the counter BulkParams::timeouts
-// points to, waits once more (bounded) for its own copies in flight and
-// returns; rr_check_timeouts() reads and clears the count.
+// Every mbarrier wait is bounded, and its outcome is the same in every thread
+// of the CTA (bulk_tile_landed).  A tile whose wait runs out (no working
+// device lets it) is skipped by the whole CTA -- nothing of it is stored --
+// and counted in BulkParams::waits[0]; one thread then waits once more
+// (bounded) for the tile's copies to land before the CTA leaves, and counts
+// the tile in waits[1] if they were not seen to land (its shared memory may
+// then still receive them after the CTA has left, so a nonzero waits[1]
+// means the device is not usable).  rr_check_timeouts() takes both counts.
 //
 // Sources: [P4] "Collective communication primitives" (ai-infra-handbooks),
 // sections "The five primitives", "Ring all-reduce and communication volume"
@@ -37,9 +41,11 @@ enum BulkMode : int { kBulkRing = 0, kBulkScatter = 1, kBulkTree = 2 };
 
 struct BulkParams {
     RankParams r;
-    unsigned int* timeouts;  // device counter of waits that ran out
-    uint32_t extra_tx;       // bytes the barrier expects beyond the copies (0; a test hook)
-    uint32_t spin;           // try_wait rounds before a wait gives up
+    unsigned int* waits;  // device counters: [0] tiles whose wait ran out, [1] of those, tiles
+                          // whose copies were not seen to land before the CTA left
+    uint32_t hold;        // test hook (0 in use): 1 makes every barrier expect one arrival
+                          // more, which is made only after the first wait has run out
+    uint32_t spin;        // try_wait rounds before a wait gives up
 };
 
 // Bytes of input tiles per CTA (N tiles of bulk_smem<N>() / N): 16 KB, 32 KB
@@ -50,14 +56,13 @@ __host__ __device__ constexpr uint32_t bulk_smem()
     return NS >= 32 ? 32768u : 16384u;
 }
 
-// The parameter block of a launch: p, the counter's address and the wait
-// bounds (rr_bulk.cu).
+// The parameter block of a launch: p, the counters' address (p.waits) and
+// the wait bounds (rr_bulk.cu).
 BulkParams bulk_params(const RankParams& p);
 
-// Whether a call can take the bulk kernels: a rank count of 2, 4, 8, 16, 32
-// or 64 (up to nmax), 16-byte aligned buffers, and segments of whole 16-byte
-// vectors (seg_bytes: bytes per segment; the ring mode allows a ragged last
-// chunk).
+// Whether a call can take the bulk kernels: the wait counters are known
+// (p.waits), a rank count of 2, 4, 8, 16, 32 or 64 (up to nmax), 16-byte
+// aligned buffers.  The callers add their own segment rules.
 bool bulk_ranks_aligned(const RankParams& p, int nmax);
 
 __device__ __forceinline__ uint32_t bulk_smem_addr(const void* ptr) { return (uint32_t)__cvta_generic_to_shared(ptr); }
@@ -74,6 +79,39 @@ __device__ __forceinline__ bool bulk_bar_wait(uint32_t bar, uint32_t parity, uin
             : "r"(bar), "r"(parity)
             : "memory");
         if (done) return true;
+    }
+    return false;
+}
+
+// Thread 0: set up a tile's barrier.  It completes once `1 + hold`
+// arrivals have been made and the copies' bytes have landed.
+__device__ __forceinline__ void bulk_bar_init(uint32_t bar, uint32_t hold)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(1u + hold) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Thread 0, once no thread waits on the barrier and no copy signals it.
+__device__ __forceinline__ void bulk_bar_inval(uint32_t bar)
+{
+    asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// Every thread of the CTA: wait (bounded) for the tile's copies.  Returns the
+// same answer in every thread: true when every thread saw them land.  On
+// false the CTA must skip the tile and leave; thread 0 has then counted the
+// tile, made the arrival the test hook withheld, and waited (bounded) for the
+// copies to land -- invalidating the barrier if they did, counting the tile
+// in waits[1] if not -- so the CTA's shared memory is not left to a copy
+// still in flight.
+__device__ __forceinline__ bool bulk_tile_landed(uint32_t bar, unsigned int* waits, uint32_t hold, uint32_t spin)
+{
+    if (__syncthreads_and(bulk_bar_wait(bar, 0, spin))) return true;
+    if (threadIdx.x == 0) {
+        atomicAdd(&waits[0], 1u);
+        if (hold) asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar) : "memory");
+        if (bulk_bar_wait(bar, 0, spin)) bulk_bar_inval(bar);
+        else atomicAdd(&waits[1], 1u);
     }
     return false;
 }
@@ -125,14 +163,11 @@ __global__ void __launch_bounds__(kThreads) bulk_fold_kernel(const __grid_consta
     const uint64_t e0 = v0 * L;                    // first element of the tile in the segment
 
     const uint32_t b = bulk_smem_addr(&bar);
-    if (threadIdx.x == 0) {
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(b) : "memory");
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
+    if (threadIdx.x == 0) bulk_bar_init(b, bp.hold);
     __syncthreads();
     if (threadIdx.x == 0) {
         asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
-                     ::"r"(b), "r"(bytes * NS + bp.extra_tx) : "memory");
+                     ::"r"(b), "r"(bytes * NS) : "memory");
 #pragma unroll
         for (int j = 0; j < NS; ++j)
             asm volatile(
@@ -140,11 +175,7 @@ __global__ void __launch_bounds__(kThreads) bulk_fold_kernel(const __grid_consta
                 ::"r"(bulk_smem_addr(sm + j * TV)), "l"(in(j) + e0), "r"(bytes), "r"(b)
                 : "memory");
     }
-    if (!bulk_bar_wait(b, 0, bp.spin)) {
-        if (threadIdx.x == 0) atomicAdd(bp.timeouts, 1u);
-        bulk_bar_wait(b, 0, bp.spin);  // once more for the copies in flight, then leave the tile
-        return;
-    }
+    if (!bulk_tile_landed(b, bp.waits, bp.hold, bp.spin)) return;  // the whole CTA skips the tile
     for (uint32_t v = threadIdx.x; v < nvt; v += kThreads) {
         Acc a[L];
         if constexpr (MODE == kBulkTree) {
@@ -196,6 +227,7 @@ __global__ void __launch_bounds__(kThreads) bulk_fold_kernel(const __grid_consta
                          : "memory");
         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
         asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // slot 0 read before the CTA leaves
+        bulk_bar_inval(b);
     }
 }
 
@@ -205,6 +237,7 @@ cudaError_t launch_bulk_fold(const RankParams& p, uint64_t seg_elems, cudaStream
 {
     constexpr uint64_t TE = (uint64_t)(bulk_smem<NS>() / NS / 16) * Ty::L;  // elements per tile
     BulkParams bp = bulk_params(p);
+    if (!bp.waits) return cudaErrorInvalidValue;  // never reached: eligibility requires the counters
     bp.r.tps = (seg_elems + TE - 1) / TE;
     const uint64_t work = bp.r.nseg * bp.r.tps;
     if (work == 0) return cudaSuccess;

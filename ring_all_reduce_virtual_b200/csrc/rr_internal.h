@@ -28,6 +28,8 @@ struct RankParams {
     uint64_t hi;    //   rank processed by this launch
     int owner_only; // one-shot all-reduce: write chunk c only to rank c (two-shot's first shot)
     int pad2_;
+    unsigned int* waits;  // the bulk-copy kernels' wait counters on the launching device
+                          // (bulk_wait_counters(); NULL keeps a call off those kernels)
 };
 
 // One segment of a table-driven step (a ring step, a tree level): fold
@@ -131,9 +133,13 @@ cudaError_t launch_step(int dtype, int op, const StepParams& p, cudaStream_t s);
 // step (wire 1: the step completes its chunks; 2: it does not).
 cudaError_t launch_oneshot_wire(int op, const RankParams& p, uint64_t work, cudaStream_t s);
 cudaError_t launch_step_wire(int op, int wire, const StepParams& p, cudaStream_t s);
-// Reads and clears the device-side count of bounded waits that ran out
-// (the bulk-copy one-shot's mbarrier waits).  Synchronous.
-cudaError_t take_bulk_timeouts(unsigned int* count);
+// The bulk-copy kernels' two wait counters on the current device (tiles whose
+// bounded wait ran out; of those, tiles whose copies were not seen to land),
+// looked up once per device; NULL if the lookup fails.
+unsigned int* bulk_wait_counters();
+// Takes (reads and clears, atomically on the device) both counters of the
+// current device.  Synchronous.
+cudaError_t take_bulk_timeouts(unsigned int* ran_out, unsigned int* in_flight);
 cudaError_t launch_bucket_pack(int grad_dtype, const BucketCopyParams& p, cudaStream_t s);
 cudaError_t launch_bucket_unpack(int grad_dtype, int op, const BucketCopyParams& p, cudaStream_t s);
 cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p, cudaStream_t s,

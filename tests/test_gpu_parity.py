@@ -597,9 +597,13 @@ def test_bulk_copy_one_shot(n, dtype, op):
 
 
 def test_bulk_copy_timeouts_are_reported_and_the_context_survives():
-    """With RR_DEBUG_BULK_TIMEOUT=1 every barrier expects 16 bytes more than
-    its copies bring, so every bounded wait runs out: the call returns, the
-    count shows up as RR_ERR_TIMEOUT, and the context still works."""
+    """With RR_DEBUG_BULK_TIMEOUT=1 every barrier expects one arrival more
+    than the copying thread makes, so every first bounded wait runs out.  The
+    whole CTA then skips its tile (the buffers keep their inputs: nothing
+    partly folded is stored), the missing arrival is made and the second wait
+    confirms that the tile's copies landed before the CTA left.  Both the
+    one-shot and the fused bucket sync report it through RR_ERR_TIMEOUT with
+    the tile count, and the context still runs another collective."""
     import os
     import subprocess
     import sys
@@ -607,13 +611,21 @@ def test_bulk_copy_timeouts_are_reported_and_the_context_survives():
     script = r'''
 import torch, numpy as np
 import ring_all_reduce_virtual_b200 as rrv
+def report():
+    try:
+        rrv.check_timeouts()
+        print("NO TIMEOUT")
+    except rrv.RRError as e:
+        print("TIMEOUT", e.status, str(e))
 x = [torch.full((2048,), float(r + 1), device="cuda") for r in range(2)]
-rrv.all_reduce(x, "sum", "oneshot")  # bulk path: aligned, C = 1024 floats
-try:
-    rrv.check_timeouts()
-    print("NO TIMEOUT")
-except rrv.RRError as e:
-    print("TIMEOUT", e.status)
+rrv.all_reduce(x, "sum", "oneshot")  # bulk path: aligned, 2 chunks of 1024 floats, one tile each
+report()
+assert torch.all(x[0] == 1.0) and torch.all(x[1] == 2.0), "a skipped tile was stored"
+plan = rrv.BucketPlan([4096], "bf16", 1 << 20)  # one bucket, 2 chunks of 2048 bf16, one tile each
+g = [[torch.full((4096,), float(r + 1), device="cuda").to(torch.bfloat16)] for r in range(2)]
+plan.all_reduce(0, g, "sum")
+report()
+assert torch.all(g[0][0] == 1.0) and torch.all(g[1][0] == 2.0), "a skipped bucket tile was stored"
 rrv.check_timeouts()  # cleared
 y = [torch.full((2048,), float(r + 1), device="cuda") for r in range(3)]
 rrv.all_reduce(y, "sum", "ring")  # another path on the same context
@@ -623,7 +635,11 @@ print("CONTEXT OK")
     env = dict(os.environ, RR_DEBUG_BULK_TIMEOUT="1")
     out = subprocess.run([sys.executable, "-c", script], env=env, capture_output=True, text=True, timeout=300)
     assert out.returncode == 0, out.stderr[-2000:]
-    assert "TIMEOUT 4" in out.stdout and "CONTEXT OK" in out.stdout, out.stdout
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("TIMEOUT")]
+    assert len(lines) == 2, out.stdout
+    for ln in lines:
+        assert ln.startswith("TIMEOUT 4") and "on 2 tiles" in ln and "not seen to land: 0" in ln, ln
+    assert "CONTEXT OK" in out.stdout, out.stdout
 
 
 @pytest.mark.parametrize("n", [2, 4, 8, 16])
