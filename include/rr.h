@@ -199,6 +199,38 @@ rr_status_t rr_allreduce_wire(void* const* bufs, int nranks, size_t count, rr_op
 rr_status_t rr_allreduce_host(void* const* host_bufs, void* const* dev_bufs, int nranks, size_t count,
                               rr_dtype_t dtype, rr_op_t op, rr_algo_t algo, cudaStream_t stream);
 
+/* The host-buffer all-reduce for callers that cannot allocate device memory.
+ * The pages have no counterpart to this call: it exists for callers that
+ * hold only host arrays and a stream and may not call cudaMalloc -- code that
+ * runs while a framework's caching allocator holds all of the device's memory,
+ * a plug-in that is handed no device buffers, or a latency-critical path that
+ * must not call cudaMalloc or cudaFree because they can synchronise the device.
+ * It does what rr_allreduce_host does with a caller's device buffers (copy
+ * host_bufs[r] in, reduce, copy the result back into every host_bufs[r]; the
+ * same bits), but stages the values in a region of device memory that the
+ * library declares statically: RR_NOALLOC_MAX_BYTES (16 MiB) on every GPU that
+ * loads the library, held until the process exits.  The call allocates
+ * nothing, on the device or the host.
+ *   - Limit: nranks slots of count elements, each rounded up to 256 bytes,
+ *     must fit in RR_NOALLOC_MAX_BYTES; a larger call returns
+ *     RR_ERR_INVALID_ARG before anything is enqueued.
+ *   - algo: AUTO or ONESHOT (the one-shot all-reduce in ring order); others
+ *     return RR_ERR_UNSUPPORTED.  Other arguments and errors as
+ *     rr_allreduce_host; host buffers must not overlap.
+ *   - The first call on a device looks up the staging region's device address
+ *     there (cudaGetSymbolAddress, with that device current) and keeps it;
+ *     make that first call before any stream capture on the device.
+ *   - Every call on a device uses the same region, which keeps the last
+ *     call's values; nothing in it needs to start at zero, because each call
+ *     overwrites the bytes it reads.  Calls whose work overlaps on the GPU --
+ *     on different streams, or from different threads, without ordering
+ *     between them -- race on the region and give wrong results.
+ *   - Host buffers should be page-locked for the copies to be asynchronous;
+ *     they hold the result once `stream` has been synchronised. */
+#define RR_NOALLOC_MAX_BYTES (16u << 20)
+rr_status_t rr_allreduce_host_noalloc(void* const* host_bufs, int nranks, size_t count, rr_dtype_t dtype,
+                                      rr_op_t op, rr_algo_t algo, cudaStream_t stream);
+
 /* One step of the ring schedule for all ranks at once (one launch), in place:
  * reduce-scatter step s has every rank r fold chunk (r-s-1) mod N received
  * from rank r-1 into its own copy (received partial on the left; AVG divides

@@ -20,7 +20,7 @@ from typing import Sequence
 from ._lib import MAX_RANKS, Cost, RingEvent, RRError, Stats, check, lib
 
 __all__ = [
-    "all_reduce", "all_reduce_wire", "all_reduce_host", "ring_step", "ring_schedule", "reduce_scatter", "all_gather", "all_to_all",
+    "all_reduce", "all_reduce_wire", "all_reduce_host", "all_reduce_host_noalloc", "ring_step", "ring_schedule", "reduce_scatter", "all_gather", "all_to_all",
     "RankSet", "BucketPlan", "GradSet", "Reducer", "cost_model", "pick_algo", "set_picker_params", "last_stats",
     "check_timeouts", "RRError",
     "OPS", "ALGOS", "MAX_RANKS",
@@ -141,6 +141,25 @@ def all_reduce_host(host: Sequence, device: Sequence, op="sum", algo="auto", str
             raise ValueError("all_reduce_host: host tensors must be contiguous CPU tensors like the device ones")
     check(lib().rr_allreduce_host(_ptr_array(host), _ptr_array(device), len(device), count, d, _op(op),
                                   _algo(algo), _stream(stream, dev)), "all_reduce_host")
+
+
+def all_reduce_host_noalloc(host: Sequence, op="sum", algo="auto", stream=None) -> None:
+    """All-reduce of host tensors for callers that cannot allocate device
+    memory (``rr_allreduce_host_noalloc``): the values are staged in the
+    library's static device region (``RR_NOALLOC_MAX_BYTES`` in all), so the
+    call allocates nothing.  ``host`` should be pinned; it holds the result
+    once the stream is synchronised."""
+    import torch
+
+    if len(host) < 1 or len(host) > MAX_RANKS:
+        raise ValueError(f"all_reduce_host_noalloc: need 1..{MAX_RANKS} host tensors")
+    h0 = host[0]
+    for h in host:
+        if h.is_cuda or not h.is_contiguous() or h.numel() != h0.numel() or h.dtype != h0.dtype:
+            raise ValueError("all_reduce_host_noalloc: host tensors must be contiguous CPU tensors alike")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    check(lib().rr_allreduce_host_noalloc(_ptr_array(host), len(host), h0.numel(), _dtype_code(h0.dtype), _op(op),
+                                          _algo(algo), _stream(stream, dev)), "all_reduce_host_noalloc")
 
 
 def ring_step(tensors, op, phase, step: int, stream=None) -> None:

@@ -56,6 +56,7 @@ def _declare(lib: ctypes.CDLL) -> None:
     sig = {
         "rr_allreduce": (st, [PP, i, sz, i, i, i, P]),
         "rr_allreduce_host": (st, [PP, PP, i, sz, i, i, i, P]),
+        "rr_allreduce_host_noalloc": (st, [PP, i, sz, i, i, i, P]),
         "rr_allreduce_wire": (st, [PP, i, sz, i, i, i, P]),
         "rr_ring_step": (st, [PP, i, sz, i, i, i, i, P]),
         "rr_ring_schedule": (st, [i, sz, i, ctypes.POINTER(RingEvent), sz, ctypes.POINTER(sz)]),

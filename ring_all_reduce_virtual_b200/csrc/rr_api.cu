@@ -460,6 +460,18 @@ rr_status_t host_pipe(HostPipe** out)
 
 }  // namespace
 
+// Hooks for entry points defined in other files of the library: record the
+// text rr_last_error() returns, and the statistics rr_get_stats() returns.
+namespace rr {
+rr_status_t record_error(rr_status_t st, const char* why)
+{
+    t_error = why;
+    return st;
+}
+
+void record_stats(const rr_stats_t& s) { t_stats = s; }
+}  // namespace rr
+
 // ================================================================ C ABI ==
 
 extern "C" {
