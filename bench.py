@@ -37,11 +37,15 @@ ELEM = 4
 SEED = 0
 FALLBACK_HBM_GBS = 6650.0
 
-# DRAM traffic of one launch of the dominant kernel per algorithmic byte,
-# from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), with the
-# hash of the dominant kernel's source files it was taken on.  The summary with its command is
-# in profiles/bulk_fold_kernel_allreduce-8x64MiB-f32.md.
-NCU_TRAFFIC = {"per_algorithmic_byte": (536886784 + 479816704) / 1073741824, "sources_sha1": "a50fff8d140ae15085d173571f96b2498ff29a4d"}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
+# the dominant kernel at the full 8 x 256 MiB size, from one ncu capture of
+# that launch in steady state:
+#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
+#       --clock-control none -k regex:bulk_fold_kernel -s 5 -c 1
+#       python bench.py --steps 3 --warmup 5 --no-extra --no-e2e --no-cpu
+# with the hash of the kernel's source files it was taken on (the bench
+# reports null once they change).
+NCU_TRAFFIC = {"bytes_per_launch": None, "sources_sha1": None}
 
 
 # The files that define the dominant kernel (bulk_fold_kernel in ring order,
@@ -78,6 +82,9 @@ def parse_args():
     ap.add_argument("--nranks", type=int, default=NRANKS, help="virtual ranks of --workload kernels")
     ap.add_argument("--reps", type=int, default=5, help="timed calls per kernel family of --workload kernels")
     ap.add_argument("--tokens", type=int, default=1024, help="tokens of the synthetic backward of --workload overlap")
+    ap.add_argument("--odd", action="store_true",
+                    help="--workload kernels: odd bucket tensor sizes, so later tensors sit out of phase with "
+                         "their gradients in the fp32 bucket")
     ap.add_argument("--count", type=int, default=COUNT,
                     help="fp32 elements per virtual rank (default 2^26 = 256 MiB); smaller for profiling")
     return ap.parse_args()
@@ -349,9 +356,10 @@ def run_ours(args, d: Dist):
     achieved = alg_bytes / t / 1e9
     peak, peak_kind = hbm_peak()
     traffic = None
-    if NCU_TRAFFIC["per_algorithmic_byte"] and NCU_TRAFFIC["sources_sha1"] == sources_sha1():
-        traffic = int(NCU_TRAFFIC["per_algorithmic_byte"] * alg_bytes)
+    if NCU_TRAFFIC["bytes_per_launch"] and NCU_TRAFFIC["sources_sha1"] == sources_sha1() and count == COUNT:
+        traffic = int(NCU_TRAFFIC["bytes_per_launch"])
 
+    copy_gbs = None if args.no_extra else time_copy_ceiling(dev, stream, NRANKS * S)
     # end to end through the public API with host buffers: H2D + all-reduce + D2H
     e2e = None
     if not args.no_e2e:
@@ -375,6 +383,9 @@ def run_ours(args, d: Dist):
                          "frac": round(achieved / peak, 4), "traffic": traffic,
                          "kernel": "bulk_fold_kernel<F32T, AVG, N 8, ring order> (bulk-copy tiles, 2 KB per rank)",
                          "algorithmic_bytes_per_launch": alg_bytes, "peak_kind": peak_kind + " (burst copy)"},
+            "copy_ceiling": None if copy_gbs is None else {
+                "copy_gbs": round(copy_gbs, 1), "frac_of_copy": round(achieved / copy_gbs, 4),
+                "what": "torch copy_ of the same 2 GiB (read + write), timed in this run like the headline"},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": int(picked["launches"]) * args.steps,
@@ -383,6 +394,27 @@ def run_ours(args, d: Dist):
         }
         print(json.dumps(line), flush=True)
     d.close()
+
+
+def time_copy_ceiling(dev, stream, nbytes):
+    """GB/s (read + write) of a plain device-to-device copy of nbytes, the
+    same traffic as one headline call, with CUDA events on the stream."""
+    import torch
+
+    src = torch.empty(nbytes // 4, dtype=torch.float32, device=dev).normal_()
+    dst = torch.empty_like(src)
+    with torch.cuda.stream(stream):
+        for _ in range(5):
+            dst.copy_(src)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(50):
+            dst.copy_(src)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    t = a.elapsed_time(b) / 50 / 1e3
+    del src, dst
+    return 2 * nbytes / t / 1e9
 
 
 def time_e2e(args, d, dev, stream, host, bufs, S):
@@ -456,33 +488,69 @@ def time_extra(dev, stream, host, S, peak):
 
 
 def fit_alpha_beta(rows):
-    """Least-squares fit of the alpha-beta model to the sweep ([P3] section 4:
-    time = steps * alpha + bytes / beta; on one GPU a step is a launch and the
-    bytes are HBM bytes): per call from Python, and per call inside a CUDA
-    graph (small sizes).  Prints one JSON line; rr_set_picker_params takes
-    such a pair."""
+    """Fit of the alpha-beta model to the sweep ([P3] section 4: time =
+    steps * alpha + bytes / beta; on one GPU a step is a launch and the bytes
+    are HBM bytes), per call from Python and per call inside a CUDA graph
+    (small sizes).  rows: (launches, HBM bytes, seconds per call, seconds per
+    call in a graph or None, L2-resident).  Each point is weighted by 1 / its
+    time, so the fit minimises relative error and the small sizes that fix
+    alpha count as much as the large ones that fix beta; points whose bytes
+    are L2-resident and not negligible (above 4 MiB) are left out, since L2
+    is faster than the HBM beta describes.  Prints one JSON line with the pair
+    and the fit's relative residuals; rr_set_picker_params takes such a pair."""
     import numpy as np
 
-    out = {"workload": "size-sweep-f32-sum", "fit": "alpha-beta, least squares over every point (launches, HBM bytes)"}
+    out = {"workload": "size-sweep-f32-sum",
+           "fit": "alpha-beta, least squares weighted by 1/time (relative error), over launch-bound points "
+                  "and HBM-resident points (L2-resident points above 4 MiB left out)"}
     for key, idx in (("per_call", 2), ("in_graph", 3)):
-        pts = [(r[0], r[1], r[idx]) for r in rows if r[idx] is not None]
+        pts = [(r[0], r[1], r[idx]) for r in rows
+               if r[idx] is not None and r[idx] > 0 and (r[1] <= 4 << 20 or not (len(r) > 4 and r[4]))]
         if len(pts) < 3:
             continue
         a = np.array([[p[0], p[1]] for p in pts], dtype=float)
         y = np.array([p[2] for p in pts], dtype=float)
-        sol = np.linalg.lstsq(a, y, rcond=None)[0]
-        if sol[1] > 0:
-            out[key] = {"alpha_us": round(sol[0] * 1e6, 3), "beta_gbs": round(1 / sol[1] / 1e9, 1), "points": len(pts)}
+        w = 1.0 / y
+        sol = np.linalg.lstsq(a * w[:, None], y * w, rcond=None)[0]
+        if sol[1] > 0 and sol[0] > 0:
+            rel = (a @ sol - y) / y
+            out[key] = {"alpha_us": round(sol[0] * 1e6, 3), "beta_gbs": round(1 / sol[1] / 1e9, 1), "points": len(pts),
+                        "rel_residual_rms": round(float(np.sqrt(np.mean(rel ** 2))), 4),
+                        "rel_residual_max": round(float(np.max(np.abs(rel))), 4)}
     print(json.dumps(out), flush=True)
+
+
+SWEEP_NS = (2, 4, 8, 16)  # the size sweep's rank counts
+SWEEP_ALGOS = ("ring", "oneshot", "two_shot", "tree", "tree_oneshot", "double_ring", "ring_steps")
+PICKER_NS = (3, 5, 6, 7, 12, 24, 32, 48, 64)  # further rank counts the picker's table covers
+PICKER_ALGOS = ("ring", "oneshot", "two_shot")  # AUTO's candidates (the ring's bits)
+PICKER_SIZES = (10, 16, 20, 24, 28, 30)  # log2 bytes per rank
+ALIGN_NS = (4, 5, 8)
+ALIGN_SIZES = (16, 24, 28)
+
+
+def _offsets(kind: str, n: int):
+    """Element offsets of each rank's buffer from a 16-byte boundary: aligned,
+    all ranks one fp32 element past it (a shared phase), or phases that
+    differ between ranks (the scalar path)."""
+    if kind == "aligned":
+        return [0] * n
+    if kind == "shared":
+        return [1] * n
+    return [r % 4 for r in range(n)]
 
 
 def run_sweep(args):
     """Message-size sweep: 1 KiB .. 1 GiB per rank, N in {2, 4, 8, 16}, fp32
-    SUM, every algorithm.  Per point: median per-call device time over 20
-    calls after 5 warm-ups, and for sizes up to 1 MiB the same through a
-    RankSet (pointers marshalled once) and the per-call time of a CUDA graph
-    holding 100 calls.  Points whose 2 N S bytes fit in L2 are
-    flagged.  The last line is the alpha-beta fit of these points."""
+    SUM, every algorithm (ring, one-shot, two-shot, tree schedule, tree-order
+    one-shot, double ring); then AUTO's candidates at further rank counts
+    (3 .. 64) and sizes, and with misaligned buffers.  Per point: median
+    per-call device time over 20 calls after 5 warm-ups, the library's own
+    host time per call (rr_get_stats host_ns, and launch_ns spent in the
+    launch calls), and for sizes up to 1 MiB the per-call time through a
+    RankSet (pointers marshalled once) and inside a CUDA graph of 100 calls.
+    Points whose 2 N S bytes fit in L2 are flagged.  The last line is the
+    alpha-beta fit of the first part's points."""
     import torch
 
     import ring_all_reduce_virtual_b200 as rrv
@@ -492,66 +560,140 @@ def run_sweep(args):
     dev = torch.device("cuda", 0)
     stream = torch.cuda.Stream(dev)
     peak, _ = hbm_peak()
-    fit_rows = []  # (launches, HBM bytes, seconds per call, seconds per call in a graph)
-    for n in (2, 4, 8, 16):
-        for e in range(10, 31):
-            nbytes = 1 << e
-            count = nbytes // ELEM
-            bufs = [torch.randn(count, device=dev) for _ in range(n)]
-            for algo in ("ring", "oneshot", "tree", "tree_oneshot"):
-                with torch.cuda.stream(stream):
-                    for _ in range(5):
+    fit_rows = []  # (launches, HBM bytes, s per call, s per call in a graph, L2-resident)
+
+    def call_of(algo, bufs, n):
+        """One all-reduce as a callable; "ring_steps" is the ring schedule as
+        2(N-1) rr_ring_step launches.  stats_of() then gives its statistics
+        (summed over the steps)."""
+        if algo != "ring_steps":
+            return (lambda: rrv.all_reduce(bufs, "sum", algo, stream)), rrv.last_stats
+        step_stats = []
+
+        def steps():
+            step_stats.clear()
+            for phase in ("reduce_scatter", "all_gather"):
+                for s_ in range(n - 1):
+                    rrv.ring_step(bufs, "sum", phase, s_, stream)
+                    step_stats.append(rrv.last_stats())
+
+        def stats_of():
+            tot = dict(step_stats[0])
+            for st_ in step_stats[1:]:
+                for key in ("launches", "hbm_bytes", "host_ns", "launch_ns"):
+                    tot[key] += st_[key]
+            return tot
+        return steps, stats_of
+
+    def point(n, nbytes, algo, bufs, align, part):
+        run, stats_of = call_of(algo, bufs, n)
+        with torch.cuda.stream(stream):
+            for _ in range(5):
+                run()
+            st = stats_of()
+            times, host_ns, launch_ns = [], [], []
+            for _ in range(20):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                run()
+                b.record(stream)
+                s2 = stats_of()
+                host_ns.append(s2["host_ns"])
+                launch_ns.append(s2["launch_ns"])
+                times.append((a, b))
+            stream.synchronize()
+            t = statistics.median(x.elapsed_time(y) for x, y in times) / 1e3
+            graph_us = rankset_us = bound_us = loop_us = None
+            if nbytes <= 16 << 20 and algo != "ring_steps":
+                # per call inside a CUDA graph of 100 calls: device time plus launch, no Python
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    for _ in range(100):
                         rrv.all_reduce(bufs, "sum", algo, stream)
-                    st = rrv.last_stats()
+                g.replay()
+                stream.synchronize()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                for _ in range(5):
+                    g.replay()
+                b.record(stream)
+                stream.synchronize()
+                graph_us = a.elapsed_time(b) * 1e3 / 500
+                del g
+            if nbytes <= 1 << 20 and algo != "ring_steps":
+                rs = rrv.RankSet(bufs)
+                bound = rs.bind("sum", algo, stream)  # arguments converted once
+                for label, fn in (("rankset", lambda: rrv.all_reduce(rs, "sum", algo, stream)), ("bound", bound)):
                     times = []
                     for _ in range(20):
                         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                         a.record(stream)
-                        rrv.all_reduce(bufs, "sum", algo, stream)
+                        fn()
                         b.record(stream)
                         times.append((a, b))
                     stream.synchronize()
-                    t = statistics.median(x.elapsed_time(y) for x, y in times) / 1e3
-                    graph_us = rankset_us = None
-                    if nbytes <= 1 << 20:
-                        # the same per-call timing through a RankSet (marshalled once)
-                        rs = rrv.RankSet(bufs)
-                        times = []
-                        for _ in range(20):
-                            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                            a.record(stream)
-                            rrv.all_reduce(rs, "sum", algo, stream)
-                            b.record(stream)
-                            times.append((a, b))
-                        stream.synchronize()
-                        rankset_us = statistics.median(x.elapsed_time(y) for x, y in times) * 1e3
-                        g = torch.cuda.CUDAGraph()
-                        with torch.cuda.graph(g, stream=stream):
-                            for _ in range(100):
-                                rrv.all_reduce(bufs, "sum", algo, stream)
-                        g.replay()
-                        stream.synchronize()
-                        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                        a.record(stream)
-                        for _ in range(5):
-                            g.replay()
-                        b.record(stream)
-                        stream.synchronize()
-                        graph_us = a.elapsed_time(b) * 1e3 / 500
-                        del g
-                algbw = nbytes / t / 1e9
-                fit_rows.append((st["launches"], st["hbm_bytes"], t, None if graph_us is None else graph_us * 1e-6))
-                print(json.dumps({
-                    "workload": "size-sweep-f32-sum", "nranks_virtual": n, "bytes_per_rank": nbytes, "algo": algo,
-                    "latency_us": round(t * 1e6, 3),
-                    "rankset_latency_us": None if rankset_us is None else round(rankset_us, 3),
-                    "graph_latency_us": None if graph_us is None else round(graph_us, 3),
-                    "algbw_gbs": round(algbw, 3), "busbw_gbs": round(algbw * 2 * (n - 1) / n, 3),
-                    "hbm_gbs": round(st["hbm_bytes"] / t / 1e9, 1), "hbm_frac": round(st["hbm_bytes"] / t / 1e9 / peak, 4),
-                    "launches": st["launches"], "l2_resident": 2 * n * nbytes <= 126 * 10**6}), flush=True)
+                    us = statistics.median(x.elapsed_time(y) for x, y in times) * 1e3
+                    if label == "rankset":
+                        rankset_us = us
+                    else:
+                        bound_us = us
+                # host-bound loop: 200 bound calls back to back, wall time per call
+                stream.synchronize()
+                t0 = time.perf_counter()
+                for _ in range(200):
+                    bound()
+                loop_us = (time.perf_counter() - t0) / 200 * 1e6
+                stream.synchronize()
+        algbw = nbytes / t / 1e9
+        l2 = 2 * n * nbytes <= 126 * 10**6
+        if part == "sizes" and algo in ("oneshot", "two_shot", "tree_oneshot", "ring_steps"):
+            # the algorithms whose algorithmic bytes are the DRAM bytes (the
+            # one-launch schedules serve most of theirs from L2)
+            fit_rows.append((st["launches"], st["hbm_bytes"], t, None if graph_us is None else graph_us * 1e-6, l2))
+        print(json.dumps({
+            "workload": "size-sweep-f32-sum", "part": part, "nranks_virtual": n, "bytes_per_rank": nbytes,
+            "algo": algo, "align": align, "latency_us": round(t * 1e6, 3),
+            "host_us": round(statistics.median(host_ns) / 1e3, 3),
+            "launch_call_us": round(statistics.median(launch_ns) / 1e3, 3),
+            "graph_latency_us": None if graph_us is None else round(graph_us, 3),
+            "rankset_latency_us": None if rankset_us is None else round(rankset_us, 3),
+            "bound_latency_us": None if bound_us is None else round(bound_us, 3),
+            "bound_loop_us": None if loop_us is None else round(loop_us, 3),
+            "algbw_gbs": round(algbw, 3), "busbw_gbs": round(algbw * 2 * (n - 1) / n, 3),
+            "hbm_gbs": round(st["hbm_bytes"] / t / 1e9, 1), "hbm_frac": round(st["hbm_bytes"] / t / 1e9 / peak, 4),
+            "launches": st["launches"], "l2_resident": l2}), flush=True)
+
+    def ranks(n, count, align):
+        offs = _offsets(align, n)
+        if align == "aligned":
+            return [torch.randn(count, device=dev) for _ in range(n)]
+        return [torch.randn(count + 4, device=dev)[o:o + count] for o in offs]
+
+    for n in SWEEP_NS:
+        for e in range(10, 31):
+            bufs = ranks(n, (1 << e) // ELEM, "aligned")
+            for algo in SWEEP_ALGOS:
+                point(n, 1 << e, algo, bufs, "aligned", "sizes")
             del bufs
             torch.cuda.empty_cache()
     fit_alpha_beta(fit_rows)
+    for n in PICKER_NS:
+        for e in PICKER_SIZES:
+            count = (1 << e) // ELEM
+            bufs = ranks(n, count, "aligned")
+            for algo in PICKER_ALGOS:
+                point(n, count * ELEM, algo, bufs, "aligned", "ranks")
+            del bufs
+            torch.cuda.empty_cache()
+    for align in ("shared", "mixed"):
+        for n in ALIGN_NS:
+            for e in ALIGN_SIZES:
+                count = (1 << e) // ELEM
+                bufs = ranks(n, count, align)
+                for algo in PICKER_ALGOS:
+                    point(n, count * ELEM, algo, bufs, align, "align")
+                del bufs
+                torch.cuda.empty_cache()
 
 
 def run_gpt_buckets(args):
@@ -702,9 +844,10 @@ def run_kernels(args):
     out = [torch.empty(count, device=dev) for _ in range(n)]
     # three tensors, two small and one large, sized in multiples of 8 elements so
     # every tensor's offset in the fp32 bucket has its gradient's 16-byte phase
-    # (a model's tensors usually do; mismatched phases take the scalar path)
+    # (a model's tensors usually do); with --odd the first two sizes are odd,
+    # so the next tensors start 1 and 2 elements out of phase
     small = (per // 3) & ~7
-    numels = [small, small, count - 2 * small]
+    numels = [small + 1, small + 1, count - 2 * small - 2] if args.odd else [small, small, count - 2 * small]
     grads = rrv.GradSet([[(torch.randn(m, device=dev, generator=gen) * 1e-3).to(torch.bfloat16) for m in numels]
                          for _ in range(n)])
     plan = rrv.BucketPlan(numels, "bf16", 2 * count)  # one bucket
@@ -721,7 +864,8 @@ def run_kernels(args):
         b.record(stream)
         torch.cuda.synchronize(dev)
         t = a.elapsed_time(b) / max(args.reps, 1) / 1e3
-        print(json.dumps({"workload": f"kernels-{n}x{count}-f32", "call": what, "ms": round(t * 1e3, 4),
+        print(json.dumps({"workload": f"kernels-{n}x{count}-f32" + ("-odd" if args.odd else ""), "call": what,
+                          "ms": round(t * 1e3, 4),
                           "hbm_gbs": round(st["hbm_bytes"] / t / 1e9, 1),
                           "hbm_frac": round(st["hbm_bytes"] / t / 1e9 / peak, 4), "launches": st["launches"]}),
               flush=True)

@@ -82,13 +82,20 @@ typedef enum rr_dtype { RR_F32 = 0, RR_BF16 = 1, RR_I32 = 2, RR_F16 = 3 } rr_dty
 typedef enum rr_op { RR_SUM = 0, RR_AVG = 1, RR_MAX = 2, RR_MIN = 3, RR_PROD = 4 } rr_op_t;
 
 /* Algorithms.
- *   RING         the ring schedule: 2(N-1) launches, one per ring step
- *                ([P4] "Ring all-reduce and communication volume"; [P3] s3)
+ *   RING         the ring schedule ([P4] "Ring all-reduce and communication
+ *                volume"; [P3] s3): its 2(N-1) steps in one launch when every
+ *                buffer has the same 16-byte phase -- each CTA carries one
+ *                tile of one chunk through all the steps in order, every step
+ *                reading the neighbour's copy and writing its own as the
+ *                schedule does (the same values, the same bytes) -- else one
+ *                launch per step
  *   ONESHOT      one launch that reads all N buffers once, folds in ring
  *                order and writes the result to all N ([P4] "alpha-beta
  *                model": one-shot reads every peer's buffer directly)
  *   TREE         the tree schedule: ceil(log2 N) pairwise reduce levels,
- *                then as many broadcast levels ([P3] s6)
+ *                then as many broadcast levels ([P3] s6); one launch like
+ *                RING (each CTA takes one tile through every level), else one
+ *                launch per level
  *   TREE_ONESHOT one launch that folds in the tree's pairwise order
  *   TWO_SHOT     two launches: a reduce-scatter by direct reads (chunk c
  *                folded in ring order into its owner, rank c), then an
@@ -99,8 +106,9 @@ typedef enum rr_op { RR_SUM = 0, RR_AVG = 1, RR_MAX = 2, RR_MIN = 3, RR_PROD = 4
  *                double ring): the first half of every buffer (H =
  *                ceil(count/2) elements) runs the RING schedule, the second
  *                half the mirror-image ring whose ranks send to the left, so
- *                a second-half chunk c folds downwards (c, c-1, ...); 2(N-1)
- *                launches, each rank sending half its bytes each way
+ *                a second-half chunk c folds downwards (c, c-1, ...); one
+ *                launch like RING, else 2(N-1); each rank sends half its
+ *                bytes each way
  *   AUTO         the picker's choice among RING, ONESHOT and TWO_SHOT
  *                (never a tree order or the double ring, whose bits differ);
  *                env RR_ALGO=ring|oneshot|tree|tree_oneshot|two_shot|
@@ -128,6 +136,9 @@ typedef struct rr_stats {
     uint64_t bytes_sent_max;   /* most bytes any one rank sent (ring: 2(N-1)/N*S when N | count) */
     uint64_t bytes_sent_total; /* bytes sent by all ranks together */
     uint64_t hbm_bytes;        /* algorithmic HBM bytes read + written by the kernels */
+    uint64_t host_ns;          /* host time of the call, entry to return (the library's share of the
+                                  per-call cost the alpha-beta model calls alpha) */
+    uint64_t launch_ns;        /* of which, time inside the kernel launch calls */
 } rr_stats_t;
 
 /* One transfer of the ring schedule: at (phase, step), `rank` sends chunk
@@ -402,6 +413,13 @@ rr_status_t rr_check_timeouts(void);
 const char* rr_status_string(rr_status_t status);
 const char* rr_last_error(void); /* detail of the last failure on this thread */
 int rr_version(void);
+
+/* The compute capability the library's device code was built for, as the
+ * CUDA runtime reports it for one of its kernels on the current device
+ * (cudaFuncGetAttributes' binaryVersion: 100 for sm_100a), in *version.
+ * RR_ERR_CUDA if the runtime cannot load the kernel there (no device, or one
+ * the code was not built for). */
+rr_status_t rr_binary_version(int* version);
 
 #ifdef __cplusplus
 }

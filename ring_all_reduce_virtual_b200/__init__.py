@@ -86,6 +86,21 @@ class RankSet:
     def __len__(self) -> int:
         return self.nranks
 
+    def bind(self, op="sum", algo="auto", stream=None):
+        """A callable that runs ``all_reduce(self, op, algo, stream)`` with
+        every argument converted to its C type once, so each call costs one
+        ctypes call: for small messages, repeated from Python, whose per-call
+        host cost is otherwise several microseconds of argument handling."""
+        f = lib().rr_allreduce
+        args = (self.ptrs, ctypes.c_int(self.nranks), ctypes.c_size_t(self.count), ctypes.c_int(self.dtype),
+                ctypes.c_int(_op(op)), ctypes.c_int(_algo(algo)), _stream(stream, self.device))
+
+        def call() -> None:
+            st = f(*args)
+            if st:
+                check(st, "all_reduce")
+        return call
+
 
 def _rank_args(tensors, what: str):
     """(pointer array, nranks, count, dtype code, device) of a list or a RankSet."""

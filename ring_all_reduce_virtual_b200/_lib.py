@@ -27,7 +27,8 @@ class Stats(ctypes.Structure):
     _fields_ = [
         ("algo", ctypes.c_int32), ("steps", ctypes.c_int32), ("launches", ctypes.c_int32),
         ("nranks", ctypes.c_int32), ("bytes_per_rank", ctypes.c_uint64), ("bytes_sent_max", ctypes.c_uint64),
-        ("bytes_sent_total", ctypes.c_uint64), ("hbm_bytes", ctypes.c_uint64),
+        ("bytes_sent_total", ctypes.c_uint64), ("hbm_bytes", ctypes.c_uint64), ("host_ns", ctypes.c_uint64),
+        ("launch_ns", ctypes.c_uint64),
     ]
 
 
@@ -84,6 +85,7 @@ def _declare(lib: ctypes.CDLL) -> None:
         "rr_status_string": (ctypes.c_char_p, [i]),
         "rr_last_error": (ctypes.c_char_p, []),
         "rr_version": (i, []),
+        "rr_binary_version": (st, [ctypes.POINTER(i)]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)

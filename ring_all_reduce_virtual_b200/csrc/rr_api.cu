@@ -10,6 +10,7 @@
 //   [P4] "Collective communication primitives" (ai-infra-handbooks)
 #include <algorithm>
 #include <atomic>
+#include <chrono>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
@@ -19,8 +20,11 @@
 #include <unordered_map>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "rr.h"
 #include "rr_internal.h"
+#include "rr_picker_table.h"
 
 using namespace rr;
 
@@ -41,9 +45,12 @@ namespace {
 thread_local rr_stats_t t_stats{};
 thread_local std::string t_error;
 
-// Picker parameters, set by rr_set_picker_params from any thread.
-std::atomic<double> g_launch_s{4e-6};    // cost of one launch
-std::atomic<double> g_hbm_bps{6.5e12};   // effective HBM bytes/s
+// Picker parameters: the sweep's alpha-beta fit until rr_set_picker_params
+// (from any thread) sets others, which also switches AUTO from the measured
+// table to the model.
+std::atomic<double> g_launch_s{kPickerAlphaS};   // cost of one launch
+std::atomic<double> g_hbm_bps{kPickerBetaBps};   // effective HBM bytes/s
+std::atomic<bool> g_use_model{false};
 
 rr_status_t fail(rr_status_t st, const std::string& why)
 {
@@ -107,9 +114,22 @@ struct Span {
     bool out;
 };
 
+// The spans of a call with one or two buffers per rank, kept on the stack so
+// that a call allocates nothing on the host either.
+struct SpanBuf {
+    Span s[2 * RR_MAX_RANKS];
+    size_t n = 0;
+    void push_back(const Span& x) { s[n++] = x; }
+    Span* begin() { return s; }
+    Span* end() { return s + n; }
+    size_t size() const { return n; }
+    Span& operator[](size_t i) { return s[i]; }
+};
+
 // Every output span must be non-NULL and overlap no other span; inputs may
 // overlap one another (they are only read).
-rr_status_t check_spans(std::vector<Span>& s)
+template <class Spans>
+rr_status_t check_spans(Spans& s)
 {
     for (const Span& a : s)
         if (a.lo == 0) return fail(RR_ERR_INVALID_ARG, "NULL buffer pointer");
@@ -117,6 +137,15 @@ rr_status_t check_spans(std::vector<Span>& s)
     for (size_t i = 0; i < s.size(); ++i)
         for (size_t j = i + 1; j < s.size() && s[j].lo < s[i].hi; ++j)
             if (s[i].out || s[j].out) return fail(RR_ERR_INVALID_ARG, "buffers overlap (or repeat)");
+    return RR_OK;
+}
+
+// Every pointer on a boundary of its element size (a device access of an
+// element at any other address faults).
+rr_status_t check_elem_aligned(const void* const* p, int n, size_t es)
+{
+    for (int i = 0; i < n; ++i)
+        if ((uintptr_t)p[i] % es != 0) return fail(RR_ERR_INVALID_ARG, "buffer not aligned to its element size");
     return RR_OK;
 }
 
@@ -143,6 +172,29 @@ rr_status_t check_device_ptrs(const void* const* p, int n)
         }
     }
     return RR_OK;
+}
+
+// Optional (RR_DEBUG=1): after a call that enqueued work, synchronise its
+// stream (unless the stream is being captured into a graph) and report a
+// kernel fault, or a bounded device wait that ran out, at the call that
+// caused it instead of at some later synchronisation.
+rr_status_t debug_check(rr_status_t st, cudaStream_t stream)
+{
+    static const bool debug = env_flag("RR_DEBUG");
+    if (!debug || st != RR_OK || t_stats.launches == 0) return st;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) {
+        cudaGetLastError();
+        return st;
+    }
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(e, "RR_DEBUG: the call's kernels failed");
+    unsigned int ran_out = 0, in_flight = 0;
+    if ((e = take_bulk_timeouts(&ran_out, &in_flight)) != cudaSuccess) return cuda_fail(e, "RR_DEBUG: reading the wait counters");
+    if (ran_out || in_flight)
+        return fail(RR_ERR_TIMEOUT, "RR_DEBUG: bounded device waits ran out on " + std::to_string(ran_out) +
+                                        " tiles during this call; copies not seen to land: " + std::to_string(in_flight));
+    return st;
 }
 
 uint64_t ceil_div(uint64_t a, uint64_t b) { return b ? (a + b - 1) / b : 0; }
@@ -192,6 +244,51 @@ void stats_begin(int algo, int n, uint64_t S)
     t_stats.bytes_per_rank = S;
 }
 
+uint64_t now_ns()
+{
+    return (uint64_t)std::chrono::duration_cast<std::chrono::nanoseconds>(
+               std::chrono::steady_clock::now().time_since_epoch())
+        .count();
+}
+
+// One API call: an NVTX range named for it (for timeline tools; a no-op
+// when none is attached), and its host time, entry to return, into the
+// call's statistics.
+struct CallTimer {
+    uint64_t t0;
+    explicit CallTimer(const char* name)
+    {
+        nvtxRangePushA(name);
+        t0 = now_ns();
+    }
+    ~CallTimer()
+    {
+        t_stats.host_ns = now_ns() - t0;
+        nvtxRangePop();
+    }
+};
+
+// An NVTX range around one launch of a step-by-step schedule.
+struct StepRange {
+    StepRange(const char* what, int phase, int step)
+    {
+        char name[64];
+        std::snprintf(name, sizeof name, "%s %s step %d", what, phase == RR_PHASE_REDUCE_SCATTER ? "RS" : "AG", step);
+        nvtxRangePushA(name);
+    }
+    ~StepRange() { nvtxRangePop(); }
+};
+
+// A launch, its host time added to the call's statistics.
+template <class F>
+cudaError_t timed_launch(F&& f)
+{
+    const uint64_t t0 = now_ns();
+    const cudaError_t e = f();
+    t_stats.launch_ns += now_ns() - t0;
+    return e;
+}
+
 // Build and launch one ring step (all ranks at once).
 rr_status_t ring_step_launch(void* const* bufs, int n, size_t count, rr_dtype_t dtype, rr_op_t op, int phase,
                              int step, cudaStream_t stream, bool wire = false)
@@ -219,30 +316,59 @@ rr_status_t ring_step_launch(void* const* bufs, int n, size_t count, rr_dtype_t 
     int op_eff = op;
     if (op == RR_AVG && !(phase == RR_PHASE_REDUCE_SCATTER && step == n - 2)) op_eff = RR_SUM;
     if (maxlen == 0) return RR_OK;
+    const StepRange range("ring", phase, step);
     cudaError_t e;
     if (wire && p.nin == 2)  // a bf16-wire reduce-scatter step; the all-gather copies wire values
-        e = launch_step_wire(op_eff, step == n - 2 ? 1 : 2, p, stream);
+        e = timed_launch([&] { return launch_step_wire(op_eff, step == n - 2 ? 1 : 2, p, stream); });
     else
-        e = launch_step(dtype, op_eff, p, stream);
+        e = timed_launch([&] { return launch_step(dtype, op_eff, p, stream); });
     if (e != cudaSuccess) return cuda_fail(e, "ring step launch");
     t_stats.launches += 1;
     return RR_OK;
 }
 
-rr_status_t run_ring(void* const* bufs, int n, size_t count, rr_dtype_t dtype, rr_op_t op, cudaStream_t stream)
+// The ring schedule in one launch (ring_chain_kernel: every tile of every
+// chunk carried through the 2(N-1) steps by one CTA) when every buffer is at
+// the same 16-byte phase; otherwise one launch per step.  wire: the bf16 wire
+// format (fp32 buffers).
+rr_status_t run_ring(void* const* bufs, int n, size_t count, rr_dtype_t dtype, rr_op_t op, cudaStream_t stream,
+                     bool wire = false)
 {
     const size_t es = esize(dtype);
-    std::vector<uint64_t> sent(n, 0);
+    if (same_phase(bufs, n)) {
+        ChainParams p{};
+        for (int r = 0; r < n; ++r) p.buf[r] = bufs[r];
+        p.n = n;
+        p.vec_ok = 1;
+        p.divisor = (float)n;
+        p.nhalf = 1;
+        p.count = count;
+        p.H = count;
+        p.C[0] = ceil_div(count, (uint64_t)n);
+        p.tps = std::max<uint64_t>(1, ceil_div(p.C[0], chain_tile_elems(dtype)));
+        cudaError_t e = timed_launch([&] { return launch_ring_chain(dtype, op, wire, p, stream); });
+        if (e != cudaSuccess) return cuda_fail(e, "ring launch");
+        t_stats.launches += 1;
+    } else {
+        for (int phase = RR_PHASE_REDUCE_SCATTER; phase <= RR_PHASE_ALL_GATHER; ++phase)
+            for (int s = 0; s < n - 1; ++s) {
+                rr_status_t st = ring_step_launch(bufs, n, count, dtype, op, phase, s, stream, wire);
+                if (st != RR_OK) return st;
+            }
+    }
+    const uint64_t wes = wire ? 2 : es;  // bytes a sent element takes on the wire
     for (int phase = RR_PHASE_REDUCE_SCATTER; phase <= RR_PHASE_ALL_GATHER; ++phase)
-        for (int s = 0; s < n - 1; ++s) {
-            rr_status_t st = ring_step_launch(bufs, n, count, dtype, op, phase, s, stream);
-            if (st != RR_OK) return st;
-            for (int r = 0; r < n; ++r) sent[r] += chunk_len(count, n, ring_send_chunk(phase, r, s, n)) * es;
-        }
+        for (int s = 0; s < n - 1; ++s)
+            for (int r = 0; r < n; ++r) {
+                const uint64_t b = chunk_len(count, n, ring_send_chunk(phase, r, s, n)) * wes;
+                t_stats.bytes_sent_total += b;
+            }
     t_stats.steps = 2 * (n - 1);
     for (int r = 0; r < n; ++r) {
-        t_stats.bytes_sent_max = std::max<uint64_t>(t_stats.bytes_sent_max, sent[r]);
-        t_stats.bytes_sent_total += sent[r];
+        uint64_t sent = 0;
+        for (int phase = RR_PHASE_REDUCE_SCATTER; phase <= RR_PHASE_ALL_GATHER; ++phase)
+            for (int s = 0; s < n - 1; ++s) sent += chunk_len(count, n, ring_send_chunk(phase, r, s, n)) * wes;
+        t_stats.bytes_sent_max = std::max<uint64_t>(t_stats.bytes_sent_max, sent);
     }
     // each reduce-scatter step reads 2 and writes 1 chunk per rank, each
     // all-gather step reads and writes 1: 5 (N-1) S in all
@@ -285,7 +411,8 @@ rr_status_t double_ring_step_launch(void* const* bufs, int n, size_t count, rr_d
     int op_eff = op;
     if (op == RR_AVG && !(phase == RR_PHASE_REDUCE_SCATTER && step == n - 2)) op_eff = RR_SUM;
     if (maxlen == 0) return RR_OK;
-    cudaError_t e = launch_step(dtype, op_eff, p, stream);
+    const StepRange range("double ring", phase, step);
+    cudaError_t e = timed_launch([&] { return launch_step(dtype, op_eff, p, stream); });
     if (e != cudaSuccess) return cuda_fail(e, "double ring step launch");
     t_stats.launches += 1;
     return RR_OK;
@@ -295,11 +422,34 @@ rr_status_t run_double_ring(void* const* bufs, int n, size_t count, rr_dtype_t d
                             cudaStream_t stream)
 {
     std::vector<uint64_t> sent(n, 0);
-    for (int phase = RR_PHASE_REDUCE_SCATTER; phase <= RR_PHASE_ALL_GATHER; ++phase)
-        for (int s = 0; s < n - 1; ++s) {
-            rr_status_t st = double_ring_step_launch(bufs, n, count, dtype, op, phase, s, stream, sent);
-            if (st != RR_OK) return st;
-        }
+    if (same_phase(bufs, n)) {  // both rings in one launch (ring_chain_kernel, two halves)
+        const uint64_t H = (count + 1) / 2, cb = count - H;
+        ChainParams p{};
+        for (int r = 0; r < n; ++r) p.buf[r] = bufs[r];
+        p.n = n;
+        p.vec_ok = 1;
+        p.divisor = (float)n;
+        p.nhalf = 2;
+        p.count = count;
+        p.H = H;
+        p.C[0] = ceil_div(H, (uint64_t)n);
+        p.C[1] = ceil_div(cb, (uint64_t)n);
+        p.tps = std::max<uint64_t>(1, ceil_div(std::max(p.C[0], p.C[1]), chain_tile_elems(dtype)));
+        cudaError_t e = timed_launch([&] { return launch_ring_chain(dtype, op, false, p, stream); });
+        if (e != cudaSuccess) return cuda_fail(e, "double ring launch");
+        t_stats.launches += 1;
+        for (int phase = RR_PHASE_REDUCE_SCATTER; phase <= RR_PHASE_ALL_GATHER; ++phase)
+            for (int s = 0; s < n - 1; ++s)
+                for (int r = 0; r < n; ++r)
+                    sent[r] += (chunk_len(H, n, ring_send_chunk(phase, r, s, n)) +
+                                chunk_len(cb, n, ccw_send_chunk(phase, r, s, n))) * esize(dtype);
+    } else {
+        for (int phase = RR_PHASE_REDUCE_SCATTER; phase <= RR_PHASE_ALL_GATHER; ++phase)
+            for (int s = 0; s < n - 1; ++s) {
+                rr_status_t st = double_ring_step_launch(bufs, n, count, dtype, op, phase, s, stream, sent);
+                if (st != RR_OK) return st;
+            }
+    }
     t_stats.steps = 2 * (n - 1);
     for (int r = 0; r < n; ++r) {
         t_stats.bytes_sent_max = std::max<uint64_t>(t_stats.bytes_sent_max, sent[r]);
@@ -325,6 +475,19 @@ rr_status_t run_tree(void* const* bufs, int n, size_t count, rr_dtype_t dtype, r
     const bool vec = same_phase(bufs, n);
     std::vector<uint64_t> sent(n, 0);
     uint64_t pairs_total = 0;
+    if (vec) {  // every level in one launch (tree_chain_kernel)
+        ChainParams p{};
+        for (int r = 0; r < n; ++r) p.buf[r] = bufs[r];
+        p.n = n;
+        p.vec_ok = 1;
+        p.divisor = (float)n;
+        p.count = count;
+        p.H = count;
+        p.tps = std::max<uint64_t>(1, ceil_div(count, chain_tile_elems(dtype)));
+        cudaError_t e = timed_launch([&] { return launch_tree_chain(dtype, op, p, stream); });
+        if (e != cudaSuccess) return cuda_fail(e, "tree launch");
+        t_stats.launches += 1;
+    }
     for (int pass = 0; pass < 2; ++pass) {
         for (int i = 0; i < L; ++i) {
             const int l = pass == 0 ? i : L - 1 - i;
@@ -349,9 +512,10 @@ rr_status_t run_tree(void* const* bufs, int n, size_t count, rr_dtype_t dtype, r
                 sg.len = count;
                 ++pairs_total;
             }
+            if (vec) continue;  // counted only: the levels ran in the one launch above
             int op_eff = op;
             if (op == RR_AVG && !(pass == 0 && l == L - 1)) op_eff = RR_SUM;
-            cudaError_t e = launch_step(dtype, op_eff, p, stream);
+            cudaError_t e = timed_launch([&] { return launch_step(dtype, op_eff, p, stream); });
             if (e != cudaSuccess) return cuda_fail(e, "tree level launch");
             t_stats.launches += 1;
         }
@@ -386,13 +550,88 @@ rr_status_t run_rank_kernel(int kind, const void* const* in, void* const* out, i
     p.hi = hi;
     p.owner_only = owner_only ? 1 : 0;
     p.waits = bulk_wait_counters();  // looked up once per launch
-    cudaError_t e = launch_rank_kernel(kind, dtype, op, p, stream);
+    cudaError_t e = timed_launch([&] { return launch_rank_kernel(kind, dtype, op, p, stream); });
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     t_stats.launches += 1;
     return RR_OK;
 }
 
-rr_algo_t resolve_algo(rr_algo_t algo, int n, size_t count, rr_dtype_t dtype)
+// Alignment class of a call's buffers, as the picker's table keys it: 0 all
+// 16-byte aligned, 1 all at one other 16-byte phase, 2 phases that differ.
+int align_class(const void* const* p, int n)
+{
+    if (!same_phase(p, n)) return 2;
+    return ((uintptr_t)p[0] & 15u) ? 1 : 0;
+}
+
+int log2_round(double x) { return x <= 1 ? 0 : (int)std::lround(std::log2(x)); }
+
+// The alpha-beta model of [P3] section 4 on one GPU: every "link" is HBM, a
+// step costs one launch, and its bytes are the HBM bytes it reads and writes
+// (ring 5(N-1) S over 2(N-1) launches -- one launch when the buffers share a
+// phase, but the model keeps the schedule's steps --, one-shot 2 N S in one,
+// two-shot (2N+1) S in two).  bf16 and fp16 always take ONESHOT: the ring
+// rounds its 16-bit partials at every hop, the fp32-accumulating one-shot
+// does not ([P1] s5.3).
+rr_algo_t model_pick(int nranks, size_t count, rr_dtype_t dtype)
+{
+    if (dtype == RR_BF16 || dtype == RR_F16 || nranks <= 1) return RR_ALGO_ONESHOT;
+    const double n = nranks, S = (double)count * (double)esize(dtype);
+    const double alpha = g_launch_s.load(), beta = g_hbm_bps.load();
+    const double ring = 2 * (n - 1) * alpha + 5 * (n - 1) * S / beta;
+    const double one = alpha + 2 * n * S / beta;
+    const double two = 2 * alpha + (2 * n + 1) * S / beta;
+    if (ring < one && ring < two) return RR_ALGO_RING;
+    return two < one ? RR_ALGO_TWO_SHOT : RR_ALGO_ONESHOT;
+}
+
+// The measured table's choice for (N, bytes per rank, alignment class): among
+// the points measured in that class (the aligned class if the table has none
+// of it), the nearest measured rank count (in log2 ratio; the smaller on a
+// tie), then the nearest measured size there.  RR_ALGO_AUTO if the table is
+// empty.
+rr_algo_t table_pick(int n, uint64_t bytes, int align)
+{
+    bool have = false;
+    for (const PickerPoint& e : kPickerTable) have = have || e.align == align;
+    if (!have) align = 0;
+    const int lb = log2_round((double)bytes);
+    double best_dn = 1e30;
+    int best_n = 0;
+    for (const PickerPoint& e : kPickerTable) {
+        if (e.align != align) continue;
+        const double dn = std::fabs(std::log2((double)e.nranks / (double)n));
+        if (dn < best_dn - 1e-12 || (std::fabs(dn - best_dn) <= 1e-12 && e.nranks < best_n)) {
+            best_dn = dn;
+            best_n = e.nranks;
+        }
+    }
+    int best_d = 1 << 30;
+    rr_algo_t pick = RR_ALGO_AUTO;
+    for (const PickerPoint& e : kPickerTable) {
+        if (e.nranks != best_n || e.align != align) continue;
+        const int d = std::abs(e.log2_bytes - lb);
+        if (d < best_d) {
+            best_d = d;
+            pick = (rr_algo_t)e.algo;
+        }
+    }
+    return pick;
+}
+
+// AUTO's choice for a call on these buffers.  bf16 and fp16 never take RING
+// (its partials would be rounded at every hop; [P1] s5.3).
+rr_algo_t pick_for(int n, size_t count, rr_dtype_t dtype, int align)
+{
+    if (n <= 1) return RR_ALGO_ONESHOT;
+    rr_algo_t a = RR_ALGO_AUTO;
+    if (!g_use_model.load(std::memory_order_relaxed)) a = table_pick(n, (uint64_t)count * esize(dtype), align);
+    if (a == RR_ALGO_AUTO) a = model_pick(n, count, dtype);
+    if (a == RR_ALGO_RING && (dtype == RR_BF16 || dtype == RR_F16)) a = RR_ALGO_ONESHOT;
+    return a;
+}
+
+rr_algo_t resolve_algo(rr_algo_t algo, int n, size_t count, rr_dtype_t dtype, const void* const* bufs)
 {
     if (algo != RR_ALGO_AUTO) return algo;
     static const int forced = [] {
@@ -407,7 +646,7 @@ rr_algo_t resolve_algo(rr_algo_t algo, int n, size_t count, rr_dtype_t dtype)
         return -1;
     }();
     if (forced >= 0) return (rr_algo_t)forced;
-    return rr_pick_algo(n, count, dtype);
+    return pick_for(n, count, dtype, bufs ? align_class(bufs, n) : 0);
 }
 
 // Slice size of the pipelined host-buffer all-reduce, per rank: 8 MiB, or
@@ -478,6 +717,17 @@ extern "C" {
 
 int rr_version(void) { return RR_VERSION; }
 
+rr_status_t rr_binary_version(int* version)
+{
+    if (!version) return fail(RR_ERR_INVALID_ARG, "NULL version pointer");
+    const cudaError_t e = kernel_binary_version(version);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return cuda_fail(e, "cudaFuncGetAttributes");
+    }
+    return RR_OK;
+}
+
 const char* rr_status_string(rr_status_t s)
 {
     switch (s) {
@@ -502,6 +752,7 @@ rr_status_t rr_get_stats(rr_stats_t* out)
 rr_status_t rr_allreduce(void* const* bufs, int nranks, size_t count, rr_dtype_t dtype, rr_op_t op,
                          rr_algo_t algo, cudaStream_t stream)
 {
+    CallTimer timer("rr_allreduce");
     rr_status_t st = check_basic(nranks, dtype, op);
     if (st != RR_OK) return st;
     if ((st = check_count(count)) != RR_OK) return st;
@@ -509,13 +760,14 @@ rr_status_t rr_allreduce(void* const* bufs, int nranks, size_t count, rr_dtype_t
     if (!bufs) return fail(RR_ERR_INVALID_ARG, "NULL bufs array");
     const int n = nranks;
     const size_t es = esize(dtype);
-    const rr_algo_t a = resolve_algo(algo, n, count, dtype);
+    const rr_algo_t a = resolve_algo(algo, n, count, dtype, count && n <= RR_MAX_RANKS ? bufs : nullptr);
     stats_begin(a, n, (uint64_t)count * es);
     if (count == 0) return RR_OK;
-    std::vector<Span> spans;
+    SpanBuf spans;
     for (int r = 0; r < n; ++r)
         spans.push_back({(uintptr_t)bufs[r], (uintptr_t)bufs[r] + count * es, true});
     if ((st = check_spans(spans)) != RR_OK) return st;
+    if ((st = check_elem_aligned(bufs, n, es)) != RR_OK) return st;
     if ((st = check_device_ptrs(bufs, n)) != RR_OK) return st;
     if (n == 1) return RR_OK;  // one rank already holds the reduction (AVG: x / 1 == x)
     const uint64_t S = (uint64_t)count * es;
@@ -576,12 +828,13 @@ rr_status_t rr_allreduce(void* const* bufs, int nranks, size_t count, rr_dtype_t
         return fail(RR_ERR_INVALID_ARG, "unknown algo");
     }
     log_call("allreduce", n, count, dtype, op, a);
-    return st;
+    return debug_check(st, stream);
 }
 
 rr_status_t rr_allreduce_wire(void* const* bufs, int nranks, size_t count, rr_op_t op, rr_dtype_t wire,
                               rr_algo_t algo, cudaStream_t stream)
 {
+    CallTimer timer("rr_allreduce_wire");
     rr_status_t st = check_basic(nranks, RR_F32, op);
     if (st != RR_OK) return st;
     if ((st = check_count(count)) != RR_OK) return st;
@@ -595,18 +848,14 @@ rr_status_t rr_allreduce_wire(void* const* bufs, int nranks, size_t count, rr_op
     const uint64_t S = (uint64_t)count * 4;
     stats_begin(a, n, S);
     if (count == 0) return RR_OK;
-    std::vector<Span> spans;
+    SpanBuf spans;
     for (int r = 0; r < n; ++r) spans.push_back({(uintptr_t)bufs[r], (uintptr_t)bufs[r] + S, true});
     if ((st = check_spans(spans)) != RR_OK) return st;
+    if ((st = check_elem_aligned(bufs, n, 4)) != RR_OK) return st;
     if ((st = check_device_ptrs(bufs, n)) != RR_OK) return st;
     if (n == 1) return RR_OK;  // nothing crosses a wire
     if (a == RR_ALGO_RING) {
-        for (int phase = RR_PHASE_REDUCE_SCATTER; phase <= RR_PHASE_ALL_GATHER; ++phase)
-            for (int s = 0; s < n - 1; ++s)
-                if ((st = ring_step_launch(bufs, n, count, RR_F32, op, phase, s, stream, true)) != RR_OK) return st;
-        t_stats.steps = 2 * (n - 1);
-        t_stats.bytes_sent_max = 2ull * (n - 1) * ceil_div(count, (uint64_t)n) * 2;  // bf16 on the wire
-        t_stats.hbm_bytes = 5ull * (uint64_t)(n - 1) * S;
+        if ((st = run_ring(bufs, n, count, RR_F32, op, stream, true)) != RR_OK) return st;
     } else {
         RankParams p{};
         for (int r = 0; r < n; ++r) p.in[r] = p.out[r] = bufs[r];
@@ -620,21 +869,22 @@ rr_status_t rr_allreduce_wire(void* const* bufs, int nranks, size_t count, rr_op
         p.lo = 0;
         p.hi = UINT64_MAX;
         p.waits = bulk_wait_counters();
-        cudaError_t e = launch_oneshot_wire(op, p, p.nseg * p.tps, stream);
+        cudaError_t e = timed_launch([&] { return launch_oneshot_wire(op, p, p.nseg * p.tps, stream); });
         if (e != cudaSuccess) return cuda_fail(e, "wire one-shot launch");
         t_stats.launches = 1;
         t_stats.steps = 1;
         t_stats.bytes_sent_max = (uint64_t)(n - 1) * count * 2;  // each rank's values go out as bf16
+        t_stats.bytes_sent_total = (uint64_t)n * t_stats.bytes_sent_max;
         t_stats.hbm_bytes = 2ull * n * S;
     }
-    t_stats.bytes_sent_total = (uint64_t)n * t_stats.bytes_sent_max;
     log_call("allreduce_wire", n, count, RR_F32, op, a);
-    return RR_OK;
+    return debug_check(RR_OK, stream);
 }
 
 rr_status_t rr_allreduce_host(void* const* host_bufs, void* const* dev_bufs, int nranks, size_t count,
                               rr_dtype_t dtype, rr_op_t op, rr_algo_t algo, cudaStream_t stream)
 {
+    CallTimer timer("rr_allreduce_host");
     rr_status_t st = check_basic(nranks, dtype, op);
     if (st != RR_OK) return st;
     if ((st = check_count(count)) != RR_OK) return st;
@@ -644,13 +894,14 @@ rr_status_t rr_allreduce_host(void* const* host_bufs, void* const* dev_bufs, int
     const size_t es = esize(dtype), bytes = count * es;
     for (int r = 0; r < n && count; ++r)
         if (!host_bufs[r]) return fail(RR_ERR_INVALID_ARG, "NULL host buffer");
-    std::vector<Span> spans;  // host buffers are written back too (one address space with UVA)
+    SpanBuf spans;  // host buffers are written back too (one address space with UVA)
     for (int r = 0; r < n && count; ++r) {
         spans.push_back({(uintptr_t)dev_bufs[r], (uintptr_t)dev_bufs[r] + bytes, true});
         spans.push_back({(uintptr_t)host_bufs[r], (uintptr_t)host_bufs[r] + bytes, true});
     }
     if ((st = check_spans(spans)) != RR_OK) return st;
-    const rr_algo_t a = resolve_algo(algo, n, count, dtype);
+    if ((st = check_elem_aligned(dev_bufs, n, es)) != RR_OK) return st;
+    const rr_algo_t a = resolve_algo(algo, n, count, dtype, count ? dev_bufs : nullptr);
     if (count == 0) return rr_allreduce(dev_bufs, n, 0, dtype, op, a, stream);
     const bool sliced = n > 1 && (a == RR_ALGO_ONESHOT || a == RR_ALGO_TREE_ONESHOT) && bytes > host_slice_bytes();
     if (!sliced) {  // copy in, reduce, copy out, all on the caller's stream
@@ -714,7 +965,9 @@ rr_status_t rr_allreduce_host(void* const* host_bufs, void* const* dev_bufs, int
     }
     if ((st = ck(cudaEventRecord(hp->done, hp->out), "event record")) != RR_OK) return st;
     if ((st = ck(cudaStreamWaitEvent(stream, hp->done, 0), "stream wait")) != RR_OK) return st;
+    const uint64_t launch_ns = t_stats.launch_ns;
     stats_begin(a, n, bytes);
+    t_stats.launch_ns = launch_ns;
     t_stats.steps = 1;
     t_stats.launches = launches;
     t_stats.bytes_sent_max = (uint64_t)(n - 1) * bytes;
@@ -727,6 +980,7 @@ rr_status_t rr_allreduce_host(void* const* host_bufs, void* const* dev_bufs, int
 rr_status_t rr_ring_step(void* const* bufs, int nranks, size_t count, rr_dtype_t dtype, rr_op_t op,
                          rr_phase_t phase, int step, cudaStream_t stream)
 {
+    CallTimer timer("rr_ring_step");
     rr_status_t st = check_basic(nranks, dtype, op);
     if (st != RR_OK) return st;
     if ((st = check_count(count)) != RR_OK) return st;
@@ -737,10 +991,11 @@ rr_status_t rr_ring_step(void* const* bufs, int nranks, size_t count, rr_dtype_t
     const size_t es = esize(dtype);
     stats_begin(RR_ALGO_RING, nranks, (uint64_t)count * es);
     if (count == 0) return RR_OK;
-    std::vector<Span> spans;
+    SpanBuf spans;
     for (int r = 0; r < nranks; ++r)
         spans.push_back({(uintptr_t)bufs[r], (uintptr_t)bufs[r] + count * es, true});
     if ((st = check_spans(spans)) != RR_OK) return st;
+    if ((st = check_elem_aligned(bufs, nranks, es)) != RR_OK) return st;
     if ((st = check_device_ptrs(bufs, nranks)) != RR_OK) return st;
     st = ring_step_launch(bufs, nranks, count, dtype, op, phase, step, stream);
     t_stats.steps = 1;
@@ -751,7 +1006,7 @@ rr_status_t rr_ring_step(void* const* bufs, int nranks, size_t count, rr_dtype_t
     }
     t_stats.hbm_bytes = (phase == RR_PHASE_REDUCE_SCATTER ? 3ull : 2ull) * count * es;
     log_call("ring_step", nranks, count, dtype, op, RR_ALGO_RING);
-    return st;
+    return debug_check(st, stream);
 }
 
 rr_status_t rr_ring_schedule(int nranks, size_t count, rr_dtype_t dtype, rr_ring_event_t* events,
@@ -782,6 +1037,7 @@ rr_status_t rr_ring_schedule(int nranks, size_t count, rr_dtype_t dtype, rr_ring
 rr_status_t rr_reduce_scatter(const void* const* send, void* const* recv, int nranks, size_t recvcount,
                               rr_dtype_t dtype, rr_op_t op, rr_algo_t algo, cudaStream_t stream)
 {
+    CallTimer timer("rr_reduce_scatter");
     rr_status_t st = check_basic(nranks, dtype, op);
     if (st != RR_OK) return st;
     if ((st = check_count(recvcount)) != RR_OK) return st;
@@ -793,12 +1049,13 @@ rr_status_t rr_reduce_scatter(const void* const* send, void* const* recv, int nr
     const uint64_t S = (uint64_t)n * recvcount * es;
     stats_begin(RR_ALGO_ONESHOT, n, S);
     if (recvcount == 0) return RR_OK;
-    std::vector<Span> spans;
+    SpanBuf spans;
     for (int r = 0; r < n; ++r) {
         spans.push_back({(uintptr_t)send[r], (uintptr_t)send[r] + S, false});
         spans.push_back({(uintptr_t)recv[r], (uintptr_t)recv[r] + recvcount * es, true});
     }
     if ((st = check_spans(spans)) != RR_OK) return st;
+    if ((st = check_elem_aligned(send, n, es)) != RR_OK || (st = check_elem_aligned(recv, n, es)) != RR_OK) return st;
     if ((st = check_device_ptrs(send, n)) != RR_OK || (st = check_device_ptrs(recv, n)) != RR_OK) return st;
     const uint64_t tps = std::max<uint64_t>(1, ceil_div(recvcount, tile_elems(dtype, reduce_vpt(n))));
     st = run_rank_kernel(kReduceScatter, send, recv, n, recvcount, (uint64_t)n * recvcount, (uint64_t)n, tps,
@@ -808,12 +1065,13 @@ rr_status_t rr_reduce_scatter(const void* const* send, void* const* recv, int nr
     t_stats.bytes_sent_total = (uint64_t)n * t_stats.bytes_sent_max;
     t_stats.hbm_bytes = (uint64_t)(n + 1) * S;
     log_call("reduce_scatter", n, recvcount, dtype, op, RR_ALGO_ONESHOT);
-    return st;
+    return debug_check(st, stream);
 }
 
 rr_status_t rr_all_gather(const void* const* send, void* const* recv, int nranks, size_t sendcount,
                           rr_dtype_t dtype, rr_algo_t algo, cudaStream_t stream)
 {
+    CallTimer timer("rr_all_gather");
     rr_status_t st = check_basic(nranks, dtype, RR_SUM);
     if (st != RR_OK) return st;
     if ((st = check_count(sendcount)) != RR_OK) return st;
@@ -825,12 +1083,13 @@ rr_status_t rr_all_gather(const void* const* send, void* const* recv, int nranks
     const uint64_t S = (uint64_t)n * sendcount * es;
     stats_begin(RR_ALGO_ONESHOT, n, S);
     if (sendcount == 0) return RR_OK;
-    std::vector<Span> spans;
+    SpanBuf spans;
     for (int r = 0; r < n; ++r) {
         spans.push_back({(uintptr_t)send[r], (uintptr_t)send[r] + sendcount * es, false});
         spans.push_back({(uintptr_t)recv[r], (uintptr_t)recv[r] + S, true});
     }
     if ((st = check_spans(spans)) != RR_OK) return st;
+    if ((st = check_elem_aligned(send, n, es)) != RR_OK || (st = check_elem_aligned(recv, n, es)) != RR_OK) return st;
     if ((st = check_device_ptrs(send, n)) != RR_OK || (st = check_device_ptrs(recv, n)) != RR_OK) return st;
     const uint64_t tps = std::max<uint64_t>(1, ceil_div(sendcount, tile_elems(dtype, kVptMove)));
     st = run_rank_kernel(kAllGather, send, recv, n, sendcount, (uint64_t)n * sendcount, (uint64_t)n, tps, dtype,
@@ -840,12 +1099,13 @@ rr_status_t rr_all_gather(const void* const* send, void* const* recv, int nranks
     t_stats.bytes_sent_total = (uint64_t)n * t_stats.bytes_sent_max;
     t_stats.hbm_bytes = (uint64_t)(n + 1) * S;
     log_call("all_gather", n, sendcount, dtype, RR_SUM, RR_ALGO_ONESHOT);
-    return st;
+    return debug_check(st, stream);
 }
 
 rr_status_t rr_all_to_all(const void* const* send, void* const* recv, int nranks, size_t count_per_peer,
                           rr_dtype_t dtype, cudaStream_t stream)
 {
+    CallTimer timer("rr_all_to_all");
     rr_status_t st = check_basic(nranks, dtype, RR_SUM);
     if (st != RR_OK) return st;
     if ((st = check_count(count_per_peer)) != RR_OK) return st;
@@ -855,12 +1115,13 @@ rr_status_t rr_all_to_all(const void* const* send, void* const* recv, int nranks
     const uint64_t S = (uint64_t)n * count_per_peer * es;
     stats_begin(RR_ALGO_ONESHOT, n, S);
     if (count_per_peer == 0) return RR_OK;
-    std::vector<Span> spans;
+    SpanBuf spans;
     for (int r = 0; r < n; ++r) {
         spans.push_back({(uintptr_t)send[r], (uintptr_t)send[r] + S, false});
         spans.push_back({(uintptr_t)recv[r], (uintptr_t)recv[r] + S, true});
     }
     if ((st = check_spans(spans)) != RR_OK) return st;
+    if ((st = check_elem_aligned(send, n, es)) != RR_OK || (st = check_elem_aligned(recv, n, es)) != RR_OK) return st;
     if ((st = check_device_ptrs(send, n)) != RR_OK || (st = check_device_ptrs(recv, n)) != RR_OK) return st;
     const uint64_t tps = std::max<uint64_t>(1, ceil_div(count_per_peer, tile_elems(dtype, kVptMove)));
     st = run_rank_kernel(kAllToAll, send, recv, n, count_per_peer, (uint64_t)n * count_per_peer,
@@ -870,7 +1131,7 @@ rr_status_t rr_all_to_all(const void* const* send, void* const* recv, int nranks
     t_stats.bytes_sent_total = (uint64_t)n * t_stats.bytes_sent_max;
     t_stats.hbm_bytes = 2ull * n * S;
     log_call("all_to_all", n, count_per_peer, dtype, RR_SUM, RR_ALGO_ONESHOT);
-    return st;
+    return debug_check(st, stream);
 }
 
 // ------------------------------------------------------------- buckets --
@@ -979,6 +1240,7 @@ rr_status_t bucket_check(const rr_bucket_plan_t* plan, int bucket, const void* c
 static rr_status_t bucket_copy(const rr_bucket_plan_t* plan, int bucket, const void* const* grads,
                                void* const* buckets, int nranks, int op, bool pack, cudaStream_t stream)
 {
+    CallTimer timer(pack ? "rr_bucket_pack" : "rr_bucket_unpack");
     int t0 = 0, nt = 0;
     rr_status_t st = bucket_check(plan, bucket, grads, nranks, &t0, &nt);
     if (st != RR_OK) return st;
@@ -1015,8 +1277,10 @@ static rr_status_t bucket_copy(const rr_bucket_plan_t* plan, int bucket, const v
         for (int r = 0; r < n; ++r) p->bucket[r] = buckets[r];
         p->vec_ok = v;
         if (maxlen == 0) continue;
-        cudaError_t e = pack ? launch_bucket_pack(plan->grad_dtype, *p, stream)
-                             : launch_bucket_unpack(plan->grad_dtype, op, *p, stream);
+        cudaError_t e = timed_launch([&] {
+            return pack ? launch_bucket_pack(plan->grad_dtype, *p, stream)
+                        : launch_bucket_unpack(plan->grad_dtype, op, *p, stream);
+        });
         if (e != cudaSuccess) {
             delete p;
             return cuda_fail(e, pack ? "bucket pack launch" : "bucket unpack launch");
@@ -1071,6 +1335,7 @@ rr_status_t rr_bucket_allreduce_range(const rr_bucket_plan_t* plan, int first_bu
 static rr_status_t bucket_fold_range(const rr_bucket_plan_t* plan, int b0, int nb, void* const* grads, int nranks,
                                      rr_op_t op, cudaStream_t stream, uint64_t max_grid)
 {
+    CallTimer timer("rr_bucket_allreduce");
     if (op != RR_SUM && op != RR_AVG) return fail(RR_ERR_UNSUPPORTED, "bucket all-reduce takes SUM or AVG");
     int t0 = 0, nt = 0;
     rr_status_t st = bucket_range_check(plan, b0, nb, grads, nranks, &t0, &nt);
@@ -1092,7 +1357,7 @@ static rr_status_t bucket_fold_range(const rr_bucket_plan_t* plan, int b0, int n
         bool v = true;
         for (int t = 0; t < ntens; ++t) v = v && same_phase(&p->grad[t * n], n);
         p->vec_ok = v;
-        cudaError_t e = launch_bucket_fold(plan->grad_dtype, op, *p, stream, max_grid);
+        cudaError_t e = timed_launch([&] { return launch_bucket_fold(plan->grad_dtype, op, *p, stream, max_grid); });
         if (e != cudaSuccess) return cuda_fail(e, "bucket all-reduce launch");
         t_stats.launches += 1;
         return RR_OK;
@@ -1125,7 +1390,7 @@ static rr_status_t bucket_fold_range(const rr_bucket_plan_t* plan, int b0, int n
     t_stats.bytes_sent_total = (uint64_t)n * t_stats.bytes_sent_max;
     t_stats.hbm_bytes = 2ull * n * total * es;
     log_call("bucket_allreduce", n, total, (rr_dtype_t)plan->grad_dtype, op, RR_ALGO_ONESHOT);
-    return st;
+    return debug_check(st, stream);
 }
 
 extern "C" {
@@ -1288,27 +1553,27 @@ rr_status_t rr_cost_model(rr_algo_t algo, int nranks, double bytes, double alpha
 
 rr_status_t rr_set_picker_params(double launch_s, double hbm_bytes_per_s)
 {
+    if (launch_s == 0 && hbm_bytes_per_s == 0) {  // back to the measured table and the sweep's fit
+        g_launch_s.store(kPickerAlphaS);
+        g_hbm_bps.store(kPickerBetaBps);
+        g_use_model.store(false);
+        return RR_OK;
+    }
     if (!(launch_s >= 0) || !(hbm_bytes_per_s > 0)) return fail(RR_ERR_INVALID_ARG, "bad picker parameters");
     g_launch_s.store(launch_s);
     g_hbm_bps.store(hbm_bytes_per_s);
+    g_use_model.store(true);
     return RR_OK;
 }
 
-// On one GPU every "link" is HBM: a step costs one launch, and its bytes are
-// the HBM bytes it reads and writes (ring 5(N-1) S over 2(N-1) launches,
-// one-shot 2 N S in one).  bf16 and fp16 always take ONESHOT: the ring rounds
-// its 16-bit partials at every hop, the fp32-accumulating one-shot does not
-// ([P1] s5.3).
 rr_algo_t rr_pick_algo(int nranks, size_t count, rr_dtype_t dtype)
 {
-    if (dtype == RR_BF16 || dtype == RR_F16 || nranks <= 1) return RR_ALGO_ONESHOT;
-    const double n = nranks, S = (double)count * (double)esize(dtype);
-    const double alpha = g_launch_s.load(), beta = g_hbm_bps.load();
-    const double ring = 2 * (n - 1) * alpha + 5 * (n - 1) * S / beta;
-    const double one = alpha + 2 * n * S / beta;
-    const double two = 2 * alpha + (2 * n + 1) * S / beta;
-    if (ring < one && ring < two) return RR_ALGO_RING;
-    return two < one ? RR_ALGO_TWO_SHOT : RR_ALGO_ONESHOT;
+    if (nranks <= 1) return RR_ALGO_ONESHOT;
+    rr_algo_t a = RR_ALGO_AUTO;
+    if (!g_use_model.load(std::memory_order_relaxed)) a = table_pick(nranks, (uint64_t)count * esize(dtype), 0);
+    if (a == RR_ALGO_AUTO) a = model_pick(nranks, count, dtype);
+    if (a == RR_ALGO_RING && (dtype == RR_BF16 || dtype == RR_F16)) a = RR_ALGO_ONESHOT;
+    return a;
 }
 
 }  // extern "C"

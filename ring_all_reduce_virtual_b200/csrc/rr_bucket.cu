@@ -31,6 +31,16 @@ struct Quad<F32T> {
     __device__ static __forceinline__ void st(float* p, const R& r) { stv(p, r); }
     __device__ static __forceinline__ void to_f(const R& r, float (&a)[4]) { F32T::unpack(r, a); }
     __device__ static __forceinline__ R from_f(const float (&a)[4]) { return F32T::pack(a); }
+    // The four elements that start d elements into the aligned window lo:hi.
+    __device__ static __forceinline__ R shift(const R& lo, const R& hi, int d)
+    {
+        switch (d) {
+        case 1: return make_uint4(lo.y, lo.z, lo.w, hi.x);
+        case 2: return make_uint4(lo.z, lo.w, hi.x, hi.y);
+        case 3: return make_uint4(lo.w, hi.x, hi.y, hi.z);
+        }
+        return lo;
+    }
 };
 
 // The 16-bit types (bf16, fp16): a quad is 8 bytes, two packed pairs.
@@ -48,6 +58,14 @@ struct Quad16 {
     {
         return make_uint2(X::pack2(a[0], a[1]), X::pack2(a[2], a[3]));
     }
+    // The four elements that start d elements into the aligned window lo:hi
+    // (element j is the low half of word j / 2 when j is even).
+    __device__ static __forceinline__ R shift(const R& lo, const R& hi, int d)
+    {
+        const uint32_t w0 = d >= 2 ? lo.y : lo.x, w1 = d >= 2 ? hi.x : lo.y, w2 = d >= 2 ? hi.y : hi.x;
+        if (d & 1) return make_uint2(__funnelshift_r(w0, w1, 16), __funnelshift_r(w1, w2, 16));
+        return make_uint2(w0, w1);
+    }
 };
 
 template <>
@@ -56,56 +74,79 @@ struct Quad<BF16T> : Quad16<BF16T> {};
 template <>
 struct Quad<F16T> : Quad16<F16T> {};
 
+// The quads of one tile of a conversion (see convert_tile), with the source
+// quads D elements out of step with the destination's: D = 0 reads one
+// aligned source quad per destination quad; D > 0 reads that quad and the
+// next and shifts them into place.  Every load of the thread is issued
+// before the first one is used, so Q (or 2Q) loads are in flight.
+template <class In, class Out, int OP, int Q, bool SHIFT>
+__device__ __forceinline__ void convert_quads(const typename In::T* s0, typename Out::T* dst, uint64_t head, uint64_t nq,
+                                              uint64_t tile, int d, float divisor)
+{
+    constexpr uint64_t TQ = (uint64_t)kThreads * Q;
+    // passes of 4 quads per thread (64 bytes of fp32 on the wider side), 2
+    // when a quad takes two loads
+    constexpr int QP = SHIFT ? 2 : 4;
+    constexpr int P = Q / QP;
+    static_assert(QP >= 1 && Q % QP == 0, "whole passes");
+    const uint64_t tid = threadIdx.x;
+#pragma unroll
+    for (int pass = 0; pass < P; ++pass) {
+        typename Quad<In>::R lo[QP], hi[QP];
+#pragma unroll
+        for (int k = 0; k < QP; ++k) {
+            const uint64_t q = tile * TQ + (uint64_t)(pass * QP + k) * kThreads + tid;
+            if (q < nq) {
+                lo[k] = Quad<In>::ld(s0 + q * 4);
+                if constexpr (SHIFT) hi[k] = Quad<In>::ld(s0 + q * 4 + 4);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < QP; ++k) {
+            const uint64_t q = tile * TQ + (uint64_t)(pass * QP + k) * kThreads + tid;
+            if (q >= nq) continue;
+            float a[4];
+            if constexpr (SHIFT) Quad<In>::to_f(Quad<In>::shift(lo[k], hi[k], d), a);
+            else Quad<In>::to_f(lo[k], a);
+#pragma unroll
+            for (int l = 0; l < 4; ++l) a[l] = finish<OP>(a[l], divisor);
+            Quad<Out>::st(dst + head + q * 4, Quad<Out>::from_f(a));
+        }
+    }
+}
+
 // Convert one tile of a segment from In's element type to Out's, dividing by
 // `divisor` first when OP is AVG.  A tile is kThreads * Q quads, Q chosen so
 // that it covers kThreads * kUnitsPerThread 16-byte vectors of the narrower
-// type (bucket_tile_elems).  When src and dst reach a quad boundary after the
-// same scalar head, the body moves quads and tile 0 also does the head and
-// the tail (< 4 elements each); otherwise every element is scalar.
+// type (bucket_tile_elems).  The quads are aligned to the destination: after
+// a scalar head up to dst's first quad boundary, every quad is one aligned
+// store, and its source elements -- which start d = (phase of src - phase of
+// dst) mod 4 elements into an aligned source quad -- are read as that quad
+// and, when d > 0, the next one, and shifted into place.  The window's second
+// quad holds at least one element of the source quad, so no load reaches
+// past the aligned block of the segment's last element (nor before the
+// block of its first).  Tile 0 also does the head and the tail (< 4 elements
+// each).
 template <class In, class Out, int OP, int Q = kUnitsPerThread * (In::L > Out::L ? In::L : Out::L) / 4>
 __device__ __forceinline__ void convert_tile(const typename In::T* src, typename Out::T* dst, uint64_t len,
-                                             uint64_t tile, bool vec_ok, float divisor)
+                                             uint64_t tile, float divisor)
 {
-    constexpr uint64_t TQ = (uint64_t)kThreads * Q;  // Q: quads per thread per tile
     const int tid = threadIdx.x;
-    const int ps = phase_of(src, 4), pd = phase_of(dst, 4);
-    auto one = [&](uint64_t e) { Out::st1(dst + e, finish<OP>((float)In::ld1(src + e), divisor)); };
-    if (!(vec_ok && ps == pd)) {
-        const uint64_t e0 = tile * TQ * 4;
-#pragma unroll 4
-        for (int k = 0; k < Q * 4; ++k) {
-            const uint64_t e = e0 + (uint64_t)k * kThreads + tid;
-            if (e < len) one(e);
-        }
-        return;
-    }
-    uint64_t head = (uint64_t)((4 - ps) & 3);
+    const int pd = phase_of(dst, 4);
+    const int d = (phase_of(src, 4) - pd) & 3;
+    uint64_t head = (uint64_t)((4 - pd) & 3);
     if (head > len) head = len;
     const uint64_t nq = (len - head) / 4;
     const uint64_t tail = len - head - nq * 4;
-    if (tile == 0 && (uint64_t)tid < head + tail)
-        one((uint64_t)tid < head ? (uint64_t)tid : head + nq * 4 + ((uint64_t)tid - head));
-    // all of this thread's loads first (Q in flight), then the conversions
-    // and stores
-    typename Quad<In>::R raw[Q];
-    uint64_t e[Q];
-    bool ok[Q];
-#pragma unroll
-    for (int k = 0; k < Q; ++k) {
-        const uint64_t q = tile * TQ + (uint64_t)k * kThreads + tid;
-        ok[k] = q < nq;
-        e[k] = head + q * 4;
-        if (ok[k]) raw[k] = Quad<In>::ld(src + e[k]);
+    if (tile == 0 && (uint64_t)tid < head + tail) {
+        const uint64_t e = (uint64_t)tid < head ? (uint64_t)tid : head + nq * 4 + ((uint64_t)tid - head);
+        Out::st1(dst + e, finish<OP>((float)In::ld1(src + e), divisor));
     }
-#pragma unroll
-    for (int k = 0; k < Q; ++k) {
-        if (!ok[k]) continue;
-        float a[4];
-        Quad<In>::to_f(raw[k], a);
-#pragma unroll
-        for (int l = 0; l < 4; ++l) a[l] = finish<OP>(a[l], divisor);
-        Quad<Out>::st(dst + e[k], Quad<Out>::from_f(a));
-    }
+    // the aligned source quad under dst's first quad (d elements before src + head)
+    const auto* s0 = reinterpret_cast<const typename In::T*>(reinterpret_cast<uintptr_t>(src + head) -
+                                                              (uintptr_t)d * sizeof(typename In::T));
+    if (d == 0) convert_quads<In, Out, OP, Q, false>(s0, dst, head, nq, tile, 0, divisor);
+    else convert_quads<In, Out, OP, Q, true>(s0, dst, head, nq, tile, d, divisor);
 }
 
 // The segment owning work item w: the last s with prefix[s] <= w (segments
@@ -144,7 +185,7 @@ __global__ void __launch_bounds__(kThreads) bucket_pack_kernel(const __grid_cons
         const uint64_t s = t * (uint64_t)p.n + r;
         const auto* src = static_cast<const typename G::T*>(p.grad[s]);
         float* dst = static_cast<float*>(p.bucket[r]) + p.toff[t];
-        convert_tile<G, F32T, kSum>(src, dst, p.tlen[t], tile, p.vec_ok, 1.0f);
+        convert_tile<G, F32T, kSum>(src, dst, p.tlen[t], tile, 1.0f);
     }
 }
 
@@ -160,7 +201,7 @@ __global__ void __launch_bounds__(kThreads) bucket_unpack_kernel(const __grid_co
         const uint64_t s = t * (uint64_t)p.n + r;
         const float* src = static_cast<const float*>(p.bucket[r]) + p.toff[t];
         auto* dst = static_cast<typename G::T*>(const_cast<void*>(p.grad[s]));
-        convert_tile<F32T, G, OP>(src, dst, p.tlen[t], tile, p.vec_ok, p.divisor);
+        convert_tile<F32T, G, OP>(src, dst, p.tlen[t], tile, p.divisor);
     }
 }
 

@@ -55,20 +55,29 @@ const BulkDebug& bulk_debug()
     return d;
 }
 
-uint64_t bulk_tile_bytes(int n) { return (n >= 32 ? 32768u : 16384u) / (uint64_t)n; }  // bulk_smem<N>() / N
-
 template <class Ty, int OP, int WIRE>
 cudaError_t launch_ring(const RankParams& p, cudaStream_t s)
 {
+    uint64_t seg = p.C;  // the longest segment: a chunk, or the launch's element range
+    const uint64_t hi = p.hi < p.count ? p.hi : p.count;
+    if (hi - p.lo < seg) seg = hi - p.lo;
     switch (p.n) {
-    case 2: return launch_bulk_fold<Ty, OP, 2, kBulkRing, WIRE>(p, p.C, s);
-    case 4: return launch_bulk_fold<Ty, OP, 4, kBulkRing, WIRE>(p, p.C, s);
-    case 8: return launch_bulk_fold<Ty, OP, 8, kBulkRing, WIRE>(p, p.C, s);
-    case 16: return launch_bulk_fold<Ty, OP, 16, kBulkRing, WIRE>(p, p.C, s);
-    case 32: return launch_bulk_fold<Ty, OP, 32, kBulkRing, WIRE>(p, p.C, s);
-    case 64: return launch_bulk_fold<Ty, OP, 64, kBulkRing, WIRE>(p, p.C, s);
+    case 2: return launch_bulk_fold<Ty, OP, 2, kBulkRing, WIRE>(p, seg, s);
+    case 4: return launch_bulk_fold<Ty, OP, 4, kBulkRing, WIRE>(p, seg, s);
+    case 8: return launch_bulk_fold<Ty, OP, 8, kBulkRing, WIRE>(p, seg, s);
+    case 16: return launch_bulk_fold<Ty, OP, 16, kBulkRing, WIRE>(p, seg, s);
+    case 32: return launch_bulk_fold<Ty, OP, 32, kBulkRing, WIRE>(p, seg, s);
+    case 64: return launch_bulk_fold<Ty, OP, 64, kBulkRing, WIRE>(p, seg, s);
     }
-    return cudaErrorInvalidValue;
+    return launch_bulk_fold<Ty, OP, 0, kBulkRing, WIRE>(p, seg, s);
+}
+
+bool pow2_rank_count(int n) { return n == 2 || n == 4 || n == 8 || n == 16 || n == 32 || n == 64; }
+
+uint64_t tiles_of(uint64_t elems, int esize, int n)
+{
+    const uint64_t te = (uint64_t)bulk_tile_vectors(n) * (16u / (uint64_t)esize);
+    return elems ? (elems + te - 1) / te : 1;
 }
 
 }  // namespace
@@ -100,10 +109,9 @@ BulkParams bulk_params(const RankParams& p)
     return bp;
 }
 
-bool bulk_ranks_aligned(const RankParams& p, int nmax)
+bool bulk_ranks_aligned(const RankParams& p, int nmax, bool pow2)
 {
-    if (p.n > nmax || (p.n != 2 && p.n != 4 && p.n != 8 && p.n != 16 && p.n != 32 && p.n != 64)) return false;
-    if (!p.waits) return false;
+    if (!p.waits || p.n < 2 || p.n > nmax || (pow2 && !pow2_rank_count(p.n))) return false;
     for (int r = 0; r < p.n; ++r)
         if ((uintptr_t)p.in[r] % 16 != 0 || (uintptr_t)p.out[r] % 16 != 0) return false;
     return true;
@@ -111,27 +119,30 @@ bool bulk_ranks_aligned(const RankParams& p, int nmax)
 
 bool bulk_eligible(const RankParams& p, int esize)
 {
-    if (!bulk_ranks_aligned(p, 64)) return false;
-    if (p.owner_only || p.lo != 0 || p.hi < p.count || p.nseg != (uint64_t)p.n) return false;
-    if ((p.C * (uint64_t)esize) % 16 != 0) return false;
-    const uint64_t tiles = (p.C * (uint64_t)esize + bulk_tile_bytes(p.n) - 1) / bulk_tile_bytes(p.n);
-    return tiles * (uint64_t)p.n <= kMaxGrid;
+    if (!p.waits || p.n < 2 || p.n > kMaxRanks || !p.vec_ok) return false;
+    // every input and output at one 16-byte phase, on element boundaries
+    const uintptr_t ph = (uintptr_t)p.in[0] % 16;
+    if ((uintptr_t)p.out[0] % 16 != ph || ph % (uintptr_t)esize != 0) return false;
+    if (p.nseg != (uint64_t)p.n || p.lo >= p.count) return false;
+    const uint64_t hi = p.hi < p.count ? p.hi : p.count;
+    const uint64_t seg = hi - p.lo < p.C ? hi - p.lo : p.C;
+    return tiles_of(seg, esize, p.n) * (uint64_t)p.n <= kMaxGrid;
 }
 
 bool bulk_scatter_eligible(const RankParams& p, int esize)
 {
-    if (!bulk_ranks_aligned(p, 16) || p.nseg != (uint64_t)p.n) return false;
-    if ((p.C * (uint64_t)esize) % 16 != 0) return false;  // every part is whole vectors
-    const uint64_t tiles = (p.C * (uint64_t)esize + bulk_tile_bytes(p.n) - 1) / bulk_tile_bytes(p.n);
-    return tiles * (uint64_t)p.n <= kMaxGrid;
+    // every input at one 16-byte phase (so part r of every rank is too), every
+    // output at one phase, all on element boundaries
+    if (!p.waits || p.n < 2 || p.n > kMaxRanks || !p.vec_ok || p.nseg != (uint64_t)p.n) return false;
+    if ((uintptr_t)p.in[0] % (uintptr_t)esize != 0 || (uintptr_t)p.out[0] % (uintptr_t)esize != 0) return false;
+    return tiles_of(p.C, esize, p.n) * (uint64_t)p.n <= kMaxGrid;
 }
 
 bool bulk_tree_eligible(const RankParams& p, int esize)
 {
-    if (!bulk_ranks_aligned(p, 16) || p.nseg != 1) return false;
+    if (!bulk_ranks_aligned(p, 16, true) || p.nseg != 1) return false;
     if ((p.count * (uint64_t)esize) % 16 != 0) return false;  // the buffer is whole vectors
-    const uint64_t tiles = (p.count * (uint64_t)esize + bulk_tile_bytes(p.n) - 1) / bulk_tile_bytes(p.n);
-    return tiles <= kMaxGrid;
+    return tiles_of(p.count, esize, p.n) <= kMaxGrid;
 }
 
 template <class Ty, int OP>
@@ -143,6 +154,14 @@ cudaError_t launch_oneshot_bulk(const RankParams& p, cudaStream_t s)
 cudaError_t launch_oneshot_wire_bulk(int op, const RankParams& p, cudaStream_t s)
 {
     return op == kAvg ? launch_ring<F32T, kAvg, 1>(p, s) : launch_ring<F32T, kSum, 1>(p, s);
+}
+
+cudaError_t kernel_binary_version(int* version)
+{
+    cudaFuncAttributes a{};
+    const cudaError_t e = cudaFuncGetAttributes(&a, take_waits_kernel);
+    if (e == cudaSuccess) *version = a.binaryVersion;
+    return e;
 }
 
 cudaError_t take_bulk_timeouts(unsigned int* ran_out, unsigned int* in_flight)

@@ -5,18 +5,27 @@
 // issues the bulk stores of the result.  Three orders and output patterns:
 //
 //   kBulkRing     the one-shot all-reduce: segment c = chunk c of every
-//                 rank, folded in ring order from rank c (optionally with the
-//                 bf16 wire format), written to every rank
+//                 rank (clipped to the launch's element range), folded in
+//                 ring order from rank c (optionally with the bf16 wire
+//                 format), written to every rank or to rank c only (the
+//                 two-shot's first shot)
 //   kBulkScatter  the reduce-scatter: segment r = part r of every rank,
 //                 folded in ring order from rank r, written to out[r] only
 //   kBulkTree     the tree-order one-shot: the whole buffer, folded in the
 //                 tree's pairwise order (N a power of two), written to every
 //                 rank
 //
-// They run where the tiles are whole 16-byte vectors at 16-byte aligned
-// addresses and the rank count is fixed at compile time (bulk_*_eligible);
-// every other call takes the per-thread-load kernels, with the same bits.
-// The fold itself uses the same apply / finish / wire steps as those kernels.
+// The ring mode runs wherever every input and output address has the same
+// 16-byte phase (a scalar head and tail per segment, whole vectors between),
+// the scatter mode wherever every input has one phase (each output stored by
+// bulk copies when it shares that phase, by the threads otherwise), both for
+// 2-64 ranks; the tree mode where the buffers are whole 16-byte vectors at
+// 16-byte aligned addresses (bulk_*_eligible).  The rank count is a
+// compile-time constant for 2, 4, 8, 16, 32 and 64 ranks (tree: 2-16) and a
+// kernel argument (NS = 0) otherwise; with the copy engine doing the loads,
+// a runtime count costs the fold no registers.  Every other call takes the
+// per-thread-load kernels, with the same bits.  The fold itself uses the
+// same apply / finish / wire steps as those kernels.
 //
 // Every mbarrier wait is bounded, and its outcome is the same in every thread
 // of the CTA (bulk_tile_landed).  A tile whose wait runs out (no working
@@ -46,6 +55,7 @@ struct BulkParams {
     uint32_t hold;        // test hook (0 in use): 1 makes every barrier expect one arrival
                           // more, which is made only after the first wait has run out
     uint32_t spin;        // try_wait rounds before a wait gives up
+    uint32_t tv;          // vectors per rank per tile (kernels whose rank count is not fixed)
 };
 
 // Bytes of input tiles per CTA (N tiles of bulk_smem<N>() / N): 16 KB, 32 KB
@@ -60,10 +70,11 @@ __host__ __device__ constexpr uint32_t bulk_smem()
 // the wait bounds (rr_bulk.cu).
 BulkParams bulk_params(const RankParams& p);
 
-// Whether a call can take the bulk kernels: the wait counters are known
-// (p.waits), a rank count of 2, 4, 8, 16, 32 or 64 (up to nmax), 16-byte
-// aligned buffers.  The callers add their own segment rules.
-bool bulk_ranks_aligned(const RankParams& p, int nmax);
+// Whether a call can take the aligned bulk kernels (scatter and tree modes):
+// the wait counters are known (p.waits), 2..nmax ranks (powers of two only
+// when pow2), 16-byte aligned buffers.  The callers add their own segment
+// rules.
+bool bulk_ranks_aligned(const RankParams& p, int nmax, bool pow2);
 
 __device__ __forceinline__ uint32_t bulk_smem_addr(const void* ptr) { return (uint32_t)__cvta_generic_to_shared(ptr); }
 
@@ -121,14 +132,14 @@ __global__ void __launch_bounds__(kThreads) bulk_fold_kernel(const __grid_consta
 {
     using T = typename Ty::T;
     using Acc = typename Ty::Acc;
-    constexpr int L = Ty::L;                       // elements per 16-byte vector
-    constexpr uint32_t TB = bulk_smem<NS>() / NS;  // bytes per rank per tile
-    constexpr uint32_t TV = TB / 16;               // vectors per tile
-    constexpr int NOUT = MODE == kBulkScatter ? 1 : NS;
-    static_assert(TB % 16 == 0 && TV >= 1, "tile of whole vectors");
-    static_assert(MODE != kBulkTree || (NS & (NS - 1)) == 0, "the pairwise tree needs a power of two");
+    constexpr int L = Ty::L;  // elements per 16-byte vector
+    static_assert(NS == 0 || (bulk_smem<NS>() / (NS > 0 ? NS : 1)) % 16 == 0, "tile of whole vectors");
+    static_assert(MODE != kBulkTree || (NS > 0 && (NS & (NS - 1)) == 0), "the pairwise tree needs a fixed power of two");
+    static_assert(MODE == kBulkRing || WIRE == 0, "the wire format is a ring-order one-shot");
     const RankParams& p = bp.r;
-    extern __shared__ __align__(128) uint4 sm[];   // [NS][TV]: slot j holds the fold's j-th input
+    const int n = NS > 0 ? NS : p.n;
+    const uint32_t TV = NS > 0 ? bulk_smem<NS>() / (NS > 0 ? NS : 1) / 16 : bp.tv;  // vectors per rank per tile
+    extern __shared__ __align__(128) uint4 sm[];                      // [n][TV]: slot j holds the fold's j-th input
     __shared__ __align__(8) uint64_t bar;
 
     const uint64_t s = blockIdx.x / p.tps, tile = blockIdx.x - s * p.tps;
@@ -136,40 +147,64 @@ __global__ void __launch_bounds__(kThreads) bulk_fold_kernel(const __grid_consta
     if constexpr (MODE == kBulkTree) {
         lo = 0;
         len = p.count;
-    } else {
+    } else if constexpr (MODE == kBulkScatter) {
         lo = s * p.C;
-        if (lo >= p.count) return;
-        len = p.C < p.count - lo ? p.C : p.count - lo;
+        len = p.C;
+    } else {  // chunk s, clipped to the launch's element range [p.lo, p.hi)
+        const uint64_t c_lo = s * p.C;
+        if (c_lo >= p.count) return;
+        const uint64_t c_hi = p.C < p.count - c_lo ? c_lo + p.C : p.count;
+        lo = c_lo > p.lo ? c_lo : p.lo;
+        const uint64_t hi = c_hi < p.hi ? c_hi : p.hi;
+        if (lo >= hi) return;
+        len = hi - lo;
     }
     const int start = MODE == kBulkTree ? 0 : (int)s;
     auto in = [&](int j) {
         int r = start + j;
-        if (r >= NS) r -= NS;
+        if (r >= n) r -= n;
         return static_cast<const T*>(p.in[r]) + lo;
     };
+    const bool one_out = MODE == kBulkScatter || (MODE == kBulkRing && p.owner_only);
+    const int nout = one_out ? 1 : n;
     auto out = [&](int o) {
         if constexpr (MODE == kBulkScatter) return static_cast<T*>(p.out[s]);
-        else return static_cast<T*>(p.out[o]) + lo;
+        else return static_cast<T*>(p.out[one_out ? start : o]) + lo;
     };
-    const uint64_t nv = len / L;                   // whole vectors of the segment
-    if constexpr (MODE == kBulkRing) {             // a ragged last chunk: its last elements
-        if (tile == 0 && (uint64_t)threadIdx.x < len - nv * L)
-            fold_one<Ty, OP, WIRE>(in, NS, out, NOUT, nv * L + threadIdx.x, p.divisor);
+    // Ring and scatter modes: every rank's copy of the segment starts at the
+    // same 16-byte phase, so the elements before the first 16-byte boundary
+    // (the head) and after the last whole vector (the tail) are folded with
+    // plain loads by tile 0, and the bulk copies move the whole vectors
+    // between.  The tree mode takes a 16-byte aligned buffer of whole vectors.
+    uint64_t head = 0;
+    if constexpr (MODE != kBulkTree) {
+        head = (uint64_t)((L - phase_of(in(0), L)) & (L - 1));
+        if (head > len) head = len;
+    }
+    // a scatter output at another phase than the inputs is stored by the
+    // threads, element by element, instead of by bulk stores
+    bool bulk_out = true;
+    if constexpr (MODE == kBulkScatter) bulk_out = phase_of(out(0), L) == phase_of(in(0), L);
+    const uint64_t nv = (len - head) / L;  // whole vectors of the segment
+    const uint64_t tail = len - head - nv * L;
+    if (tile == 0 && (uint64_t)threadIdx.x < head + tail) {
+        const uint64_t e = (uint64_t)threadIdx.x < head ? (uint64_t)threadIdx.x : head + nv * L + (threadIdx.x - head);
+        fold_one<Ty, OP, WIRE>(in, n, out, nout, e, p.divisor);
     }
     const uint64_t v0 = tile * TV;
     if (v0 >= nv) return;
     const uint32_t nvt = (uint32_t)(nv - v0 < TV ? nv - v0 : TV);  // vectors in this tile
     const uint32_t bytes = nvt * 16u;
-    const uint64_t e0 = v0 * L;                    // first element of the tile in the segment
+    const uint64_t e0 = head + v0 * L;     // first element of the tile: 16-byte aligned in every copy
 
     const uint32_t b = bulk_smem_addr(&bar);
     if (threadIdx.x == 0) bulk_bar_init(b, bp.hold);
     __syncthreads();
     if (threadIdx.x == 0) {
         asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
-                     ::"r"(b), "r"(bytes * NS) : "memory");
+                     ::"r"(b), "r"(bytes * (uint32_t)n) : "memory");
 #pragma unroll
-        for (int j = 0; j < NS; ++j)
+        for (int j = 0; j < (NS > 0 ? NS : n); ++j)
             asm volatile(
                 "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                 ::"r"(bulk_smem_addr(sm + j * TV)), "l"(in(j) + e0), "r"(bytes), "r"(b)
@@ -205,8 +240,8 @@ __global__ void __launch_bounds__(kThreads) bulk_fold_kernel(const __grid_consta
             for (int l = 0; l < L; ++l) a[l] = stack[LV - 1][l];  // N = 2^(LV-1): one block of all ranks
         } else {
             Ty::unpack(sm[v], a);
-#pragma unroll
-            for (int j = 1; j < NS; ++j) {
+#pragma unroll 4
+            for (int j = 1; j < (NS > 0 ? NS : n); ++j) {
                 Acc x[L];
                 Ty::unpack(sm[j * TV + v], x);
 #pragma unroll
@@ -219,9 +254,13 @@ __global__ void __launch_bounds__(kThreads) bulk_fold_kernel(const __grid_consta
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the generic writes, before the bulk reads
     __syncthreads();
+    if (!bulk_out) {
+        for (uint32_t v = threadIdx.x; v < nvt; v += kThreads) st_lanes(out(0) + e0 + (uint64_t)v * L, sm[v]);
+        if (threadIdx.x == 0) bulk_bar_inval(b);
+        return;
+    }
     if (threadIdx.x == 0) {
-#pragma unroll
-        for (int o = 0; o < NOUT; ++o)
+        for (int o = 0; o < nout; ++o)
             asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
                          ::"l"(out(o) + e0), "r"(bulk_smem_addr(sm)), "r"(bytes)
                          : "memory");
@@ -231,18 +270,26 @@ __global__ void __launch_bounds__(kThreads) bulk_fold_kernel(const __grid_consta
     }
 }
 
-// One CTA per (segment, tile): nseg segments of seg_elems elements each.
+// Vectors per rank per tile when the rank count is not fixed at compile
+// time: the rank's share of 16 KB (32 KB from 32 ranks on), whole vectors.
+inline uint32_t bulk_tile_vectors(int n) { return (uint32_t)((n >= 32 ? 32768u : 16384u) / (uint32_t)n / 16u); }
+
+// One CTA per (segment, tile): nseg segments of at most seg_elems elements
+// each.  NS = 0 runs the rank count p.n.
 template <class Ty, int OP, int NS, int MODE, int WIRE>
 cudaError_t launch_bulk_fold(const RankParams& p, uint64_t seg_elems, cudaStream_t s)
 {
-    constexpr uint64_t TE = (uint64_t)(bulk_smem<NS>() / NS / 16) * Ty::L;  // elements per tile
     BulkParams bp = bulk_params(p);
     if (!bp.waits) return cudaErrorInvalidValue;  // never reached: eligibility requires the counters
-    bp.r.tps = (seg_elems + TE - 1) / TE;
+    const uint32_t tv = NS > 0 ? bulk_smem<NS>() / (NS > 0 ? NS : 1) / 16 : bulk_tile_vectors(p.n);
+    const uint64_t te = (uint64_t)tv * Ty::L;  // elements per tile
+    bp.tv = tv;
+    bp.r.tps = seg_elems ? (seg_elems + te - 1) / te : 1;
     const uint64_t work = bp.r.nseg * bp.r.tps;
     if (work == 0) return cudaSuccess;
     if (work > kMaxGrid) return cudaErrorInvalidValue;  // never reached: the eligibility checks cap it
-    bulk_fold_kernel<Ty, OP, NS, MODE, WIRE><<<(unsigned)work, kThreads, bulk_smem<NS>(), s>>>(bp);
+    const uint32_t smem = tv * 16u * (uint32_t)p.n;
+    bulk_fold_kernel<Ty, OP, NS, MODE, WIRE><<<(unsigned)work, kThreads, smem, s>>>(bp);
     return cudaGetLastError();
 }
 

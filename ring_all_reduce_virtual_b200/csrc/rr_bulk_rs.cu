@@ -20,7 +20,7 @@ cudaError_t launch_scatter_bulk(const RankParams& p, cudaStream_t s)
     case 8: return launch_bulk_fold<Ty, OP, 8, kBulkScatter, 0>(p, p.C, s);
     case 16: return launch_bulk_fold<Ty, OP, 16, kBulkScatter, 0>(p, p.C, s);
     }
-    return cudaErrorInvalidValue;
+    return launch_bulk_fold<Ty, OP, 0, kBulkScatter, 0>(p, p.C, s);
 }
 
 #define RR_INSTANTIATE(TY, OP) template cudaError_t launch_scatter_bulk<TY, OP>(const RankParams&, cudaStream_t);

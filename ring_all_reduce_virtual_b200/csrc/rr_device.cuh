@@ -241,6 +241,17 @@ __device__ __forceinline__ int phase_of(const T* p, int L)
     return (int)(((uintptr_t)p / sizeof(T)) & (uintptr_t)(L - 1));
 }
 
+// Store the elements of one 16-byte vector one by one (at an address that is
+// not 16-byte aligned): the bits as they are.
+template <class T>
+__device__ __forceinline__ void st_lanes(T* q, const uint4& r)
+{
+    constexpr int L = 16 / (int)sizeof(T);
+    const T* e = reinterpret_cast<const T*>(&r);
+#pragma unroll
+    for (int l = 0; l < L; ++l) q[l] = e[l];
+}
+
 // --------------------------------------------------------------- the tile
 
 // Scalar fold of element e of a segment.
@@ -263,12 +274,13 @@ __device__ __forceinline__ void fold_one(const InF& in, int nin, const OutF& out
 // selects the bf16 wire format (see wire_in / wire_out).  in(j) /
 // out(o) return the segment's base pointers.  vec_ok says
 // that every in(j) has the same address modulo 16 as in(0), and every out(o)
-// the same as out(0) (checked by the host); when in(0) and out(0) also agree,
-// the segment splits into a scalar head up to the first 16-byte boundary, a
-// body of 16-byte vectors and a scalar tail, otherwise every element is
-// scalar.  Tile t covers body vectors [t*TV, (t+1)*TV), TV = kThreads*VPT, or
-// the same number of elements on the scalar path; tile 0 also does the head
-// and tail.
+// the same as out(0) (checked by the host); then the segment splits into a
+// scalar head up to the inputs' first 16-byte boundary, a body of 16-byte
+// vectors and a scalar tail -- each vector stored whole when out(0) has the
+// inputs' phase, element by element otherwise -- and without vec_ok every
+// element is scalar.  Tile t covers body vectors [t*TV, (t+1)*TV), TV =
+// kThreads*VPT, or the same number of elements on the scalar path; tile 0
+// also does the head and tail.
 template <class Ty, int OP, int VPT, int G, int NS = 0, int WIRE = 0, class InF, class OutF>
 __device__ __forceinline__ void fold_tile(const InF& in, int nin, const OutF& out, int nout, uint64_t len,
                                           uint64_t tile, bool vec_ok, float divisor)
@@ -280,7 +292,8 @@ __device__ __forceinline__ void fold_tile(const InF& in, int nin, const OutF& ou
     const int tid = threadIdx.x;
     const int pin = phase_of(in(0), L);
     const int pout = phase_of(out(0), L);
-    if (!(vec_ok && pin == pout)) {
+    const bool whole = pin == pout;  // results stored as whole vectors
+    if (!vec_ok) {
         const uint64_t e0 = tile * TV * L;
 #pragma unroll 4
         for (int k = 0; k < VPT * L; ++k) {
@@ -318,7 +331,10 @@ __device__ __forceinline__ void fold_tile(const InF& in, int nin, const OutF& ou
             T* q = out(o);
 #pragma unroll
             for (int u = 0; u < VPT; ++u)
-                if (ok[u]) stv(q + off[u], raw[u]);
+                if (ok[u]) {
+                    if (whole) stv(q + off[u], raw[u]);
+                    else st_lanes(q + off[u], raw[u]);
+                }
         }
         return;
     }
@@ -365,7 +381,10 @@ __device__ __forceinline__ void fold_tile(const InF& in, int nin, const OutF& ou
         T* q = out(o);
 #pragma unroll
         for (int u = 0; u < VPT; ++u)
-            if (ok[u]) stv(q + off[u], res[u]);
+            if (ok[u]) {
+                if (whole) stv(q + off[u], res[u]);
+                else st_lanes(q + off[u], res[u]);
+            }
     }
 }
 

@@ -51,6 +51,25 @@ struct StepParams {
     uint64_t tps;
 };
 
+// The ring, double-ring and tree schedules in one launch.  The schedules'
+// data dependencies run along (chunk, tile) chains: tile t of chunk k at
+// ring step s reads only what step s-1 wrote to tile t of chunk k (on the
+// previous rank), and a tree level reads only what the level below wrote to
+// the same elements.  So one CTA carries its tile through every step, each
+// thread on the same elements at every step (it reads what it wrote itself),
+// and no CTA waits for another.
+struct ChainParams {
+    void* buf[kMaxRanksH];
+    int n;
+    int vec_ok;      // every buffer at the same 16-byte phase (required: the chains run the vector path)
+    float divisor;   // AVG's divisor
+    int nhalf;       // ring: 1 (the whole buffer, clockwise); double ring: 2 (half 1 counter-clockwise)
+    uint64_t count;  // elements per rank
+    uint64_t H;      // the double ring's first element of half 1 (count for the ring)
+    uint64_t C[2];   // chunk size of each half
+    uint64_t tps;    // tiles per chunk (ring) or per buffer (tree)
+};
+
 // Bucket launches: one launch covers up to kMaxBucketTensors tensors of one
 // bucket and up to kMaxBucketPtrs gradient pointers (tensor-major: entry
 // t * n + r is rank r's copy of the launch's t-th tensor).
@@ -129,6 +148,12 @@ constexpr uint64_t kMaxGrid = 0x7fffffffull;
 // Launchers: return the launch's cudaError_t.  `op` is an rr_op_t value.
 cudaError_t launch_rank_kernel(int kind, int dtype, int op, const RankParams& p, cudaStream_t s);
 cudaError_t launch_step(int dtype, int op, const StepParams& p, cudaStream_t s);
+// The whole ring schedule (p.nhalf 1) or double ring (2) in one launch, and
+// the whole tree schedule (reduce levels, then broadcast levels) in one launch;
+// wire: the ring's bf16 wire format (fp32 buffers, SUM or AVG).
+cudaError_t launch_ring_chain(int dtype, int op, bool wire, const ChainParams& p, cudaStream_t s);
+uint64_t chain_tile_elems(int dtype);  // elements of one chain tile (ChainParams::tps counts these)
+cudaError_t launch_tree_chain(int dtype, int op, const ChainParams& p, cudaStream_t s);
 // bf16 wire (fp32 buffers, SUM or AVG): the fused one-shot, and a reduce-scatter
 // step (wire 1: the step completes its chunks; 2: it does not).
 cudaError_t launch_oneshot_wire(int op, const RankParams& p, uint64_t work, cudaStream_t s);
@@ -140,6 +165,8 @@ unsigned int* bulk_wait_counters();
 // Takes (reads and clears, atomically on the device) both counters of the
 // current device.  Synchronous.
 cudaError_t take_bulk_timeouts(unsigned int* ran_out, unsigned int* in_flight);
+// cudaFuncGetAttributes(...).binaryVersion of one of the library's kernels.
+cudaError_t kernel_binary_version(int* version);
 cudaError_t launch_bucket_pack(int grad_dtype, const BucketCopyParams& p, cudaStream_t s);
 cudaError_t launch_bucket_unpack(int grad_dtype, int op, const BucketCopyParams& p, cudaStream_t s);
 cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p, cudaStream_t s,
@@ -151,6 +178,7 @@ namespace rr {
 // Kernel parameter blocks must fit the 32,764-byte kernel parameter limit.
 static_assert(sizeof(RankParams) <= 32764, "RankParams too large");
 static_assert(sizeof(StepParams) <= 32764, "StepParams too large");
+static_assert(sizeof(ChainParams) <= 32764, "ChainParams too large");
 static_assert(sizeof(BucketCopyParams) <= 32764, "BucketCopyParams too large");
 static_assert(sizeof(BucketFoldParams) <= 32764, "BucketFoldParams too large");
 }  // namespace rr

@@ -18,7 +18,7 @@ from dataclasses import dataclass
 import numpy as np
 
 #: value distributions of the workloads
-DISTS = ("uniform", "normal", "prod", "int", "arange", "pow2")
+DISTS = ("uniform", "full", "normal", "prod", "int", "arange", "pow2")
 
 
 def rank_values(seed: int, rank: int, count: int, dist: str = "uniform", dtype: str = "f32",
@@ -26,7 +26,11 @@ def rank_values(seed: int, rank: int, count: int, dist: str = "uniform", dtype: 
     """Draw ``count`` values for one rank.
 
     dist:
-      - ``uniform``: uniform on [-1, 1)
+      - ``uniform``: uniform on [-1, 1) (numpy's float32 draws: multiples of
+        2^-23, so a sum of two is always exact)
+      - ``full``: uniform on [-1, 1) drawn in float64 and rounded to float32,
+        so every value has a full 24-bit mantissa and short sums round: each
+        fold order gives its own bits
       - ``normal``: normal(0, 1e-3)
       - ``prod``: uniform on [0.99, 1.01) (keeps long products finite)
       - ``int``: integers in [-1024, 1024), exact in fp32 and bf16 sums of a
@@ -40,6 +44,8 @@ def rank_values(seed: int, rank: int, count: int, dist: str = "uniform", dtype: 
     rng = np.random.default_rng(key)
     if dist == "uniform":
         v = rng.random(count, dtype=np.float32) * np.float32(2.0) - np.float32(1.0)
+    elif dist == "full":
+        v = (rng.random(count) * 2.0 - 1.0).astype(np.float32)
     elif dist == "normal":
         v = rng.standard_normal(count, dtype=np.float32) * np.float32(1e-3)
     elif dist == "prod":

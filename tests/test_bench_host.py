@@ -71,10 +71,13 @@ def test_reference_arm_other_ranks_exit_quietly():
 def test_alpha_beta_fit_recovers_known_terms(capsys):
     """The sweep's least-squares fit of time = launches * alpha + bytes / beta
     returns the alpha and beta that generated exact points."""
-    rows = [(k, b, k * 3e-6 + b / 7e12, (k * 1.5e-6 + b / 7e12) if b < 1e7 else None)
+    rows = [(k, b, k * 3e-6 + b / 7e12, (k * 1.5e-6 + b / 7e12) if b < 1e7 else None, False)
             for k in (1, 6, 14, 30) for b in (1e4, 1e6, 1e8, 1e10)]
+    # L2-resident points above 4 MiB would pull beta up: they are left out
+    rows += [(1, 5e7, 1e-6, None, True), (2, 9e7, 2e-6, None, True)]
     bench.fit_alpha_beta(rows)
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["per_call"]["alpha_us"] == pytest.approx(3.0, rel=1e-6)
     assert line["per_call"]["beta_gbs"] == pytest.approx(7000.0, rel=1e-6)
     assert line["in_graph"]["alpha_us"] == pytest.approx(1.5, rel=1e-6)
+    assert line["per_call"]["rel_residual_max"] < 1e-6

@@ -177,28 +177,85 @@ def test_gpt_like_bucketed_sync(gpt_grads, path):
 
 # ------------------------------------------------------------ workload 4 --
 
+SWEEP_ALGOS = ("ring", "oneshot", "two_shot", "tree", "tree_oneshot", "double_ring")
+SWEEP_ORACLE = {  # fp32: the stepping schedules give their definitions' bits (pinned on the CPU)
+    "ring": oracle.fold_ring_order, "oneshot": oracle.fold_ring_order, "two_shot": oracle.fold_ring_order,
+    "tree": oracle.tree_schedule, "tree_oneshot": oracle.tree_fold, "double_ring": oracle.fold_double_ring,
+}
+
+
+def _check_sampled_tree(host, dev, seed):
+    """The tree order is element-wise: the oracle's tree fold of the sampled
+    [N, m] rows is the result at those elements."""
+    n, count = len(host), host[0].size
+    idx = _sample_idx(count, n, 20000, seed)
+    rows = [np.ascontiguousarray(a[idx]) for a in host]
+    oracle.tree_fold(rows, "sum")
+    got = _gather(dev, idx)
+    for r in range(n):
+        assert_bits_equal([got[r]], [rows[0]], f"sampled tree rank {r}")
+
+
+def _check_sampled_double_ring(host, dev, seed):
+    """The double ring (reading 13): element i < H = ceil(count/2) is chunk
+    i // ceil(H/N) of the clockwise ring, folded upwards from that rank;
+    element i >= H is chunk c = (i - H) // ceil((count - H)/N) of the mirror
+    ring, folded downwards c, c-1, ..., c+1 -- the upward fold of the
+    rank-reversed rows from N-1-c.  Both through the oracle's sampled fold."""
+    n, count = len(host), host[0].size
+    H = (count + 1) // 2
+    CA, CB = -(-H // n), -(-(count - H) // n)
+    idx = _sample_idx(count, n, 20000, seed)
+    idx = np.unique(np.concatenate([idx, [H - 1, H, H + 1]]))
+    idx = idx[(idx >= 0) & (idx < count)]
+    a, b = idx[idx < H], idx[idx >= H]
+    want = np.empty(idx.size, dtype=np.float32)
+    want[idx < H] = oracle.fold_samples(np.stack([x[a] for x in host]), (a // CA).astype(np.int32), "sum")
+    rev = np.stack([x[b] for x in host][::-1])
+    want[idx >= H] = oracle.fold_samples(rev, (n - 1 - (b - H) // CB).astype(np.int32), "sum")
+    got = _gather(dev, idx)
+    for r in range(n):
+        assert_bits_equal([got[r]], [want], f"sampled double ring rank {r}")
+
+
 @pytest.mark.parametrize("n", [2, 4, 8, 16])
 @pytest.mark.parametrize("nbytes", [1 << 10, 1 << 20, 1 << 26, 1 << 30])
 def test_size_sweep_points(n, nbytes):
-    """Sweep points (1 KiB .. 1 GiB per rank, fp32 SUM): ring, one-shot and
-    tree order against the oracle (every element up to 64 MiB, sampled at
-    1 GiB), and ring == one-shot bit for bit."""
+    """Sweep points (1 KiB .. 1 GiB per rank, fp32 SUM) for every schedule:
+    ring, one-shot and two-shot (ring order), the tree schedule and the
+    tree-order one-shot, and the double ring, against the oracle -- every
+    element up to 64 MiB, sampled elements (chunk boundaries included) at
+    1 GiB -- with all ranks identical, and the ring-order ones equal to each
+    other bit for bit."""
     count = nbytes // 4
-    x = synth.ranks(4, n, count, "uniform")
-    outs = {}
-    for algo in ("ring", "oneshot", "tree_oneshot"):
-        d = to_dev(x)
+    # normal(0, 1e-3): full mantissas, so every fold order gives its own bits
+    # (uniform[-1, 1) draws are multiples of 2^-23, whose short sums are exact)
+    x = synth.ranks(4, n, count, "normal")
+    pristine = to_dev(x)
+    ring_sample = None
+    for algo in SWEEP_ALGOS:
+        d = [t.clone() for t in pristine]
         rrv.all_reduce(d, "sum", algo)
         if nbytes <= 1 << 26:
             want = [a.copy() for a in x]
-            (oracle.tree_fold if algo == "tree_oneshot" else oracle.fold_ring_order)(want, "sum")
+            SWEEP_ORACLE[algo](want, "sum")
             assert_bits_equal(to_host(d), want, algo)
-        elif algo != "tree_oneshot":
+        elif algo in ("ring", "oneshot", "two_shot"):
             _check_sampled_fold(x, d, "sum", seed=n, k=20000)
-        outs[algo] = d
+        elif algo in ("tree", "tree_oneshot"):
+            _check_sampled_tree(x, d, seed=n + 1)
+        else:
+            _check_sampled_double_ring(x, d, seed=n + 2)
         _all_ranks_equal(d)
-    assert torch.equal(outs["ring"][0].view(torch.int32), outs["oneshot"][0].view(torch.int32))
-    del outs
+        if algo in ("ring", "oneshot", "two_shot"):  # one ring order: the same bits
+            first = d[0][: min(count, 1 << 22)].clone()
+            if ring_sample is None:
+                ring_sample = first
+            else:
+                assert torch.equal(first.view(torch.int32), ring_sample.view(torch.int32)), algo
+        del d
+    del pristine
+    torch.cuda.empty_cache()
 
 
 # ------------------------------------------------------------ workload 5 --

@@ -37,6 +37,8 @@ TILE_MOVE = {"f32": 4096, "bf16": 8192, "f16": 8192, "i32": 4096}  # per tile of
 def _dist(op, dtype):
     if dtype == "i32":
         return "int"
+    if op in ("sum", "avg"):
+        return "full"  # full mantissas: a fold in the wrong order gives other bits
     return "prod" if op == "prod" else "uniform"
 
 
@@ -58,6 +60,18 @@ def _cuda():
     from ring_all_reduce_virtual_b200.build import build
 
     build()
+
+
+def test_library_runs_sm100a_code():
+    """The runtime loads the library's kernels as code built for compute
+    capability 10.0 (sm_100a)."""
+    import ctypes
+
+    from ring_all_reduce_virtual_b200 import _lib
+
+    v = ctypes.c_int(0)
+    _lib.check(_lib.lib().rr_binary_version(ctypes.byref(v)), "rr_binary_version")
+    assert v.value == 100
 
 
 # -------------------------------------------------------- worked example --
@@ -203,9 +217,10 @@ def test_ring_steps_track_the_oracle_state(n, dtype, op):
 def test_ring_stats_match_the_schedule():
     n, count = 4, 1024
     d = to_dev(synth.ranks(7, n, count, "uniform"))
-    rrv.all_reduce(d, "sum", "ring")
+    rrv.all_reduce(d, "sum", "ring")  # buffers at one 16-byte phase: the whole schedule in one launch
     st = rrv.last_stats()
-    assert st["algo"] == "ring" and st["steps"] == 6 and st["launches"] == 6
+    assert st["algo"] == "ring" and st["steps"] == 6 and st["launches"] == 1
+    assert 0 < st["launch_ns"] <= st["host_ns"]
     assert st["bytes_sent_max"] == 6144  # [P4]: 2(n-1)/n x 4096 bytes
     assert st["hbm_bytes"] == 5 * 3 * 4096
     rrv.all_reduce(d, "sum", "oneshot")
@@ -217,7 +232,17 @@ def test_ring_stats_match_the_schedule():
     rrv.all_reduce(d, "sum", "double_ring")  # the same volume, half to each neighbour
     st = rrv.last_stats()
     want = oracle.double_ring_allreduce(synth.ranks(7, n, count, "uniform"))
-    assert st["launches"] == 6 and st["bytes_sent_max"] == int(want.max()) == 6144
+    assert st["launches"] == 1 and st["bytes_sent_max"] == int(want.max()) == 6144
+    rrv.all_reduce(d, "sum", "tree")
+    st = rrv.last_stats()
+    assert st["launches"] == 1 and st["steps"] == 4
+    # buffers at different 16-byte phases: one launch per step, the same counts
+    m = to_dev(synth.ranks(7, n, count, "uniform"), offsets=[0, 1, 2, 3])
+    rrv.all_reduce(m, "sum", "ring")
+    st = rrv.last_stats()
+    assert st["launches"] == 6 and st["steps"] == 6 and st["bytes_sent_max"] == 6144
+    rrv.all_reduce(m, "sum", "tree")
+    assert rrv.last_stats()["launches"] == 4
 
 
 # --------------------------------------------- reduce-scatter, all-gather --
@@ -520,6 +545,50 @@ def test_rank_set_matches_the_oracle_across_reuse(algo):
     assert_bits_equal(to_host(d), want, f"rank set {algo} reused")
 
 
+@pytest.mark.parametrize("algo", ["oneshot", "ring", "auto"])
+def test_rank_set_bound_call_matches_the_oracle(algo):
+    """RankSet.bind converts the arguments once; calling it twice reduces
+    twice (the second call reduces the first one's result)."""
+    n, count = 8, 8 * 1000 + 3
+    x = synth.ranks(33, n, count, "full")
+    d = to_dev(x)
+    call = rrv.RankSet(d).bind("avg", algo)
+    call()
+    call()
+    want = [a.copy() for a in x]
+    oracle.fold_ring_order(want, "avg")
+    oracle.fold_ring_order(want, "avg")
+    assert_bits_equal(to_host(d), want, f"bound {algo}")
+
+
+def test_auto_picks_by_the_table_for_the_buffers_alignment():
+    """AUTO takes the measured table's choice for the call's rank count, size
+    and alignment class -- aligned buffers the aligned points, buffers whose
+    16-byte phases differ the points measured with such buffers -- and the
+    result has the ring's bits either way."""
+    from conftest import picker_table
+
+    _, rows, _ = picker_table()
+    mixed = [r for r in rows if r[2] == 2]
+    for n in (2, 3, 8):
+        count = 1000 * n + 3
+        x = synth.ranks(35 + n, n, count, "full")
+        want = [a.copy() for a in x]
+        oracle.fold_ring_order(want, "sum")
+        d = to_dev(x)
+        rrv.all_reduce(d, "sum", "auto")
+        assert rrv.last_stats()["algo"] == rrv.pick_algo(n, count, "f32")
+        assert_bits_equal(to_host(d), want, f"auto aligned n={n}")
+        m = to_dev(x, offsets=[r % 4 for r in range(n)])
+        rrv.all_reduce(m, "sum", "auto")
+        if mixed:
+            near = min({r[0] for r in mixed}, key=lambda k: (abs(np.log2(k / n)), k))
+            pts = {r[1]: r[3] for r in mixed if r[0] == near}
+            lb = int(round(np.log2(count * 4)))
+            assert rrv.last_stats()["algo"] == pts[min(pts, key=lambda b: (abs(b - lb), b))]
+        assert_bits_equal(to_host(m), want, f"auto mixed n={n}")
+
+
 def test_rank_set_ring_steps_and_wire():
     n, count = 4, 5000
     x = synth.ranks(23, n, count, "uniform")
@@ -580,19 +649,51 @@ def test_bucket_calls_refuse_gradients_that_do_not_match_the_plan():
 
 # ------------------------------------------------- bulk-copy one-shot path --
 
-@pytest.mark.parametrize("n", [2, 4, 8, 16, 32, 64])
+@pytest.mark.parametrize("n", [2, 3, 4, 5, 7, 8, 12, 16, 24, 32, 48, 64])
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16", "i32"])
 @pytest.mark.parametrize("op", ["sum", "avg", "max", "min", "prod"])
 def test_bulk_copy_one_shot(n, dtype, op):
-    """Aligned buffers and chunks of whole 16-byte vectors take the one-shot
-    that stages tiles with bulk async copies.  count = n*C - (n-1) with C a
-    multiple of 8 makes the last chunk end n-1 elements short, inside a
-    vector, so the elements past its last whole vector take plain loads."""
+    """Aligned buffers take the one-shot that stages tiles with bulk async
+    copies (rank counts 2, 4, 8, 16, 32, 64 fixed at compile time, the others
+    as a kernel argument).  count = n*C - (n-1) with C a multiple of 8 makes
+    the last chunk end n-1 elements short, inside a vector, so the elements
+    past its last whole vector take plain loads."""
     if dtype == "i32" and op == "avg":
         pytest.skip("AVG is not defined for int32")
     C = 8 * 2000
     count = n * C - (n - 1)
     x, _ = _run(n, count, dtype, op, "oneshot", seed=50 + n)
+    rrv.check_timeouts()
+
+
+@pytest.mark.parametrize("n", [3, 4, 6, 8, 24])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("off", [1, 2, 3])
+def test_bulk_copy_one_shot_shared_phase(n, dtype, off):
+    """Every rank's buffer `off` elements past a 16-byte boundary, and chunks
+    whose length is not a whole number of vectors: each chunk's segment has
+    its own scalar head and tail around the bulk-copied vectors, for the
+    one-shot (SUM and AVG) and the two-shot's first shot (owner only)."""
+    count = n * 3001 + 5
+    _run(n, count, dtype, "avg", "oneshot", seed=40 + n, offsets=[off] * n)
+    _run(n, count, dtype, "sum", "two_shot", seed=41 + n, offsets=[off] * n)
+    rrv.check_timeouts()
+
+
+@pytest.mark.parametrize("n", [3, 8])
+def test_bulk_copy_host_slices(n):
+    """The host-buffer all-reduce folds each 8 MiB slice as its own launch
+    over an element range that cuts chunks: the bulk-copy fold clipped to
+    [lo, hi), against the oracle's whole-buffer fold."""
+    count = (8 << 20) // 4 * 2 + 4099  # three slices, the last one short
+    x = synth.ranks(44 + n, n, count, "full")
+    want = [a.copy() for a in x]
+    oracle.fold_ring_order(want, "sum")
+    host = [torch.from_numpy(a.copy()).pin_memory() for a in x]
+    dev = [torch.empty(count, device="cuda") for _ in range(n)]
+    rrv.all_reduce_host(host, dev, "sum", "oneshot")
+    torch.cuda.synchronize()
+    assert_bits_equal([h.numpy() for h in host], want, f"host slices n={n}")
     rrv.check_timeouts()
 
 
@@ -642,12 +743,13 @@ print("CONTEXT OK")
     assert "CONTEXT OK" in out.stdout, out.stdout
 
 
-@pytest.mark.parametrize("n", [2, 4, 8, 16])
+@pytest.mark.parametrize("n", [2, 3, 4, 6, 8, 16, 24])
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16", "i32"])
 @pytest.mark.parametrize("op", ["sum", "avg", "max", "min", "prod"])
 def test_bulk_copy_reduce_scatter_and_tree_order(n, dtype, op):
-    """Parts (reduce-scatter) and buffers (tree order) of whole 16-byte vectors
-    at aligned addresses take the bulk-copy kernels: same bits as the oracle."""
+    """Parts (reduce-scatter, any rank count) and buffers (tree order, powers
+    of two up to 16) of whole 16-byte vectors at aligned addresses take the
+    bulk-copy kernels: same bits as the oracle."""
     if dtype == "i32" and op == "avg":
         pytest.skip("AVG is not defined for int32")
     per = 8 * 1500
@@ -673,7 +775,7 @@ def test_bulk_copy_bf16_wire(n, op):
     rrv.check_timeouts()
 
 
-@pytest.mark.parametrize("n", [2, 3, 8, 64])
+@pytest.mark.parametrize("n", [2, 3, 5, 8, 64])
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16", "i32"])
 def test_aligned_all_gather_and_two_shot(n, dtype):
     """Parts of whole 16-byte vectors at aligned addresses (the vector path
