@@ -383,8 +383,10 @@ def run_ours(args, d: Dist):
                          "kernel": "bulk_fold_kernel<F32T, AVG, N 8, ring order> (bulk-copy tiles, 2 KB per rank)",
                          "algorithmic_bytes_per_launch": alg_bytes, "peak_kind": peak_kind + " (burst copy)"},
             "copy_ceiling": None if copy_gbs is None else {
-                "copy_gbs": round(copy_gbs, 1), "frac_of_copy": round(achieved / copy_gbs, 4),
-                "what": "torch copy_ of the same 2 GiB (read + write), timed in this run like the headline"},
+                "copy_gbs": round(copy_gbs[0], 1), "frac_of_copy": round(achieved / copy_gbs[0], 4),
+                "own_copy_gbs": round(copy_gbs[1], 1), "frac_of_own_copy": round(achieved / copy_gbs[1], 4),
+                "what": "copies of the same 2 GiB (read + write), timed in this run like the headline: torch "
+                        "copy_, and the library's own copy kernel (all-to-all of one rank)"},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": int(picked["launches"]) * args.steps,
@@ -396,24 +398,33 @@ def run_ours(args, d: Dist):
 
 
 def time_copy_ceiling(dev, stream, nbytes):
-    """GB/s (read + write) of a plain device-to-device copy of nbytes, the
-    same traffic as one headline call, with CUDA events on the stream."""
+    """GB/s (read + write) of plain device-to-device copies of nbytes, the
+    same traffic as one headline call, with CUDA events on the stream: torch's
+    copy_, and the library's own copy kernel (an all-to-all of one rank, which
+    copies its buffer)."""
     import torch
+
+    import ring_all_reduce_virtual_b200 as rrv
 
     src = torch.empty(nbytes // 4, dtype=torch.float32, device=dev).normal_()
     dst = torch.empty_like(src)
-    with torch.cuda.stream(stream):
-        for _ in range(5):
-            dst.copy_(src)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(50):
-            dst.copy_(src)
-        b.record(stream)
-    torch.cuda.synchronize(dev)
-    t = a.elapsed_time(b) / 50 / 1e3
+
+    def rate(fn):
+        with torch.cuda.stream(stream):
+            for _ in range(5):
+                fn()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(50):
+                fn()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        return 2 * nbytes / (a.elapsed_time(b) / 50 / 1e3) / 1e9
+
+    torch_gbs = rate(lambda: dst.copy_(src))
+    own_gbs = rate(lambda: rrv.all_to_all([src], [dst], stream))
     del src, dst
-    return 2 * nbytes / t / 1e9
+    return torch_gbs, own_gbs
 
 
 def time_e2e(args, d, dev, stream, host, bufs, S):

@@ -26,15 +26,19 @@
  *     enqueued on `stream` and the call returns.  A CUDA launch error is
  *     returned as RR_ERR_CUDA (detail in rr_last_error()).
  *   - Argument errors are returned before anything is enqueued:
- *     RR_ERR_INVALID_ARG for a NULL or repeated device pointer, nranks
+ *     RR_ERR_INVALID_ARG for a NULL, repeated or misaligned device pointer, nranks
  *     outside 1..RR_MAX_RANKS, overlapping buffers, a bad enum, an element
  *     count above 2^48 (far past any device memory; it keeps byte ranges
  *     from wrapping) or a count that the operation cannot split;
  *     RR_ERR_UNSUPPORTED for a valid but unsupported combination (AVG on
  *     int32).
- *   - count == 0 is RR_OK and enqueues nothing.  Any pointer alignment is
- *     accepted; buffers whose addresses agree modulo 16 bytes take the
- *     128-bit vector path, the rest a scalar path.
+ *   - count == 0 is RR_OK and enqueues nothing.  A device pointer must sit on
+ *     a boundary of its element size (RR_ERR_INVALID_ARG otherwise); any such
+ *     alignment is accepted.  Buffers whose addresses agree modulo 16 bytes
+ *     take 128-bit vector or bulk-copy access after a scalar head per
+ *     segment; a copy or conversion whose output sits at another 16-byte
+ *     phase than its input is realigned through shared memory; only a
+ *     one-shot over ranks at different phases runs element by element.
  *   - Chunking: chunk size C = ceil(count / N); chunk k is the element range
  *     [k*C, min((k+1)*C, count)), possibly short or empty ([P4] "Ring
  *     all-reduce and communication volume": the tensor is split with
@@ -386,9 +390,20 @@ void rr_reducer_free(rr_reducer_t* red);
 rr_status_t rr_cost_model(rr_algo_t algo, int nranks, double bytes_per_rank, double alpha_s,
                           double beta_bytes_per_s, rr_cost_t* out);
 
-/* The algorithm AUTO runs for this call shape (RING or ONESHOT), from the
- * same model applied to one GPU's launch cost and HBM traffic, with the
- * parameters set by rr_set_picker_params (defaults: 4 us, 6.5 TB/s). */
+/* The algorithm AUTO runs for this call shape on 16-byte aligned buffers
+ * (RING, ONESHOT or TWO_SHOT: the schedules whose results carry the ring's
+ * bits).  It is measured, not modelled: a sweep of every candidate on the GPU
+ * the library is built for gives a table of the fastest per (rank count, bytes
+ * per rank, alignment class), and a call takes the nearest measured rank
+ * count (in log2 ratio) and size ([P3] s4 and [P4] "alpha-beta model" say
+ * which should win for small and large messages; the table is that
+ * measurement).  AUTO itself also keys the table on the call's buffers:
+ * 16-byte aligned, all at one other 16-byte phase, or at phases that differ.
+ * bf16 and fp16 never take RING (its partials round at every hop).
+ * rr_set_picker_params(alpha, beta) makes AUTO use the model instead -- the
+ * rr_cost_model of one GPU, a launch costing alpha seconds and HBM moving beta
+ * bytes per second -- and rr_set_picker_params(0, 0) returns to the table
+ * (whose sweep also fitted the model's default alpha and beta). */
 rr_algo_t rr_pick_algo(int nranks, size_t count, rr_dtype_t dtype);
 rr_status_t rr_set_picker_params(double launch_s, double hbm_bytes_per_s);
 

@@ -356,20 +356,16 @@ rr_status_t run_ring(void* const* bufs, int n, size_t count, rr_dtype_t dtype, r
                 if (st != RR_OK) return st;
             }
     }
+    // over the reduce-scatter rank r sends chunks r, r-1, ..., r+2 (every chunk
+    // but r+1), over the all-gather chunks r+1, r, ..., r+3 (every chunk but r+2)
     const uint64_t wes = wire ? 2 : es;  // bytes a sent element takes on the wire
-    for (int phase = RR_PHASE_REDUCE_SCATTER; phase <= RR_PHASE_ALL_GATHER; ++phase)
-        for (int s = 0; s < n - 1; ++s)
-            for (int r = 0; r < n; ++r) {
-                const uint64_t b = chunk_len(count, n, ring_send_chunk(phase, r, s, n)) * wes;
-                t_stats.bytes_sent_total += b;
-            }
-    t_stats.steps = 2 * (n - 1);
     for (int r = 0; r < n; ++r) {
-        uint64_t sent = 0;
-        for (int phase = RR_PHASE_REDUCE_SCATTER; phase <= RR_PHASE_ALL_GATHER; ++phase)
-            for (int s = 0; s < n - 1; ++s) sent += chunk_len(count, n, ring_send_chunk(phase, r, s, n)) * wes;
+        const uint64_t sent =
+            (2 * (uint64_t)count - chunk_len(count, n, imod(r + 1, n)) - chunk_len(count, n, imod(r + 2, n))) * wes;
         t_stats.bytes_sent_max = std::max<uint64_t>(t_stats.bytes_sent_max, sent);
+        t_stats.bytes_sent_total += sent;
     }
+    t_stats.steps = 2 * (n - 1);
     // each reduce-scatter step reads 2 and writes 1 chunk per rank, each
     // all-gather step reads and writes 1: 5 (N-1) S in all
     t_stats.hbm_bytes = 5ull * (uint64_t)(n - 1) * count * es;
@@ -438,11 +434,11 @@ rr_status_t run_double_ring(void* const* bufs, int n, size_t count, rr_dtype_t d
         cudaError_t e = timed_launch([&] { return launch_ring_chain(dtype, op, false, p, stream); });
         if (e != cudaSuccess) return cuda_fail(e, "double ring launch");
         t_stats.launches += 1;
-        for (int phase = RR_PHASE_REDUCE_SCATTER; phase <= RR_PHASE_ALL_GATHER; ++phase)
-            for (int s = 0; s < n - 1; ++s)
-                for (int r = 0; r < n; ++r)
-                    sent[r] += (chunk_len(H, n, ring_send_chunk(phase, r, s, n)) +
-                                chunk_len(cb, n, ccw_send_chunk(phase, r, s, n))) * esize(dtype);
+        // each half as the ring: the clockwise half skips chunks r+1 and r+2, the
+        // mirror ring (chunks sent downwards) chunks r-1 and r-2
+        for (int r = 0; r < n; ++r)
+            sent[r] = (2 * H - chunk_len(H, n, imod(r + 1, n)) - chunk_len(H, n, imod(r + 2, n)) + 2 * cb -
+                       chunk_len(cb, n, imod(r - 1, n)) - chunk_len(cb, n, imod(r - 2, n))) * esize(dtype);
     } else {
         for (int phase = RR_PHASE_REDUCE_SCATTER; phase <= RR_PHASE_ALL_GATHER; ++phase)
             for (int s = 0; s < n - 1; ++s) {
@@ -1224,6 +1220,7 @@ rr_status_t bucket_range_check(const rr_bucket_plan_t* plan, int b0, int nb, con
         for (int t = *t0; t < *t0 + *nt; ++t) {
             const void* g = grads[(size_t)r * plan->ntensors + t];
             if (plan->numel[t] == 0) continue;
+            if ((uintptr_t)g % es != 0) return fail(RR_ERR_INVALID_ARG, "gradient not aligned to its element size");
             spans.push_back({(uintptr_t)g, (uintptr_t)g + plan->numel[t] * es, true});
         }
     return check_spans(spans);
@@ -1252,7 +1249,7 @@ static rr_status_t bucket_copy(const rr_bucket_plan_t* plan, int bucket, const v
     for (int r = 0; r < n; ++r)
         spans.push_back({(uintptr_t)buckets[r], (uintptr_t)buckets[r] + plan->bnumel[bucket] * 4, true});
     if (plan->bnumel[bucket] && (st = check_spans(spans)) != RR_OK) return st;
-    bool vec = same_phase(buckets, n);
+    if ((st = check_elem_aligned(buckets, n, 4)) != RR_OK) return st;
     const int per_launch = std::max(1, std::min(kMaxBucketTensors, kMaxBucketPtrs / n));
     auto* p = new BucketCopyParams();
     for (int g0 = 0; g0 < nt; g0 += per_launch) {
@@ -1262,20 +1259,17 @@ static rr_status_t bucket_copy(const rr_bucket_plan_t* plan, int bucket, const v
         p->nt = g1 - g0;
         p->divisor = (float)n;
         uint64_t maxlen = 0;
-        bool v = vec;
         const uint64_t te = bucket_tile_elems(plan->grad_dtype);
         p->tile0[0] = 0;
         for (int t = g0; t < g1; ++t) {
             const int gt = t0 + t;
             for (int r = 0; r < n; ++r) p->grad[(t - g0) * n + r] = grads[(size_t)r * plan->ntensors + gt];
-            v = v && same_phase(&p->grad[(t - g0) * n], n);
             p->toff[t - g0] = plan->offset[gt];
             p->tlen[t - g0] = plan->numel[gt];
             p->tile0[t - g0 + 1] = p->tile0[t - g0] + (uint64_t)n * ceil_div(plan->numel[gt], te);
             maxlen = std::max<uint64_t>(maxlen, plan->numel[gt]);
         }
         for (int r = 0; r < n; ++r) p->bucket[r] = buckets[r];
-        p->vec_ok = v;
         if (maxlen == 0) continue;
         cudaError_t e = timed_launch([&] {
             return pack ? launch_bucket_pack(plan->grad_dtype, *p, stream)

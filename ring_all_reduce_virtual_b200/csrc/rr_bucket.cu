@@ -74,45 +74,71 @@ struct Quad<BF16T> : Quad16<BF16T> {};
 template <>
 struct Quad<F16T> : Quad16<F16T> {};
 
-// The quads of one tile of a conversion (see convert_tile), with the source
-// quads D elements out of step with the destination's: D = 0 reads one
-// aligned source quad per destination quad; D > 0 reads that quad and the
-// next and shifts them into place.  Every load of the thread is issued
-// before the first one is used, so Q (or 2Q) loads are in flight.
-template <class In, class Out, int OP, int Q, bool SHIFT>
+// The quads of one tile of a conversion (see convert_tile) whose source
+// quads are in step with the destination's: one aligned load per quad, Q per
+// thread all issued before the first one is used.
+template <class In, class Out, int OP, int Q>
 __device__ __forceinline__ void convert_quads(const typename In::T* s0, typename Out::T* dst, uint64_t head, uint64_t nq,
-                                              uint64_t tile, int d, float divisor)
+                                              uint64_t tile, float divisor)
 {
     constexpr uint64_t TQ = (uint64_t)kThreads * Q;
-    // passes of 4 quads per thread (64 bytes of fp32 on the wider side), 2
-    // when a quad takes two loads
-    constexpr int QP = SHIFT ? 2 : 4;
-    constexpr int P = Q / QP;
-    static_assert(QP >= 1 && Q % QP == 0, "whole passes");
+    constexpr int QP = 4;  // quads per pass: 64 bytes of fp32 on the wider side
+    static_assert(Q % QP == 0, "whole passes");
     const uint64_t tid = threadIdx.x;
 #pragma unroll
-    for (int pass = 0; pass < P; ++pass) {
-        typename Quad<In>::R lo[QP], hi[QP];
+    for (int pass = 0; pass < Q / QP; ++pass) {
+        typename Quad<In>::R raw[QP];
 #pragma unroll
         for (int k = 0; k < QP; ++k) {
             const uint64_t q = tile * TQ + (uint64_t)(pass * QP + k) * kThreads + tid;
-            if (q < nq) {
-                lo[k] = Quad<In>::ld(s0 + q * 4);
-                if constexpr (SHIFT) hi[k] = Quad<In>::ld(s0 + q * 4 + 4);
-            }
+            if (q < nq) raw[k] = Quad<In>::ld(s0 + q * 4);
         }
 #pragma unroll
         for (int k = 0; k < QP; ++k) {
             const uint64_t q = tile * TQ + (uint64_t)(pass * QP + k) * kThreads + tid;
             if (q >= nq) continue;
             float a[4];
-            if constexpr (SHIFT) Quad<In>::to_f(Quad<In>::shift(lo[k], hi[k], d), a);
-            else Quad<In>::to_f(lo[k], a);
+            Quad<In>::to_f(raw[k], a);
 #pragma unroll
             for (int l = 0; l < 4; ++l) a[l] = finish<OP>(a[l], divisor);
             Quad<Out>::st(dst + head + q * 4, Quad<Out>::from_f(a));
         }
     }
+}
+
+// The same when the source quads are d = 1..3 elements out of step: the
+// tile's source quads (and the one after, which holds the last few elements)
+// are loaded aligned -- one load per quad, all in flight -- into shared
+// memory, and each destination quad reads the two stage quads it straddles
+// and shifts them in registers, so no global load is issued twice.  Every thread of the CTA takes
+// part (the tile is the CTA's).
+template <class In, class Out, int OP, int Q>
+__device__ __forceinline__ void convert_quads_staged(const typename In::T* s0, typename Out::T* dst, uint64_t head,
+                                                     uint64_t nq, uint64_t tile, int d, float divisor)
+{
+    using R = typename Quad<In>::R;
+    constexpr uint32_t TQ = (uint32_t)kThreads * Q;
+    __shared__ R stage[TQ + 1];
+    const uint64_t q0 = tile * TQ;
+    if (q0 >= nq) return;
+    const uint32_t nqt = nq - q0 < TQ ? (uint32_t)(nq - q0) : TQ;  // destination quads of this tile
+#pragma unroll
+    for (int k = 0; k <= Q; ++k) {
+        const uint32_t i = (uint32_t)k * kThreads + threadIdx.x;
+        if (i <= nqt) stage[i] = Quad<In>::ld(s0 + (q0 + i) * 4);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < Q; ++k) {
+        const uint32_t i = (uint32_t)k * kThreads + threadIdx.x;
+        if (i >= nqt) continue;
+        float a[4];
+        Quad<In>::to_f(Quad<In>::shift(stage[i], stage[i + 1], d), a);  // two aligned stage reads, shifted
+#pragma unroll
+        for (int l = 0; l < 4; ++l) a[l] = finish<OP>(a[l], divisor);
+        Quad<Out>::st(dst + head + (q0 + i) * 4, Quad<Out>::from_f(a));
+    }
+    __syncthreads();  // the stage is free for the CTA's next tile
 }
 
 // Convert one tile of a segment from In's element type to Out's, dividing by
@@ -121,12 +147,12 @@ __device__ __forceinline__ void convert_quads(const typename In::T* s0, typename
 // type (bucket_tile_elems).  The quads are aligned to the destination: after
 // a scalar head up to dst's first quad boundary, every quad is one aligned
 // store, and its source elements -- which start d = (phase of src - phase of
-// dst) mod 4 elements into an aligned source quad -- are read as that quad
-// and, when d > 0, the next one, and shifted into place.  The window's second
-// quad holds at least one element of the source quad, so no load reaches
-// past the aligned block of the segment's last element (nor before the
-// block of its first).  Tile 0 also does the head and the tail (< 4 elements
-// each).
+// dst) mod 4 elements into an aligned source quad -- are read from that quad
+// and, when d > 0, the next one, through shared memory (convert_quads_staged).
+// Every source quad loaded holds at least one element of the segment, so no
+// load reaches past the aligned block of the segment's last element (nor
+// before the block of its first).  Tile 0 also does the head and the tail
+// (< 4 elements each).  Every thread of the CTA calls this for the same tile.
 template <class In, class Out, int OP, int Q = kUnitsPerThread * (In::L > Out::L ? In::L : Out::L) / 4>
 __device__ __forceinline__ void convert_tile(const typename In::T* src, typename Out::T* dst, uint64_t len,
                                              uint64_t tile, float divisor)
@@ -145,8 +171,8 @@ __device__ __forceinline__ void convert_tile(const typename In::T* src, typename
     // the aligned source quad under dst's first quad (d elements before src + head)
     const auto* s0 = reinterpret_cast<const typename In::T*>(reinterpret_cast<uintptr_t>(src + head) -
                                                               (uintptr_t)d * sizeof(typename In::T));
-    if (d == 0) convert_quads<In, Out, OP, Q, false>(s0, dst, head, nq, tile, 0, divisor);
-    else convert_quads<In, Out, OP, Q, true>(s0, dst, head, nq, tile, d, divisor);
+    if (d == 0) convert_quads<In, Out, OP, Q>(s0, dst, head, nq, tile, divisor);
+    else convert_quads_staged<In, Out, OP, Q>(s0, dst, head, nq, tile, d, divisor);
 }
 
 // The segment owning work item w: the last s with prefix[s] <= w (segments
@@ -238,12 +264,14 @@ __global__ void __launch_bounds__(kThreads) bucket_fold_kernel(const __grid_cons
 // at any element, so tile 0 folds the elements before the segment's first
 // 16-byte boundary and after its last whole vector with plain loads, and the
 // bulk copies move the whole vectors between.  Needs every rank's copy of a
-// tensor at the same address modulo 16 (vec_ok) and N = 2, 4, 8 or 16.
+// tensor at the same address modulo 16 (vec_ok) and 2-16 ranks (2, 4, 8 and
+// 16 fixed at compile time, the others a kernel argument).
 struct BucketBulkParams {
     BucketFoldParams f;  // tile0 counts bulk tiles (bucket_bulk_tile_elems)
     unsigned int* waits; // as BulkParams (rr_bulk.cuh): the wait counters, the test hook, the bound
     uint32_t hold;
     uint32_t spin;
+    uint32_t tv;         // vectors per rank per tile (kernels whose rank count is not fixed)
 };
 static_assert(sizeof(BucketBulkParams) <= 32764, "BucketBulkParams too large");
 
@@ -253,20 +281,21 @@ __global__ void __launch_bounds__(kThreads) bucket_bulk_kernel(const __grid_cons
     using T = typename G::T;
     using Acc = typename G::Acc;
     constexpr int L = G::L;
-    constexpr uint32_t TV = bulk_smem<NS>() / NS / 16;  // vectors per rank per tile
     const BucketFoldParams& p = bp.f;
-    extern __shared__ __align__(128) uint4 sm[];       // [NS][TV]: slot j holds rank (c + j) mod N
+    const int n = NS > 0 ? NS : p.n;
+    const uint32_t TV = NS > 0 ? bulk_smem<NS>() / (NS > 0 ? NS : 1) / 16 : bp.tv;  // vectors per rank per tile
+    extern __shared__ __align__(128) uint4 sm[];       // [n][TV]: slot j holds rank (c + j) mod N
     __shared__ __align__(8) uint64_t bar;
 
     const uint64_t w = blockIdx.x;
     const int s = find_segment(p.tile0, p.nseg, w);
     const uint64_t tile = w - p.tile0[s];
     const BucketSeg& sg = p.seg[s];
-    const int base = (int)sg.t * NS;
+    const int base = (int)sg.t * n;
     const int start = (int)sg.c;
     auto in = [&](int j) {
         int r = start + j;
-        if (r >= NS) r -= NS;
+        if (r >= n) r -= n;
         return static_cast<const T*>(p.grad[base + r]) + sg.off;
     };
     auto out = [&](int o) { return static_cast<T*>(p.grad[base + o]) + sg.off; };
@@ -277,7 +306,7 @@ __global__ void __launch_bounds__(kThreads) bucket_bulk_kernel(const __grid_cons
     const uint64_t tail = len - head - nv * L;
     if (tile == 0 && (uint64_t)threadIdx.x < head + tail) {
         const uint64_t e = (uint64_t)threadIdx.x < head ? (uint64_t)threadIdx.x : head + nv * L + (threadIdx.x - head);
-        fold_one<G, OP, 0>(in, NS, out, NS, e, p.divisor);
+        fold_one<G, OP, 0>(in, n, out, n, e, p.divisor);
     }
     const uint64_t v0 = tile * TV;
     if (v0 >= nv) return;
@@ -290,9 +319,9 @@ __global__ void __launch_bounds__(kThreads) bucket_bulk_kernel(const __grid_cons
     __syncthreads();
     if (threadIdx.x == 0) {
         asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
-                     ::"r"(b), "r"(bytes * NS) : "memory");
+                     ::"r"(b), "r"(bytes * (uint32_t)n) : "memory");
 #pragma unroll
-        for (int j = 0; j < NS; ++j)
+        for (int j = 0; j < (NS > 0 ? NS : n); ++j)
             asm volatile(
                 "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                 ::"r"(bulk_smem_addr(sm + j * TV)), "l"(in(j) + e0), "r"(bytes), "r"(b)
@@ -302,8 +331,8 @@ __global__ void __launch_bounds__(kThreads) bucket_bulk_kernel(const __grid_cons
     for (uint32_t v = threadIdx.x; v < nvt; v += kThreads) {
         Acc a[L];
         G::unpack(sm[v], a);
-#pragma unroll
-        for (int j = 1; j < NS; ++j) {
+#pragma unroll 4
+        for (int j = 1; j < (NS > 0 ? NS : n); ++j) {
             Acc x[L];
             G::unpack(sm[j * TV + v], x);
 #pragma unroll
@@ -316,8 +345,7 @@ __global__ void __launch_bounds__(kThreads) bucket_bulk_kernel(const __grid_cons
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
     if (threadIdx.x == 0) {
-#pragma unroll
-        for (int o = 0; o < NS; ++o)
+        for (int o = 0; o < n; ++o)
             asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
                          ::"l"(out(o) + e0), "r"(bulk_smem_addr(sm)), "r"(bytes)
                          : "memory");
@@ -331,8 +359,7 @@ __global__ void __launch_bounds__(kThreads) bucket_bulk_kernel(const __grid_cons
 // share of bulk_smem<N>().
 uint64_t bucket_bulk_tile_elems(int grad_dtype, int n)
 {
-    const uint64_t bytes = (n >= 32 ? 32768u : 16384u) / (uint64_t)n;
-    return bytes / 16 * (grad_dtype == kF32 ? 4u : 8u);
+    return (uint64_t)bulk_tile_vectors(n) * (grad_dtype == kF32 ? 4u : 8u);
 }
 
 template <class G, int OP>
@@ -356,14 +383,16 @@ cudaError_t launch_bucket_bulk(const BucketFoldParams& p, int grad_dtype, cudaSt
     cudaError_t e = cudaSuccess;
     if (work > 0 && work <= kMaxGrid) {
         *launched = true;
+        bp->tv = bulk_tile_vectors(p.n);
         switch (p.n) {
         case 2: bucket_bulk_kernel<G, OP, 2><<<(unsigned)work, kThreads, bulk_smem<2>(), s>>>(*bp); break;
         case 4: bucket_bulk_kernel<G, OP, 4><<<(unsigned)work, kThreads, bulk_smem<4>(), s>>>(*bp); break;
         case 8: bucket_bulk_kernel<G, OP, 8><<<(unsigned)work, kThreads, bulk_smem<8>(), s>>>(*bp); break;
         case 16: bucket_bulk_kernel<G, OP, 16><<<(unsigned)work, kThreads, bulk_smem<16>(), s>>>(*bp); break;
-        default: *launched = false;
+        default:
+            bucket_bulk_kernel<G, OP, 0><<<(unsigned)work, kThreads, bp->tv * 16u * (uint32_t)p.n, s>>>(*bp);
         }
-        if (*launched) e = cudaGetLastError();
+        e = cudaGetLastError();
     } else if (work == 0) {
         *launched = true;
     }
@@ -431,7 +460,7 @@ cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p
     const uint64_t work = p.tile0[p.nseg];
     const bool avg = op == kAvg;
     // the bulk-copy fold when it applies (no CTA cap: one CTA per tile)
-    if (max_grid >= kMaxGrid && p.vec_ok && (p.n == 2 || p.n == 4 || p.n == 8 || p.n == 16)) {
+    if (max_grid >= kMaxGrid && p.vec_ok && p.n >= 2 && p.n <= 16) {
         bool launched = false;
         cudaError_t e = cudaSuccess;
         if (grad_dtype == kBF16)

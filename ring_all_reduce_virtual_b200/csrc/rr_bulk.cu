@@ -132,15 +132,18 @@ bool bulk_eligible(const RankParams& p, int esize)
 bool bulk_scatter_eligible(const RankParams& p, int esize)
 {
     // every input at one 16-byte phase (so part r of every rank is too), every
-    // output at one phase, all on element boundaries
-    if (!p.waits || p.n < 2 || p.n > kMaxRanks || !p.vec_ok || p.nseg != (uint64_t)p.n) return false;
+    // output at one phase, all on element boundaries; up to 16 ranks (beyond,
+    // a rank's tile is under 1 KB, too few threads fold each tile and a part
+    // has one small output to hide that: 64 ranks ran at 0.71 of the copy peak
+    // against 1.10 with per-thread loads)
+    if (!p.waits || p.n < 2 || p.n > 16 || !p.vec_ok || p.nseg != (uint64_t)p.n) return false;
     if ((uintptr_t)p.in[0] % (uintptr_t)esize != 0 || (uintptr_t)p.out[0] % (uintptr_t)esize != 0) return false;
     return tiles_of(p.C, esize, p.n) * (uint64_t)p.n <= kMaxGrid;
 }
 
 bool bulk_tree_eligible(const RankParams& p, int esize)
 {
-    if (!bulk_ranks_aligned(p, 16, true) || p.nseg != 1) return false;
+    if (!bulk_ranks_aligned(p, 16, false) || p.nseg != 1 || (p.n > 8 && p.n != 16)) return false;
     if ((p.count * (uint64_t)esize) % 16 != 0) return false;  // the buffer is whole vectors
     return tiles_of(p.count, esize, p.n) <= kMaxGrid;
 }

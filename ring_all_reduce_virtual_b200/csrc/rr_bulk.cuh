@@ -12,8 +12,8 @@
 //   kBulkScatter  the reduce-scatter: segment r = part r of every rank,
 //                 folded in ring order from rank r, written to out[r] only
 //   kBulkTree     the tree-order one-shot: the whole buffer, folded in the
-//                 tree's pairwise order (N a power of two), written to every
-//                 rank
+//                 tree's pairwise order (an unpaired rank carried up), written
+//                 to every rank
 //
 // The ring mode runs wherever every input and output address has the same
 // 16-byte phase (a scalar head and tail per segment, whole vectors between),
@@ -21,7 +21,7 @@
 // bulk copies when it shares that phase, by the threads otherwise), both for
 // 2-64 ranks; the tree mode where the buffers are whole 16-byte vectors at
 // 16-byte aligned addresses (bulk_*_eligible).  The rank count is a
-// compile-time constant for 2, 4, 8, 16, 32 and 64 ranks (tree: 2-16) and a
+// compile-time constant for 2, 4, 8, 16, 32 and 64 ranks (tree: 2-8 and 16) and a
 // kernel argument (NS = 0) otherwise; with the copy engine doing the loads,
 // a runtime count costs the fold no registers.  Every other call takes the
 // per-thread-load kernels, with the same bits.  The fold itself uses the
@@ -133,8 +133,8 @@ __global__ void __launch_bounds__(kThreads) bulk_fold_kernel(const __grid_consta
     using T = typename Ty::T;
     using Acc = typename Ty::Acc;
     constexpr int L = Ty::L;  // elements per 16-byte vector
-    static_assert(NS == 0 || (bulk_smem<NS>() / (NS > 0 ? NS : 1)) % 16 == 0, "tile of whole vectors");
-    static_assert(MODE != kBulkTree || (NS > 0 && (NS & (NS - 1)) == 0), "the pairwise tree needs a fixed power of two");
+    static_assert(NS == 0 || bulk_smem<NS>() / (NS > 0 ? NS : 1) >= 16, "a tile of at least one vector per rank");
+    static_assert(MODE != kBulkTree || NS > 0, "the pairwise tree needs a fixed rank count");
     static_assert(MODE == kBulkRing || WIRE == 0, "the wire format is a ring-order one-shot");
     const RankParams& p = bp.r;
     const int n = NS > 0 ? NS : p.n;
@@ -215,7 +215,12 @@ __global__ void __launch_bounds__(kThreads) bulk_fold_kernel(const __grid_consta
         Acc a[L];
         if constexpr (MODE == kBulkTree) {
             // pairwise order with fp32 partials: slot j joins a stack whose
-            // level b holds a finished block of 2^b ranks (no rounding between levels)
+            // level b holds a finished block of 2^b ranks (no rounding between
+            // levels).  After the last slot the stack holds one block per set
+            // bit of N; the tree carries an unpaired block up until a level
+            // pairs it, so the blocks combine from the lowest level upwards,
+            // each higher block on the left (one block of all ranks when N is
+            // a power of two).
             constexpr int LV = NS <= 2 ? 2 : NS <= 4 ? 3 : NS <= 8 ? 4 : NS <= 16 ? 5 : NS <= 32 ? 6 : 7;
             Acc stack[LV][L];
 #pragma unroll
@@ -236,8 +241,14 @@ __global__ void __launch_bounds__(kThreads) bulk_fold_kernel(const __grid_consta
 #pragma unroll
                         for (int l = 0; l < L; ++l) stack[bb][l] = a[l];
             }
+            bool have = false;
 #pragma unroll
-            for (int l = 0; l < L; ++l) a[l] = stack[LV - 1][l];  // N = 2^(LV-1): one block of all ranks
+            for (int bb = 0; bb < LV; ++bb) {
+                if (!((NS >> bb) & 1)) continue;
+#pragma unroll
+                for (int l = 0; l < L; ++l) a[l] = have ? apply<OP>(stack[bb][l], a[l]) : stack[bb][l];
+                have = true;
+            }
         } else {
             Ty::unpack(sm[v], a);
 #pragma unroll 4

@@ -252,6 +252,23 @@ __device__ __forceinline__ void st_lanes(T* q, const uint4& r)
     for (int l = 0; l < L; ++l) q[l] = e[l];
 }
 
+// The 16 bytes that start b bytes into the 32-byte window lo:hi (0 < b < 16,
+// b even: a whole number of 16- or 32-bit elements).
+__device__ __forceinline__ uint4 shift_window(const uint4& lo, const uint4& hi, int b)
+{
+    uint32_t w0, w1, w2, w3, w4;  // five words from word b / 4 on
+    switch (b >> 2) {
+    case 0: w0 = lo.x; w1 = lo.y; w2 = lo.z; w3 = lo.w; w4 = hi.x; break;
+    case 1: w0 = lo.y; w1 = lo.z; w2 = lo.w; w3 = hi.x; w4 = hi.y; break;
+    case 2: w0 = lo.z; w1 = lo.w; w2 = hi.x; w3 = hi.y; w4 = hi.z; break;
+    default: w0 = lo.w; w1 = hi.x; w2 = hi.y; w3 = hi.z; w4 = hi.w; break;
+    }
+    if (b & 3)
+        return make_uint4(__funnelshift_r(w0, w1, 16), __funnelshift_r(w1, w2, 16), __funnelshift_r(w2, w3, 16),
+                          __funnelshift_r(w3, w4, 16));
+    return make_uint4(w0, w1, w2, w3);
+}
+
 // --------------------------------------------------------------- the tile
 
 // Scalar fold of element e of a segment.

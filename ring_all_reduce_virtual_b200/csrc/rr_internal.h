@@ -89,8 +89,8 @@ struct BucketCopyParams {
     uint64_t tile0[kMaxBucketTensors + 1]; // first work item of tensor t (n ranks x its tiles)
     int n;
     int nt;
-    int vec_ok;
     float divisor;
+    int pad_;
 };
 
 // A fused bucket segment: elements [off, off + len) of launch tensor t, all

@@ -17,6 +17,66 @@ namespace rr {
 namespace {
 
 
+// Copy tile `tile` of a segment of `len` elements, in -> out, the bits as
+// they are; tiles as fold_tile's with VPT vectors per thread.  When in and
+// out have the same 16-byte phase: whole vectors (fold_tile's copy path).
+// Otherwise the tile's vectors are aligned to the output, and their source
+// elements, d = (phase of in - phase of out) mod L elements into an aligned
+// input vector, are copied aligned -- one asynchronous copy per input vector,
+// plus the one after, which holds the last few elements -- into shared
+// memory; each
+// output vector reads the two stage vectors it straddles and shifts them in
+// registers, so every access is a whole aligned vector and no global load is
+// issued twice.  Every thread of the CTA calls this for the same tile.
+template <class Ty, int VPT>
+__device__ __forceinline__ void copy_tile(const typename Ty::T* in, typename Ty::T* out, uint64_t len, uint64_t tile)
+{
+    using T = typename Ty::T;
+    constexpr int L = Ty::L;
+    constexpr uint32_t TV = (uint32_t)kThreads * VPT;
+    const int pin = phase_of(in, L), pout = phase_of(out, L);
+    if (pin == pout) {
+        auto i0 = [&](int) { return in; };
+        auto o0 = [&](int) { return out; };
+        fold_tile<Ty, kSum, VPT, 1>(i0, 1, o0, 1, len, tile, true, 1.0f);
+        return;
+    }
+    uint64_t head = (uint64_t)((L - pout) & (L - 1));
+    if (head > len) head = len;
+    const uint64_t nv = (len - head) / L, tail = len - head - nv * L;
+    if (tile == 0 && (uint64_t)threadIdx.x < head + tail) {
+        const uint64_t e = (uint64_t)threadIdx.x < head ? (uint64_t)threadIdx.x : head + nv * L + (threadIdx.x - head);
+        out[e] = in[e];
+    }
+    const uint64_t v0 = tile * TV;
+    if (v0 >= nv) return;
+    const uint32_t nvt = nv - v0 < TV ? (uint32_t)(nv - v0) : TV;
+    const int d = (pin - pout) & (L - 1);
+    const T* ib = reinterpret_cast<const T*>(reinterpret_cast<uintptr_t>(in + head + v0 * L) - (uintptr_t)d * sizeof(T));
+    __shared__ __align__(16) uint4 stage[TV + 1];
+    // global -> shared without passing through registers (the one-to-many
+    // copies run at 32 registers a thread), all of the thread's copies in flight
+#pragma unroll
+    for (int k = 0; k <= VPT; ++k) {
+        const uint32_t i = (uint32_t)k * kThreads + threadIdx.x;
+        if (i <= nvt)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(&stage[i])),
+                         "l"(ib + (uint64_t)i * L)
+                         : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+#pragma unroll 1
+    for (int k = 0; k < VPT; ++k) {
+        const uint32_t i = (uint32_t)k * kThreads + threadIdx.x;
+        if (i >= nvt) continue;
+        // two aligned 16-byte reads of the stage, shifted in registers
+        stv(out + head + (v0 + i) * L, shift_window(stage[i], stage[i + 1], d * (int)sizeof(T)));
+    }
+    __syncthreads();  // the stage is free for the CTA's next tile
+}
+
 // The one-to-many copies below give each CTA one tile of one output (16 KB
 // in, 16 KB out): such short-lived CTAs keep enough bytes in flight only at
 // full occupancy, so they are held to the registers of 8 CTAs per SM
@@ -45,9 +105,7 @@ __global__ void __launch_bounds__(kThreads, kSmallCtasPerSm) chunk_bcast_kernel(
         const uint64_t len = p.count - lo < p.C ? p.count - lo : p.C;
         const int owner = (int)c;
         const int dst = (int)k < owner ? (int)k : (int)k + 1;
-        auto in = [&](int) { return static_cast<const T*>(p.in[owner]) + lo; };
-        auto out = [&](int) { return static_cast<T*>(p.out[dst]) + lo; };
-        fold_tile<Ty, kSum, kVptMove, 1>(in, 1, out, 1, len, tile, p.vec_ok, 1.0f);
+        copy_tile<Ty, kVptMove>(static_cast<const T*>(p.in[owner]) + lo, static_cast<T*>(p.out[dst]) + lo, len, tile);
     }
 }
 
@@ -89,9 +147,7 @@ __global__ void __launch_bounds__(kThreads, kSmallCtasPerSm) all_gather_kernel(c
     for (uint64_t w = blockIdx.x; w < total; w += gridDim.x) {
         const uint64_t st = w / n, o = w - st * n;
         const uint64_t q = st / p.tps, tile = st - q * p.tps;
-        auto in = [&](int) { return static_cast<const T*>(p.in[q]); };
-        auto out = [&](int) { return static_cast<T*>(p.out[o]) + q * p.C; };
-        fold_tile<Ty, kSum, kVptMove, 1>(in, 1, out, 1, p.C, tile, p.vec_ok, 1.0f);
+        copy_tile<Ty, kVptMove>(static_cast<const T*>(p.in[q]), static_cast<T*>(p.out[o]) + q * p.C, p.C, tile);
     }
 }
 
@@ -105,9 +161,7 @@ __global__ void __launch_bounds__(kThreads) all_to_all_kernel(const __grid_const
     for (uint64_t w = blockIdx.x; w < total; w += gridDim.x) {
         const uint64_t s = w / p.tps, tile = w - s * p.tps;
         const uint64_t r = s / (uint64_t)p.n, q = s - r * (uint64_t)p.n;
-        auto in = [&](int) { return static_cast<const T*>(p.in[q]) + r * p.C; };
-        auto out = [&](int) { return static_cast<T*>(p.out[r]) + q * p.C; };
-        fold_tile<Ty, kSum, kVptMove, 1>(in, 1, out, 1, p.C, tile, 1, 1.0f);
+        copy_tile<Ty, kVptMove>(static_cast<const T*>(p.in[q]) + r * p.C, static_cast<T*>(p.out[r]) + q * p.C, p.C, tile);
     }
 }
 

@@ -179,6 +179,26 @@ def test_fold_order_fixture():
     assert to_host(d)[0][0] == 1.0
 
 
+@pytest.mark.parametrize("algo", ["tree", "tree_oneshot"])
+@pytest.mark.parametrize("count", [4, 4096, 5])
+def test_tree_order_with_unpaired_ranks_golden(algo, count):
+    """The hand-derived fixture of the tree's order for N = 3, 5, 6, 7 (an
+    unpaired rank carried up to the next level), on every element of buffers
+    of one vector, of many tiles (bulk-copy tree fold and the single-launch
+    tree schedule) and of a ragged size."""
+    from conftest import golden_lines
+
+    for ln in golden_lines("tree_order_unpaired.txt"):
+        n_s, xs, want = ln.split(":")
+        vals = [np.float32(float(v)) for v in xs.split()]
+        x = [np.full(count, v, dtype=np.float32) for v in vals]
+        d = to_dev(x)
+        rrv.all_reduce(d, "sum", algo)
+        for r, g in enumerate(to_host(d)):
+            assert np.all(g == np.float32(float(want))), (algo, n_s, r, g[:4])
+    rrv.check_timeouts()
+
+
 def test_max_signed_zero_ties_follow_the_fold():
     n = 4
     x = [np.full(n, -1.0, dtype=np.float32) for _ in range(n)]
@@ -263,6 +283,45 @@ def test_reduce_scatter_all_gather_all_to_all(n, dtype):
     a2a = empty_like_ranks(n, n * per, dtype)
     rrv.all_to_all(d, a2a)
     assert_bits_equal(to_host(a2a), oracle.all_to_all(x), "a2a")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16", "i32"])
+@pytest.mark.parametrize("shift", [1, 2, 3, 5, 7])
+def test_copies_to_another_phase(dtype, shift):
+    """All-gather and all-to-all blocks of a length that is `shift` elements
+    past a whole number of 16-byte vectors, over several tiles: block q lands
+    q * shift elements out of phase with its source, so the copies take the
+    shift through shared memory; and the fused/staged bucket paths on tensors
+    whose bucket offsets take every phase."""
+    L = 4 if dtype in ("f32", "i32") else 8
+    if shift >= L:
+        pytest.skip("shift within one vector")
+    n = 3
+    per = 3 * TILE_MOVE[dtype] + shift
+    x = synth.ranks(11 + shift, n, per, "int" if dtype == "i32" else "full", dtype)
+    ag = empty_like_ranks(n, n * per, dtype)
+    rrv.all_gather(to_dev(x), ag)
+    assert_bits_equal(to_host(ag), oracle.all_gather(x), f"ag shift {shift}")
+    y = synth.ranks(12 + shift, n, n * per, "int" if dtype == "i32" else "full", dtype)
+    a2a = empty_like_ranks(n, n * per, dtype)
+    rrv.all_to_all(to_dev(y), a2a)
+    assert_bits_equal(to_host(a2a), oracle.all_to_all(y), f"a2a shift {shift}")
+    if dtype == "i32":
+        return
+    numels = [shift, 20000 + shift, 3, 30001, 17]  # later tensors start at every phase, over several tiles
+    host = _grad_set(13 + shift, n, numels, dtype)
+    want = [[g.copy() for g in rank] for rank in host]
+    cap = 1 << 30
+    oracle.bucket_sync(want, cap, "avg")
+    plan = rrv.BucketPlan(numels, dtype, cap)
+    grads = [to_dev(rank) for rank in host]
+    numel = plan.info(0)[2]
+    buckets = [torch.empty(numel, dtype=torch.float32, device="cuda") for _ in range(n)]
+    plan.pack(0, grads, buckets)
+    rrv.all_reduce(buckets, "sum", "oneshot")
+    plan.unpack(0, buckets, grads, "avg")
+    for r in range(n):
+        assert_bits_equal(to_host(grads[r]), want[r], f"staged bucket rank {r}")
 
 
 @pytest.mark.parametrize("op", ["sum", "avg", "min", "prod"])
@@ -743,13 +802,13 @@ print("CONTEXT OK")
     assert "CONTEXT OK" in out.stdout, out.stdout
 
 
-@pytest.mark.parametrize("n", [2, 3, 4, 6, 8, 16, 24])
+@pytest.mark.parametrize("n", [2, 3, 4, 5, 6, 7, 8, 16, 24])
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16", "i32"])
 @pytest.mark.parametrize("op", ["sum", "avg", "max", "min", "prod"])
 def test_bulk_copy_reduce_scatter_and_tree_order(n, dtype, op):
-    """Parts (reduce-scatter, any rank count) and buffers (tree order, powers
-    of two up to 16) of whole 16-byte vectors at aligned addresses take the
-    bulk-copy kernels: same bits as the oracle."""
+    """Parts (reduce-scatter, any rank count) and buffers (tree order, 2-8
+    and 16 ranks, an unpaired rank carried up) of whole 16-byte vectors at
+    aligned addresses take the bulk-copy kernels: same bits as the oracle."""
     if dtype == "i32" and op == "avg":
         pytest.skip("AVG is not defined for int32")
     per = 8 * 1500
@@ -792,7 +851,7 @@ def test_aligned_all_gather_and_two_shot(n, dtype):
     rrv.check_timeouts()
 
 
-@pytest.mark.parametrize("n", [2, 4, 8, 16])
+@pytest.mark.parametrize("n", [2, 3, 4, 5, 8, 12, 16])
 @pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
 def test_bucket_sync_bulk_path_with_heads_and_tails(n, dtype):
     """Tensors at odd element offsets, the same on every rank: the fused
