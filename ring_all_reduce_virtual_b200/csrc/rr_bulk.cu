@@ -124,6 +124,9 @@ bool bulk_eligible(const RankParams& p, int esize)
     const uintptr_t ph = (uintptr_t)p.in[0] % 16;
     if ((uintptr_t)p.out[0] % 16 != ph || ph % (uintptr_t)esize != 0) return false;
     if (p.nseg != (uint64_t)p.n || p.lo >= p.count) return false;
+    // one output per chunk (the two-shot's first shot) past 16 ranks: as for the
+    // reduce-scatter, too few threads fold each small tile for one small output
+    if (p.owner_only && p.n > 16) return false;
     const uint64_t hi = p.hi < p.count ? p.hi : p.count;
     const uint64_t seg = hi - p.lo < p.C ? hi - p.lo : p.C;
     return tiles_of(seg, esize, p.n) * (uint64_t)p.n <= kMaxGrid;
