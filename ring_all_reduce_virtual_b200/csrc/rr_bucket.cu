@@ -264,8 +264,8 @@ __global__ void __launch_bounds__(kThreads) bucket_fold_kernel(const __grid_cons
 // at any element, so tile 0 folds the elements before the segment's first
 // 16-byte boundary and after its last whole vector with plain loads, and the
 // bulk copies move the whole vectors between.  Needs every rank's copy of a
-// tensor at the same address modulo 16 (vec_ok) and 2-16 ranks (2, 4, 8 and
-// 16 fixed at compile time, the others a kernel argument).
+// tensor at the same address modulo 16 (vec_ok) and 2 or more ranks (2, 4, 8
+// and 16 fixed at compile time, the others a kernel argument).
 struct BucketBulkParams {
     BucketFoldParams f;  // tile0 counts bulk tiles (bucket_bulk_tile_elems)
     unsigned int* waits; // as BulkParams (rr_bulk.cuh): the wait counters, the test hook, the bound
@@ -460,7 +460,7 @@ cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p
     const uint64_t work = p.tile0[p.nseg];
     const bool avg = op == kAvg;
     // the bulk-copy fold when it applies (no CTA cap: one CTA per tile)
-    if (max_grid >= kMaxGrid && p.vec_ok && p.n >= 2 && p.n <= 16) {
+    if (max_grid >= kMaxGrid && p.vec_ok && p.n >= 2) {
         bool launched = false;
         cudaError_t e = cudaSuccess;
         if (grad_dtype == kBF16)

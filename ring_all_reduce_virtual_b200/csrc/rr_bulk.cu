@@ -146,7 +146,7 @@ bool bulk_scatter_eligible(const RankParams& p, int esize)
 
 bool bulk_tree_eligible(const RankParams& p, int esize)
 {
-    if (!bulk_ranks_aligned(p, 16, false) || p.nseg != 1 || (p.n > 8 && p.n != 16)) return false;
+    if (!bulk_ranks_aligned(p, 16, false) || p.nseg != 1 || (p.n > 8 && p.n != 12 && p.n != 16)) return false;
     if ((p.count * (uint64_t)esize) % 16 != 0) return false;  // the buffer is whole vectors
     return tiles_of(p.count, esize, p.n) <= kMaxGrid;
 }

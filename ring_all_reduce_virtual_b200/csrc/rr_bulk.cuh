@@ -21,7 +21,7 @@
 // bulk copies when it shares that phase, by the threads otherwise), both for
 // 2-64 ranks; the tree mode where the buffers are whole 16-byte vectors at
 // 16-byte aligned addresses (bulk_*_eligible).  The rank count is a
-// compile-time constant for 2, 4, 8, 16, 32 and 64 ranks (tree: 2-8 and 16) and a
+// compile-time constant for 2, 4, 8, 16, 32 and 64 ranks (tree: 2-8, 12 and 16) and a
 // kernel argument (NS = 0) otherwise; with the copy engine doing the loads,
 // a runtime count costs the fold no registers.  Every other call takes the
 // per-thread-load kernels, with the same bits.  The fold itself uses the

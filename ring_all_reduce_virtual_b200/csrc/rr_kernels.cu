@@ -77,8 +77,70 @@ __device__ __forceinline__ void copy_tile(const typename Ty::T* in, typename Ty:
     __syncthreads();  // the stage is free for the CTA's next tile
 }
 
-// The one-to-many copies below give each CTA one tile of one output (16 KB
-// in, 16 KB out): such short-lived CTAs keep enough bytes in flight only at
+// Copy tile `tile` of `in` to nout outputs out(0..nout-1), all at one 16-byte
+// phase: the tile is staged in shared memory once (cp.async, whole aligned
+// vectors) and each vector, shifted to the outputs' phase, is stored to every
+// output.  Every thread of the CTA calls this for the same tile.
+template <class Ty, int VPT, class Out>
+__device__ __forceinline__ void fan_tile(const typename Ty::T* in, Out out, int nout, uint64_t len, uint64_t tile)
+{
+    using T = typename Ty::T;
+    constexpr int L = Ty::L;
+    constexpr uint32_t TV = (uint32_t)kThreads * VPT;
+    const int pout = phase_of(out(0), L);
+    const int pin = phase_of(in, L);
+    uint64_t head = (uint64_t)((L - pout) & (L - 1));
+    if (head > len) head = len;
+    const uint64_t nv = (len - head) / L, tail = len - head - nv * L;
+    if (tile == 0 && (uint64_t)threadIdx.x < head + tail) {
+        const uint64_t e = (uint64_t)threadIdx.x < head ? (uint64_t)threadIdx.x : head + nv * L + (threadIdx.x - head);
+        const T x = in[e];
+        for (int j = 0; j < nout; ++j) out(j)[e] = x;
+    }
+    const uint64_t v0 = tile * TV;
+    if (v0 >= nv) return;
+    const uint32_t nvt = nv - v0 < TV ? (uint32_t)(nv - v0) : TV;
+    const int d = (pin - pout) & (L - 1);
+    // d == 0: the tile's own vectors; otherwise one more, for the last shift
+    const uint32_t nst = d ? nvt + 1 : nvt;
+    const T* ib = reinterpret_cast<const T*>(reinterpret_cast<uintptr_t>(in + head + v0 * L) - (uintptr_t)d * sizeof(T));
+    __shared__ __align__(16) uint4 stage[TV + 1];
+#pragma unroll
+    for (int k = 0; k <= VPT; ++k) {
+        const uint32_t i = (uint32_t)k * kThreads + threadIdx.x;
+        if (i < nst)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(&stage[i])),
+                         "l"(ib + (uint64_t)i * L)
+                         : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+#pragma unroll 1
+    for (int k = 0; k < VPT; ++k) {
+        const uint32_t i = (uint32_t)k * kThreads + threadIdx.x;
+        if (i >= nvt) continue;
+        const uint4 v = d ? shift_window(stage[i], stage[i + 1], d * (int)sizeof(T)) : stage[i];
+        const uint64_t e = head + (v0 + i) * L;
+        for (int j = 0; j < nout; ++j) stv(out(j) + e, v);
+    }
+    __syncthreads();  // the stage is free for the CTA's next tile
+}
+
+// Outputs written per work item by the fan-out forms of the one-to-many
+// copies (all-gather, the two-shot's broadcast).  Measured on 2-48 ranks x
+// 256 MiB fp32 outputs, whole-vector and odd-sized parts: the all-gather at
+// 1 / 2 / 4 / 8 outputs per item ran at 0.87-0.99 / 0.98-1.00 / 0.93-0.98 /
+// 0.89-0.98 of the copy peak (one output per item fell off with the rank
+// count on odd parts: each item stages and shifts its tile for 16 KB of
+// output); the two-shot moved by at most 2 % between 1 and 2.
+#ifndef RR_FAN
+#define RR_FAN 2
+#endif
+constexpr int kFan = RR_FAN;
+
+// The one-to-many copies below give each CTA one tile of one or kFan
+// outputs (16 KB in, 16 or 32 KB out): such short-lived CTAs keep enough bytes in flight only at
 // full occupancy, so they are held to the registers of 8 CTAs per SM
 // (measured on the 64-rank all-gather: 6 CTAs per SM ran at 0.86 of the copy
 // peak, 8 at 1.03).  The all-to-all reads a separate tile per CTA and ran
@@ -87,7 +149,8 @@ constexpr int kSmallCtasPerSm = 8;
 
 // ------------------------------------------------- chunk broadcast
 // Two-shot's second shot: segment c = chunk c, read from its owner (rank c)
-// and written to chunk c of the N-1 other ranks.  One output per work item:
+// and written to chunk c of the N-1 other ranks.  One output per work item
+// (ranks at different 16-byte phases):
 // item w = (c * tps + tile) * (N-1) + k writes rank k (k < c) or k+1, so the
 // N-1 CTAs of a tile run side by side and all but the first read the owner's
 // tile from L2 (HBM reads it once).
@@ -106,6 +169,31 @@ __global__ void __launch_bounds__(kThreads, kSmallCtasPerSm) chunk_bcast_kernel(
         const int owner = (int)c;
         const int dst = (int)k < owner ? (int)k : (int)k + 1;
         copy_tile<Ty, kVptMove>(static_cast<const T*>(p.in[owner]) + lo, static_cast<T*>(p.out[dst]) + lo, len, tile);
+    }
+}
+
+// The same copies with kFan outputs per work item, when every rank's buffer
+// sits at one 16-byte phase: item w = (c * tps + tile) * G + g writes ranks
+// g*kFan ... of the N-1 others (G groups), the owner's tile read once per item.
+template <class Ty>
+__global__ void __launch_bounds__(kThreads, kSmallCtasPerSm) chunk_bcast_fan_kernel(const __grid_constant__ RankParams p)
+{
+    using T = typename Ty::T;
+    const uint64_t m = (uint64_t)p.n - 1, ng = (m + kFan - 1) / kFan;
+    const uint64_t total = p.nseg * p.tps * ng;
+    for (uint64_t w = blockIdx.x; w < total; w += gridDim.x) {
+        const uint64_t st = w / ng, g = w - st * ng;
+        const uint64_t c = st / p.tps, tile = st - c * p.tps;
+        const uint64_t lo = c * p.C;
+        if (lo >= p.count) continue;
+        const uint64_t len = p.count - lo < p.C ? p.count - lo : p.C;
+        const int owner = (int)c, k0 = (int)g * kFan;
+        const int nout = (int)m - k0 < kFan ? (int)m - k0 : kFan;
+        auto out = [&](int j) {
+            const int k = k0 + j;
+            return static_cast<T*>(p.out[k < owner ? k : k + 1]) + lo;
+        };
+        fan_tile<Ty, kVptMove>(static_cast<const T*>(p.in[owner]) + lo, out, nout, len, tile);
     }
 }
 
@@ -134,10 +222,10 @@ __global__ void __launch_bounds__(kThreads) reduce_scatter_kernel(const __grid_c
 
 // ------------------------------------------------------ all-gather
 // Segment q = rank q's part, written to offset q*C of every output.  One
-// output per work item: item w = (q * tps + tile) * N + o, so the N CTAs of
-// a tile run side by side and HBM reads the source tile once (the others hit
-// L2).  Writing all N outputs from one CTA measured 0.94 of the copy peak at
-// 8 ranks x 256 MiB, this map 0.99.
+// output per work item (outputs at different 16-byte phases): item
+// w = (q * tps + tile) * N + o, so the N CTAs of a tile run side by side and
+// HBM reads the source tile once (the others hit L2).  Writing all N outputs
+// from one CTA measured 0.94 of the copy peak at 8 ranks x 256 MiB.
 template <class Ty>
 __global__ void __launch_bounds__(kThreads, kSmallCtasPerSm) all_gather_kernel(const __grid_constant__ RankParams p)
 {
@@ -148,6 +236,24 @@ __global__ void __launch_bounds__(kThreads, kSmallCtasPerSm) all_gather_kernel(c
         const uint64_t st = w / n, o = w - st * n;
         const uint64_t q = st / p.tps, tile = st - q * p.tps;
         copy_tile<Ty, kVptMove>(static_cast<const T*>(p.in[q]), static_cast<T*>(p.out[o]) + q * p.C, p.C, tile);
+    }
+}
+
+// The same copies with kFan outputs per work item, when every output sits at
+// one 16-byte phase: item w = (q * tps + tile) * G + g writes outputs
+// g*kFan ... (G groups), the source tile read once per item.
+template <class Ty>
+__global__ void __launch_bounds__(kThreads, kSmallCtasPerSm) all_gather_fan_kernel(const __grid_constant__ RankParams p)
+{
+    using T = typename Ty::T;
+    const uint64_t n = (uint64_t)p.n, ng = (n + kFan - 1) / kFan;
+    const uint64_t total = p.nseg * p.tps * ng;
+    for (uint64_t w = blockIdx.x; w < total; w += gridDim.x) {
+        const uint64_t st = w / ng, g = w - st * ng;
+        const uint64_t q = st / p.tps, tile = st - q * p.tps;
+        const int o0 = (int)g * kFan, nout = (int)n - o0 < kFan ? (int)n - o0 : kFan;
+        auto out = [&](int j) { return static_cast<T*>(p.out[o0 + j]) + q * p.C; };
+        fan_tile<Ty, kVptMove>(static_cast<const T*>(p.in[q]), out, nout, p.C, tile);
     }
 }
 
@@ -194,11 +300,23 @@ uint64_t tile_elems(int dtype, int vpt)
     return (uint64_t)kThreads * (uint64_t)vpt * (dtype == kBF16 || dtype == kF16 ? 8u : 4u);
 }
 
+namespace {
+bool outs_same_phase(const RankParams& p)
+{
+    for (int r = 1; r < p.n; ++r)
+        if ((uintptr_t)p.out[r] % 16 != (uintptr_t)p.out[0] % 16) return false;
+    return true;
+}
+}  // namespace
+
 cudaError_t launch_rank_kernel(int kind, int dtype, int op, const RankParams& p, cudaStream_t s)
 {
     uint64_t work = kind == kOneshotTree ? p.tps : p.nseg * p.tps;
-    if (kind == kAllGather) work *= (uint64_t)p.n;  // one output per work item
-    if (kind == kChunkBroadcast) work *= (uint64_t)(p.n - 1);
+    // one output per work item, or kFan when the outputs share a 16-byte phase
+    const bool fan = kFan > 1 && outs_same_phase(p);
+    const uint64_t per = fan ? (uint64_t)kFan : 1;
+    if (kind == kAllGather) work *= ((uint64_t)p.n + per - 1) / per;
+    if (kind == kChunkBroadcast) work *= ((uint64_t)p.n - 1 + per - 1) / per;
     if (kind == kAllGather || kind == kAllToAll || kind == kChunkBroadcast) op = kSum;
     const int n = p.n;
     constexpr int V = kVptReduce;
@@ -214,9 +332,11 @@ cudaError_t launch_rank_kernel(int kind, int dtype, int op, const RankParams& p,
             }
             return launch_all(reduce_scatter_kernel<Ty, OP, V, kGroup, 0>, p, work, s);
         case kOneshotTree: return launch_oneshot_tree<Ty, OP>(p, work, s);
-        case kAllGather: return launch_all(all_gather_kernel<Ty>, p, work, s);
+        case kAllGather:
+            return launch_all(fan ? all_gather_fan_kernel<Ty> : all_gather_kernel<Ty>, p, work, s);
         case kAllToAll: return launch_all(all_to_all_kernel<Ty>, p, work, s);
-        case kChunkBroadcast: return launch_all(chunk_bcast_kernel<Ty>, p, work, s);
+        case kChunkBroadcast:
+            return launch_all(fan ? chunk_bcast_fan_kernel<Ty> : chunk_bcast_kernel<Ty>, p, work, s);
         }
         return cudaErrorInvalidValue;
     });

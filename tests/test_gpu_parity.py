@@ -802,12 +802,12 @@ print("CONTEXT OK")
     assert "CONTEXT OK" in out.stdout, out.stdout
 
 
-@pytest.mark.parametrize("n", [2, 3, 4, 5, 6, 7, 8, 16, 24])
+@pytest.mark.parametrize("n", [2, 3, 4, 5, 6, 7, 8, 12, 16, 24])
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16", "i32"])
 @pytest.mark.parametrize("op", ["sum", "avg", "max", "min", "prod"])
 def test_bulk_copy_reduce_scatter_and_tree_order(n, dtype, op):
-    """Parts (reduce-scatter, any rank count) and buffers (tree order, 2-8
-    and 16 ranks, an unpaired rank carried up) of whole 16-byte vectors at
+    """Parts (reduce-scatter, any rank count) and buffers (tree order, 2-8,
+    12 and 16 ranks, an unpaired block carried up) of whole 16-byte vectors at
     aligned addresses take the bulk-copy kernels: same bits as the oracle."""
     if dtype == "i32" and op == "avg":
         pytest.skip("AVG is not defined for int32")
@@ -851,7 +851,29 @@ def test_aligned_all_gather_and_two_shot(n, dtype):
     rrv.check_timeouts()
 
 
-@pytest.mark.parametrize("n", [2, 3, 4, 5, 8, 12, 16])
+@pytest.mark.parametrize("n", [2, 5, 9, 13])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "i32"])
+@pytest.mark.parametrize("layout", ["same", "mixed"])
+def test_one_to_many_copies_by_output_phase(n, dtype, layout):
+    """The all-gather and the two-shot's broadcast write several outputs per
+    work item when every output sits at one 16-byte phase ("same": all one
+    element past a boundary, so each block has a scalar head) and one output
+    per item otherwise ("mixed"); rank counts that leave a partial last group
+    of outputs, sources at other phases, parts over several tiles."""
+    L = 4 if dtype in ("f32", "i32") else 8
+    per = 2 * TILE_MOVE[dtype] + 3
+    src_off = [(3 * r + 2) % L for r in range(n)]
+    out_off = [1] * n if layout == "same" else [r % L for r in range(n)]
+    x = synth.ranks(140 + n, n, per, "int" if dtype == "i32" else "full", dtype)
+    zero = [np.zeros(n * per, dtype=a.dtype) for a in x]
+    ag = to_dev(zero, offsets=out_off)
+    rrv.all_gather(to_dev(x, offsets=src_off), ag)
+    assert_bits_equal(to_host(ag), oracle.all_gather(x), f"ag {layout} n={n}")
+    count = n * per - 5
+    _run(n, count, dtype, "sum", "two_shot", seed=150 + n, offsets=out_off)
+
+
+@pytest.mark.parametrize("n", [2, 3, 4, 5, 8, 12, 16, 24, 33, 64])
 @pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
 def test_bucket_sync_bulk_path_with_heads_and_tails(n, dtype):
     """Tensors at odd element offsets, the same on every rank: the fused
