@@ -266,13 +266,14 @@ class BucketPlan:
         check(lib().rr_bucket_plan(arr, len(numels), _dtype_code(grad_dtype), int(cap_bytes),
                                    ctypes.byref(handle)), "bucket_plan")
         self._h = handle
+        self._free = lib().rr_bucket_plan_free  # held: module globals may be gone when __del__ runs at exit
         self.numels = [int(m) for m in numels]
         self.grad_dtype = _dtype_code(grad_dtype)
 
     def __del__(self):
         h = getattr(self, "_h", None)
         if h is not None and h.value:
-            lib().rr_bucket_plan_free(h)
+            self._free(h)
             self._h = None
 
     @property
@@ -380,12 +381,13 @@ class Reducer:
         check(lib().rr_reducer_create(plan._h, g.ptrs, g.nranks, _op(op), _stream(self.comm, g.device),
                                       int(max_ctas), ctypes.byref(handle)), "reducer_create")
         self._h = handle
+        self._free = lib().rr_reducer_free  # held: module globals may be gone when __del__ runs at exit
         self._device = g.device
 
     def __del__(self):
         h = getattr(self, "_h", None)
         if h is not None and h.value:
-            lib().rr_reducer_free(h)
+            self._free(h)
             self._h = None
 
     def ready(self, tensor: int, stream=None) -> None:

@@ -72,8 +72,6 @@ cudaError_t launch_ring(const RankParams& p, cudaStream_t s)
     return launch_bulk_fold<Ty, OP, 0, kBulkRing, WIRE>(p, seg, s);
 }
 
-bool pow2_rank_count(int n) { return n == 2 || n == 4 || n == 8 || n == 16 || n == 32 || n == 64; }
-
 uint64_t tiles_of(uint64_t elems, int esize, int n)
 {
     const uint64_t te = (uint64_t)bulk_tile_vectors(n) * (16u / (uint64_t)esize);
@@ -109,14 +107,6 @@ BulkParams bulk_params(const RankParams& p)
     return bp;
 }
 
-bool bulk_ranks_aligned(const RankParams& p, int nmax, bool pow2)
-{
-    if (!p.waits || p.n < 2 || p.n > nmax || (pow2 && !pow2_rank_count(p.n))) return false;
-    for (int r = 0; r < p.n; ++r)
-        if ((uintptr_t)p.in[r] % 16 != 0 || (uintptr_t)p.out[r] % 16 != 0) return false;
-    return true;
-}
-
 bool bulk_eligible(const RankParams& p, int esize)
 {
     if (!p.waits || p.n < 2 || p.n > kMaxRanks || !p.vec_ok) return false;
@@ -146,8 +136,10 @@ bool bulk_scatter_eligible(const RankParams& p, int esize)
 
 bool bulk_tree_eligible(const RankParams& p, int esize)
 {
-    if (!bulk_ranks_aligned(p, 16, false) || p.nseg != 1 || (p.n > 8 && p.n != 12 && p.n != 16)) return false;
-    if ((p.count * (uint64_t)esize) % 16 != 0) return false;  // the buffer is whole vectors
+    if (!p.waits || p.n < 2 || p.nseg != 1 || (p.n > 8 && p.n != 12 && p.n != 16) || !p.vec_ok) return false;
+    // every buffer at one 16-byte phase, on element boundaries
+    const uintptr_t ph = (uintptr_t)p.in[0] % 16;
+    if ((uintptr_t)p.out[0] % 16 != ph || ph % (uintptr_t)esize != 0) return false;
     return tiles_of(p.count, esize, p.n) <= kMaxGrid;
 }
 

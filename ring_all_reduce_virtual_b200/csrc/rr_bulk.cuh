@@ -15,14 +15,14 @@
 //                 tree's pairwise order (an unpaired rank carried up), written
 //                 to every rank
 //
-// The ring mode runs wherever every input and output address has the same
-// 16-byte phase (a scalar head and tail per segment, whole vectors between),
-// the scatter mode wherever every input has one phase (each output stored by
-// bulk copies when it shares that phase, by the threads otherwise), both for
-// 2-64 ranks; the tree mode where the buffers are whole 16-byte vectors at
-// 16-byte aligned addresses (bulk_*_eligible).  The rank count is a
-// compile-time constant for 2, 4, 8, 16, 32 and 64 ranks (tree: 2-8, 12 and 16) and a
-// kernel argument (NS = 0) otherwise; with the copy engine doing the loads,
+// The ring and tree modes run wherever every input and output address has
+// the same 16-byte phase (a scalar head and tail per segment, whole vectors
+// between), the scatter mode wherever every input has one phase (each output
+// stored by bulk copies when it shares that phase, by the threads
+// otherwise); ring and scatter for 2-64 ranks, tree for 2-8, 12 and 16
+// (bulk_*_eligible).  The rank count is a compile-time constant for 2, 4, 8,
+// 16, 32 and 64 ranks (tree: 2-8, 12 and 16) and a kernel argument (NS = 0)
+// otherwise; with the copy engine doing the loads,
 // a runtime count costs the fold no registers.  Every other call takes the
 // per-thread-load kernels, with the same bits.  The fold itself uses the
 // same apply / finish / wire steps as those kernels.
@@ -59,11 +59,16 @@ struct BulkParams {
 };
 
 // Bytes of input tiles per CTA (N tiles of bulk_smem<N>() / N): 16 KB, 32 KB
-// from 32 ranks on so that each rank's tile stays at least 512 bytes.
+// from kBulkWideRanks ranks on so that each rank's tile stays at least 512 bytes.
+#ifndef RR_BULK_WIDE_RANKS
+#define RR_BULK_WIDE_RANKS 9
+#endif
+constexpr int kBulkWideRanks = RR_BULK_WIDE_RANKS;
+
 template <int NS>
 __host__ __device__ constexpr uint32_t bulk_smem()
 {
-    return NS >= 32 ? 32768u : 16384u;
+    return NS >= kBulkWideRanks ? 32768u : 16384u;
 }
 
 // The parameter block of a launch: p, the counters' address (p.waits) and
@@ -171,16 +176,13 @@ __global__ void __launch_bounds__(kThreads) bulk_fold_kernel(const __grid_consta
         if constexpr (MODE == kBulkScatter) return static_cast<T*>(p.out[s]);
         else return static_cast<T*>(p.out[one_out ? start : o]) + lo;
     };
-    // Ring and scatter modes: every rank's copy of the segment starts at the
-    // same 16-byte phase, so the elements before the first 16-byte boundary
-    // (the head) and after the last whole vector (the tail) are folded with
-    // plain loads by tile 0, and the bulk copies move the whole vectors
-    // between.  The tree mode takes a 16-byte aligned buffer of whole vectors.
-    uint64_t head = 0;
-    if constexpr (MODE != kBulkTree) {
-        head = (uint64_t)((L - phase_of(in(0), L)) & (L - 1));
-        if (head > len) head = len;
-    }
+    // Every rank's copy of the segment starts at the same 16-byte phase, so
+    // the elements before the first 16-byte boundary (the head) and after the
+    // last whole vector (the tail) are folded with plain loads by tile 0 (in
+    // the tree's order in tree mode), and the bulk copies move the whole
+    // vectors between.
+    uint64_t head = (uint64_t)((L - phase_of(in(0), L)) & (L - 1));
+    if (head > len) head = len;
     // a scatter output at another phase than the inputs is stored by the
     // threads, element by element, instead of by bulk stores
     bool bulk_out = true;
@@ -189,7 +191,8 @@ __global__ void __launch_bounds__(kThreads) bulk_fold_kernel(const __grid_consta
     const uint64_t tail = len - head - nv * L;
     if (tile == 0 && (uint64_t)threadIdx.x < head + tail) {
         const uint64_t e = (uint64_t)threadIdx.x < head ? (uint64_t)threadIdx.x : head + nv * L + (threadIdx.x - head);
-        fold_one<Ty, OP, WIRE>(in, n, out, nout, e, p.divisor);
+        if constexpr (MODE == kBulkTree) tree_fold_lanes<Ty, OP, 1, NS>(p, e, false);  // lo = 0
+        else fold_one<Ty, OP, WIRE>(in, n, out, nout, e, p.divisor);
     }
     const uint64_t v0 = tile * TV;
     if (v0 >= nv) return;
@@ -282,8 +285,8 @@ __global__ void __launch_bounds__(kThreads) bulk_fold_kernel(const __grid_consta
 }
 
 // Vectors per rank per tile when the rank count is not fixed at compile
-// time: the rank's share of 16 KB (32 KB from 32 ranks on), whole vectors.
-inline uint32_t bulk_tile_vectors(int n) { return (uint32_t)((n >= 32 ? 32768u : 16384u) / (uint32_t)n / 16u); }
+// time: the rank's share of 16 KB (32 KB from kBulkWideRanks ranks on), whole vectors.
+inline uint32_t bulk_tile_vectors(int n) { return (uint32_t)((n >= kBulkWideRanks ? 32768u : 16384u) / (uint32_t)n / 16u); }
 
 // One CTA per (segment, tile): nseg segments of at most seg_elems elements
 // each.  NS = 0 runs the rank count p.n.

@@ -10,85 +10,8 @@ namespace rr {
 namespace {
 
 // ------------------------------------------------ one-shot, tree order
-// The tree's pairwise order ([P3] section 6: ranks pair up, pairs pair up,
-// log2 N levels) folded per element in registers.  Ranks are pushed in order
-// 0..N-1 onto a stack of partial blocks: pushing rank j combines it with the
-// blocks it completes (one per trailing one bit of j, earlier block on the
-// left), so slot[b] always holds a block of 2^b ranks.  At the end the blocks
-// for the set bits of N are combined from the smallest upwards, each larger
-// (earlier) block on the left: exactly the level schedule in which a rank
-// without a partner carries its value up.
-template <class Ty, int OP, int W, int NMAX>
-__device__ __forceinline__ void tree_fold_lanes(const RankParams& p, uint64_t e0, bool vec)
-{
-    using T = typename Ty::T;
-    using Acc = typename Ty::Acc;
-    constexpr int LV = NMAX <= 2 ? 2 : (NMAX <= 4 ? 3 : (NMAX <= 8 ? 4 : 7));  // log2(NMAX) + 1
-    Acc slot[LV][W];
-    Acc cur[W];
-    const int n = p.n;
-#pragma unroll
-    for (int g = 0; g < NMAX; g += kGroup) {
-        if (g < n) {
-            Acc v[kGroup][W];
-#pragma unroll
-            for (int k = 0; k < kGroup; ++k) {
-                if (g + k < n && g + k < NMAX) {
-                    const T* src = static_cast<const T*>(p.in[g + k]) + e0;
-                    if constexpr (W == Ty::L) {
-                        if (vec) {
-                            Ty::unpack(ldv(src), v[k]);
-                            continue;
-                        }
-                    }
-                    v[k][0] = Ty::ld1(src);
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < kGroup; ++k) {
-                const int j = g + k;
-                if (j < n && j < NMAX) {
-#pragma unroll
-                    for (int l = 0; l < W; ++l) cur[l] = v[k][l];
-                    int lvl = 0;
-#pragma unroll
-                    for (int b = 0; b < LV - 1; ++b) {
-                        if (((j >> b) & 1) && lvl == b) {
-#pragma unroll
-                            for (int l = 0; l < W; ++l) cur[l] = apply<OP>(slot[b][l], cur[l]);
-                            lvl = b + 1;
-                        }
-                    }
-#pragma unroll
-                    for (int b = 0; b < LV; ++b)
-                        if (b == lvl)
-#pragma unroll
-                            for (int l = 0; l < W; ++l) slot[b][l] = cur[l];
-                }
-            }
-        }
-    }
-    bool have = false;
-#pragma unroll
-    for (int b = 0; b < LV; ++b) {
-        if ((n >> b) & 1) {
-#pragma unroll
-            for (int l = 0; l < W; ++l) cur[l] = have ? apply<OP>(slot[b][l], cur[l]) : slot[b][l];
-            have = true;
-        }
-    }
-#pragma unroll
-    for (int l = 0; l < W; ++l) cur[l] = finish<OP>(cur[l], p.divisor);
-    if constexpr (W == Ty::L) {
-        if (vec) {
-            const uint4 r = Ty::pack(cur);
-#pragma unroll 4
-            for (int o = 0; o < n; ++o) stv(static_cast<T*>(p.out[o]) + e0, r);
-            return;
-        }
-    }
-    for (int o = 0; o < n; ++o) Ty::st1(static_cast<T*>(p.out[o]) + e0, cur[0]);
-}
+// tree_fold_lanes (rr_oneshot.cuh) folds one element or one vector per
+// thread; tree_vectors below keeps several vectors in flight.
 
 // For N <= NMAX <= 8: every rank's vectors for VPT vectors are loaded first
 // (N * VPT loads in flight per thread), then each vector is folded in tree

@@ -851,6 +851,23 @@ def test_aligned_all_gather_and_two_shot(n, dtype):
     rrv.check_timeouts()
 
 
+@pytest.mark.parametrize("n", [3, 5, 8, 12, 16])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("off", [0, 1, 3])
+def test_tree_order_bulk_heads_and_tails(n, dtype, off):
+    """The tree-order one-shot on the bulk-copy fold with every buffer at one
+    16-byte phase: a scalar head (buffers `off` elements past a boundary) and
+    a ragged tail, folded in the tree's order by tile 0, whole vectors
+    between, over several tiles."""
+    L = 4 if dtype == "f32" else 8
+    if off >= L:
+        pytest.skip("offset within one vector")
+    count = 3 * TILE[dtype] + 5
+    for op in ("sum", "avg"):
+        _run(n, count, dtype, op, "tree_oneshot", seed=170 + n + off, offsets=[off] * n)
+    rrv.check_timeouts()
+
+
 @pytest.mark.parametrize("n", [2, 5, 9, 13])
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "i32"])
 @pytest.mark.parametrize("layout", ["same", "mixed"])
