@@ -411,10 +411,11 @@ rr_status_t rr_set_picker_params(double launch_s, double hbm_bytes_per_s);
 
 rr_status_t rr_get_stats(rr_stats_t* out); /* last call on this host thread */
 
-/* Bounded waits.  The one-shot all-reduce (rank count 2, 4, 8, 16, 32 or 64),
- * the reduce-scatter, the tree-order one-shot and the fused bucket sync (2-16
- * ranks) stage their tiles in shared memory with bulk async copies when the
- * buffers are 16-byte aligned; their threads wait on an mbarrier for those
+/* Bounded waits.  The one-shot all-reduce (2-64 ranks), the reduce-scatter
+ * (2-16 ranks), the tree-order one-shot (2-8, 12 and 16 ranks) and the fused
+ * bucket sync (2-64 ranks) stage their tiles in shared memory with bulk async
+ * copies when every rank's buffer sits at one 16-byte phase (on element
+ * boundaries); their threads wait on an mbarrier for those
  * copies with an iteration limit instead of forever.  A wait that runs out --
  * no working device lets it -- makes the whole CTA skip its tile (nothing of
  * that tile's result is written) and is counted on the device; one thread
