@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(kThreads) bucket_bulk_kernel(const __grid_cons
 }
 
 // Elements per bulk tile of the bucket sync: the whole vectors of one rank's
-// share of bulk_smem<N>().
+// share of the tile bytes (the compiled counts 2, 4, 8 and 16 tile alike).
 uint64_t bucket_bulk_tile_elems(int grad_dtype, int n)
 {
     return (uint64_t)bulk_tile_vectors(n) * (grad_dtype == kF32 ? 4u : 8u);

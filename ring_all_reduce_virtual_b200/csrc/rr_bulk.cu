@@ -74,7 +74,7 @@ cudaError_t launch_ring(const RankParams& p, cudaStream_t s)
 
 uint64_t tiles_of(uint64_t elems, int esize, int n)
 {
-    const uint64_t te = (uint64_t)bulk_tile_vectors(n) * (16u / (uint64_t)esize);
+    const uint64_t te = (uint64_t)bulk_launch_tile_vectors(n) * (16u / (uint64_t)esize);
     return elems ? (elems + te - 1) / te : 1;
 }
 

@@ -58,13 +58,24 @@ struct BulkParams {
     uint32_t tv;          // vectors per rank per tile (kernels whose rank count is not fixed)
 };
 
-// Bytes of input tiles per CTA (N tiles of bulk_smem<N>() / N): 16 KB, 32 KB
-// from kBulkWideRanks ranks on so that each rank's tile stays at least 512 bytes.
+// Bytes of input tiles per CTA (N tiles of a share each): 16 KB, 32 KB from
+// kBulkWideRanks ranks on (so that a CTA keeps enough bytes in flight while
+// it folds), and for a rank count given at run time kBulkManyBytes from 32
+// ranks on.  Measured on 64 Mi fp32 per rank: 32 KB from 9 ranks instead of
+// from 32 took 17-31 ranks from 0.83-0.97 to 1.00 of the copy peak; 40 KB
+// took the run-time-count folds at 40-64 ranks up by 1-3 % and the
+// compiled 32- and 64-rank ones down by 2 %.
 #ifndef RR_BULK_WIDE_RANKS
 #define RR_BULK_WIDE_RANKS 9
 #endif
+#ifndef RR_BULK_MANY_BYTES
+#define RR_BULK_MANY_BYTES 40960
+#endif
 constexpr int kBulkWideRanks = RR_BULK_WIDE_RANKS;
+constexpr uint32_t kBulkManyBytes = RR_BULK_MANY_BYTES;
+static_assert(kBulkManyBytes + 64 <= 48 * 1024, "within the default dynamic shared memory of a CTA");
 
+// Compiled rank counts.
 template <int NS>
 __host__ __device__ constexpr uint32_t bulk_smem()
 {
@@ -285,8 +296,21 @@ __global__ void __launch_bounds__(kThreads) bulk_fold_kernel(const __grid_consta
 }
 
 // Vectors per rank per tile when the rank count is not fixed at compile
-// time: the rank's share of 16 KB (32 KB from kBulkWideRanks ranks on), whole vectors.
-inline uint32_t bulk_tile_vectors(int n) { return (uint32_t)((n >= kBulkWideRanks ? 32768u : 16384u) / (uint32_t)n / 16u); }
+// time: the rank's share of the tile bytes, whole vectors.
+inline uint32_t bulk_tile_vectors(int n)
+{
+    const uint32_t bytes = n >= 32 ? kBulkManyBytes : n >= kBulkWideRanks ? 32768u : 16384u;
+    return bytes / (uint32_t)n / 16u;
+}
+
+// The same for a launch that may take a compiled rank count (the ring mode
+// compiles 32 and 64 ranks; below 32 the two tilings agree).
+inline uint32_t bulk_launch_tile_vectors(int n)
+{
+    if (n == 32) return bulk_smem<32>() / 32u / 16u;
+    if (n == 64) return bulk_smem<64>() / 64u / 16u;
+    return bulk_tile_vectors(n);
+}
 
 // One CTA per (segment, tile): nseg segments of at most seg_elems elements
 // each.  NS = 0 runs the rank count p.n.
