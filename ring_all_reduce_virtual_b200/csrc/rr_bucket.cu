@@ -106,27 +106,38 @@ __device__ __forceinline__ void convert_quads(const typename In::T* s0, typename
     }
 }
 
-// The same when the source quads are d = 1..3 elements out of step: the
-// tile's source quads (and the one after, which holds the last few elements)
-// are loaded aligned -- one load per quad, all in flight -- into shared
-// memory, and each destination quad reads the two stage quads it straddles
-// and shifts them in registers, so no global load is issued twice.  Every thread of the CTA takes
-// part (the tile is the CTA's).
+// The same when the source quads are d = 1..3 elements out of step (fp32
+// sources): the tile's source quads (and the one after, which holds the last
+// few elements) are copied aligned by cp.async -- one copy per quad, all in
+// flight, none through registers -- into shared memory, and each destination
+// quad reads the two stage quads it straddles and shifts them in registers,
+// so no global load is issued twice.  Every thread of the CTA takes part (the
+// tile is the CTA's).  Measured on the unpack of 2-8 ranks x 64 Mi bf16
+// parameters 1 and 2 elements out of phase: 0.93-1.06 of the copy peak,
+// against 0.82-0.97 with the stage filled through registers.
 template <class In, class Out, int OP, int Q>
 __device__ __forceinline__ void convert_quads_staged(const typename In::T* s0, typename Out::T* dst, uint64_t head,
                                                      uint64_t nq, uint64_t tile, int d, float divisor)
 {
     using R = typename Quad<In>::R;
+    static_assert(sizeof(R) == 16, "16-byte source quads (fp32): the 16-bit sources take convert_quads_shfl");
     constexpr uint32_t TQ = (uint32_t)kThreads * Q;
     __shared__ R stage[TQ + 1];
     const uint64_t q0 = tile * TQ;
     if (q0 >= nq) return;
     const uint32_t nqt = nq - q0 < TQ ? (uint32_t)(nq - q0) : TQ;  // destination quads of this tile
+    // global -> shared without passing through registers, all of the
+    // thread's copies in flight
 #pragma unroll
     for (int k = 0; k <= Q; ++k) {
         const uint32_t i = (uint32_t)k * kThreads + threadIdx.x;
-        if (i <= nqt) stage[i] = Quad<In>::ld(s0 + (q0 + i) * 4);
+        if (i <= nqt)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(&stage[i])),
+                         "l"(s0 + (q0 + i) * 4)
+                         : "memory");
     }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();
 #pragma unroll
     for (int k = 0; k < Q; ++k) {
@@ -139,6 +150,54 @@ __device__ __forceinline__ void convert_quads_staged(const typename In::T* s0, t
         Quad<Out>::st(dst + head + (q0 + i) * 4, Quad<Out>::from_f(a));
     }
     __syncthreads();  // the stage is free for the CTA's next tile
+}
+
+// The same with the shift done across lanes instead of through shared
+// memory: each warp takes a run of 32 * Q destination quads (32 consecutive
+// quads per access, all Q loads in flight), and a lane takes the source quad
+// after its own from lane + 1 by warp shuffle -- lane 31 from lane 0 of the
+// next access, or for the warp's last access from one more load.
+template <class In, class Out, int OP, int Q>
+__device__ __forceinline__ void convert_quads_shfl(const typename In::T* s0, typename Out::T* dst, uint64_t head,
+                                                   uint64_t nq, uint64_t tile, int d, float divisor)
+{
+    using R = typename Quad<In>::R;
+    constexpr uint32_t TQ = (uint32_t)kThreads * Q;
+    constexpr int W = sizeof(R) / 4;  // 32-bit words per quad
+    const uint64_t q0 = tile * TQ;
+    if (q0 >= nq) return;
+    const uint32_t nqt = nq - q0 < TQ ? (uint32_t)(nq - q0) : TQ;  // destination quads of this tile
+    const uint32_t lane = threadIdx.x & 31u, b = (threadIdx.x >> 5) * 32u * Q;  // the warp's first quad
+    R cur[Q], after{};
+#pragma unroll
+    for (int k = 0; k < Q; ++k) {
+        const uint32_t i = b + (uint32_t)k * 32u + lane;
+        cur[k] = R{};
+        if (i <= nqt) cur[k] = Quad<In>::ld(s0 + (q0 + i) * 4);
+    }
+    const uint32_t ia = b + 32u * Q;  // the quad after the warp's run
+    if (lane == 31u && ia <= nqt) after = Quad<In>::ld(s0 + (q0 + ia) * 4);
+#pragma unroll
+    for (int k = 0; k < Q; ++k) {
+        R nb;
+        const R& nx = k + 1 < Q ? cur[k + 1 < Q ? k + 1 : k] : after;
+        uint32_t* o = reinterpret_cast<uint32_t*>(&nb);
+        const uint32_t* c = reinterpret_cast<const uint32_t*>(&cur[k]);
+        const uint32_t* x = reinterpret_cast<const uint32_t*>(&nx);
+#pragma unroll
+        for (int w = 0; w < W; ++w) {
+            const uint32_t up = __shfl_sync(0xffffffffu, c[w], (lane + 1u) & 31u);
+            const uint32_t first = __shfl_sync(0xffffffffu, x[w], 0);
+            o[w] = lane == 31u ? (k + 1 < Q ? first : x[w]) : up;
+        }
+        const uint32_t i = b + (uint32_t)k * 32u + lane;
+        if (i >= nqt) continue;
+        float a[4];
+        Quad<In>::to_f(Quad<In>::shift(cur[k], nb, d), a);
+#pragma unroll
+        for (int l = 0; l < 4; ++l) a[l] = finish<OP>(a[l], divisor);
+        Quad<Out>::st(dst + head + (q0 + i) * 4, Quad<Out>::from_f(a));
+    }
 }
 
 // Convert one tile of a segment from In's element type to Out's, dividing by
@@ -171,7 +230,14 @@ __device__ __forceinline__ void convert_tile(const typename In::T* src, typename
     // the aligned source quad under dst's first quad (d elements before src + head)
     const auto* s0 = reinterpret_cast<const typename In::T*>(reinterpret_cast<uintptr_t>(src + head) -
                                                               (uintptr_t)d * sizeof(typename In::T));
+    // shifted quads of a 16-bit source (the pack) by warp shuffle, of an fp32
+    // source (the unpack) through shared memory: measured on 8 x 64 Mi bf16
+    // parameters 1 and 2 elements out of phase, the shuffles ran the pack at
+    // 1.005 of the copy peak against 1.002 with a register-filled stage, but
+    // the unpack at 0.90 against 0.97 (holding eight 16-byte quads a thread
+    // took 74 registers), and 1.06 with the cp.async stage
     if (d == 0) convert_quads<In, Out, OP, Q>(s0, dst, head, nq, tile, divisor);
+    else if constexpr (sizeof(typename Quad<In>::R) == 8) convert_quads_shfl<In, Out, OP, Q>(s0, dst, head, nq, tile, d, divisor);
     else convert_quads_staged<In, Out, OP, Q>(s0, dst, head, nq, tile, d, divisor);
 }
 

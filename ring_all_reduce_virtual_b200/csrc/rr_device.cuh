@@ -170,11 +170,30 @@ __device__ __forceinline__ bool is_pow2(float d)
     return (u & 0x007fffffu) == 0u && d >= 1.0f;  // positive, normal, zero mantissa
 }
 
+// Any other whole rank count N (below 2^24) takes no division either: the
+// fp64 product of a and the correctly rounded fp64 reciprocal of N, rounded
+// once to fp32, is a / N correctly rounded.  The product's relative error is
+// below 2^-52; the exact quotient's relative distance to the nearest fp32
+// rounding boundary is at least 2^-25 / N, because a boundary m (a midpoint
+// between neighbouring fp32 values) is an odd multiple of its binade's step
+// 2^(E-24), a (whose binade is not below E) and N * m are multiples of that
+// step, and a == N * m is impossible: for N not a power of two, N * m has
+// more than 24 significant bits.  So both roundings land on the same side of
+// every boundary, for subnormal quotients, zeros and infinities too.  (The
+// division sequence this replaces cost up to 20 % of the time of a bucket
+// unpack at 3, 5 or 6 ranks, where it runs once per element per rank.)
+__device__ __forceinline__ bool is_whole_count(float d)
+{
+    return d >= 1.0f && d < 16777216.0f && d == truncf(d);
+}
+
 template <int OP>
 __device__ __forceinline__ float finish(float a, float divisor)
 {
     if constexpr (OP == kAvg) {
         if (is_pow2(divisor)) return __fmul_rn(a, __frcp_rn(divisor));
+        if (is_whole_count(divisor))
+            return __double2float_rn(__dmul_rn((double)a, __drcp_rn((double)divisor)));
         return __fdiv_rn(a, divisor);
     } else {
         return a;

@@ -341,3 +341,32 @@ def test_grad_set_checks_its_tensors():
         rrv.GradSet([[]])
     with pytest.raises(ValueError):
         rrv.GradSet([[torch.zeros(4)], [torch.zeros(4)]])  # not CUDA tensors
+
+
+# ------------------------------------------- AVG's division, in numbers --
+
+def test_avg_quotient_through_fp64_equals_ieee_division():
+    """The kernels compute a / N for a rank count N that is not a power of
+    two as the fp64 product of a and the fp64 reciprocal of N, rounded once
+    to fp32.  That is IEEE a / N in fp32 for every a (the argument: the
+    product's error is far below the quotient's distance to a rounding
+    boundary).  Checked here with numpy's IEEE arithmetic on random bit
+    patterns of every binade, on the values nearest to N times a rounding
+    midpoint (the hardest cases), and on zeros, subnormals and infinities."""
+    rng = np.random.default_rng(20261203)
+    bits = rng.integers(0, 0x7F800000, size=1 << 16, dtype=np.uint32)
+    bits = np.concatenate([bits, bits | np.uint32(0x80000000)])  # both signs, every finite binade
+    x = bits.view(np.float32)
+    special = np.array([0.0, -0.0, np.inf, -np.inf, 1e-45, -1e-45, 1.1754942e-38, 3.4028235e38, 1.0, 3.0],
+                       dtype=np.float32)
+    for n in [k for k in range(3, 65) if k & (k - 1)]:
+        # fp32 values next to n * m, m a midpoint between neighbouring fp32 values
+        m_lo = rng.integers(1 << 23, 1 << 24, size=1 << 13).astype(np.float64)
+        e = rng.integers(-140, 100, size=m_lo.size)
+        m = (m_lo + 0.5) * np.exp2(e - 23.0)
+        near = (m * n).astype(np.float32)
+        near = np.concatenate([near, np.nextafter(near, np.float32(np.inf)), np.nextafter(near, np.float32(0))])
+        a = np.concatenate([x, special, near[np.isfinite(near)]])
+        want = a / np.float32(n)
+        got = (a.astype(np.float64) * (1.0 / n)).astype(np.float32)
+        assert np.array_equal(got.view(np.uint32), want.view(np.uint32)), n

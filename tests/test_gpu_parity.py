@@ -851,6 +851,43 @@ def test_aligned_all_gather_and_two_shot(n, dtype):
     rrv.check_timeouts()
 
 
+def _near_midpoints(rng, n, size):
+    """fp32 values next to n * m, m a midpoint between neighbouring fp32
+    values: the quotients closest to a rounding boundary."""
+    m = (rng.integers(1 << 23, 1 << 24, size=size) + 0.5) * np.exp2(rng.integers(-140, 100, size=size) - 23.0)
+    near = (m * n).astype(np.float32)
+    near = np.concatenate([near, np.nextafter(near, np.float32(np.inf)), np.nextafter(near, np.float32(0))])
+    return near[np.isfinite(near)]
+
+
+@pytest.mark.parametrize("n", [3, 5, 6, 7, 12, 24, 48, 63])
+@pytest.mark.parametrize("algo", ["oneshot", "two_shot", "ring"])
+def test_avg_quotient_hard_cases(n, algo):
+    """AVG's quotient for rank counts that are not powers of two, on the
+    values whose quotient lies closest to an fp32 rounding boundary, on
+    subnormals, zeros, infinities and random bits of every binade: rank 0
+    holds the values, every other rank zeros, so each element's fold is the
+    value itself and the result is its quotient by N -- IEEE's, bit for bit,
+    and the oracle's."""
+    rng = np.random.default_rng(300 + n)
+    bits = rng.integers(0, 0x7F800000, size=4096, dtype=np.uint32) | (rng.integers(0, 2, 4096, dtype=np.uint32) << 31)
+    special = np.array([0.0, np.inf, -np.inf, 1e-45, -1e-45, 1.1754942e-38, 3.4028235e38, 1.0, 3.0], dtype=np.float32)
+    x0 = np.concatenate([bits.view(np.float32), special, _near_midpoints(rng, n, 2048)]).astype(np.float32)
+    x = [x0] + [np.zeros_like(x0) for _ in range(n - 1)]
+    want = [a.copy() for a in x]
+    oracle.fold_ring_order(want, "avg")
+    quot = x0 / np.float32(n)
+    for w in want:
+        assert np.array_equal(bits_of(w), bits_of(quot))  # the oracle: IEEE's quotient
+    d = to_dev(x)
+    rrv.all_reduce(d, "avg", algo)
+    assert_bits_equal(to_host(d), want, f"avg {algo} n={n}")
+
+
+def bits_of(a):
+    return np.ascontiguousarray(a).view(np.uint32)
+
+
 @pytest.mark.parametrize("n", [3, 5, 8, 12, 16])
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("off", [0, 1, 3])
