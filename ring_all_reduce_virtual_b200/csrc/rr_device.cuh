@@ -170,6 +170,26 @@ __device__ __forceinline__ bool is_pow2(float d)
     return (u & 0x007fffffu) == 0u && d >= 1.0f;  // positive, normal, zero mantissa
 }
 
+// The exact reciprocal of a power of two 2^k (|k| < 126): the exponent
+// negated, no reciprocal instruction.
+__device__ __forceinline__ float pow2_reciprocal(float d)
+{
+    return __uint_as_float(0x7f000000u - (__float_as_uint(d) & 0x7f800000u));
+}
+
+// The correctly rounded fp64 reciprocals of the rank counts 1..kMaxRanks,
+// evaluated by the compiler (IEEE division in a constant expression).
+struct CountReciprocals {
+    double v[kMaxRanks + 1];
+};
+constexpr CountReciprocals count_reciprocals()
+{
+    CountReciprocals r{};
+    for (int i = 1; i <= kMaxRanks; ++i) r.v[i] = 1.0 / (double)i;
+    return r;
+}
+static __constant__ CountReciprocals kCountReciprocals = count_reciprocals();
+
 // Any other whole rank count N (below 2^24) takes no division either: the
 // fp64 product of a and the correctly rounded fp64 reciprocal of N, rounded
 // once to fp32, is a / N correctly rounded.  The product's relative error is
@@ -191,9 +211,12 @@ template <int OP>
 __device__ __forceinline__ float finish(float a, float divisor)
 {
     if constexpr (OP == kAvg) {
-        if (is_pow2(divisor)) return __fmul_rn(a, __frcp_rn(divisor));
-        if (is_whole_count(divisor))
-            return __double2float_rn(__dmul_rn((double)a, __drcp_rn((double)divisor)));
+        if (is_pow2(divisor)) return __fmul_rn(a, pow2_reciprocal(divisor));
+        if (is_whole_count(divisor)) {
+            const uint32_t k = (uint32_t)divisor;
+            const double r = k <= (uint32_t)kMaxRanks ? kCountReciprocals.v[k] : __drcp_rn((double)divisor);
+            return __double2float_rn(__dmul_rn((double)a, r));
+        }
         return __fdiv_rn(a, divisor);
     } else {
         return a;

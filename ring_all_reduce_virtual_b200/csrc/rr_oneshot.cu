@@ -46,6 +46,7 @@ template <class Ty, int OP>
 cudaError_t launch_oneshot_ring(const RankParams& p, uint64_t work, cudaStream_t s)
 {
     if (bulk_eligible(p, (int)sizeof(typename Ty::T))) return launch_oneshot_bulk<Ty, OP>(p, s);
+    if (!p.vec_ok && mixed_eligible(p, (int)sizeof(typename Ty::T))) return launch_oneshot_mixed<Ty, OP>(p, s);
     const int n = p.n;
     constexpr int V = kVptReduce;
     switch (n) {

@@ -30,6 +30,14 @@ template <class Ty, int OP>
 cudaError_t launch_tree_bulk(const RankParams& p, cudaStream_t s);
 cudaError_t launch_oneshot_wire_bulk(int op, const RankParams& p, cudaStream_t s);
 
+// The one-shot over rank buffers at different 16-byte phases (rr_mixed.cu):
+// every rank's tile staged at its own shift, whole-vector stores to every
+// output at its own phase.  mixed_eligible: a plain call of 2-16 ranks on
+// element boundaries.
+bool mixed_eligible(const RankParams& p, int esize);
+template <class Ty, int OP>
+cudaError_t launch_oneshot_mixed(const RankParams& p, cudaStream_t s);
+
 // The tree's pairwise order ([P3] section 6: ranks pair up, pairs pair up,
 // log2 N levels) folded per element in registers.  Ranks are pushed in order
 // 0..N-1 onto a stack of partial blocks: pushing rank j combines it with the

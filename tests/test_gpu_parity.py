@@ -851,6 +851,25 @@ def test_aligned_all_gather_and_two_shot(n, dtype):
     rrv.check_timeouts()
 
 
+@pytest.mark.parametrize("n", [2, 3, 5, 8, 16, 64])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16", "i32"])
+def test_one_shot_over_ranks_at_different_phases(n, dtype):
+    """Rank buffers whose addresses differ modulo 16 bytes: each rank's tile is
+    staged at its own shift and every output gets whole vectors at its own
+    phase (plus scalar heads and tails); ragged chunks over several tiles,
+    every op, the two-shot's owner-only first shot too."""
+    L = 4 if dtype in ("f32", "i32") else 8
+    offsets = [(3 * r + 1) % L for r in range(n)]
+    if len(set(offsets)) == 1:
+        offsets[0] = (offsets[0] + 1) % L
+    count = n * 1500 + 7
+    ops = ("sum", "max", "min", "prod") if dtype == "i32" else ("sum", "avg", "max", "prod")
+    for op in ops:
+        _run(n, count, dtype, op, "oneshot", seed=400 + n, offsets=offsets)
+    _run(n, count, dtype, "sum", "two_shot", seed=410 + n, offsets=offsets)
+    _run(n, 3, dtype, "sum", "oneshot", seed=420 + n, offsets=offsets)  # fewer elements than ranks
+
+
 def _near_midpoints(rng, n, size):
     """fp32 values next to n * m, m a midpoint between neighbouring fp32
     values: the quotients closest to a rounding boundary."""
