@@ -30,10 +30,6 @@ uint32_t mixed_tile_vectors(int n)
     return bulk_tile_vectors(n);
 }
 
-#ifndef RR_MIXED_STORE_WALK
-#define RR_MIXED_STORE_WALK 0
-#endif
-
 struct MixedParams {
     RankParams r;
     uint32_t tv;  // vectors per rank per tile; every slot holds tv + 1
@@ -118,22 +114,13 @@ __global__ void __launch_bounds__(kThreads) oneshot_mixed_kernel(const __grid_co
 
     // 3. every output: whole aligned vectors shifted out of the result (item
     // q = vector m of output o, all outputs' vectors spread over the CTA), and
-    // scalars before the first 16-byte boundary and after the last whole vector
-#if RR_MIXED_STORE_WALK == 2
-    for (int o = 0; o < nout; ++o) {
-        T* ob = out(o);
-        uint32_t h = (uint32_t)((L - phase_of(ob, L)) & (L - 1));
-        if (h > te) h = te;
-        const uint32_t nv = (te - h) / L;
-        for (uint32_t m = threadIdx.x; m < nv; m += kThreads) {
-            const uint4 v = h ? shift_window(resv[m], resv[m + 1], (int)(h * sizeof(T))) : resv[m];
-            stv(ob + h + (uint64_t)m * L, v);
-        }
-    }
-#elif RR_MIXED_STORE_WALK == 1
+    // scalars before the first 16-byte boundary and after the last whole vector.
+    // Measured at 2 / 4 / 8 / 16 ranks x 256 MiB fp32: this walk 1.00 / 0.93 /
+    // 0.89 / 0.955 of the copy peak; the same items found by a division per
+    // item 0.82 / 0.80 / 0.78 / 0.96; one output after the other 1.01 / 0.96 /
+    // 0.86 / 0.93.  Thread t takes items t, t + kThreads, ... of the (output,
+    // vector) sequence, stepping through it without a division.
     {
-        // thread t takes items t, t + kThreads, ... of the (output, vector)
-        // sequence, stepping through it without a division
         int o = 0;
         uint32_t m = threadIdx.x;
         while (o < nout && m >= nvt) m -= nvt, ++o;
@@ -150,17 +137,6 @@ __global__ void __launch_bounds__(kThreads) oneshot_mixed_kernel(const __grid_co
             while (o < nout && m >= nvt) m -= nvt, ++o;
         }
     }
-#else
-    for (uint32_t q = threadIdx.x; q < (uint32_t)nout * nvt; q += kThreads) {
-        const uint32_t o = q / nvt, m = q - o * nvt;
-        T* ob = out((int)o);
-        uint32_t h = (uint32_t)((L - phase_of(ob, L)) & (L - 1));
-        if (h > te) h = te;
-        if (m >= (te - h) / L) continue;  // past the output's last whole vector
-        const uint4 v = h ? shift_window(resv[m], resv[m + 1], (int)(h * sizeof(T))) : resv[m];
-        stv(ob + h + (uint64_t)m * L, v);
-    }
-#endif
     for (uint32_t q = threadIdx.x; q < (uint32_t)nout * 2u * L; q += kThreads) {
         const uint32_t o = q / (2u * L), k = q - o * (2u * L);
         T* ob = out((int)o);
