@@ -84,6 +84,9 @@ def parse_args():
     ap.add_argument("--odd", action="store_true",
                     help="--workload kernels: odd bucket tensor sizes, so later tensors sit out of phase with "
                          "their gradients in the fp32 bucket")
+    ap.add_argument("--mixed", action="store_true",
+                    help="--workload kernels: rank buffers of the all-reduces at different 16-byte phases "
+                         "(rank r starts (3r + 1) mod 4 elements past a boundary)")
     ap.add_argument("--count", type=int, default=COUNT,
                     help="fp32 elements per virtual rank (default 2^26 = 256 MiB); smaller for profiling")
     return ap.parse_args()
@@ -848,7 +851,10 @@ def run_kernels(args):
     S = count * ELEM
     peak, _ = hbm_peak()
     gen = torch.Generator(device=dev).manual_seed(SEED)
-    x = [torch.randn(count, device=dev, generator=gen) * 1e-3 for _ in range(n)]
+    if args.mixed:  # views at unequal offsets: no two ranks share a 16-byte phase (up to 4 ranks)
+        x = [(torch.randn(count + 4, device=dev, generator=gen) * 1e-3)[(3 * r + 1) % 4:][:count] for r in range(n)]
+    else:
+        x = [torch.randn(count, device=dev, generator=gen) * 1e-3 for _ in range(n)]
     per = count // n
     rs = [torch.empty(per, device=dev) for _ in range(n)]
     out = [torch.empty(count, device=dev) for _ in range(n)]
@@ -874,7 +880,8 @@ def run_kernels(args):
         b.record(stream)
         torch.cuda.synchronize(dev)
         t = a.elapsed_time(b) / max(args.reps, 1) / 1e3
-        print(json.dumps({"workload": f"kernels-{n}x{count}-f32" + ("-odd" if args.odd else ""), "call": what,
+        print(json.dumps({"workload": f"kernels-{n}x{count}-f32" + ("-odd" if args.odd else "")
+                          + ("-mixed" if args.mixed else ""), "call": what,
                           "ms": round(t * 1e3, 4),
                           "hbm_gbs": round(st["hbm_bytes"] / t / 1e9, 1),
                           "hbm_frac": round(st["hbm_bytes"] / t / 1e9 / peak, 4), "launches": st["launches"]}),
