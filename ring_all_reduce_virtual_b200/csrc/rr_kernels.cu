@@ -325,6 +325,7 @@ cudaError_t launch_rank_kernel(int kind, int dtype, int op, const RankParams& p,
         case kOneshotRing: return launch_oneshot_ring<Ty, OP>(p, work, s);
         case kReduceScatter:
             if (bulk_scatter_eligible(p, (int)sizeof(typename Ty::T))) return launch_scatter_bulk<Ty, OP>(p, s);
+            if (!p.vec_ok && mixed_eligible(p, (int)sizeof(typename Ty::T))) return launch_scatter_mixed<Ty, OP>(p, s);
             switch (n) {
             case 2: return launch_all(reduce_scatter_kernel<Ty, OP, V, 1, 2>, p, work, s);
             case 4: return launch_all(reduce_scatter_kernel<Ty, OP, V, 3, 4>, p, work, s);

@@ -36,7 +36,14 @@ struct MixedParams {
     uint32_t pad_;
 };
 
-template <class Ty, int OP>
+// MODE kMixedRing: segment c = chunk c of every rank, folded from rank c,
+// written to every rank (or to rank c only: the two-shot's first shot);
+// kMixedScatter: segment r = part r (offset r*C) of every rank, folded from
+// rank r, written to out[r] (the reduce-scatter).  WIRE: the bf16 wire format
+// of the ring-order one-shot (rr_device.cuh).
+enum MixedMode : int { kMixedRing = 0, kMixedScatter = 1 };
+
+template <class Ty, int OP, int MODE, int WIRE>
 __global__ void __launch_bounds__(kThreads) oneshot_mixed_kernel(const __grid_constant__ MixedParams mp)
 {
     using T = typename Ty::T;
@@ -50,12 +57,17 @@ __global__ void __launch_bounds__(kThreads) oneshot_mixed_kernel(const __grid_co
     __shared__ uint32_t shift[kMaxRanks];        // slot j's first element of the tile
 
     const uint64_t c = blockIdx.x / p.tps, tile = blockIdx.x - c * p.tps;
-    // chunk c clipped to this launch's element range
-    const uint64_t c_lo = c * p.C;
-    if (c_lo >= p.count) return;
-    const uint64_t c_hi = p.C < p.count - c_lo ? c_lo + p.C : p.count;
-    const uint64_t lo = c_lo > p.lo ? c_lo : p.lo;
-    const uint64_t hi = c_hi < p.hi ? c_hi : p.hi;
+    uint64_t lo, hi;
+    if constexpr (MODE == kMixedScatter) {
+        lo = c * p.C;
+        hi = lo + p.C;
+    } else {  // chunk c clipped to this launch's element range
+        const uint64_t c_lo = c * p.C;
+        if (c_lo >= p.count) return;
+        const uint64_t c_hi = p.C < p.count - c_lo ? c_lo + p.C : p.count;
+        lo = c_lo > p.lo ? c_lo : p.lo;
+        hi = c_hi < p.hi ? c_hi : p.hi;
+    }
     const uint64_t start = lo + tile * TE;
     if (lo >= hi || start >= hi) return;
     const uint32_t te = (uint32_t)(hi - start < TE ? hi - start : TE);  // elements of this tile
@@ -65,8 +77,11 @@ __global__ void __launch_bounds__(kThreads) oneshot_mixed_kernel(const __grid_co
         if (r >= n) r -= n;
         return static_cast<const T*>(p.in[r]) + start;
     };
-    const int nout = p.owner_only ? 1 : n;
-    auto out = [&](int o) { return static_cast<T*>(p.out[p.owner_only ? first : o]) + start; };
+    const int nout = MODE == kMixedScatter || p.owner_only ? 1 : n;
+    auto out = [&](int o) {
+        if constexpr (MODE == kMixedScatter) return static_cast<T*>(p.out[first]) + (start - lo);
+        else return static_cast<T*>(p.out[p.owner_only ? first : o]) + start;
+    };
 
     // 1. stage: slot j holds rank (c + j) mod N, from the aligned vector at or
     // below the tile's first element up to the one holding its last element;
@@ -104,10 +119,10 @@ __global__ void __launch_bounds__(kThreads) oneshot_mixed_kernel(const __grid_co
             Acc x[L];
             Ty::unpack(slot_vec(j, m), x);
 #pragma unroll
-            for (int l = 0; l < L; ++l) a[l] = apply<OP>(a[l], x[l]);
+            for (int l = 0; l < L; ++l) a[l] = apply<OP>(wire_in<WIRE>(a[l]), x[l]);
         }
 #pragma unroll
-        for (int l = 0; l < L; ++l) a[l] = finish<OP>(a[l], p.divisor);
+        for (int l = 0; l < L; ++l) a[l] = wire_out<WIRE>(finish<OP>(a[l], p.divisor));
         resv[m] = Ty::pack(a);
     }
     __syncthreads();
@@ -166,25 +181,53 @@ bool mixed_eligible(const RankParams& p, int esize)
     return (seg + te - 1) / te * (uint64_t)p.n <= kMaxGrid;
 }
 
-template <class Ty, int OP>
-cudaError_t launch_oneshot_mixed(const RankParams& p, cudaStream_t s)
+namespace {
+
+// One CTA per (segment, tile); a segment is a chunk clipped to the launch's
+// element range (ring mode) or a part (scatter mode).
+template <class Ty, int OP, int MODE, int WIRE>
+cudaError_t launch_mixed(const RankParams& p, cudaStream_t s)
 {
     MixedParams mp{};
     mp.r = p;
     mp.tv = mixed_tile_vectors(p.n);
     const uint64_t te = (uint64_t)mp.tv * Ty::L;
-    const uint64_t hi = p.hi < p.count ? p.hi : p.count;
-    const uint64_t seg = hi - p.lo < p.C ? hi - p.lo : p.C;
+    uint64_t seg = p.C;
+    if constexpr (MODE == kMixedRing) {
+        const uint64_t hi = p.hi < p.count ? p.hi : p.count;
+        seg = hi - p.lo < p.C ? hi - p.lo : p.C;
+    }
     mp.r.tps = seg ? (seg + te - 1) / te : 1;
     const uint64_t work = (uint64_t)p.n * mp.r.tps;
     if (work == 0) return cudaSuccess;
     if (work > kMaxGrid) return cudaErrorInvalidValue;  // never reached: mixed_eligible caps it
     const uint32_t smem = ((uint32_t)p.n + 1u) * (mp.tv + 1u) * 16u;
-    oneshot_mixed_kernel<Ty, OP><<<(unsigned)work, kThreads, smem, s>>>(mp);
+    oneshot_mixed_kernel<Ty, OP, MODE, WIRE><<<(unsigned)work, kThreads, smem, s>>>(mp);
     return cudaGetLastError();
 }
 
-#define RR_INSTANTIATE(TY, OP) template cudaError_t launch_oneshot_mixed<TY, OP>(const RankParams&, cudaStream_t);
+}  // namespace
+
+template <class Ty, int OP>
+cudaError_t launch_oneshot_mixed(const RankParams& p, cudaStream_t s)
+{
+    return launch_mixed<Ty, OP, kMixedRing, 0>(p, s);
+}
+
+template <class Ty, int OP>
+cudaError_t launch_scatter_mixed(const RankParams& p, cudaStream_t s)
+{
+    return launch_mixed<Ty, OP, kMixedScatter, 0>(p, s);
+}
+
+cudaError_t launch_oneshot_wire_mixed(int op, const RankParams& p, cudaStream_t s)
+{
+    return op == kAvg ? launch_mixed<F32T, kAvg, kMixedRing, 1>(p, s) : launch_mixed<F32T, kSum, kMixedRing, 1>(p, s);
+}
+
+#define RR_INSTANTIATE(TY, OP)                                                                   \
+    template cudaError_t launch_oneshot_mixed<TY, OP>(const RankParams&, cudaStream_t);           \
+    template cudaError_t launch_scatter_mixed<TY, OP>(const RankParams&, cudaStream_t);
 RR_FOR_EACH_TYPE_OP(RR_INSTANTIATE)
 #undef RR_INSTANTIATE
 

@@ -77,6 +77,7 @@ cudaError_t launch_oneshot_wire_op(const RankParams& p, uint64_t work, cudaStrea
 cudaError_t launch_oneshot_wire(int op, const RankParams& p, uint64_t work, cudaStream_t s)
 {
     if (bulk_eligible(p, (int)sizeof(float))) return launch_oneshot_wire_bulk(op, p, s);
+    if (!p.vec_ok && mixed_eligible(p, (int)sizeof(float))) return launch_oneshot_wire_mixed(op, p, s);
     return op == kAvg ? launch_oneshot_wire_op<kAvg>(p, work, s) : launch_oneshot_wire_op<kSum>(p, work, s);
 }
 

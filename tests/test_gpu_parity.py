@@ -868,6 +868,20 @@ def test_one_shot_over_ranks_at_different_phases(n, dtype):
         _run(n, count, dtype, op, "oneshot", seed=400 + n, offsets=offsets)
     _run(n, count, dtype, "sum", "two_shot", seed=410 + n, offsets=offsets)
     _run(n, 3, dtype, "sum", "oneshot", seed=420 + n, offsets=offsets)  # fewer elements than ranks
+    # the reduce-scatter: inputs at the ranks' phases, outputs at other ones
+    per = 1500 + 3
+    x = synth.ranks(430 + n, n, n * per, _dist("sum", dtype), dtype)
+    rs = to_dev([np.zeros(per, dtype=a.dtype) for a in x], offsets=offsets[::-1])
+    op = "max" if dtype == "i32" else "avg"
+    rrv.reduce_scatter(to_dev(x, offsets=offsets), rs, op)
+    assert_bits_equal(to_host(rs), oracle.reduce_scatter([a.copy() for a in x], op), f"rs {op} n={n}")
+    if dtype == "f32":  # the bf16 wire format of the one-shot
+        y = synth.ranks(440 + n, n, count, "full")
+        want = [a.copy() for a in y]
+        oracle.fold_wire(want, "avg")
+        d = to_dev(y, offsets=offsets)
+        rrv.all_reduce_wire(d, "avg", "bf16", "oneshot")
+        assert_bits_equal(to_host(d), want, f"wire n={n}")
 
 
 def _near_midpoints(rng, n, size):
