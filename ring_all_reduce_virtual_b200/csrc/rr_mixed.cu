@@ -39,9 +39,11 @@ struct MixedParams {
 // MODE kMixedRing: segment c = chunk c of every rank, folded from rank c,
 // written to every rank (or to rank c only: the two-shot's first shot);
 // kMixedScatter: segment r = part r (offset r*C) of every rank, folded from
-// rank r, written to out[r] (the reduce-scatter).  WIRE: the bf16 wire format
-// of the ring-order one-shot (rr_device.cuh).
-enum MixedMode : int { kMixedRing = 0, kMixedScatter = 1 };
+// rank r, written to out[r] (the reduce-scatter); kMixedTree: the whole
+// buffer as one segment, folded in the tree's pairwise order (up to 16
+// ranks), written to every rank.  WIRE: the bf16 wire format of the
+// ring-order one-shot (rr_device.cuh).
+enum MixedMode : int { kMixedRing = 0, kMixedScatter = 1, kMixedTree = 2 };
 
 template <class Ty, int OP, int MODE, int WIRE>
 __global__ void __launch_bounds__(kThreads) oneshot_mixed_kernel(const __grid_constant__ MixedParams mp)
@@ -61,6 +63,9 @@ __global__ void __launch_bounds__(kThreads) oneshot_mixed_kernel(const __grid_co
     if constexpr (MODE == kMixedScatter) {
         lo = c * p.C;
         hi = lo + p.C;
+    } else if constexpr (MODE == kMixedTree) {
+        lo = 0;
+        hi = p.count;
     } else {  // chunk c clipped to this launch's element range
         const uint64_t c_lo = c * p.C;
         if (c_lo >= p.count) return;
@@ -77,9 +82,10 @@ __global__ void __launch_bounds__(kThreads) oneshot_mixed_kernel(const __grid_co
         if (r >= n) r -= n;
         return static_cast<const T*>(p.in[r]) + start;
     };
-    const int nout = MODE == kMixedScatter || p.owner_only ? 1 : n;
+    const int nout = MODE == kMixedScatter || (MODE == kMixedRing && p.owner_only) ? 1 : n;
     auto out = [&](int o) {
         if constexpr (MODE == kMixedScatter) return static_cast<T*>(p.out[first]) + (start - lo);
+        else if constexpr (MODE == kMixedTree) return static_cast<T*>(p.out[o]) + start;
         else return static_cast<T*>(p.out[p.owner_only ? first : o]) + start;
     };
 
@@ -114,12 +120,48 @@ __global__ void __launch_bounds__(kThreads) oneshot_mixed_kernel(const __grid_co
     };
     for (uint32_t m = threadIdx.x; m < nvt; m += kThreads) {
         Acc a[L];
-        Ty::unpack(slot_vec(0, m), a);
-        for (int j = 1; j < n; ++j) {
-            Acc x[L];
-            Ty::unpack(slot_vec(j, m), x);
+        if constexpr (MODE == kMixedTree) {
+            // the tree's pairwise order with fp32 partials: slot j joins a
+            // stack whose level b holds a finished block of 2^b ranks; after
+            // the last slot the blocks of the set bits of N combine from the
+            // lowest level up, each higher (earlier) block on the left
+            constexpr int LV = 5;  // up to 16 ranks
+            Acc stack[LV][L];
 #pragma unroll
-            for (int l = 0; l < L; ++l) a[l] = apply<OP>(wire_in<WIRE>(a[l]), x[l]);
+            for (int j = 0; j < 16; ++j) {
+                if (j >= n) break;
+                Ty::unpack(slot_vec(j, m), a);
+                int lvl = 0;
+#pragma unroll
+                for (int bb = 0; bb < LV - 1; ++bb) {
+                    if (((j >> bb) & 1) && lvl == bb) {
+#pragma unroll
+                        for (int l = 0; l < L; ++l) a[l] = apply<OP>(stack[bb][l], a[l]);
+                        lvl = bb + 1;
+                    }
+                }
+#pragma unroll
+                for (int bb = 0; bb < LV; ++bb)
+                    if (bb == lvl)
+#pragma unroll
+                        for (int l = 0; l < L; ++l) stack[bb][l] = a[l];
+            }
+            bool have = false;
+#pragma unroll
+            for (int bb = 0; bb < LV; ++bb) {
+                if (!((n >> bb) & 1)) continue;
+#pragma unroll
+                for (int l = 0; l < L; ++l) a[l] = have ? apply<OP>(stack[bb][l], a[l]) : stack[bb][l];
+                have = true;
+            }
+        } else {
+            Ty::unpack(slot_vec(0, m), a);
+            for (int j = 1; j < n; ++j) {
+                Acc x[L];
+                Ty::unpack(slot_vec(j, m), x);
+#pragma unroll
+                for (int l = 0; l < L; ++l) a[l] = apply<OP>(wire_in<WIRE>(a[l]), x[l]);
+            }
         }
 #pragma unroll
         for (int l = 0; l < L; ++l) a[l] = wire_out<WIRE>(finish<OP>(a[l], p.divisor));
@@ -181,10 +223,20 @@ bool mixed_eligible(const RankParams& p, int esize)
     return (seg + te - 1) / te * (uint64_t)p.n <= kMaxGrid;
 }
 
+bool mixed_tree_eligible(const RankParams& p, int esize)
+{
+    if (p.n < 2 || p.n > 16 || p.nseg != 1) return false;
+    for (int r = 0; r < p.n; ++r)
+        if ((uintptr_t)p.in[r] % (uintptr_t)esize || (uintptr_t)p.out[r] % (uintptr_t)esize) return false;
+    const uint64_t te = (uint64_t)mixed_tile_vectors(p.n) * (16u / (uint64_t)esize);
+    return (p.count + te - 1) / te <= kMaxGrid;
+}
+
 namespace {
 
 // One CTA per (segment, tile); a segment is a chunk clipped to the launch's
-// element range (ring mode) or a part (scatter mode).
+// element range (ring mode), a part (scatter mode) or the whole buffer (tree
+// mode).
 template <class Ty, int OP, int MODE, int WIRE>
 cudaError_t launch_mixed(const RankParams& p, cudaStream_t s)
 {
@@ -192,13 +244,13 @@ cudaError_t launch_mixed(const RankParams& p, cudaStream_t s)
     mp.r = p;
     mp.tv = mixed_tile_vectors(p.n);
     const uint64_t te = (uint64_t)mp.tv * Ty::L;
-    uint64_t seg = p.C;
+    uint64_t seg = MODE == kMixedTree ? p.count : p.C;
     if constexpr (MODE == kMixedRing) {
         const uint64_t hi = p.hi < p.count ? p.hi : p.count;
         seg = hi - p.lo < p.C ? hi - p.lo : p.C;
     }
     mp.r.tps = seg ? (seg + te - 1) / te : 1;
-    const uint64_t work = (uint64_t)p.n * mp.r.tps;
+    const uint64_t work = p.nseg * mp.r.tps;
     if (work == 0) return cudaSuccess;
     if (work > kMaxGrid) return cudaErrorInvalidValue;  // never reached: mixed_eligible caps it
     const uint32_t smem = ((uint32_t)p.n + 1u) * (mp.tv + 1u) * 16u;
@@ -220,6 +272,12 @@ cudaError_t launch_scatter_mixed(const RankParams& p, cudaStream_t s)
     return launch_mixed<Ty, OP, kMixedScatter, 0>(p, s);
 }
 
+template <class Ty, int OP>
+cudaError_t launch_tree_mixed(const RankParams& p, cudaStream_t s)
+{
+    return launch_mixed<Ty, OP, kMixedTree, 0>(p, s);
+}
+
 cudaError_t launch_oneshot_wire_mixed(int op, const RankParams& p, cudaStream_t s)
 {
     return op == kAvg ? launch_mixed<F32T, kAvg, kMixedRing, 1>(p, s) : launch_mixed<F32T, kSum, kMixedRing, 1>(p, s);
@@ -227,7 +285,8 @@ cudaError_t launch_oneshot_wire_mixed(int op, const RankParams& p, cudaStream_t 
 
 #define RR_INSTANTIATE(TY, OP)                                                                   \
     template cudaError_t launch_oneshot_mixed<TY, OP>(const RankParams&, cudaStream_t);           \
-    template cudaError_t launch_scatter_mixed<TY, OP>(const RankParams&, cudaStream_t);
+    template cudaError_t launch_scatter_mixed<TY, OP>(const RankParams&, cudaStream_t);            \
+    template cudaError_t launch_tree_mixed<TY, OP>(const RankParams&, cudaStream_t);
 RR_FOR_EACH_TYPE_OP(RR_INSTANTIATE)
 #undef RR_INSTANTIATE
 

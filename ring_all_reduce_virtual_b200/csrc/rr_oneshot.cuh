@@ -30,8 +30,9 @@ template <class Ty, int OP>
 cudaError_t launch_tree_bulk(const RankParams& p, cudaStream_t s);
 cudaError_t launch_oneshot_wire_bulk(int op, const RankParams& p, cudaStream_t s);
 
-// The one-shot, the reduce-scatter and the bf16-wire one-shot over rank
-// buffers at different 16-byte phases (rr_mixed.cu): every rank's tile staged
+// The one-shot, the reduce-scatter, the bf16-wire one-shot and the
+// tree-order one-shot over rank buffers at different 16-byte phases
+// (rr_mixed.cu): every rank's tile staged
 // at its own shift, whole-vector stores to every output at its own phase.
 // mixed_eligible: a plain call of 2-16 ranks on element boundaries.
 bool mixed_eligible(const RankParams& p, int esize);
@@ -40,6 +41,10 @@ cudaError_t launch_oneshot_mixed(const RankParams& p, cudaStream_t s);
 template <class Ty, int OP>
 cudaError_t launch_scatter_mixed(const RankParams& p, cudaStream_t s);
 cudaError_t launch_oneshot_wire_mixed(int op, const RankParams& p, cudaStream_t s);
+// the tree-order one-shot the same way (2-16 ranks; the whole buffer is one segment)
+bool mixed_tree_eligible(const RankParams& p, int esize);
+template <class Ty, int OP>
+cudaError_t launch_tree_mixed(const RankParams& p, cudaStream_t s);
 
 // The tree's pairwise order ([P3] section 6: ranks pair up, pairs pair up,
 // log2 N levels) folded per element in registers.  Ranks are pushed in order

@@ -126,6 +126,7 @@ template <class Ty, int OP>
 cudaError_t launch_oneshot_tree(const RankParams& p, uint64_t work, cudaStream_t s)
 {
     if (bulk_tree_eligible(p, (int)sizeof(typename Ty::T))) return launch_tree_bulk<Ty, OP>(p, s);
+    if (!p.vec_ok && mixed_tree_eligible(p, (int)sizeof(typename Ty::T))) return launch_tree_mixed<Ty, OP>(p, s);
     const int n = p.n;
     constexpr int V = kVptReduce;
     switch (n) {

@@ -857,7 +857,8 @@ def test_one_shot_over_ranks_at_different_phases(n, dtype):
     """Rank buffers whose addresses differ modulo 16 bytes: each rank's tile is
     staged at its own shift and every output gets whole vectors at its own
     phase (plus scalar heads and tails); ragged chunks over several tiles,
-    every op, the two-shot's owner-only first shot too."""
+    every op, the two-shot's owner-only first shot, the tree's order, the
+    reduce-scatter and the bf16 wire too."""
     L = 4 if dtype in ("f32", "i32") else 8
     offsets = [(3 * r + 1) % L for r in range(n)]
     if len(set(offsets)) == 1:
@@ -868,6 +869,8 @@ def test_one_shot_over_ranks_at_different_phases(n, dtype):
         _run(n, count, dtype, op, "oneshot", seed=400 + n, offsets=offsets)
     _run(n, count, dtype, "sum", "two_shot", seed=410 + n, offsets=offsets)
     _run(n, 3, dtype, "sum", "oneshot", seed=420 + n, offsets=offsets)  # fewer elements than ranks
+    for op in ops[:2]:  # the tree's pairwise order, staged the same way (up to 16 ranks)
+        _run(n, count, dtype, op, "tree_oneshot", seed=450 + n, offsets=offsets)
     # the reduce-scatter: inputs at the ranks' phases, outputs at other ones
     per = 1500 + 3
     x = synth.ranks(430 + n, n, n * per, _dist("sum", dtype), dtype)
