@@ -1,9 +1,10 @@
 // rr_kernels.cu -- the collectives' kernels and their launchers.
 //
 // All kernels are HBM-bound streaming kernels: each input byte is read once
-// and each output byte written once per launch, with 128-bit vector access
-// and a grid-stride loop over (segment, tile) work items sized to one wave of
-// resident CTAs.  No kernel waits on another CTA or another launch.
+// and each output byte written once per launch (a source tile that several
+// outputs need is read from L2 after the first), with 128-bit vector access
+// and one CTA per (segment, tile) work item (a grid-stride loop covers grids
+// past the launch limit).  No kernel waits on another CTA or another launch.
 //
 // Sources: [P4] "Collective communication primitives" (ai-infra-handbooks),
 // sections "The five primitives", "Ring all-reduce and communication volume"
