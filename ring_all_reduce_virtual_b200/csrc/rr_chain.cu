@@ -93,6 +93,55 @@ __device__ __forceinline__ void chain_fold(const ChainLanes<Ty>& ln, const typen
         }
 }
 
+// The next reduce-scatter step's own operand (the receiving rank's copy,
+// which nothing writes before that step) copied by cp.async into this
+// thread's shared-memory slots, so that the step waits only for the
+// neighbour's partial.  Each thread reads only the slots it filled, after its
+// own cp.async.wait_group: no barrier.  Used by the bf16-wire ring, whose
+// rounding steps lengthen each step: measured at 3 / 8 / 24 / 48 ranks x
+// 256 MiB, 0.317 / 0.818 / 3.53 / 7.86 ms without and 0.291 / 0.711 / 3.37 /
+// 7.47 ms with it; the plain ring, bound by the read of the partial it has
+// just stored, moved by -1 to +2 % and keeps its loads.
+template <class Ty>
+__device__ __forceinline__ void chain_stage(const ChainLanes<Ty>& ln, const typename Ty::T* own, uint4* slot)
+{
+#pragma unroll
+    for (int u = 0; u < kChainVpt; ++u)
+        if (ln.ok[u])
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                             (uint32_t)__cvta_generic_to_shared(slot + u * kThreads + threadIdx.x)),
+                         "l"(own + ln.vec[u])
+                         : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// chain_fold with the own operand taken from the stage slots.
+template <class Ty, int OP, int WIRE>
+__device__ __forceinline__ void chain_fold_staged(const ChainLanes<Ty>& ln, const typename Ty::T* src,
+                                                  typename Ty::T* dst, const uint4* slot, float divisor)
+{
+    using Acc = typename Ty::Acc;
+    constexpr int L = Ty::L;
+    if (ln.has_one) {
+        Acc a = apply<OP>(wire_in<WIRE>(Ty::ld1(src + ln.one)), Ty::ld1(dst + ln.one));
+        Ty::st1(dst + ln.one, wire_out<WIRE>(finish<OP>(a, divisor)));
+    }
+    uint4 x[kChainVpt];
+#pragma unroll
+    for (int u = 0; u < kChainVpt; ++u)
+        if (ln.ok[u]) x[u] = ldv(src + ln.vec[u]);
+#pragma unroll
+    for (int u = 0; u < kChainVpt; ++u)
+        if (ln.ok[u]) {
+            Acc a[L], b[L];
+            Ty::unpack(x[u], a);
+            Ty::unpack(slot[u * kThreads + threadIdx.x], b);
+#pragma unroll
+            for (int l = 0; l < L; ++l) a[l] = wire_out<WIRE>(finish<OP>(apply<OP>(wire_in<WIRE>(a[l]), b[l]), divisor));
+            stv(dst + ln.vec[u], Ty::pack(a));
+        }
+}
+
 // One all-gather (or broadcast) step on a thread's lanes: dst = src, bits.
 template <class Ty>
 __device__ __forceinline__ void chain_copy(const ChainLanes<Ty>& ln, const typename Ty::T* src, typename Ty::T* dst)
@@ -169,13 +218,32 @@ __global__ void __launch_bounds__(kThreads) ring_chain_kernel(const __grid_const
         const ChainLanes<Ty> ln(static_cast<const T*>(p.buf[k]) + lo, len, tile);
         if (!ln.has_one && !ln.ok[0]) continue;
         // reduce-scatter step s: rank k + dir (s + 1) folds its neighbour's partial into its copy
+        if constexpr (WIRE) {
+            __shared__ uint4 stage[2][kChainVpt * kThreads];
+            chain_stage<Ty>(ln, static_cast<const T*>(p.buf[wrap(k + dir, n)]) + lo, stage[0]);
 #pragma unroll 1
-        for (int s = 0; s < n - 1; ++s) {
-            const int r = wrap(k + dir * (s + 1), n), from = wrap(r - dir, n);
-            const T* src = static_cast<const T*>(p.buf[from]) + lo;
-            T* dst = static_cast<T*>(p.buf[r]) + lo;
-            if (s == n - 2) chain_fold<Ty, OP, WIRE ? 1 : 0>(ln, src, dst, p.divisor);
-            else chain_fold<Ty, OPP, WIRE ? 2 : 0>(ln, src, dst, p.divisor);
+            for (int s = 0; s < n - 1; ++s) {
+                const int r = wrap(k + dir * (s + 1), n), from = wrap(r - dir, n);
+                const T* src = static_cast<const T*>(p.buf[from]) + lo;
+                T* dst = static_cast<T*>(p.buf[r]) + lo;
+                if (s + 1 < n - 1) {
+                    chain_stage<Ty>(ln, static_cast<const T*>(p.buf[wrap(r + dir, n)]) + lo, stage[(s + 1) & 1]);
+                    asm volatile("cp.async.wait_group 1;" ::: "memory");
+                } else {
+                    asm volatile("cp.async.wait_group 0;" ::: "memory");
+                }
+                if (s == n - 2) chain_fold_staged<Ty, OP, 1>(ln, src, dst, stage[s & 1], p.divisor);
+                else chain_fold_staged<Ty, OPP, 2>(ln, src, dst, stage[s & 1], p.divisor);
+            }
+        } else {
+#pragma unroll 1
+            for (int s = 0; s < n - 1; ++s) {
+                const int r = wrap(k + dir * (s + 1), n), from = wrap(r - dir, n);
+                const T* src = static_cast<const T*>(p.buf[from]) + lo;
+                T* dst = static_cast<T*>(p.buf[r]) + lo;
+                if (s == n - 2) chain_fold<Ty, OP, 0>(ln, src, dst, p.divisor);
+                else chain_fold<Ty, OPP, 0>(ln, src, dst, p.divisor);
+            }
         }
         // all-gather step s: rank k + dir s copies the finished chunk from its neighbour
 #pragma unroll 1
