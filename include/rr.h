@@ -328,7 +328,13 @@ rr_status_t rr_bucket_unpack(const rr_bucket_plan_t* plan, int bucket, const voi
  * with the bits of pack -> rr_allreduce(SUM, ring order over the bucket's
  * flat index) -> unpack(op), but reading and writing each gradient once
  * (4 bytes per bf16 parameter per rank instead of 20).  op: SUM or AVG.
- * One launch. */
+ * One launch.  Where every rank's copy of a tensor shares a 16-byte phase
+ * the launch is a programmatic dependent of the stream's previous kernel:
+ * it waits for that kernel and its memory before reading, and a previous
+ * sync of this library lets its CTAs be scheduled while it drains (so
+ * back-to-back syncs of many buckets lose less to ramp-up); for syncs that
+ * should run beside other work on the GPU, the reducer below launches
+ * plainly. */
 rr_status_t rr_bucket_allreduce(const rr_bucket_plan_t* plan, int bucket, void* const* grads,
                                 int nranks, rr_op_t op, cudaStream_t stream);
 

@@ -1304,18 +1304,18 @@ rr_status_t rr_bucket_unpack(const rr_bucket_plan_t* plan, int bucket, const voi
 }
 
 static rr_status_t bucket_fold_range(const rr_bucket_plan_t* plan, int b0, int nb, void* const* grads, int nranks,
-                                     rr_op_t op, cudaStream_t stream, uint64_t max_grid);
+                                     rr_op_t op, cudaStream_t stream, uint64_t max_grid, bool pdl);
 
 rr_status_t rr_bucket_allreduce(const rr_bucket_plan_t* plan, int bucket, void* const* grads, int nranks,
                                 rr_op_t op, cudaStream_t stream)
 {
-    return bucket_fold_range(plan, bucket, 1, grads, nranks, op, stream, kMaxGrid);
+    return bucket_fold_range(plan, bucket, 1, grads, nranks, op, stream, kMaxGrid, true);
 }
 
 rr_status_t rr_bucket_allreduce_range(const rr_bucket_plan_t* plan, int first_bucket, int nbuckets, void* const* grads,
                                       int nranks, rr_op_t op, cudaStream_t stream)
 {
-    return bucket_fold_range(plan, first_bucket, nbuckets, grads, nranks, op, stream, kMaxGrid);
+    return bucket_fold_range(plan, first_bucket, nbuckets, grads, nranks, op, stream, kMaxGrid, true);
 }
 
 }  // extern "C"
@@ -1327,7 +1327,7 @@ rr_status_t rr_bucket_allreduce_range(const rr_bucket_plan_t* plan, int first_bu
 // until the parameter block is full, so a range costs a few launches instead
 // of one per bucket, with the same bits.
 static rr_status_t bucket_fold_range(const rr_bucket_plan_t* plan, int b0, int nb, void* const* grads, int nranks,
-                                     rr_op_t op, cudaStream_t stream, uint64_t max_grid)
+                                     rr_op_t op, cudaStream_t stream, uint64_t max_grid, bool pdl)
 {
     CallTimer timer("rr_bucket_allreduce");
     if (op != RR_SUM && op != RR_AVG) return fail(RR_ERR_UNSUPPORTED, "bucket all-reduce takes SUM or AVG");
@@ -1351,7 +1351,8 @@ static rr_status_t bucket_fold_range(const rr_bucket_plan_t* plan, int b0, int n
         bool v = true;
         for (int t = 0; t < ntens; ++t) v = v && same_phase(&p->grad[t * n], n);
         p->vec_ok = v;
-        cudaError_t e = timed_launch([&] { return launch_bucket_fold(plan->grad_dtype, op, *p, stream, max_grid); });
+        cudaError_t e =
+            timed_launch([&] { return launch_bucket_fold(plan->grad_dtype, op, *p, stream, max_grid, pdl); });
         if (e != cudaSuccess) return cuda_fail(e, "bucket all-reduce launch");
         t_stats.launches += 1;
         return RR_OK;
@@ -1472,7 +1473,7 @@ rr_status_t rr_reducer_ready(rr_reducer_t* red, int tensor, cudaStream_t produce
     cudaError_t e = cudaEventRecord(red->ready[b], producer);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(red->comm, red->ready[b], 0);
     if (e != cudaSuccess) return cuda_fail(e, "ordering the bucket sync after its gradients");
-    return bucket_fold_range(red->plan, b, 1, red->grads.data(), red->n, red->op, red->comm, red->max_grid);
+    return bucket_fold_range(red->plan, b, 1, red->grads.data(), red->n, red->op, red->comm, red->max_grid, false);
 }
 
 rr_status_t rr_check_timeouts(void)

@@ -347,6 +347,12 @@ __global__ void __launch_bounds__(kThreads) bucket_bulk_kernel(const __grid_cons
     using T = typename G::T;
     using Acc = typename G::Acc;
     constexpr int L = G::L;
+    // When launched as a programmatic dependent of the stream's previous
+    // kernel (direct bucket-sync calls): wait for that kernel and its memory
+    // before touching the gradients, and let the next sync's CTAs be
+    // scheduled while this grid drains.  Launched plainly, both are no-ops.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const BucketFoldParams& p = bp.f;
     const int n = NS > 0 ? NS : p.n;
     const uint32_t TV = NS > 0 ? bulk_smem<NS>() / (NS > 0 ? NS : 1) / 16 : bp.tv;  // vectors per rank per tile
@@ -429,7 +435,7 @@ uint64_t bucket_bulk_tile_elems(int grad_dtype, int n)
 }
 
 template <class G, int OP>
-cudaError_t launch_bucket_bulk(const BucketFoldParams& p, int grad_dtype, cudaStream_t s, bool* launched)
+cudaError_t launch_bucket_bulk(const BucketFoldParams& p, int grad_dtype, cudaStream_t s, bool pdl, bool* launched)
 {
     *launched = false;
     RankParams rp{};
@@ -450,15 +456,27 @@ cudaError_t launch_bucket_bulk(const BucketFoldParams& p, int grad_dtype, cudaSt
     if (work > 0 && work <= kMaxGrid) {
         *launched = true;
         bp->tv = bulk_tile_vectors(p.n);
+        auto go = [&](void (*kernel)(BucketBulkParams), uint32_t smem) {
+            cudaLaunchAttribute attr{};
+            attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr.val.programmaticStreamSerializationAllowed = 1;
+            cudaLaunchConfig_t cfg{};
+            cfg.gridDim = dim3((unsigned)work);
+            cfg.blockDim = dim3(kThreads);
+            cfg.dynamicSmemBytes = smem;
+            cfg.stream = s;
+            cfg.attrs = &attr;
+            cfg.numAttrs = pdl ? 1 : 0;
+            return cudaLaunchKernelEx(&cfg, kernel, *bp);
+        };
         switch (p.n) {
-        case 2: bucket_bulk_kernel<G, OP, 2><<<(unsigned)work, kThreads, bulk_smem<2>(), s>>>(*bp); break;
-        case 4: bucket_bulk_kernel<G, OP, 4><<<(unsigned)work, kThreads, bulk_smem<4>(), s>>>(*bp); break;
-        case 8: bucket_bulk_kernel<G, OP, 8><<<(unsigned)work, kThreads, bulk_smem<8>(), s>>>(*bp); break;
-        case 16: bucket_bulk_kernel<G, OP, 16><<<(unsigned)work, kThreads, bulk_smem<16>(), s>>>(*bp); break;
-        default:
-            bucket_bulk_kernel<G, OP, 0><<<(unsigned)work, kThreads, bp->tv * 16u * (uint32_t)p.n, s>>>(*bp);
+        case 2: e = go(bucket_bulk_kernel<G, OP, 2>, bulk_smem<2>()); break;
+        case 4: e = go(bucket_bulk_kernel<G, OP, 4>, bulk_smem<4>()); break;
+        case 8: e = go(bucket_bulk_kernel<G, OP, 8>, bulk_smem<8>()); break;
+        case 16: e = go(bucket_bulk_kernel<G, OP, 16>, bulk_smem<16>()); break;
+        default: e = go(bucket_bulk_kernel<G, OP, 0>, bp->tv * 16u * (uint32_t)p.n);
         }
-        e = cudaGetLastError();
+        if (e == cudaSuccess) e = cudaGetLastError();
     } else if (work == 0) {
         *launched = true;
     }
@@ -521,7 +539,8 @@ cudaError_t launch_bucket_unpack(int grad_dtype, int op, const BucketCopyParams&
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p, cudaStream_t s, uint64_t max_grid)
+cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p, cudaStream_t s, uint64_t max_grid,
+                               bool pdl)
 {
     const uint64_t work = p.tile0[p.nseg];
     const bool avg = op == kAvg;
@@ -530,14 +549,14 @@ cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p
         bool launched = false;
         cudaError_t e = cudaSuccess;
         if (grad_dtype == kBF16)
-            e = avg ? launch_bucket_bulk<BF16T, kAvg>(p, grad_dtype, s, &launched)
-                    : launch_bucket_bulk<BF16T, kSum>(p, grad_dtype, s, &launched);
+            e = avg ? launch_bucket_bulk<BF16T, kAvg>(p, grad_dtype, s, pdl, &launched)
+                    : launch_bucket_bulk<BF16T, kSum>(p, grad_dtype, s, pdl, &launched);
         else if (grad_dtype == kF16)
-            e = avg ? launch_bucket_bulk<F16T, kAvg>(p, grad_dtype, s, &launched)
-                    : launch_bucket_bulk<F16T, kSum>(p, grad_dtype, s, &launched);
+            e = avg ? launch_bucket_bulk<F16T, kAvg>(p, grad_dtype, s, pdl, &launched)
+                    : launch_bucket_bulk<F16T, kSum>(p, grad_dtype, s, pdl, &launched);
         else if (grad_dtype == kF32)
-            e = avg ? launch_bucket_bulk<F32T, kAvg>(p, grad_dtype, s, &launched)
-                    : launch_bucket_bulk<F32T, kSum>(p, grad_dtype, s, &launched);
+            e = avg ? launch_bucket_bulk<F32T, kAvg>(p, grad_dtype, s, pdl, &launched)
+                    : launch_bucket_bulk<F32T, kSum>(p, grad_dtype, s, pdl, &launched);
         if (e != cudaSuccess || launched) return e;
     }
     if (grad_dtype == kBF16)

@@ -169,8 +169,12 @@ cudaError_t take_bulk_timeouts(unsigned int* ran_out, unsigned int* in_flight);
 cudaError_t kernel_binary_version(int* version);
 cudaError_t launch_bucket_pack(int grad_dtype, const BucketCopyParams& p, cudaStream_t s);
 cudaError_t launch_bucket_unpack(int grad_dtype, int op, const BucketCopyParams& p, cudaStream_t s);
+// pdl: launch the bulk-copy sync as a programmatic dependent of the stream's
+// previous kernel (its CTAs scheduled while a previous sync drains): for
+// back-to-back syncs, not for syncs that run beside other work (the reducer),
+// whose waiting CTAs would hold SMs that work could use.
 cudaError_t launch_bucket_fold(int grad_dtype, int op, const BucketFoldParams& p, cudaStream_t s,
-                               uint64_t max_grid = kMaxGrid);
+                               uint64_t max_grid = kMaxGrid, bool pdl = false);
 
 }  // namespace rr
 
