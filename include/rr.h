@@ -38,10 +38,11 @@
  *     take 128-bit vector or bulk-copy access after a scalar head per
  *     segment; a copy or conversion whose output sits at another 16-byte
  *     phase than its input is realigned through shared memory or across
- *     lanes; a one-shot over 2-16 ranks at different phases stages every
- *     rank's tile at its own shift, and only such a one-shot over more ranks
- *     (and the schedules' steps over ranks at different phases, one launch
- *     per step) run element by element.
+ *     lanes; a one-shot or reduce-scatter over ranks at different phases
+ *     stages every rank's tile at its own shift (the tree-order one-shot up
+ *     to 16 ranks), and only the schedules' steps over ranks at different
+ *     phases (one launch per step) and a tree-order one-shot over more ranks
+ *     run element by element.
  *   - Chunking: chunk size C = ceil(count / N); chunk k is the element range
  *     [k*C, min((k+1)*C, count)), possibly short or empty ([P4] "Ring
  *     all-reduce and communication volume": the tensor is split with

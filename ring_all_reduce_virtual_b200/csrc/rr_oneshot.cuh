@@ -34,7 +34,7 @@ cudaError_t launch_oneshot_wire_bulk(int op, const RankParams& p, cudaStream_t s
 // tree-order one-shot over rank buffers at different 16-byte phases
 // (rr_mixed.cu): every rank's tile staged
 // at its own shift, whole-vector stores to every output at its own phase.
-// mixed_eligible: a plain call of 2-16 ranks on element boundaries.
+// mixed_eligible: a plain call of 2-64 ranks on element boundaries.
 bool mixed_eligible(const RankParams& p, int esize);
 template <class Ty, int OP>
 cudaError_t launch_oneshot_mixed(const RankParams& p, cudaStream_t s);
