@@ -29,6 +29,26 @@ namespace rr {
 namespace {
 
 constexpr int kChainVpt = 2;  // 16-byte vectors per thread per tile (about 30 registers each)
+
+// The chains' 16-byte accesses: streaming hints (CACHE 0, evict first), or
+// default caching (CACHE 1).  Every chain reads back only what its own thread
+// wrote, so either is coherent.  Measured per schedule at 3 / 8 / 24 ranks x
+// 256 MiB fp32, streaming / cached: ring 0.273 / 0.728 / 3.34 against 0.290 /
+// 0.782 / 3.30 ms; tree 0.269 / 0.810 / 2.83 against 0.243 / 0.719 / 2.58 ms;
+// bf16-wire ring 0.291 / 0.713 / 3.37 against 0.283 / 0.703 / 3.34 ms.  So
+// the plain ring streams, the tree and the wire ring cache.
+template <int CACHE>
+__device__ __forceinline__ uint4 chain_ld(const void* p)
+{
+    if constexpr (CACHE) return *reinterpret_cast<const uint4*>(p);
+    else return ldv(p);
+}
+template <int CACHE>
+__device__ __forceinline__ void chain_st(void* p, const uint4& v)
+{
+    if constexpr (CACHE) *reinterpret_cast<uint4*>(p) = v;
+    else stv(p, v);
+}
 constexpr uint64_t kChainTileVecs = (uint64_t)kThreads * kChainVpt;
 
 // The elements one thread owns in one tile of a segment of `len` elements
@@ -64,7 +84,7 @@ struct ChainLanes {
 // arriving partial on the left), then AVG's division and the wire rounding
 // where the step completes the chunk.  WIRE: 0 none, 1 completing step, 2
 // partial step (see wire_in / wire_out).
-template <class Ty, int OP, int WIRE>
+template <class Ty, int OP, int WIRE, int CACHE>
 __device__ __forceinline__ void chain_fold(const ChainLanes<Ty>& ln, const typename Ty::T* src, typename Ty::T* dst,
                                            float divisor)
 {
@@ -78,8 +98,8 @@ __device__ __forceinline__ void chain_fold(const ChainLanes<Ty>& ln, const typen
 #pragma unroll
     for (int u = 0; u < kChainVpt; ++u)
         if (ln.ok[u]) {
-            x[u] = ldv(src + ln.vec[u]);
-            y[u] = ldv(dst + ln.vec[u]);
+            x[u] = chain_ld<CACHE>(src + ln.vec[u]);
+            y[u] = chain_ld<CACHE>(dst + ln.vec[u]);
         }
 #pragma unroll
     for (int u = 0; u < kChainVpt; ++u)
@@ -89,7 +109,7 @@ __device__ __forceinline__ void chain_fold(const ChainLanes<Ty>& ln, const typen
             Ty::unpack(y[u], b);
 #pragma unroll
             for (int l = 0; l < L; ++l) a[l] = wire_out<WIRE>(finish<OP>(apply<OP>(wire_in<WIRE>(a[l]), b[l]), divisor));
-            stv(dst + ln.vec[u], Ty::pack(a));
+            chain_st<CACHE>(dst + ln.vec[u], Ty::pack(a));
         }
 }
 
@@ -116,7 +136,7 @@ __device__ __forceinline__ void chain_stage(const ChainLanes<Ty>& ln, const type
 }
 
 // chain_fold with the own operand taken from the stage slots.
-template <class Ty, int OP, int WIRE>
+template <class Ty, int OP, int WIRE, int CACHE>
 __device__ __forceinline__ void chain_fold_staged(const ChainLanes<Ty>& ln, const typename Ty::T* src,
                                                   typename Ty::T* dst, const uint4* slot, float divisor)
 {
@@ -129,7 +149,7 @@ __device__ __forceinline__ void chain_fold_staged(const ChainLanes<Ty>& ln, cons
     uint4 x[kChainVpt];
 #pragma unroll
     for (int u = 0; u < kChainVpt; ++u)
-        if (ln.ok[u]) x[u] = ldv(src + ln.vec[u]);
+        if (ln.ok[u]) x[u] = chain_ld<CACHE>(src + ln.vec[u]);
 #pragma unroll
     for (int u = 0; u < kChainVpt; ++u)
         if (ln.ok[u]) {
@@ -138,26 +158,26 @@ __device__ __forceinline__ void chain_fold_staged(const ChainLanes<Ty>& ln, cons
             Ty::unpack(slot[u * kThreads + threadIdx.x], b);
 #pragma unroll
             for (int l = 0; l < L; ++l) a[l] = wire_out<WIRE>(finish<OP>(apply<OP>(wire_in<WIRE>(a[l]), b[l]), divisor));
-            stv(dst + ln.vec[u], Ty::pack(a));
+            chain_st<CACHE>(dst + ln.vec[u], Ty::pack(a));
         }
 }
 
 // One all-gather (or broadcast) step on a thread's lanes: dst = src, bits.
-template <class Ty>
+template <class Ty, int CACHE>
 __device__ __forceinline__ void chain_copy(const ChainLanes<Ty>& ln, const typename Ty::T* src, typename Ty::T* dst)
 {
     if (ln.has_one) dst[ln.one] = src[ln.one];
     uint4 x[kChainVpt];
 #pragma unroll
     for (int u = 0; u < kChainVpt; ++u)
-        if (ln.ok[u]) x[u] = ldv(src + ln.vec[u]);
+        if (ln.ok[u]) x[u] = chain_ld<CACHE>(src + ln.vec[u]);
 #pragma unroll
     for (int u = 0; u < kChainVpt; ++u)
-        if (ln.ok[u]) stv(dst + ln.vec[u], x[u]);
+        if (ln.ok[u]) chain_st<CACHE>(dst + ln.vec[u], x[u]);
 }
 
 // One tree reduce step on a thread's lanes: out = a op b (a on the left).
-template <class Ty, int OP>
+template <class Ty, int OP, int CACHE>
 __device__ __forceinline__ void tree_fold_pair(const ChainLanes<Ty>& ln, const typename Ty::T* a_, const typename Ty::T* b_,
                                                typename Ty::T* out, float divisor)
 {
@@ -168,8 +188,8 @@ __device__ __forceinline__ void tree_fold_pair(const ChainLanes<Ty>& ln, const t
 #pragma unroll
     for (int u = 0; u < kChainVpt; ++u)
         if (ln.ok[u]) {
-            x[u] = ldv(a_ + ln.vec[u]);
-            y[u] = ldv(b_ + ln.vec[u]);
+            x[u] = chain_ld<CACHE>(a_ + ln.vec[u]);
+            y[u] = chain_ld<CACHE>(b_ + ln.vec[u]);
         }
 #pragma unroll
     for (int u = 0; u < kChainVpt; ++u)
@@ -179,7 +199,7 @@ __device__ __forceinline__ void tree_fold_pair(const ChainLanes<Ty>& ln, const t
             Ty::unpack(y[u], b);
 #pragma unroll
             for (int l = 0; l < L; ++l) a[l] = finish<OP>(apply<OP>(a[l], b[l]), divisor);
-            stv(out + ln.vec[u], Ty::pack(a));
+            chain_st<CACHE>(out + ln.vec[u], Ty::pack(a));
         }
 }
 
@@ -232,8 +252,8 @@ __global__ void __launch_bounds__(kThreads) ring_chain_kernel(const __grid_const
                 } else {
                     asm volatile("cp.async.wait_group 0;" ::: "memory");
                 }
-                if (s == n - 2) chain_fold_staged<Ty, OP, 1>(ln, src, dst, stage[s & 1], p.divisor);
-                else chain_fold_staged<Ty, OPP, 2>(ln, src, dst, stage[s & 1], p.divisor);
+                if (s == n - 2) chain_fold_staged<Ty, OP, 1, 1>(ln, src, dst, stage[s & 1], p.divisor);
+                else chain_fold_staged<Ty, OPP, 2, 1>(ln, src, dst, stage[s & 1], p.divisor);
             }
         } else {
 #pragma unroll 1
@@ -241,15 +261,15 @@ __global__ void __launch_bounds__(kThreads) ring_chain_kernel(const __grid_const
                 const int r = wrap(k + dir * (s + 1), n), from = wrap(r - dir, n);
                 const T* src = static_cast<const T*>(p.buf[from]) + lo;
                 T* dst = static_cast<T*>(p.buf[r]) + lo;
-                if (s == n - 2) chain_fold<Ty, OP, 0>(ln, src, dst, p.divisor);
-                else chain_fold<Ty, OPP, 0>(ln, src, dst, p.divisor);
+                if (s == n - 2) chain_fold<Ty, OP, 0, 0>(ln, src, dst, p.divisor);
+                else chain_fold<Ty, OPP, 0, 0>(ln, src, dst, p.divisor);
             }
         }
         // all-gather step s: rank k + dir s copies the finished chunk from its neighbour
 #pragma unroll 1
         for (int s = 0; s < n - 1; ++s) {
             const int r = wrap(k + dir * s, n), from = wrap(r - dir, n);
-            chain_copy<Ty>(ln, static_cast<const T*>(p.buf[from]) + lo, static_cast<T*>(p.buf[r]) + lo);
+            chain_copy<Ty, WIRE ? 1 : 0>(ln, static_cast<const T*>(p.buf[from]) + lo, static_cast<T*>(p.buf[r]) + lo);
         }
     }
 }
@@ -273,8 +293,8 @@ __global__ void __launch_bounds__(kThreads) tree_chain_kernel(const __grid_const
                 // chain_fold folds src into dst with src on the left: here x_a is the left operand
                 const T* xa = static_cast<const T*>(p.buf[a]);
                 T* xb = static_cast<T*>(p.buf[a + h]);
-                if (l == levels - 1) tree_fold_pair<Ty, OP>(ln, xa, xb, static_cast<T*>(p.buf[a]), p.divisor);
-                else tree_fold_pair<Ty, OPP>(ln, xa, xb, static_cast<T*>(p.buf[a]), p.divisor);
+                if (l == levels - 1) tree_fold_pair<Ty, OP, 1>(ln, xa, xb, static_cast<T*>(p.buf[a]), p.divisor);
+                else tree_fold_pair<Ty, OPP, 1>(ln, xa, xb, static_cast<T*>(p.buf[a]), p.divisor);
             }
         }
 #pragma unroll 1
@@ -282,7 +302,7 @@ __global__ void __launch_bounds__(kThreads) tree_chain_kernel(const __grid_const
             const int h = 1 << l;
 #pragma unroll 1
             for (int a = 0; a + h < n; a += 2 * h)
-                chain_copy<Ty>(ln, static_cast<const T*>(p.buf[a]), static_cast<T*>(p.buf[a + h]));
+                chain_copy<Ty, 1>(ln, static_cast<const T*>(p.buf[a]), static_cast<T*>(p.buf[a + h]));
         }
     }
 }
