@@ -740,16 +740,21 @@ def test_bulk_copy_one_shot_shared_phase(n, dtype, off):
 
 
 @pytest.mark.parametrize("n", [3, 8])
-def test_bulk_copy_host_slices(n):
+@pytest.mark.parametrize("layout", ["aligned", "mixed"])
+def test_bulk_copy_host_slices(n, layout):
     """The host-buffer all-reduce folds each 8 MiB slice as its own launch
-    over an element range that cuts chunks: the bulk-copy fold clipped to
+    over an element range that cuts chunks: the bulk-copy fold (or, with
+    device buffers at different 16-byte phases, the staged kernel) clipped to
     [lo, hi), against the oracle's whole-buffer fold."""
     count = (8 << 20) // 4 * 2 + 4099  # three slices, the last one short
     x = synth.ranks(44 + n, n, count, "full")
     want = [a.copy() for a in x]
     oracle.fold_ring_order(want, "sum")
     host = [torch.from_numpy(a.copy()).pin_memory() for a in x]
-    dev = [torch.empty(count, device="cuda") for _ in range(n)]
+    if layout == "aligned":
+        dev = [torch.empty(count, device="cuda") for _ in range(n)]
+    else:
+        dev = [torch.empty(count + 4, device="cuda")[(3 * r + 1) % 4:][:count] for r in range(n)]
     rrv.all_reduce_host(host, dev, "sum", "oneshot")
     torch.cuda.synchronize()
     assert_bits_equal([h.numpy() for h in host], want, f"host slices n={n}")
