@@ -1,6 +1,7 @@
-// rr_mixed.cu -- the one-shot all-reduce in ring order over rank buffers
-// whose addresses differ modulo 16 bytes (views at unequal offsets): no
-// 16-byte vector of one rank lines up with the same elements of another.
+// rr_mixed.cu -- the one-shot all-reduce (ring order, its two-shot first
+// shot and bf16-wire form, and tree order) and the reduce-scatter over rank
+// buffers whose addresses differ modulo 16 bytes (views at unequal offsets):
+// no 16-byte vector of one rank lines up with the same elements of another.
 //
 // Each CTA takes one tile of one chunk.  Every rank's elements of the tile
 // are copied by cp.async into a shared-memory slot of its own, as the aligned
@@ -11,11 +12,14 @@
 // gets whole aligned 16-byte stores, every vector shifted out of two result
 // vectors to the output's phase, plus scalar stores for the elements before
 // its first 16-byte boundary and after its last whole vector.  Same bits as
-// every other one-shot (the fold, finish and rounding steps of rr_device.cuh).
+// the aligned kernels (the fold, finish and rounding steps of rr_device.cuh).
 //
 // Sources: [P4] "Collective communication primitives" (ai-infra-handbooks),
-// sections "Ring all-reduce and communication volume" and "alpha-beta model"
-// (one-shot: every rank reads every peer's buffer directly).
+// sections "The five primitives", "Ring all-reduce and communication volume"
+// and "alpha-beta model" (one-shot: every rank reads every peer's buffer
+// directly); [P3] "Training gradient sync and collective communication"
+// (geek-doc.cn), section 6 (tree order); [P1] "How all-reduce keeps every card
+// identical" (mhpq.cn), section 7.3 (low-precision gradients on the wire).
 #include "rr_bulk.cuh"
 
 namespace rr {
