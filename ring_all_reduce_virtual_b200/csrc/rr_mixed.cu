@@ -3,9 +3,10 @@
 // buffers whose addresses differ modulo 16 bytes (views at unequal offsets):
 // no 16-byte vector of one rank lines up with the same elements of another.
 //
-// Each CTA takes one tile of one chunk.  Every rank's elements of the tile
-// are copied by cp.async into a shared-memory slot of its own, as the aligned
-// 16-byte vectors that cover them (the slot remembers where the first element
+// Each CTA takes one tile of one segment (a chunk, a part, or in tree order
+// the whole buffer).  Every rank's elements of the tile are copied by
+// cp.async into a shared-memory slot of its own, as the aligned 16-byte
+// vectors that cover them (the slot remembers where the first element
 // sits); the fold takes the tile's m-th vector of elements from every slot --
 // shifted out of the two slot vectors it straddles -- in ring order and
 // writes the rounded result into a result slot, element 0 first; each output
