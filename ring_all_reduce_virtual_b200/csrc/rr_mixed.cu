@@ -50,7 +50,9 @@ struct MixedParams {
 // ring-order one-shot (rr_device.cuh).
 enum MixedMode : int { kMixedRing = 0, kMixedScatter = 1, kMixedTree = 2 };
 
-template <class Ty, int OP, int MODE, int WIRE>
+// TMAX: the most ranks a tree-mode instance folds (8 or 16; its stack holds
+// one level per power of two).
+template <class Ty, int OP, int MODE, int WIRE, int TMAX = 16>
 __global__ void __launch_bounds__(kThreads) oneshot_mixed_kernel(const __grid_constant__ MixedParams mp)
 {
     using T = typename Ty::T;
@@ -130,10 +132,10 @@ __global__ void __launch_bounds__(kThreads) oneshot_mixed_kernel(const __grid_co
             // stack whose level b holds a finished block of 2^b ranks; after
             // the last slot the blocks of the set bits of N combine from the
             // lowest level up, each higher (earlier) block on the left
-            constexpr int LV = 5;  // up to 16 ranks
+            constexpr int LV = TMAX <= 8 ? 4 : 5;  // log2(TMAX) + 1 levels
             Acc stack[LV][L];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
+            for (int j = 0; j < TMAX; ++j) {
                 if (j >= n) break;
                 Ty::unpack(slot_vec(j, m), a);
                 int lvl = 0;
@@ -242,7 +244,7 @@ namespace {
 // One CTA per (segment, tile); a segment is a chunk clipped to the launch's
 // element range (ring mode), a part (scatter mode) or the whole buffer (tree
 // mode).
-template <class Ty, int OP, int MODE, int WIRE>
+template <class Ty, int OP, int MODE, int WIRE, int TMAX = 16>
 cudaError_t launch_mixed(const RankParams& p, cudaStream_t s)
 {
     MixedParams mp{};
@@ -259,7 +261,7 @@ cudaError_t launch_mixed(const RankParams& p, cudaStream_t s)
     if (work == 0) return cudaSuccess;
     if (work > kMaxGrid) return cudaErrorInvalidValue;  // never reached: mixed_eligible caps it
     const uint32_t smem = ((uint32_t)p.n + 1u) * (mp.tv + 1u) * 16u;
-    oneshot_mixed_kernel<Ty, OP, MODE, WIRE><<<(unsigned)work, kThreads, smem, s>>>(mp);
+    oneshot_mixed_kernel<Ty, OP, MODE, WIRE, TMAX><<<(unsigned)work, kThreads, smem, s>>>(mp);
     return cudaGetLastError();
 }
 
@@ -280,7 +282,8 @@ cudaError_t launch_scatter_mixed(const RankParams& p, cudaStream_t s)
 template <class Ty, int OP>
 cudaError_t launch_tree_mixed(const RankParams& p, cudaStream_t s)
 {
-    return launch_mixed<Ty, OP, kMixedTree, 0>(p, s);
+    // a stack of 4 levels up to 8 ranks: 48 registers instead of 64 (fp32)
+    return p.n <= 8 ? launch_mixed<Ty, OP, kMixedTree, 0, 8>(p, s) : launch_mixed<Ty, OP, kMixedTree, 0, 16>(p, s);
 }
 
 cudaError_t launch_oneshot_wire_mixed(int op, const RankParams& p, cudaStream_t s)
