@@ -370,3 +370,61 @@ def test_avg_quotient_through_fp64_equals_ieee_division():
         want = a / np.float32(n)
         got = (a.astype(np.float64) * (1.0 / n)).astype(np.float32)
         assert np.array_equal(got.view(np.uint32), want.view(np.uint32)), n
+
+
+# ----------------------------------------------- the boundary from plain C --
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "rr.h"
+
+int main(void)
+{
+    /* host-only entry points of the C ABI, called from C99/C11 code */
+    if (rr_version() != RR_VERSION) return 1;
+    if (strcmp(rr_status_string(RR_OK), "ok") != 0) return 2;
+    rr_ring_event_t ev[64];
+    size_t nev = 0;
+    if (rr_ring_schedule(4, 4096, RR_F32, ev, 64, &nev) != RR_OK || nev != 2 * 3 * 4) return 3;
+    size_t sent = 0;  /* the pages' 4-rank example: 2(N-1)/N of 16 KiB per rank */
+    for (size_t i = 0; i < nev; ++i)
+        if (ev[i].rank == 0) sent += ev[i].bytes;
+    if (sent != 24576) return 4;
+    rr_cost_t cost;
+    if (rr_cost_model(RR_ALGO_RING, 8, 1.0e9, 1.0e-6, 1.0e11, &cost) != RR_OK || cost.steps != 14.0) return 5;
+    const size_t numels[4] = {100, 5000, 3, 777};
+    rr_bucket_plan_t* plan = NULL;
+    if (rr_bucket_plan(numels, 4, RR_BF16, 4096, &plan) != RR_OK || plan == NULL) return 6;
+    int first = -1, nt = -1;
+    size_t numel = 0;
+    if (rr_bucket_count(plan) < 1 || rr_bucket_info(plan, 0, &first, &nt, &numel) != RR_OK || first != 0) return 7;
+    rr_bucket_plan_free(plan);
+    if (rr_allreduce(NULL, 4, 16, RR_F32, RR_SUM, RR_ALGO_AUTO, 0) != RR_ERR_INVALID_ARG) return 8;
+    printf("c client ok\n");
+    return 0;
+}
+"""
+
+
+def test_c_client_compiles_links_and_runs_host_calls(tmp_path):
+    """The boundary is plain C: a C11 program including rr.h compiles with
+    warnings as errors, links against the library and runs the host-only
+    calls (schedule, cost model, bucket plan, argument errors)."""
+    import shutil
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    cuda_inc, cuda_lib = "/usr/local/cuda/include", "/usr/local/cuda/lib64"
+    lib_dir = os.path.dirname(_lib.LIB_PATH)
+    cmd = [gcc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+           "-I", cuda_inc, str(src), "-o", str(exe), "-L", lib_dir, "-lrr_virtual", "-L", cuda_lib, "-lcudart",
+           f"-Wl,-rpath,{lib_dir}", f"-Wl,-rpath,{cuda_lib}"]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0 and "c client ok" in run.stdout, (run.returncode, run.stderr)
