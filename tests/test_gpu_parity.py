@@ -997,3 +997,78 @@ def test_bucket_sync_bulk_path_with_heads_and_tails(n, dtype):
     for r in range(n):
         assert_bits_equal(to_host(grads[r]), want[r], f"rank {r}")
     rrv.check_timeouts()
+
+
+C_GPU_CLIENT = r"""
+#include <stdio.h>
+#include <cuda_runtime_api.h>
+#include "rr.h"
+
+/* The pages' 4-rank example from plain C: x_r = arange(4) + 10 r; the
+ * all-reduce (SUM) is [60, 64, 68, 72] on every rank, the reduce-scatter
+ * gives rank r element r of it, and the all-gather of those parts is the
+ * all-reduce again. */
+int main(void)
+{
+    enum { N = 4, C = 4 };
+    float* d[N];
+    float* part[N];
+    float* ag[N];
+    for (int r = 0; r < N; ++r) {
+        float h[C];
+        for (int i = 0; i < C; ++i) h[i] = (float)(i + 10 * r);
+        if (cudaMalloc((void**)&d[r], sizeof h) != cudaSuccess) return 1;
+        if (cudaMalloc((void**)&part[r], sizeof(float)) != cudaSuccess) return 1;
+        if (cudaMalloc((void**)&ag[r], sizeof h) != cudaSuccess) return 1;
+        cudaMemcpy(d[r], h, sizeof h, cudaMemcpyHostToDevice);
+    }
+    if (rr_reduce_scatter((const void* const*)d, (void* const*)part, N, 1, RR_F32, RR_SUM, RR_ALGO_AUTO, 0) != RR_OK)
+        return 2;
+    if (rr_allreduce((void* const*)d, N, C, RR_F32, RR_SUM, RR_ALGO_RING, 0) != RR_OK) return 3;
+    if (rr_all_gather((const void* const*)part, (void* const*)ag, N, 1, RR_F32, RR_ALGO_AUTO, 0) != RR_OK) return 4;
+    if (cudaDeviceSynchronize() != cudaSuccess) return 5;
+    const float want[C] = {60.f, 64.f, 68.f, 72.f};
+    for (int r = 0; r < N; ++r) {
+        float h[C], g[C], p;
+        cudaMemcpy(h, d[r], sizeof h, cudaMemcpyDeviceToHost);
+        cudaMemcpy(g, ag[r], sizeof g, cudaMemcpyDeviceToHost);
+        cudaMemcpy(&p, part[r], sizeof p, cudaMemcpyDeviceToHost);
+        for (int i = 0; i < C; ++i)
+            if (h[i] != want[i] || g[i] != want[i]) return 6;
+        if (p != want[r]) return 7;
+        cudaFree(d[r]);
+        cudaFree(part[r]);
+        cudaFree(ag[r]);
+    }
+    printf("c gpu client ok\n");
+    return 0;
+}
+"""
+
+
+def test_c_client_reproduces_the_four_rank_example(tmp_path):
+    """The boundary from plain C on the GPU (no Python, no torch): cudaMalloc'd
+    rank buffers, the ring all-reduce, reduce-scatter and all-gather of the
+    pages' 4-rank worked example."""
+    import os
+    import shutil
+    import subprocess
+
+    from ring_all_reduce_virtual_b200 import _lib
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "client_gpu.c"
+    src.write_text(C_GPU_CLIENT)
+    exe = tmp_path / "client_gpu"
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    lib_dir = os.path.dirname(_lib.LIB_PATH)
+    cuda_lib = "/usr/local/cuda/lib64"
+    r = subprocess.run([gcc, "-std=c11", "-Wall", "-Werror", "-I", os.path.join(root, "include"),
+                        "-I", "/usr/local/cuda/include", str(src), "-o", str(exe), "-L", lib_dir, "-lrr_virtual",
+                        "-L", cuda_lib, "-lcudart", f"-Wl,-rpath,{lib_dir}", f"-Wl,-rpath,{cuda_lib}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0 and "c gpu client ok" in run.stdout, (run.returncode, run.stdout, run.stderr)
